@@ -1,0 +1,184 @@
+/*
+ * pararnn.h -- C ABI of the B200 (sm_100a) ParaGRU / ParaLSTM Newton-scan
+ * solver.
+ *
+ * The problem (from "Параллельность RNN?", §1.1): given the initial state s_0
+ * and the inputs, the states s_1..s_T of the recurrence s_t = f(s_{t-1}, x_t)
+ * are the unique root of the residual r_t = s_t - f(s_{t-1}, x_t).  The
+ * solvers find it by Newton iterations (§1.2) whose linear systems have a
+ * block-bidiagonal Jacobian (§1.3); each system is the linear recurrence
+ * ds_t = A_t ds_{t-1} - r_t, solved by an associative scan over affine pairs
+ * (A, b) (§1.3, "Уровень 2").  The cells have diagonal recurrent weights, so
+ * A_t is diagonal for ParaGRU and 2x2 block-diagonal per channel for ParaLSTM
+ * ("Apple научила классические RNN масштабироваться до 7B параметров...",
+ * "Что именно сделали технически", item 3).  The interface mirrors the
+ * pages' step signature recurrence_step(h, x, system_parameters) ("Как
+ * запустить"): x is the precomputed gate input projection u, the system
+ * parameters are the diagonal weights a and the biases.
+ *
+ * Cells (every product is elementwise; sig = logistic sigmoid):
+ *   ParaGRU  gates (z, r, c):
+ *     z = sig(a_z h + u_z + b_z)   r = sig(a_r h + u_r + b_r)
+ *     c = tanh(a_c (r h) + u_c + b_c)          h' = (1 - z) h + z c
+ *   ParaLSTM gates (i, f, g, o), state (c, h):
+ *     i = sig(a_i h + u_i + b_i)   f = sig(a_f h + u_f + b_f)
+ *     g = tanh(a_g h + u_g + b_g)  o = sig(a_o h + u_o + b_o)
+ *     c' = f c + i g               h' = o tanh(c')
+ *
+ * Layouts (row-major, channel index d fastest, all contiguous):
+ *   u        [B][T][G][D]  G = 3 (GRU) or 4 (LSTM); bf16 or fp32
+ *   a, bias  [G][D]        fp32
+ *   h0, c0   [B][D]        fp32
+ *   h, c     [B][T][D]     fp32, state after step t at index t-1
+ *   dLdh     [B][T][D]     fp32
+ *   du       [B][T][G][D]  fp32
+ *   da,dbias [G][D]        fp32
+ *
+ * Conventions shared by every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory and keeps no global state.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Device-written results (states, stats, status) are
+ *     valid once the stream reaches that point; reading them is the caller's
+ *     synchronisation.
+ *   - Host-detectable errors return a negative PARARNN_ERR_* code before any
+ *     work is enqueued.  Outcomes decided on the device go to a status word.
+ *   - Requirements: B, T, D >= 1; D % 8 == 0; u, h, c, du, dLdh 16-byte
+ *     aligned; a, bias, h0, c0, da, dbias, dc0, dh0 4-byte aligned.
+ *   - The workspace: size from pararnn_workspace_size(); it must be
+ *     zero-filled once before its first use (pararnn_workspace_init), after
+ *     which the library keeps it consistent across calls (each call bumps an
+ *     epoch counter stored in it).  One call at a time may use a workspace.
+ *   - No entry point traps, asserts or waits without bound on the device:
+ *     every cross-block wait gives up after opts.timeout_us microseconds and
+ *     reports PARARNN_STATUS_TIMEOUT.
+ */
+#ifndef PARARNN_H
+#define PARARNN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including CUDA headers */
+typedef struct CUstream_st* pararnn_stream_t;
+
+/* element type of u */
+enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 };
+/* cell selector */
+enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
+
+/* host return codes */
+#define PARARNN_OK 0
+#define PARARNN_ERR_INVALID_ARG (-1)
+#define PARARNN_ERR_UNSUPPORTED_DTYPE (-2)
+#define PARARNN_ERR_WORKSPACE_TOO_SMALL (-3)
+#define PARARNN_ERR_CUDA (-4)
+#define PARARNN_ERR_MISALIGNED (-5)
+#define PARARNN_ERR_TOO_LARGE (-6)
+
+/* device status word values (pararnn_stats.status, adjoint *status) */
+#define PARARNN_STATUS_CONVERGED 0
+#define PARARNN_STATUS_NOT_CONVERGED 1
+#define PARARNN_STATUS_NONFINITE 2
+#define PARARNN_STATUS_TIMEOUT 3
+
+/* opts.flags */
+#define PARARNN_FLAG_INJECT_WITHHOLD 1u /* testing: chunk `inject_chunk` never
+                                           publishes its look-back record */
+
+typedef struct {
+  float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
+  int max_iters;      /* cap on Newton updates; <= 0 -> 64 (the workspace is
+                         sized for this value) */
+  unsigned flags;     /* PARARNN_FLAG_* */
+  int inject_chunk;   /* chunk index for PARARNN_FLAG_INJECT_WITHHOLD */
+  unsigned timeout_us;/* bound on any cross-block wait; 0 -> 2,000,000 */
+  int max_cluster;    /* cap on CTAs per thread-block cluster (2..16);
+                         0 -> the largest the device can keep resident */
+} pararnn_opts;
+
+/* Device-resident solve statistics (written by the solve; zeroed by it at
+ * the start of the call). */
+typedef struct {
+  int iters;          /* Newton updates applied (max over sequence chunks) */
+  float max_residual; /* max|r| at the last evaluated iterate, before the
+                         final update (max over chunks) */
+  int status;         /* PARARNN_STATUS_* (max over chunks) */
+  int evals;          /* cell evaluations per element (max over chunks) */
+} pararnn_stats;
+
+/* Bytes of workspace a call needs.  `adjoint` = 0 for the forward solves,
+ * 1 for pararnn_adjoint.  max_iters as in pararnn_opts (<= 0 -> default).
+ * Returns 0 on invalid sizes. */
+size_t pararnn_workspace_size(int cell, int B, int T, int D, int max_iters,
+                              int adjoint);
+
+/* Zero-fill a workspace (stream-ordered).  Needed once before first use. */
+int pararnn_workspace_init(void* workspace, size_t ws_bytes,
+                           pararnn_stream_t stream);
+
+/* ParaGRU forward solve.
+ * In:  u [B][T][3][D] (z, r, c projections; dtype u_dtype), a [3][D],
+ *      bias [3][D] or NULL (zeros), h0 [B][D] or NULL (zeros).
+ * Out: h [B][T][D] states; *stats (device); iter_hist [max_iters+2] or NULL:
+ *      iter_hist[k], k <= max_iters, counts the (b, d) channels whose own
+ *      max_t |r_t| is below tol from evaluation k onwards (k = updates applied
+ *      before that evaluation); iter_hist[max_iters+1] counts channels that
+ *      never got there within the cap.
+ * Newton starts from h = 0 at every t, applies the page's update until the
+ * residual of an iterate is below tol everywhere upstream (and then applies
+ * that last update), or until max_iters updates have been applied. */
+int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
+                      const float* bias, const float* h0, float* h, int B,
+                      int T, int D, const pararnn_opts* opts,
+                      pararnn_stats* stats, int* iter_hist, void* workspace,
+                      size_t ws_bytes, pararnn_stream_t stream);
+
+/* ParaLSTM forward solve.  As pararnn_gru_solve with u [B][T][4][D]
+ * (i, f, g, o), a/bias [4][D], initial cell state c0 (NULL = zeros) and both
+ * state trajectories out: c [B][T][D], h [B][T][D].  The residual norm is the
+ * max over both components. */
+int pararnn_lstm_solve(const void* u, int u_dtype, const float* a,
+                       const float* bias, const float* c0, const float* h0,
+                       float* c, float* h, int B, int T, int D,
+                       const pararnn_opts* opts, pararnn_stats* stats,
+                       int* iter_hist, void* workspace, size_t ws_bytes,
+                       pararnn_stream_t stream);
+
+/* Adjoint (backward) of a solved trajectory: the reverse scan
+ *   lambda_t = g_t + A_{t+1}^T lambda_{t+1},  lambda_T = g_T
+ * on the transposed Jacobians (Jacobian structure from "Параллельность
+ * RNN?", §1.3), with g_t = dL/dh_t (dL/dc_t = 0 for ParaLSTM).  Outputs
+ *   du_t = (df_t/du_t)^T lambda_t                [B][T][G][D]
+ *   da   = sum_{b,t} (df_t/da)^T lambda_t        [G][D]
+ *   dbias= sum_{b,t} du_t  (NULL to skip)        [G][D]
+ *   dh0  = d L / d h0, dc0 = d L / d c0 (LSTM; NULL to skip) [B][D]
+ * c0 and c must be NULL for ParaGRU and non-NULL for ParaLSTM.  The sums over
+ * (b, t) are reduced in a fixed order (bitwise reproducible).
+ * *status (device int) receives PARARNN_STATUS_CONVERGED (0) on success,
+ * NONFINITE or TIMEOUT otherwise. */
+int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
+                    const float* bias, const float* c0, const float* h0,
+                    const float* c, const float* h, const float* dLdh,
+                    float* du, float* da, float* dbias, float* dc0, float* dh0,
+                    int B, int T, int D, int* status, void* workspace,
+                    size_t ws_bytes, pararnn_stream_t stream);
+
+/* Naive step-by-step GPU evaluation (one thread per (b, d) channel looping
+ * over t) -- the sequential baseline the parallel solve is compared with.
+ * c0/c must be NULL for ParaGRU.  No workspace. */
+int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a,
+                         const float* bias, const float* c0, const float* h0,
+                         float* c, float* h, int B, int T, int D,
+                         pararnn_stream_t stream);
+
+/* Human-readable text for a return code. */
+const char* pararnn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PARARNN_H */

@@ -1,0 +1,311 @@
+// api.cu -- the C ABI (include/pararnn.h): argument checks, workspace layout,
+// TMA descriptors and kernel launches.  Host code only; every step of the
+// solve runs in the kernels.
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace pararnn {
+int launch_gru_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
+                   cudaStream_t stream);
+int gru_chunk_steps();
+int gru_max_cluster(bool bf16);
+int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
+                    cudaStream_t stream);
+int lstm_chunk_steps();
+int lstm_max_cluster(bool bf16);
+int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, const float* bias,
+                        const float* c0, const float* h0, float* c, float* h, int B, int T,
+                        int D, cudaStream_t stream);
+struct AdjParams;
+int adjoint_chunk_steps(int cell);
+size_t adjoint_ws_bytes(int cell, int B, int T, int D);
+int launch_adjoint(int cell, bool bf16, const CUtensorMap& tmap_u, const void* u, const float* a,
+                   const float* bias, const float* c0, const float* h0, const float* c,
+                   const float* h, const float* dLdh, float* du, float* da, float* dbias,
+                   float* dc0, float* dh0, int B, int T, int D, int* status, void* ws,
+                   cudaStream_t stream);
+}  // namespace pararnn
+
+using namespace pararnn;
+
+namespace {
+
+constexpr int kDefaultMaxIters = 64;
+constexpr float kDefaultTol = 1e-6f;
+constexpr unsigned kDefaultTimeoutUs = 2000000u;
+constexpr int kMaxItersLimit = 1 << 16;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cdiv(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+int resolve_max_iters(int m) { return m <= 0 ? kDefaultMaxIters : m; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Tensor map over u [B][T][G][D] with a box of 32 channels x G gates x tc steps.
+int make_u_map(CUtensorMap* map, const void* u, bool bf16, int B, int T, int G, int D, int tc) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return PARARNN_ERR_CUDA;
+  const cuuint64_t es = bf16 ? 2 : 4;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {D * es, (cuuint64_t)G * D * es, (cuuint64_t)T * G * D * es};
+  cuuint32_t box[4] = {(cuuint32_t)kChan, (cuuint32_t)G, (cuuint32_t)tc, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                  const_cast<void*>(u), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+int check_sizes(int B, int T, int D) {
+  if (B < 1 || T < 1 || D < 1 || (D % 8) != 0) return PARARNN_ERR_INVALID_ARG;
+  if ((long long)B * T * D > (1LL << 40)) return PARARNN_ERR_TOO_LARGE;
+  return PARARNN_OK;
+}
+
+int rec_floats(int cell) { return cell == PARARNN_GRU ? 4 : 8; }
+
+int chunk_steps(int cell) { return cell == PARARNN_GRU ? gru_chunk_steps() : lstm_chunk_steps(); }
+
+// Records are kept per cluster chunk; the workspace is sized for clusters of
+// at least kMinCluster CTAs (the launch checks the size it actually needs).
+constexpr int kMinCluster = 8;
+
+long long cluster_chunks(int cell, int B, int T, int D, int CL) {
+  const int nC = cdiv(T, chunk_steps(cell));
+  const int cl = std::min(nC, CL);
+  return (long long)B * cdiv(D, kChan) * cdiv(nC, cl);
+}
+
+size_t fwd_ws(int cell, int B, int T, int D, int max_iters) {
+  return fwd_ws_layout((size_t)cluster_chunks(cell, B, T, D, kMinCluster), max_iters,
+                       rec_floats(cell), (size_t)B * D)
+      .total;
+}
+
+// Largest usable cluster size for a cell's kernel on the current device.
+int max_cluster(int cell, bool bf16) {
+  static int cache[2][2][64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int& c = cache[cell][bf16 ? 1 : 0][dev];
+  if (c == 0) c = cell == PARARNN_GRU ? gru_max_cluster(bf16) : lstm_max_cluster(bf16);
+  return c;
+}
+
+__global__ void fwd_init_kernel(WsHeader* hdr, pararnn_stats* stats, int* chan_k, size_t nch,
+                                int* hist, int nhist) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    unsigned e = (hdr->epoch + 1u) & 0x1fffffffu;
+    if (e == 0u) e = 1u;
+    hdr->epoch = e;
+    hdr->ticket = 0u;
+    stats->iters = 0;
+    stats->max_residual = 0.f;
+    stats->status = 0;
+    stats->evals = 0;
+  }
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (chan_k)
+    for (size_t i = i0; i < nch; i += stride) chan_k[i] = 0;
+  if (hist)
+    for (size_t i = i0; i < (size_t)nhist; i += stride) hist[i] = 0;
+}
+
+__global__ void hist_kernel(const int* __restrict__ chan_k, size_t n, int* hist, int max_iters) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  int k = chan_k[i];
+  if (k > max_iters) k = max_iters + 1;  // never below tol within the cap
+  atomicAdd(&hist[k], 1);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA; }
+
+int forward(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+            const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
+            const pararnn_opts* opts, pararnn_stats* stats, int* iter_hist, void* workspace,
+            size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_sizes(B, T, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  if (!u || !a || !h || !stats || !workspace) return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_LSTM && !c) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(u, 16) || !aligned(h, 16) || (c && !aligned(c, 16)) || !aligned(a, 4) ||
+      (bias && !aligned(bias, 4)) || (h0 && !aligned(h0, 4)) || (c0 && !aligned(c0, 4)) ||
+      !aligned(stats, 4) || !aligned(workspace, 256) || (iter_hist && !aligned(iter_hist, 4)))
+    return PARARNN_ERR_MISALIGNED;
+  const float tol = (opts && opts->tol > 0.f) ? opts->tol : kDefaultTol;
+  const int max_iters = resolve_max_iters(opts ? opts->max_iters : 0);
+  if (max_iters > kMaxItersLimit) return PARARNN_ERR_INVALID_ARG;
+  const int G = cell == PARARNN_GRU ? 3 : 4;
+  const int tc = chunk_steps(cell);
+  const int nDT = cdiv(D, kChan), nC = cdiv(T, tc);
+  int clmax = max_cluster(cell, u_dtype == PARARNN_BF16);
+  if (clmax <= 0) return PARARNN_ERR_CUDA;
+  if (opts && opts->max_cluster > 0) clmax = std::min(clmax, opts->max_cluster);
+  const int CL = std::min(nC, clmax);
+  const int nCC = cdiv(nC, CL);
+  const long long nctas = (long long)B * nDT * nCC * CL;
+  if (nctas >= (1LL << 31)) return PARARNN_ERR_TOO_LARGE;
+  const long long ncc = (long long)B * nDT * nCC;
+  const FwdWsLayout L = fwd_ws_layout((size_t)ncc, max_iters, rec_floats(cell), (size_t)B * D);
+  if (ws_bytes < L.total) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
+
+  CUtensorMap map;
+  rc = make_u_map(&map, u, u_dtype == PARARNN_BF16, B, T, G, D, tc);
+  if (rc) return rc;
+
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  FwdParams p;
+  p.a = a;
+  p.bias = bias;
+  p.h0 = h0;
+  p.c0 = c0;
+  p.h = h;
+  p.c = c;
+  p.B = B;
+  p.T = T;
+  p.D = D;
+  p.nDT = nDT;
+  p.nC = nC;
+  p.CL = CL;
+  p.nCC = nCC;
+  p.max_iters = max_iters;
+  p.tol = tol;
+  p.flags = opts ? opts->flags : 0u;
+  p.inject_chunk = opts ? opts->inject_chunk : -1;
+  p.timeout_ns = 1000ull * ((opts && opts->timeout_us) ? opts->timeout_us : kDefaultTimeoutUs);
+  p.hdr = reinterpret_cast<WsHeader*>(ws);
+  p.rec_flags = reinterpret_cast<unsigned*>(ws + L.flags);
+  p.rec_vals = reinterpret_cast<float*>(ws + L.vals);
+  p.chan_k = iter_hist ? reinterpret_cast<int*>(ws + L.chan_k) : nullptr;
+  p.stats = stats;
+
+  const size_t nch = (size_t)B * D;
+  const int nhist = max_iters + 2;
+  const unsigned igrid = iter_hist ? (unsigned)std::min<size_t>((nch + 255) / 256, 1024) : 1u;
+  fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
+  if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+  const int e = cell == PARARNN_GRU
+                    ? launch_gru_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream)
+                    : launch_lstm_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream);
+  if (e != 0) return PARARNN_ERR_CUDA;
+  if (iter_hist) {
+    hist_kernel<<<(unsigned)((nch + 255) / 256), 256, 0, stream>>>(p.chan_k, nch, iter_hist,
+                                                                     max_iters);
+    if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+  }
+  return PARARNN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pararnn_workspace_size(int cell, int B, int T, int D, int max_iters, int adjoint) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return 0;
+  if (check_sizes(B, T, D) != PARARNN_OK) return 0;
+  if (adjoint) return adjoint_ws_bytes(cell, B, T, D);
+  const int m = resolve_max_iters(max_iters);
+  if (m > kMaxItersLimit) return 0;
+  return fwd_ws(cell, B, T, D, m);
+}
+
+int pararnn_workspace_init(void* workspace, size_t ws_bytes, pararnn_stream_t stream) {
+  if (!workspace) return PARARNN_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+int pararnn_gru_solve(const void* u, int u_dtype, const float* a, const float* bias,
+                      const float* h0, float* h, int B, int T, int D, const pararnn_opts* opts,
+                      pararnn_stats* stats, int* iter_hist, void* workspace, size_t ws_bytes,
+                      pararnn_stream_t stream) {
+  return forward(PARARNN_GRU, u, u_dtype, a, bias, nullptr, h0, nullptr, h, B, T, D, opts, stats,
+                 iter_hist, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+int pararnn_lstm_solve(const void* u, int u_dtype, const float* a, const float* bias,
+                       const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
+                       const pararnn_opts* opts, pararnn_stats* stats, int* iter_hist,
+                       void* workspace, size_t ws_bytes, pararnn_stream_t stream) {
+  return forward(PARARNN_LSTM, u, u_dtype, a, bias, c0, h0, c, h, B, T, D, opts, stats, iter_hist,
+                 workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+                    const float* c0, const float* h0, const float* c, const float* h,
+                    const float* dLdh, float* du, float* da, float* dbias, float* dc0, float* dh0,
+                    int B, int T, int D, int* status, void* workspace, size_t ws_bytes,
+                    pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, T, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  if (!u || !a || !h || !dLdh || !du || !da || !status || !workspace)
+    return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_LSTM && !c) return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_GRU && (c || c0 || dc0)) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(u, 16) || !aligned(h, 16) || !aligned(dLdh, 16) || !aligned(du, 16) ||
+      (c && !aligned(c, 16)) || !aligned(a, 4) || !aligned(da, 4) || (bias && !aligned(bias, 4)) ||
+      (dbias && !aligned(dbias, 4)) || (h0 && !aligned(h0, 4)) || (c0 && !aligned(c0, 4)) ||
+      (dh0 && !aligned(dh0, 4)) || (dc0 && !aligned(dc0, 4)) || !aligned(status, 4) ||
+      !aligned(workspace, 256))
+    return PARARNN_ERR_MISALIGNED;
+  if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
+  const int G = cell == PARARNN_GRU ? 3 : 4;
+  CUtensorMap map;
+  rc = make_u_map(&map, u, u_dtype == PARARNN_BF16, B, T, G, D, adjoint_chunk_steps(cell));
+  if (rc) return rc;
+  const int e = launch_adjoint(cell, u_dtype == PARARNN_BF16, map, u, a, bias, c0, h0, c, h, dLdh,
+                               du, da, dbias, dc0, dh0, B, T, D, status, workspace,
+                               (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+                         const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
+                         pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, T, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  if (!u || !a || !h || (cell == PARARNN_LSTM && !c)) return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_GRU && (c || c0)) return PARARNN_ERR_INVALID_ARG;
+  const int e = launch_seq_baseline(cell, u_dtype == PARARNN_BF16, u, a, bias, c0, h0, c, h, B, T,
+                                    D, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+const char* pararnn_strerror(int code) {
+  switch (code) {
+    case PARARNN_OK: return "ok";
+    case PARARNN_ERR_INVALID_ARG: return "invalid argument (null pointer, size or cell)";
+    case PARARNN_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype for u (want f32 or bf16)";
+    case PARARNN_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than pararnn_workspace_size()";
+    case PARARNN_ERR_CUDA: return "CUDA error while setting up or launching a kernel";
+    case PARARNN_ERR_MISALIGNED: return "pointer misaligned (16 B for tensors, 4 B for vectors)";
+    case PARARNN_ERR_TOO_LARGE: return "problem too large for the index types";
+    default: return "unknown pararnn error code";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,166 @@
+// common.cuh -- device helpers shared by the solver kernels (sm_100a only).
+//
+// PTX wrappers for the special-function unit, NaN-propagating max, the
+// acquire/release flag protocol of the cross-block look-back, mbarriers and
+// TMA bulk-tensor loads, plus the workspace layout the host and the kernels
+// agree on.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pararnn.h"
+
+namespace pararnn {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kChan = 32;  // channels per tile (one warp width)
+
+// ------------------------------------------------------------ arithmetic --
+// 2^x on the MUFU pipe (ftz).  Saturates to +inf / 0.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 1/x on the MUFU pipe (ftz); rcp(inf) = 0.
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// max that returns NaN if either operand is NaN (so a NaN residual can never
+// look converged).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
+
+// ------------------------------------------------------- memory ordering --
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ float2 ld_relaxed_f2(const float2* p) {
+  float2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];"
+               : "=f"(v.x), "=f"(v.y) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_relaxed_f4(const float4* p) {
+  float4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ------------------------------------------------------ mbarrier and TMA --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on an mbarrier phase; false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity,
+                                                  uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+// 4-D tiled bulk-tensor load (no multicast) completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// ------------------------------------------------------------ workspace --
+// Forward-solve workspace:
+//   [0, 256)           header: epoch, ticket counter
+//   flags  u32 [nrec]  look-back record flags, nrec = cluster chunks * (max_iters+1)
+//   vals   f32 [nrec][kChan][RW]  record payload (RW floats per channel)
+//   chan_k int [B*D]   per-channel convergence iterate (histogram input)
+// A record flag is (epoch << 3) | (kind << 1) | ok.
+struct WsHeader {
+  unsigned epoch;
+  unsigned ticket;
+  unsigned pad[62];
+};
+enum : unsigned { kRecAgg = 1, kRecIncl = 2 };
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct FwdWsLayout {
+  size_t flags, vals, chan_k, total;
+};
+__host__ __device__ inline FwdWsLayout fwd_ws_layout(size_t nchunks, int max_iters, int rec_floats,
+                                                     size_t BD) {
+  FwdWsLayout L;
+  size_t nrec = nchunks * (size_t)(max_iters + 1);
+  L.flags = 256;
+  L.vals = L.flags + align256(nrec * 4);
+  L.chan_k = L.vals + align256(nrec * kChan * rec_floats * 4);
+  L.total = L.chan_k + align256(BD * 4);
+  return L;
+}
+
+// Everything a forward-solve kernel needs besides the tensor map.
+struct FwdParams {
+  const float* a;     // [G][D]
+  const float* bias;  // [G][D] or null
+  const float* h0;    // [B][D] or null
+  const float* c0;    // [B][D] or null (LSTM)
+  float* h;           // [B][T][D]
+  float* c;           // [B][T][D] (LSTM)
+  int B, T, D;
+  int nDT;            // channel tiles per batch row: ceil(D / 32)
+  int nC;             // sequence chunks (CTAs) per tile
+  int CL;             // CTAs per cluster (consecutive chunks of one tile)
+  int nCC;            // cluster chunks per tile: ceil(nC / CL)
+  int max_iters;
+  float tol;
+  unsigned flags;
+  int inject_chunk;
+  uint64_t timeout_ns;
+  WsHeader* hdr;
+  unsigned* rec_flags;
+  float* rec_vals;
+  int* chan_k;        // [B*D] or null
+  pararnn_stats* stats;
+};
+
+}  // namespace pararnn

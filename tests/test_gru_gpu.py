@@ -1,0 +1,158 @@
+"""GPU parity of the fused ParaGRU Newton-scan solve against the fp64 oracle.
+
+States must match the sequential fp64 recurrence within max-abs 1e-4
+(fp32 state, fp32 or bf16 inputs).  Inputs are the seeded synthetic ones
+both sides read (bf16 values widen exactly to fp64 for the oracle).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nonlinear_rnn_paragru_b200 as pr
+from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_STATE = 1e-4
+
+
+def _solve(x, **kw):
+    dev = "cuda"
+    u = x["u"].to(dev)
+    a = x["a"].to(dev)
+    bias = x["bias"].to(dev)
+    h0 = x["h0"].to(dev)
+    h, stats, hist = pr.gru_solve(u, a, bias, h0, **kw)
+    torch.cuda.synchronize()
+    return h.cpu().numpy(), pr.read_stats(stats), (hist.cpu().numpy() if hist is not None else None)
+
+
+def _ref(x):
+    return oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+
+
+def test_config1_full(cuda_ok):
+    w = WORKLOADS[1]
+    x = make_inputs(w)
+    h, st, _ = _solve(x, max_iters=w.T)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, err
+    assert st["status"] == "converged" and st["max_residual"] < 1e-6
+    assert 1 <= st["iters"] <= 12
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 1000, 96), (1, 257, 64), (3, 256, 32),
+                                   (1, 1, 8), (2, 5, 40), (1, 2049, 128)])
+def test_ragged_shapes_bf16(cuda_ok, B, T, D):
+    x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
+    h, st, _ = _solve(x)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, (err, st)
+    assert st["status"] == "converged"
+
+
+@pytest.mark.parametrize("B,T,D", [(1, 3000, 64), (2, 700, 48)])
+def test_long_fp32(cuda_ok, B, T, D):
+    x = make_inputs(WORKLOADS[4].scaled(B=B, T=T, D=D))
+    h, st, hist = _solve(x, hist=True)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, (err, st)
+    assert hist.sum() == B * D
+    assert hist[-1] == 0   # every channel converged within the cap
+
+
+def test_nonzero_h0(cuda_ok):
+    x = make_inputs(WORKLOADS[2].scaled(B=2, T=600, D=64))
+    x["h0"] = torch.randn((2, 64), generator=torch.Generator().manual_seed(5)) * 0.5
+    h, st, _ = _solve(x)
+    assert np.abs(h - _ref(x)).max() < TOL_STATE
+
+
+def test_config2_full_size(cuda_ok):
+    w = WORKLOADS[2]
+    x = make_inputs(w)
+    h, st, _ = _solve(x)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, (err, st)
+    assert st["status"] == "converged"
+    assert st["max_residual"] < 1e-6
+
+
+def test_residual_of_result_is_small(cuda_ok):
+    # property that holds at any size: the returned trajectory's residual
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=4096, D=256))
+    h, st, _ = _solve(x)
+    res = oracle.gru_residual(x["u"], x["a"], x["bias"], x["h0"], h)
+    assert np.abs(res).max() < 2e-6
+
+
+def test_iteration_histogram_matches_oracle_counts(cuda_ok):
+    x = make_inputs(WORKLOADS[4].scaled(B=1, T=2048, D=64))
+    _, st, hist = _solve(x, hist=True, max_iters=32)
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=32)
+    # counts are reported, not asserted equal: fp32 vs fp64 may differ by one
+    ks = np.nonzero(hist)[0]
+    assert ks.max() <= r["chan_k"].max() + 1
+    assert abs(st["evals"] - (r["iters"] + 1)) <= 1
+
+
+@pytest.mark.parametrize("n", [1, 2, 3])
+def test_capped_iterates_match_oracle_newton(cuda_ok, n):
+    # with the cap at n updates the solver returns the n-th Newton iterate
+    # (states after n updates of the page's scheme) and NOT_CONVERGED
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=1300, D=64))
+    h, st, _ = _solve(x, max_iters=n)
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=n)
+    assert st["status"] == "not_converged"
+    assert st["iters"] == n and st["evals"] == n + 1
+    assert np.abs(h - r["h"]).max() < TOL_STATE
+    assert st["max_residual"] == pytest.approx(r["trace"][n], rel=1e-2)
+
+
+def test_withheld_record_times_out_without_hanging(cuda_ok):
+    # host-injected fault: cluster chunk 0 of the first tile never publishes
+    # (T = 5000 needs two 16-CTA cluster chunks), so its successor's bounded
+    # wait expires and the solve reports TIMEOUT.
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=5000, D=32))
+    opts = pr._opts(1e-6, 16, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD,
+                    inject_chunk=0, timeout_us=20000)
+    h, st, _ = _solve(x, max_iters=16, opts=opts)
+    assert st["status"] == "timeout"
+    # and the context is still usable
+    h2, st2, _ = _solve(x, max_iters=16)
+    assert st2["status"] == "converged"
+
+
+def test_seq_baseline_matches_oracle(cuda_ok):
+    x = make_inputs(WORKLOADS[2].scaled(B=2, T=512, D=64))
+    _, h = pr.seq_baseline(pr.PARARNN_GRU, x["u"].cuda(), x["a"].cuda(),
+                           x["bias"].cuda(), None, x["h0"].cuda())
+    torch.cuda.synchronize()
+    assert np.abs(h.cpu().numpy() - _ref(x)).max() < TOL_STATE
+
+
+def test_repeat_calls_reuse_workspace(cuda_ok):
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=1500, D=64))
+    ws = pr.Workspace("cuda")
+    outs = []
+    for _ in range(3):
+        h, st, _ = _solve(x, workspace=ws)
+        outs.append(h)
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
+
+
+def test_multi_cluster_lookback_fp32(cuda_ok):
+    # T spans several 16-CTA cluster chunks: exercises the cross-cluster
+    # decoupled look-back (plus a ragged tail chunk).
+    x = make_inputs(WORKLOADS[4].scaled(B=1, T=20000, D=64))
+    h, st, hist = _solve(x, hist=True)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, (err, st)
+    assert st["status"] == "converged"
+
+
+def test_binding_rejects_wrong_dtype(cuda_ok):
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=64, D=32))
+    with pytest.raises(TypeError):
+        pr.gru_solve(x["u"].cuda(), x["a"].double().cuda(), None, None)

@@ -12,7 +12,6 @@ import torch
 import oracle
 from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs
 
-torch.set_default_dtype(torch.float64)
 
 
 def _rand_gru(B, T, D, seed, a_range=1.0, bias_std=0.3):
@@ -41,8 +40,8 @@ def _torch_gru_cell(a, D):
     gate is 1 - z, so its z-row carries -a_z and the input -(u_z + b_z))."""
     cell = torch.nn.GRUCell(3 * D, D, bias=False, dtype=torch.float64)
     with torch.no_grad():
-        cell.weight_ih.copy_(torch.eye(3 * D))     # gate rows r, z, n
-        whh = torch.zeros(3 * D, D)
+        cell.weight_ih.copy_(torch.eye(3 * D, dtype=torch.float64))     # gate rows r, z, n
+        whh = torch.zeros(3 * D, D, dtype=torch.float64)
         a = torch.as_tensor(a)
         whh[0:D] = torch.diag(a[1])        # r
         whh[D:2 * D] = torch.diag(-a[0])   # torch z = 1 - our z
@@ -73,8 +72,8 @@ def _torch_gru_seq(u, a, bias, h0):
 def _torch_lstm_cell(a, D):
     cell = torch.nn.LSTMCell(4 * D, D, bias=False, dtype=torch.float64)
     with torch.no_grad():
-        cell.weight_ih.copy_(torch.eye(4 * D))     # gate rows i, f, g, o
-        whh = torch.zeros(4 * D, D)
+        cell.weight_ih.copy_(torch.eye(4 * D, dtype=torch.float64))     # gate rows i, f, g, o
+        whh = torch.zeros(4 * D, D, dtype=torch.float64)
         a = torch.as_tensor(a)
         for q in range(4):
             whh[q * D:(q + 1) * D] = torch.diag(a[q])
@@ -192,7 +191,7 @@ def _gru_functional(h, u, a, b):
     D = h.shape[1]
     w_hh = torch.cat([torch.diag(a[1]), torch.diag(-a[0]), torch.diag(a[2])])
     x = torch.cat([u[:, 1] + b[1], -(u[:, 0] + b[0]), u[:, 2] + b[2]], dim=1)
-    return torch._VF.gru_cell(x, h, torch.eye(3 * D), w_hh, None, None)
+    return torch._VF.gru_cell(x, h, torch.eye(3 * D, dtype=torch.float64), w_hh, None, None)
 
 
 def test_lstm_step_derivatives_vs_central_differences():
@@ -262,7 +261,7 @@ def test_lstm_bptt_vs_torch_autograd():
     hs = []
     for t in range(T):
         xt = (u[:, t] + b).reshape(B, 4 * D)
-        hh, cc = torch._VF.lstm_cell(xt, (hh, cc), torch.eye(4 * D), w_hh, None, None)
+        hh, cc = torch._VF.lstm_cell(xt, (hh, cc), torch.eye(4 * D, dtype=torch.float64), w_hh, None, None)
         hs.append(hh)
     L = (torch.stack(hs, 1) * torch.tensor(g)).sum()
     gu, ga, gb, gc0, gh0 = torch.autograd.grad(L, (u, a, b, c0, h0))
