@@ -80,7 +80,7 @@ int check_sizes(int B, int T, int D) {
   return PARARNN_OK;
 }
 
-int rec_floats(int cell) { return cell == PARARNN_GRU ? 4 : 8; }
+int rec_floats(int cell) { return cell == PARARNN_GRU ? 4 : 12; }
 
 int chunk_steps(int cell) { return cell == PARARNN_GRU ? gru_chunk_steps() : lstm_chunk_steps(); }
 

@@ -52,13 +52,18 @@ struct GruSlot {
   Aff1 agg[kMaxCluster][kChan];  // aggregate of cluster rank r (r < own rank)
   float cmax[kMaxCluster];       // max|r| of every rank
   float dinc[kChan];             // incoming delta of the cluster chunk
+  float plast[kChan];            // last state (pre-update) of CTA rank-1
+  float clast[kChan];            // last state (pre-update) of the previous cluster chunk
   int upok;                      // upstream cluster chunks all below tol
   int timeout;                   // the look-back gave up
+  int haveclast;                 // clast is valid this iteration
 };
 
 struct GruShared {
   float2 agg[kGruNW][kChan];   // warp aggregates, then exclusive warp prefixes
   float din[kGruNW][kChan];    // incoming delta of each warp's sub-chunk
+  float hlo[kGruNW][kChan];    // each warp's last state before the update
+  float bnd[kGruNW][kChan];    // each warp's boundary state for the next iteration
   float chmax[kGruNW][kChan];  // per (warp, channel) max|r|
   float wmax[kGruNW];
   GruSlot slot[2];
@@ -238,14 +243,17 @@ __global__ void __launch_bounds__(kGruThreads, 2)
   int last_bad = -1;        // warp 0: last evaluation whose channel max|r| >= tol
   float final_m = 0.f;
   int updates = 0, k = 0;
-  // h_{t-1} before this warp's first step: warp 0 holds the CTA boundary, the
-  // others the last state of the previous warp (initial guess 0); each moves
-  // by its incoming delta every iteration, so no exchange is needed.
+  // h_{t-1} before this warp's first step (warp 0: the CTA boundary).  Each
+  // iteration it is re-anchored to the owner's last state before the update
+  // plus this iteration's incoming delta, so it tracks the stored state to
+  // within one update's rounding; the previous warp's / CTA's / cluster
+  // chunk's pre-update last state travels with the aggregates.
   float hb = (warp == 0) ? hbnd : 0.f;
 
   for (;; ++k) {
     const bool cap = (k >= p.max_iters);
     const int par = k & 1;
+    sh.hlo[warp][lane] = h[kGruL - 1];
     float dl, Pw, m;
     if (cap)
       m = gru_pass<false>(rows, lane, hb, h, P, az, ar, ac, az2, ar2, ac2, dl, Pw);
@@ -281,6 +289,7 @@ __global__ void __launch_bounds__(kGruThreads, 2)
         if (r == rank) continue;
         GruSlot* peer = cluster.map_shared_rank(&sh.slot[par], r);
         if (r > rank) peer->agg[rank][lane] = cta;
+        if (r == rank + 1) peer->plast[lane] = sh.hlo[kGruNW - 1][lane];
         if (lane == 0) peer->cmax[rank] = cm;
       }
     }
@@ -303,15 +312,18 @@ __global__ void __launch_bounds__(kGruThreads, 2)
         const Aff1 clus = sl.agg[rank][lane].after(ex);
         const size_t rec = (size_t)ticket * rec_stride + k;
         float* rv = p.rec_vals + rec * (size_t)(kChan * 4);
-        float dinc = 0.f;
-        bool up_ok = true, to = false;
+        float dinc = 0.f, clast = 0.f;
+        bool up_ok = true, to = false, have = false;
+        if (publisher) rec_put_last(rv, lane, sh.hlo[kGruNW - 1][lane]);
         if (!frozen) {
           if (publisher) {
             rec_put_agg(rv, lane, clus);
             publish_flag(&p.rec_flags[rec], make_flag(epoch, kRecAgg, own_ok));
           }
-          if (!lookback<Aff1, float>(p.rec_flags, p.rec_vals, ticket0, jc, k, rec_stride, epoch,
-                                     p.timeout_ns, dinc, up_ok)) {
+          if (lookback<Aff1, float>(p.rec_flags, p.rec_vals, ticket0, jc, k, rec_stride, epoch,
+                                    p.timeout_ns, dinc, up_ok, &clast)) {
+            have = true;
+          } else {
             dinc = 0.f;
             up_ok = true;
             to = true;
@@ -324,9 +336,11 @@ __global__ void __launch_bounds__(kGruThreads, 2)
         for (int r = 0; r < CL; ++r) {
           GruSlot* peer = (r == rank) ? &sh.slot[par] : cluster.map_shared_rank(&sh.slot[par], r);
           peer->dinc[lane] = dinc;
+          peer->clast[lane] = clast;
           if (lane == 0) {
             peer->upok = up_ok ? 1 : 0;
             peer->timeout = to ? 1 : 0;
+            peer->haveclast = have ? 1 : 0;
           }
         }
       }
@@ -342,11 +356,14 @@ __global__ void __launch_bounds__(kGruThreads, 2)
       } else {
         float dinc = 0.f;
         bool up_ok = true;
+        float base = hb;  // this CTA's boundary before the update
         if (multi) {
           dinc = sh.slot[par].dinc[lane];
           up_ok = sh.slot[par].upok != 0;
           if (sh.slot[par].timeout) status = PARARNN_STATUS_TIMEOUT;
+          if (rank == 0 && sh.slot[par].haveclast) base = sh.slot[par].clast[lane];
         }
+        if (rank > 0) base = sh.slot[par].plast[lane];
         if (up_ok) frozen = true;
         const float din = ex.apply(dinc);  // incoming delta of this CTA
         stop = (up_ok && own_ok) ? 1 : 0;
@@ -354,7 +371,9 @@ __global__ void __launch_bounds__(kGruThreads, 2)
 #pragma unroll
         for (int w = 0; w < kGruNW; ++w) {
           const float2 e = sh.agg[w][lane];
-          sh.din[w][lane] = fmaf(e.x, din, e.y);
+          const float dw = fmaf(e.x, din, e.y);
+          sh.din[w][lane] = dw;
+          sh.bnd[w][lane] = (w == 0 ? base : sh.hlo[w - 1][lane]) + dw;
         }
       }
       if (lane == 0) sh.ctl[2] = stop;
@@ -362,7 +381,7 @@ __global__ void __launch_bounds__(kGruThreads, 2)
     __syncthreads();
     if (!cap) {
       const float din = sh.din[warp][lane];
-      hb += din;
+      hb = sh.bnd[warp][lane];
 #pragma unroll
       for (int i = 0; i < kGruL; ++i) h[i] = fmaf(P[i], din, h[i]);
     }

@@ -59,7 +59,12 @@ struct Aff2 {
 };
 
 // Global record payload per lane: AGG fields and INCL fields never overlap,
-// so a reader that saw either flag value reads consistent data.
+// so a reader that saw either flag value reads consistent data.  Both kinds
+// also carry the chunk's last state before this iteration's update ("last",
+// written before the first flag), from which the successor re-anchors its
+// boundary state each iteration.
+//   Aff1: [P, d, incl, last]              (4 floats per lane)
+//   Aff2: [m00 m01 m10 m11 | d0 d1 incl.c incl.h | last.c last.h - -] (12)
 __device__ __forceinline__ void rec_put_agg(float* rec, int lane, const Aff1& e) {
   float* p = rec + lane * 4;
   *reinterpret_cast<float2*>(p) = make_float2(e.P, e.d);
@@ -73,23 +78,33 @@ __device__ __forceinline__ void rec_get_agg(const float* rec, int lane, Aff1& e)
 __device__ __forceinline__ void rec_get_incl(const float* rec, int lane, float& v) {
   v = __ldcg(rec + lane * 4 + 2);
 }
+__device__ __forceinline__ void rec_put_last(float* rec, int lane, float v) { rec[lane * 4 + 3] = v; }
+__device__ __forceinline__ void rec_get_last(const float* rec, int lane, float& v) {
+  v = __ldcg(rec + lane * 4 + 3);
+}
 __device__ __forceinline__ void rec_put_agg(float* rec, int lane, const Aff2& e) {
-  float* p = rec + lane * 8;
+  float* p = rec + lane * 12;
   *reinterpret_cast<float4*>(p) = make_float4(e.m00, e.m01, e.m10, e.m11);
   *reinterpret_cast<float2*>(p + 4) = make_float2(e.d0, e.d1);
 }
 __device__ __forceinline__ void rec_put_incl(float* rec, int lane, float2 v) {
-  *reinterpret_cast<float2*>(rec + lane * 8 + 6) = v;
+  *reinterpret_cast<float2*>(rec + lane * 12 + 6) = v;
+}
+__device__ __forceinline__ void rec_put_last(float* rec, int lane, float2 v) {
+  *reinterpret_cast<float2*>(rec + lane * 12 + 8) = v;
+}
+__device__ __forceinline__ void rec_get_last(const float* rec, int lane, float2& v) {
+  v = __ldcg(reinterpret_cast<const float2*>(rec + lane * 12 + 8));
 }
 __device__ __forceinline__ void rec_get_agg(const float* rec, int lane, Aff2& e) {
-  const float4 m = __ldcg(reinterpret_cast<const float4*>(rec + lane * 8));
-  const float2 d = __ldcg(reinterpret_cast<const float2*>(rec + lane * 8 + 4));
+  const float4 m = __ldcg(reinterpret_cast<const float4*>(rec + lane * 12));
+  const float2 d = __ldcg(reinterpret_cast<const float2*>(rec + lane * 12 + 4));
   e = {m.x, m.y, m.z, m.w, d.x, d.y};
 }
 __device__ __forceinline__ void rec_get_incl(const float* rec, int lane, float2& v) {
-  v = __ldcg(reinterpret_cast<const float2*>(rec + lane * 8 + 6));
+  v = __ldcg(reinterpret_cast<const float2*>(rec + lane * 12 + 6));
 }
-template <class E> __host__ __device__ constexpr int rec_floats() { return sizeof(E) == sizeof(Aff1) ? 4 : 8; }
+template <class E> __host__ __device__ constexpr int rec_floats() { return sizeof(E) == sizeof(Aff1) ? 4 : 12; }
 
 __device__ __forceinline__ unsigned make_flag(unsigned epoch, unsigned kind, bool ok) {
   return (epoch << 3) | (kind << 1) | (ok ? 1u : 0u);
@@ -107,10 +122,13 @@ __device__ __forceinline__ void publish_flag(unsigned* fl, unsigned flag) {
 // Decoupled look-back over the predecessors of cluster chunk `jc` (records of
 // chunk q live at rec_base[(ticket0 + q) * stride + k]).  Warp-uniform.
 // Returns false on timeout.  On success `din` is the incoming delta of chunk
-// jc and `up_ok` tells whether every upstream chunk was below tol at k.
+// jc, `up_ok` tells whether every upstream chunk was below tol at k, and
+// `plast` (if not null) is the immediate predecessor's last state before its
+// update of iteration k.
 template <class E, class V>
 __device__ bool lookback(const unsigned* flags, const float* vals, int ticket0, int jc, int k,
-                         int stride, unsigned epoch, uint64_t timeout_ns, V& din, bool& up_ok) {
+                         int stride, unsigned epoch, uint64_t timeout_ns, V& din, bool& up_ok,
+                         V* plast = nullptr) {
   const int lane = threadIdx.x & 31;
   constexpr int RF = rec_floats<E>();
   E acc = E::id();
@@ -161,6 +179,7 @@ __device__ bool lookback(const unsigned* flags, const float* vals, int ticket0, 
     for (int q = 0; q < window; ++q) {
       const size_t r = (size_t)(ticket0 + jc - 1 - q0 - q) * stride + k;
       const float* rec = vals + r * (size_t)(kChan * RF);
+      if (plast != nullptr && q0 == 0 && q == 0) rec_get_last(rec, lane, *plast);
       if (q == incl_at) {
         V v;
         rec_get_incl(rec, lane, v);

@@ -1,0 +1,90 @@
+"""GPU parity of the fused ParaLSTM Newton-scan solve against the fp64 oracle
+(max-abs 1e-4 on both c and h)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nonlinear_rnn_paragru_b200 as pr
+from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_STATE = 1e-4
+
+
+def _solve(x, **kw):
+    d = "cuda"
+    c, h, st, hist = pr.lstm_solve(x["u"].to(d), x["a"].to(d), x["bias"].to(d),
+                                   x["c0"].to(d), x["h0"].to(d), **kw)
+    torch.cuda.synchronize()
+    return (c.cpu().numpy(), h.cpu().numpy(), pr.read_stats(st),
+            hist.cpu().numpy() if hist is not None else None)
+
+
+def _ref(x):
+    return oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+
+
+def _check(x, **kw):
+    c, h, st, hist = _solve(x, **kw)
+    rc, rh = _ref(x)
+    err = max(np.abs(c - rc).max(), np.abs(h - rh).max())
+    assert err < TOL_STATE, (err, st)
+    assert st["status"] == "converged", st
+    return st, hist
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 1000, 96), (1, 129, 64), (1, 1, 8),
+                                   (3, 128, 32), (1, 2200, 40)])
+def test_ragged_shapes_bf16(cuda_ok, B, T, D):
+    _check(make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D)))
+
+
+def test_fp32_inputs(cuda_ok):
+    w = WORKLOADS[3].scaled(B=1, T=700, D=64)
+    x = make_inputs(w)
+    x["u"] = x["u"].float()
+    _check(x)
+
+
+def test_nonzero_initial_state(cuda_ok):
+    x = make_inputs(WORKLOADS[3].scaled(B=2, T=600, D=64))
+    g = torch.Generator().manual_seed(7)
+    x["c0"] = torch.randn((2, 64), generator=g, dtype=torch.float32)
+    x["h0"] = torch.randn((2, 64), generator=g, dtype=torch.float32) * 0.5
+    _check(x)
+
+
+def test_config5_shape_scaled(cuda_ok):
+    st, _ = _check(make_inputs(WORKLOADS[5].scaled(B=2, T=2048, D=128)))
+
+
+def test_config3_full_size(cuda_ok):
+    st, _ = _check(make_inputs(WORKLOADS[3]))
+    assert st["max_residual"] < 1e-6
+
+
+def test_multi_cluster_chunks(cuda_ok):
+    # T = 5000 spans several 16-CTA cluster chunks of 2048 steps
+    st, hist = _check(make_inputs(WORKLOADS[3].scaled(B=1, T=5000, D=64)), hist=True)
+    assert hist.sum() == 64 and hist[-1] == 0
+
+
+@pytest.mark.parametrize("n", [1, 2])
+def test_capped_iterates_match_oracle_newton(cuda_ok, n):
+    x = make_inputs(WORKLOADS[3].scaled(B=1, T=900, D=64))
+    c, h, st, _ = _solve(x, max_iters=n)
+    r = oracle.lstm_newton(x["u"], x["a"], x["bias"], x["c0"], x["h0"], tol=0.0,
+                           max_iters=n)
+    assert st["status"] == "not_converged" and st["iters"] == n
+    assert max(np.abs(c - r["c"]).max(), np.abs(h - r["h"]).max()) < TOL_STATE
+
+
+def test_seq_baseline_matches_oracle(cuda_ok):
+    x = make_inputs(WORKLOADS[3].scaled(B=2, T=300, D=64))
+    c, h = pr.seq_baseline(pr.PARARNN_LSTM, x["u"].cuda(), x["a"].cuda(),
+                           x["bias"].cuda(), x["c0"].cuda(), x["h0"].cuda())
+    torch.cuda.synchronize()
+    rc, rh = _ref(x)
+    assert max(np.abs(c.cpu().numpy() - rc).max(), np.abs(h.cpu().numpy() - rh).max()) < TOL_STATE
