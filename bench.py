@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the ParaGRU / ParaLSTM Newton-scan hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1..5]
+                    [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the workload:
+the fused Newton-scan forward solve and, for workloads with a backward pass,
+the reverse adjoint scan.  The default workload is ParaGRU B=8, T=4096,
+D=1024 with bf16 input projections (forward + adjoint), the layer shape the
+throughput metric is quoted on.  Inputs are seeded synthetic tensors of that
+shape; u alone (201 MB) is larger than the 126 MB L2, so no flush is needed
+between timed steps.
+
+Under torchrun (N > 1) every rank solves its own independent problem of the
+same size (weak scaling, no data-path collective); the time is the max over
+ranks and `value` counts the token-channels of all ranks.  `--impl reference`
+times the fp64 CPU oracle (sequential recurrence + BPTT) on a bounded sample
+of the same workload.  Rank 0 prints one JSON line.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Newton-solved token*channels/s (fwd+bwd)"
+UNIT = "tokch/s"
+# Counters of the dominant kernel taken with ncu on this build (one launch of
+# the default workload; see profiles/).  None when not captured for the
+# kernel as it stands.
+NCU_TRAFFIC_BYTES = {}
+# special-function (MUFU) operations per element and cell evaluation, as the
+# kernels issue them: ParaGRU 3 ex2 + 2 rcp; ParaLSTM 5 ex2 + 3 rcp
+MUFU_PER_EVAL = {"gru": 5, "lstm": 8}
+# algorithmic HBM bytes per token-channel: inputs read once, outputs written once
+def fwd_bytes(w):
+    ue = 2 if w.u_dtype == "bf16" else 4
+    return w.G * ue + (4 if w.cell == "gru" else 8)
+
+
+def adj_bytes(w):
+    ue = 2 if w.u_dtype == "bf16" else 4
+    states = 4 if w.cell == "gru" else 8
+    return w.G * ue + states + 4 + 4 * w.G   # u, states, dL/dh in; du out
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------- distributed --
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a per-rank scalar over all ranks (timing is the slowest rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world, units_per_rank, ms_max):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
+def rank_seed(rank):
+    """Each rank solves its own independent problem."""
+    return 1000 * rank
+
+
+# ---------------------------------------------------------------- clocks --
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.mhz, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._th = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks stay unreported
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.mhz.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._th is not None:
+            self._th.join()
+
+    def summary(self):
+        if not self.mhz:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.mhz)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+# ------------------------------------------------------------- our path --
+class Path:
+    """Device buffers and the step (forward solve + adjoint) of one workload."""
+
+    def __init__(self, w, x, pr):
+        self.w, self.x, self.pr = w, x, pr
+        d = "cuda"
+        B, T, D, G = w.B, w.T, w.D, w.G
+        self.lstm = w.cell == "lstm"
+        self.h = torch.empty((B, T, D), dtype=torch.float32, device=d)
+        self.c = torch.empty((B, T, D), dtype=torch.float32, device=d) if self.lstm else None
+        self.stats = torch.zeros(4, dtype=torch.int32, device=d)
+        self.hist = (torch.empty(66, dtype=torch.int32, device=d) if w.histogram else None)
+        self.ws = pr.Workspace(d)
+        self.wsa = pr.Workspace(d)
+        self.opts = pr._opts(1e-6, 64)
+        cell = pr.PARARNN_LSTM if self.lstm else pr.PARARNN_GRU
+        self.fbuf = self.ws.get(pr.pararnn_workspace_size(cell, B, T, D, 64, 0))
+        if w.adjoint:
+            self.du = torch.empty((B, T, G, D), dtype=torch.float32, device=d)
+            self.da = torch.empty((G, D), dtype=torch.float32, device=d)
+            self.db = torch.empty((G, D), dtype=torch.float32, device=d)
+            self.dh0 = torch.empty((B, D), dtype=torch.float32, device=d)
+            self.dc0 = torch.empty((B, D), dtype=torch.float32, device=d) if self.lstm else None
+            self.status = torch.zeros(1, dtype=torch.int32, device=d)
+            self.abuf = self.wsa.get(pr.pararnn_workspace_size(cell, B, T, D, 0, 1))
+
+    def launches_per_step(self):
+        n = 2 + (1 if self.hist is not None else 0)        # init, solve, [hist]
+        return n + (3 if self.w.adjoint else 0)            # init, adjoint, reduce
+
+    def forward(self, x=None):
+        x = x or self.x
+        pr = self.pr
+        if self.lstm:
+            pr.pararnn_lstm_solve(x["u"], x["a"], x["bias"], x["c0"], x["h0"], self.c,
+                                  self.h, self.opts, self.stats, self.hist, self.fbuf)
+        else:
+            pr.pararnn_gru_solve(x["u"], x["a"], x["bias"], x["h0"], self.h, self.opts,
+                                 self.stats, self.hist, self.fbuf)
+
+    def backward(self, x=None):
+        x = x or self.x
+        pr = self.pr
+        cell = pr.PARARNN_LSTM if self.lstm else pr.PARARNN_GRU
+        pr.pararnn_adjoint(cell, x["u"], x["a"], x["bias"], x.get("c0"), x["h0"], self.c,
+                           self.h, x["dLdh"], self.du, self.da, self.db, self.dc0, self.dh0,
+                           self.status, self.abuf)
+
+    def step(self, x=None):
+        self.forward(x)
+        if self.w.adjoint:
+            self.backward(x)
+
+
+def time_events(fn, n):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n  # ms
+
+
+def cpu_baseline(w, seconds_hint=10.0):
+    """The fp64 oracle (sequential recurrence + BPTT) on a bounded sample of
+    the workload: all of T, a slice of the channels."""
+    import oracle
+    Dk = 64
+    ws = w.scaled(B=1, D=Dk)
+    x = make_inputs(ws, with_grad=True)
+    reps, t_total, n = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while True:
+        t1 = time.perf_counter()
+        if w.cell == "gru":
+            h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+            if w.adjoint:
+                oracle.gru_bptt(x["u"], x["a"], x["bias"], x["h0"], h, x["dLdh"])
+        else:
+            c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+            if w.adjoint:
+                oracle.lstm_bptt(x["u"], x["a"], x["bias"], x["c0"], x["h0"], c, h, x["dLdh"])
+        t_total += time.perf_counter() - t1
+        n += ws.tokch
+        reps += 1
+        if time.perf_counter() - t0 > seconds_hint or reps >= 2000:
+            break
+    return {"value": n / t_total, "unit": UNIT, "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"B=1, T={w.T}, D={Dk} slice of {w.name}, fp64 sequential "
+                      f"{'recurrence + BPTT' if w.adjoint else 'recurrence'}, "
+                      f"{reps} repetition(s), {t_total:.1f} s"}
+
+
+def run_ours(args, world, rank):
+    import nonlinear_rnn_paragru_b200 as pr
+    pr.load_library()  # fails loudly when the CUDA library is missing
+    w = WORKLOADS[args.workload]
+    x = make_inputs(w, seed=rank_seed(rank), device="cuda", with_grad=w.adjoint)
+    path = Path(w, x, pr)
+    for _ in range(max(args.warmup, 3)):
+        path.step()
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler = ClockSampler(torch.cuda.current_device())
+    with sampler:
+        ms = time_events(path.step, args.steps)
+        barrier(world)
+    ms_max = max_over_ranks(ms, world)
+    st = pr.read_stats(path.stats)
+    value = weak_value(world, w.tokch, ms_max)
+
+    # per-kernel timing (same stream, CUDA events) for the roofline
+    fwd_ms = time_events(path.forward, max(3, args.steps // 2))
+    adj_ms = time_events(path.backward, max(3, args.steps // 2)) if w.adjoint else 0.0
+    clk = sampler.summary()
+    peaks, src = measured_peaks()
+    f_mhz = clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    mufu_peak = 148 * 16 * f_mhz * 1e6 / 1e12          # Tops/s
+    mufu_done = w.tokch * st["evals"] * MUFU_PER_EVAL[w.cell] / (fwd_ms * 1e-3) / 1e12
+    hbm_ach = w.tokch * fwd_bytes(w) / (fwd_ms * 1e-3) / 1e9
+    kern = ("lstm_newton_fused" if w.cell == "lstm" else "gru_newton_fused")
+    traffic = NCU_TRAFFIC_BYTES.get((kern, w.name))
+    roofline = {"bound": "alu", "kernel": kern, "achieved": round(mufu_done, 3),
+                "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
+                "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
+                "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
+                "ops_per_launch": w.tokch * st["evals"] * MUFU_PER_EVAL[w.cell]}
+    hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
+           "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,
+           "fwd_bytes_per_tokch": fwd_bytes(w)}
+    if w.adjoint:
+        adj_gbs = w.tokch * adj_bytes(w) / (adj_ms * 1e-3) / 1e9
+        hbm.update({"adj_achieved_gbs": round(adj_gbs, 1),
+                    "adj_frac": round(adj_gbs / peaks["hbm_gbs"], 4),
+                    "adj_bytes_per_tokch": adj_bytes(w)})
+
+    # naive step-by-step GPU loop (forward only), same inputs
+    cell = pr.PARARNN_LSTM if path.lstm else pr.PARARNN_GRU
+    seq_ms = time_events(lambda: pr.pararnn_seq_baseline(cell, x["u"], x["a"], x["bias"],
+                                                        x.get("c0"), x["h0"], path.c, path.h),
+                         2)
+
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the step, D2H of its outputs, all inside the timed region
+    host = {k: v.cpu().pin_memory() for k, v in x.items()}
+    dev = {k: torch.empty_like(v) for k, v in x.items()}
+    outs = [path.h] + ([path.c] if path.lstm else [])
+    if w.adjoint:
+        outs += [path.du, path.da, path.db, path.dh0] + ([path.dc0] if path.lstm else [])
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+
+    def e2e_step():
+        for k in dev:
+            dev[k].copy_(host[k], non_blocking=True)
+        path.step(dev)
+        for ho, o in zip(host_out, outs):
+            ho.copy_(o, non_blocking=True)
+
+    e2e_step()
+    barrier(world)
+    e2e_ms = max_over_ranks(time_events(e2e_step, args.e2e_steps), world)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name + (" fwd+adjoint" if w.adjoint else " fwd"),
+                   "cell": w.cell, "B": w.B, "T": w.T, "D": w.D, "u_dtype": w.u_dtype,
+                   "tol": 1e-6, "l2": "inputs larger than L2 (u alone exceeds 126 MB)",
+                   "parallelism": f"{world} independent replica(s)"},
+        "newton": {"iters": st["iters"], "evals": st["evals"],
+                   "max_residual": st["max_residual"], "status": st["status"]},
+        "fwd_ms": round(fwd_ms, 4), "adj_ms": round(adj_ms, 4),
+        "fwd_tokch_per_s": w.tokch / (fwd_ms * 1e-3),
+        "roofline": roofline, "hbm_roofline": hbm,
+        "seq_gpu_baseline": {"fwd_ms": round(seq_ms, 3),
+                             "speedup_fused_fwd": round(seq_ms / fwd_ms, 2),
+                             "pages_claim": "up to 665x over sequential (hardware not stated)"},
+        "e2e": {"value": weak_value(world, w.tokch, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 3)},
+        "clocks": clk,
+        "gpu_launches": path.launches_per_step() * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w)
+    return out
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS[args.workload]
+    cb = cpu_baseline(w, seconds_hint=10.0)
+    t = w.tokch / cb["value"]
+    return {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name + (" fwd+adjoint" if w.adjoint else " fwd"),
+                       "cell": w.cell, "B": w.B, "T": w.T, "D": w.D},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), 0)),
+              flush=True)
+        return 0
+    world, rank, _ = dist_setup()
+    out = run_ours(args, world, rank)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
