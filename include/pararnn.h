@@ -167,6 +167,31 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
                     int B, int T, int D, int* status, void* workspace,
                     size_t ws_bytes, pararnn_stream_t stream);
 
+/* Adjoint without a caller-supplied workspace.  (The pages have no
+ * counterpart; this is a library convenience.)  For callers that cannot hand
+ * the library scratch memory -- because an allocator they do not control owns
+ * the device memory, or because cudaMalloc's latency and implicit
+ * synchronisation are not acceptable on their path.  Same arguments and
+ * results as pararnn_adjoint minus the workspace: the scratch is a fixed
+ * PARARNN_NOALLOC_SCRATCH_BYTES array inside the library, held in device
+ * memory by every GPU that loads the library until the process exits.  The
+ * call allocates nothing.  The first call on a device looks the array up and
+ * clears it (a synchronous step), so make that first call before any stream
+ * capture.  All calls on a device share the array: calls that overlap on the
+ * GPU race and must not be made.  Problems that need more scratch than the
+ * array holds (pararnn_workspace_size(cell, B, T, D, 0, 1) above the limit:
+ * about 6500 ParaGRU chunks of 32 channels x 256 steps, i.e.
+ * B*ceil(D/32)*ceil(T/256), or about 3200 ParaLSTM chunks of 32 x 128) return
+ * PARARNN_ERR_WORKSPACE_TOO_SMALL without launching anything. */
+#define PARARNN_NOALLOC_SCRATCH_BYTES (8u << 20)
+int pararnn_adjoint_noalloc(int cell, const void* u, int u_dtype,
+                            const float* a, const float* bias,
+                            const float* c0, const float* h0, const float* c,
+                            const float* h, const float* dLdh, float* du,
+                            float* da, float* dbias, float* dc0, float* dh0,
+                            int B, int T, int D, int* status,
+                            pararnn_stream_t stream);
+
 /* Naive step-by-step GPU evaluation (one thread per (b, d) channel looping
  * over t) -- the sequential baseline the parallel solve is compared with.
  * c0/c must be NULL for ParaGRU.  No workspace. */

@@ -21,7 +21,8 @@ __all__ = [
     "PARARNN_F32", "PARARNN_BF16", "PARARNN_GRU", "PARARNN_LSTM",
     "PararnnOpts", "PararnnError", "library_path", "load_library",
     "pararnn_workspace_size", "pararnn_workspace_init", "pararnn_gru_solve",
-    "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_seq_baseline",
+    "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_noalloc",
+    "pararnn_seq_baseline",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
     "Workspace", "read_stats",
 ]
@@ -77,6 +78,8 @@ def load_library():
                                 fp, fp, fp, i, i, i, ip, vp, sz, vp]),
         "pararnn_seq_baseline": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i,
                                      i, vp]),
+        "pararnn_adjoint_noalloc": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, fp,
+                                        fp, fp, fp, fp, fp, i, i, i, ip, vp]),
         "pararnn_strerror": (ctypes.c_char_p, [i]),
     }
     for name, (res, args) in sigs.items():
@@ -181,6 +184,17 @@ def pararnn_adjoint(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, dbias, dc0,
         _iptr(status), _wptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)),
         "pararnn_adjoint")
+
+
+def pararnn_adjoint_noalloc(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, dbias,
+                            dc0, dh0, status, stream=None):
+    """pararnn_adjoint with the library's built-in scratch instead of a
+    workspace: for callers that cannot provide device scratch memory."""
+    _check(load_library().pararnn_adjoint_noalloc(
+        cell, _uptr(u), _dtype_code(u), _ptr(a), _ptr(bias), _ptr(c0),
+        _ptr(h0), _ptr(c), _ptr(h), _ptr(dLdh), _ptr(du), _ptr(da),
+        _ptr(dbias), _ptr(dc0), _ptr(dh0), u.shape[0], u.shape[1], u.shape[3],
+        _iptr(status), _stream(stream)), "pararnn_adjoint_noalloc")
 
 
 def pararnn_seq_baseline(cell, u, a, bias, c0, h0, c, h, stream=None):
