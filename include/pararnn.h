@@ -180,10 +180,10 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * capture.  All calls on a device share the array: calls that overlap on the
  * GPU race and must not be made.  Problems that need more scratch than the
  * array holds (pararnn_workspace_size(cell, B, T, D, 0, 1) above the limit:
- * about 6500 ParaGRU chunks of 32 channels x 256 steps, i.e.
- * B*ceil(D/32)*ceil(T/256), or about 3200 ParaLSTM chunks of 32 x 128) return
+ * about 13000 ParaGRU chunks of 32 channels x 128 steps, i.e.
+ * B*ceil(D/32)*ceil(T/128), or about 6500 ParaLSTM chunks of 32 x 64) return
  * PARARNN_ERR_WORKSPACE_TOO_SMALL without launching anything. */
-#define PARARNN_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define PARARNN_NOALLOC_SCRATCH_BYTES (16u << 20)
 int pararnn_adjoint_noalloc(int cell, const void* u, int u_dtype,
                             const float* a, const float* bias,
                             const float* c0, const float* h0, const float* c,

@@ -18,9 +18,10 @@
 //     per chunk; chunks take tickets from the last one backwards);
 //   pass 2 (reverse): re-evaluate the cell, run the exact recurrence from the
 //     true incoming carry, write du and accumulate da / dbias partials.
-// The gate projections arrive by TMA; states and dL/dh are read with
-// coalesced loads (the second pass hits L2).  Per-CTA partial sums of da and
-// dbias are reduced by a second kernel in a fixed order (reproducible).
+// u, the states and dL/dh of the chunk arrive by TMA bulk-tensor loads into
+// shared memory (one mbarrier), so both passes read on-chip data.  Per-CTA
+// partial sums of da and dbias are reduced by a second kernel in a fixed
+// order (reproducible).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -39,7 +40,8 @@ __device__ __forceinline__ float tanhx(float x) {
 
 struct GruCell {
   static constexpr int G = 3;
-  static constexpr int L = 32;
+  static constexpr int L = 16;
+  static constexpr int kMinBlocks = 3;
   using E = Aff1;
   using V = float;
   struct S {  // state s_{t-1}
@@ -76,7 +78,8 @@ struct GruCell {
 
 struct LstmCell {
   static constexpr int G = 4;
-  static constexpr int L = 16;
+  static constexpr int L = 8;
+  static constexpr int kMinBlocks = 2;
   using E = Aff2;
   using V = float2;  // (lambda_c, lambda_h)
   struct S {
@@ -138,24 +141,38 @@ struct AdjParams {
   int* status;
 };
 
+// State before the chunk (global), and states inside it (shared memory).
 template <class Cell>
-__device__ __forceinline__ typename Cell::S load_state(const AdjParams& p, int b, int t, int d,
-                                                       bool dval);
+__device__ __forceinline__ typename Cell::S boundary_state(const AdjParams& p, int b, int t0,
+                                                           int d, bool dval);
 template <>
-__device__ __forceinline__ GruCell::S load_state<GruCell>(const AdjParams& p, int b, int t, int d,
-                                                          bool dval) {
-  if (!dval || t >= p.T) return {0.f};
-  if (t < 0) return {p.h0 ? p.h0[(size_t)b * p.D + d] : 0.f};
-  return {p.h[((size_t)b * p.T + t) * p.D + d]};
+__device__ __forceinline__ GruCell::S boundary_state<GruCell>(const AdjParams& p, int b, int t0,
+                                                              int d, bool dval) {
+  if (!dval) return {0.f};
+  if (t0 == 0) return {p.h0 ? p.h0[(size_t)b * p.D + d] : 0.f};
+  return {p.h[((size_t)b * p.T + t0 - 1) * p.D + d]};
 }
 template <>
-__device__ __forceinline__ LstmCell::S load_state<LstmCell>(const AdjParams& p, int b, int t,
-                                                            int d, bool dval) {
-  if (!dval || t >= p.T) return {0.f, 0.f};
-  if (t < 0)
+__device__ __forceinline__ LstmCell::S boundary_state<LstmCell>(const AdjParams& p, int b, int t0,
+                                                                int d, bool dval) {
+  if (!dval) return {0.f, 0.f};
+  if (t0 == 0)
     return {p.c0 ? p.c0[(size_t)b * p.D + d] : 0.f, p.h0 ? p.h0[(size_t)b * p.D + d] : 0.f};
-  const size_t i = ((size_t)b * p.T + t) * p.D + d;
+  const size_t i = ((size_t)b * p.T + t0 - 1) * p.D + d;
   return {p.c[i], p.h[i]};
+}
+template <class Cell>
+__device__ __forceinline__ typename Cell::S tile_state(const float* hs, const float* cs, int s,
+                                                       int lane);
+template <>
+__device__ __forceinline__ GruCell::S tile_state<GruCell>(const float* hs, const float*, int s,
+                                                          int lane) {
+  return {hs[s * kChan + lane]};
+}
+template <>
+__device__ __forceinline__ LstmCell::S tile_state<LstmCell>(const float* hs, const float* cs,
+                                                            int s, int lane) {
+  return {cs[s * kChan + lane], hs[s * kChan + lane]};
 }
 
 template <class Cell, bool kBF16>
@@ -171,14 +188,31 @@ __device__ __forceinline__ void load_u(const unsigned char* tile, int s, int lan
   if (Cell::G == 3) u[3] = 0.f;
 }
 
+// Shared-memory tiles of one chunk: u [TC][G][32] (bf16 or fp32), then the
+// fp32 tiles h [TC][32], c [TC][32] (ParaLSTM) and dL/dh [TC][32].
 template <class Cell, bool kBF16>
-__global__ void __launch_bounds__(kAdjThreads, 2)
-    adjoint_kernel(const __grid_constant__ CUtensorMap tmap, const AdjParams p) {
+struct AdjTiles {
+  static constexpr int TC = kAdjNW * Cell::L;
+  static constexpr int kU = TC * Cell::G * kChan * (kBF16 ? 2 : 4);
+  static constexpr int kS = TC * kChan * 4;
+  static constexpr int kNS = (Cell::G == 4) ? 3 : 2;  // state/grad tiles
+  static constexpr int kBytes = kU + kNS * kS;
+};
+
+template <class Cell, bool kBF16>
+__global__ void __launch_bounds__(kAdjThreads, Cell::kMinBlocks)
+    adjoint_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap tmh,
+                   const __grid_constant__ CUtensorMap tmc, const __grid_constant__ CUtensorMap tmg,
+                   const AdjParams p) {
   using E = typename Cell::E;
   using V = typename Cell::V;
   using S = typename Cell::S;
+  using Tiles = AdjTiles<Cell, kBF16>;
   constexpr int L = Cell::L, G = Cell::G, TC = kAdjNW * L;
   extern __shared__ __align__(1024) unsigned char tile[];
+  const float* h_t = reinterpret_cast<const float*>(tile + Tiles::kU);
+  const float* g_t = reinterpret_cast<const float*>(tile + Tiles::kU + Tiles::kS);
+  const float* c_t = reinterpret_cast<const float*>(tile + Tiles::kU + 2 * Tiles::kS);
   __shared__ E agg[kAdjNW][kChan];
   __shared__ float red[kAdjNW][2 * G][kChan];
   __shared__ int ctl[4];
@@ -200,11 +234,15 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
   const int t0 = j * TC;
   const int d = d0 + lane;
   const bool dval = d < p.D;
-  constexpr unsigned kBytes = TC * G * kChan * (kBF16 ? 2 : 4);
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bar, kBytes);
+    mbar_arrive_expect_tx(&bar, (unsigned)Tiles::kBytes);
     tma_load_4d(tile, &tmap, &bar, d0, 0, t0, b);
+    tma_load_3d(tile + Tiles::kU, &tmh, &bar, d0, t0, b);
+    tma_load_3d(tile + Tiles::kU + Tiles::kS, &tmg, &bar, d0, t0, b);
+    if (G == 4) tma_load_3d(tile + Tiles::kU + 2 * Tiles::kS, &tmc, &bar, d0, t0, b);
   }
+  // the state before this thread's first step
+  const S s_before_chunk = boundary_state<Cell>(p, b, t0, d, dval);
   typename Cell::K K;
 #pragma unroll
   for (int q = 0; q < G; ++q) {
@@ -216,8 +254,10 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
 
   const int a0 = warp * L;             // first local step of this thread
   const int nvalid = min(L, p.T - (t0 + a0));
-  auto gval = [&](int s) -> float {    // dL/dh at local step s (0 past the end)
-    return (dval && s < nvalid) ? p.dLdh[((size_t)b * p.T + t0 + a0 + s) * p.D + d] : 0.f;
+  // dL/dh and states past the end of the sequence arrive as zeros (TMA fill)
+  auto gval = [&](int s) -> float { return g_t[(a0 + s) * kChan + lane]; };
+  auto state_at = [&](int s) -> S {   // state after local step s of this thread
+    return (a0 + s < 0) ? s_before_chunk : tile_state<Cell>(h_t, c_t, a0 + s, lane);
   };
 
   // ---- pass 1: compose this range's carry map (reverse).  accm maps the
@@ -225,11 +265,11 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
   // the carry leaving the current step.
   E accm = E::id();
   {
-    S sp = load_state<Cell>(p, b, t0 + a0 + L - 2, d, dval);  // state before step L-1
+#pragma unroll 4
     for (int s = L - 1; s >= 0; --s) {
       float u[4];
       load_u<Cell, kBF16>(tile, a0 + s, lane, u);
-      const S spn = (s > 0) ? load_state<Cell>(p, b, t0 + a0 + s - 2, d, dval) : sp;
+      const S sp = state_at(s - 1);
       if constexpr (G == 3) {
         float A;
         Cell::template eval<false>(sp, u, K, A, nullptr, nullptr);
@@ -241,7 +281,6 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
         accm = Aff2{1.f, 0.f, 0.f, 1.f, 0.f, gval(s)}.after(accm);
         accm = mat_only(A).after(accm);
       }
-      sp = spn;
     }
   }
   agg[warp][lane] = accm;  // carry into this range -> carry out of its first step
@@ -291,11 +330,11 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
   for (int q = 0; q < G; ++q) sa[q] = sb[q] = 0.f;
   bool bad = false;
   {
-    S sp = load_state<Cell>(p, b, t0 + a0 + L - 2, d, dval);
+#pragma unroll 2
     for (int s = L - 1; s >= 0; --s) {
       float u[4];
       load_u<Cell, kBF16>(tile, a0 + s, lane, u);
-      const S spn = (s > 0) ? load_state<Cell>(p, b, t0 + a0 + s - 2, d, dval) : sp;
+      const S sp = state_at(s - 1);
       const float gs = gval(s);
       float du_c[8], da_c[3];
       float out[4];
@@ -330,7 +369,6 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
           bad |= !isfinite(out[q]);
         }
       }
-      sp = spn;
     }
   }
   // d L / d s_0: the carry out of the first step of the sequence
@@ -361,22 +399,34 @@ __global__ void __launch_bounds__(kAdjThreads, 2)
   if (tid == 0 && ctl[3]) atomicMax(p.status, ctl[3]);
 }
 
-// da[q][d] = sum over (b, chunk) of the per-CTA partials, in a fixed order.
+// da[q][d] = sum over (b, chunk) of the per-CTA partials, in a fixed order:
+// block (q, channel tile), warp w sums chunks w, w + 8, ... of every batch
+// row in order, then the 8 warp sums are added in warp order.
 __global__ void adjoint_reduce(const float* __restrict__ part, float* da, float* dbias, int B,
                                int D, int nDT, int nC, int G) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 2 * G * D) return;
-  const int q = i / D, d = i - q * D;
-  const int dt = d / kChan, lane = d - dt * kChan;
+  __shared__ float ws[kAdjNW][kChan];
+  const int q = blockIdx.x / nDT, dt = blockIdx.x - q * nDT;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float acc = 0.f;
   for (int b = 0; b < B; ++b) {
     const size_t tl = (size_t)b * nDT + dt;
-    for (int v = 0; v < nC; ++v) acc += part[(((tl * nC + v) * 2 * G) + q) * kChan + lane];
+    for (int v = warp; v < nC; v += kAdjNW)
+      acc += part[(((tl * nC + v) * 2 * G) + q) * kChan + lane];
   }
-  if (q < G)
-    da[q * D + d] = acc;
-  else if (dbias)
-    dbias[(q - G) * D + d] = acc;
+  ws[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAdjNW; ++w) t += ws[w][lane];
+    const int d = dt * kChan + lane;
+    if (d < D) {
+      if (q < G)
+        da[q * D + d] = t;
+      else if (dbias)
+        dbias[(q - G) * D + d] = t;
+    }
+  }
 }
 
 __global__ void adjoint_init(WsHeader* hdr, int* status) {
@@ -410,17 +460,17 @@ static AdjLayout adj_layout(int cell, int B, int T, int D) {
 size_t adjoint_ws_bytes(int cell, int B, int T, int D) { return adj_layout(cell, B, T, D).total; }
 
 template <class Cell, bool kBF16>
-static int launch_adj_t(const CUtensorMap& tmap, const AdjParams& p, int nch, cudaStream_t stream) {
-  constexpr int TC = kAdjNW * Cell::L;
-  const int smem = TC * Cell::G * kChan * (kBF16 ? 2 : 4);
+static int launch_adj_t(const CUtensorMap* maps, const AdjParams& p, int nch,
+                        cudaStream_t stream) {
+  const int smem = AdjTiles<Cell, kBF16>::kBytes;
   auto kern = adjoint_kernel<Cell, kBF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
-  kern<<<nch, kAdjThreads, smem, stream>>>(tmap, p);
+  kern<<<nch, kAdjThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], p);
   return (int)cudaGetLastError();
 }
 
-int launch_adjoint(int cell, bool bf16, const CUtensorMap& tmap_u, const void* u, const float* a,
+int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, const float* a,
                    const float* bias, const float* c0, const float* h0, const float* c,
                    const float* h, const float* dLdh, float* du, float* da, float* dbias,
                    float* dc0, float* dh0, int B, int T, int D, int* status, void* ws,
@@ -460,14 +510,14 @@ int launch_adjoint(int cell, bool bf16, const CUtensorMap& tmap_u, const void* u
   if (cudaGetLastError() != cudaSuccess) return 1;
   int e;
   if (cell == PARARNN_GRU)
-    e = bf16 ? launch_adj_t<GruCell, true>(tmap_u, p, (int)nch, stream)
-             : launch_adj_t<GruCell, false>(tmap_u, p, (int)nch, stream);
+    e = bf16 ? launch_adj_t<GruCell, true>(maps, p, (int)nch, stream)
+             : launch_adj_t<GruCell, false>(maps, p, (int)nch, stream);
   else
-    e = bf16 ? launch_adj_t<LstmCell, true>(tmap_u, p, (int)nch, stream)
-             : launch_adj_t<LstmCell, false>(tmap_u, p, (int)nch, stream);
+    e = bf16 ? launch_adj_t<LstmCell, true>(maps, p, (int)nch, stream)
+             : launch_adj_t<LstmCell, false>(maps, p, (int)nch, stream);
   if (e) return e;
-  const int n = 2 * G * D;
-  adjoint_reduce<<<(n + 255) / 256, 256, 0, stream>>>(p.part, da, dbias, B, D, p.nDT, p.nC, G);
+  adjoint_reduce<<<2 * G * p.nDT, kAdjThreads, 0, stream>>>(p.part, da, dbias, B, D, p.nDT, p.nC,
+                                                             G);
   return (int)cudaGetLastError();
 }
 

@@ -23,7 +23,7 @@ int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, cons
 struct AdjParams;
 int adjoint_chunk_steps(int cell);
 size_t adjoint_ws_bytes(int cell, int B, int T, int D);
-int launch_adjoint(int cell, bool bf16, const CUtensorMap& tmap_u, const void* u, const float* a,
+int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, const float* a,
                    const float* bias, const float* c0, const float* h0, const float* c,
                    const float* h, const float* dLdh, float* du, float* da, float* dbias,
                    float* dc0, float* dh0, int B, int T, int D, int* status, void* ws,
@@ -71,6 +71,20 @@ int make_u_map(CUtensorMap* map, const void* u, bool bf16, int B, int T, int G, 
                   const_cast<void*>(u), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+// Tensor map over an fp32 [B][T][D] array with a box of 32 channels x tc steps.
+int make_s_map(CUtensorMap* map, const float* x, int B, int T, int D, int tc) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return PARARNN_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
+  cuuint32_t box[3] = {(cuuint32_t)kChan, (cuuint32_t)tc, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 
@@ -272,10 +286,14 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
     return PARARNN_ERR_MISALIGNED;
   if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const int G = cell == PARARNN_GRU ? 3 : 4;
-  CUtensorMap map;
-  rc = make_u_map(&map, u, u_dtype == PARARNN_BF16, B, T, G, D, adjoint_chunk_steps(cell));
+  const int tc = adjoint_chunk_steps(cell);
+  CUtensorMap maps[4];  // u, h, c (ParaLSTM; h again for ParaGRU), dL/dh
+  rc = make_u_map(&maps[0], u, u_dtype == PARARNN_BF16, B, T, G, D, tc);
+  if (!rc) rc = make_s_map(&maps[1], h, B, T, D, tc);
+  if (!rc) rc = make_s_map(&maps[2], c ? c : h, B, T, D, tc);
+  if (!rc) rc = make_s_map(&maps[3], dLdh, B, T, D, tc);
   if (rc) return rc;
-  const int e = launch_adjoint(cell, u_dtype == PARARNN_BF16, map, u, a, bias, c0, h0, c, h, dLdh,
+  const int e = launch_adjoint(cell, u_dtype == PARARNN_BF16, maps, u, a, bias, c0, h0, c, h, dLdh,
                                du, da, dbias, dc0, dh0, B, T, D, status, workspace,
                                (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;

@@ -54,10 +54,10 @@ def test_noalloc_adjoint_matches_workspace_adjoint_twice(cuda_ok, shape):
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch(cuda_ok):
-    # ParaLSTM B=4, T=2048, D=4096 needs about 20 MiB of scratch: refused
+    # ParaLSTM B=4, T=2048, D=4096 needs about 40 MiB of scratch: refused
     # with PARARNN_ERR_WORKSPACE_TOO_SMALL before anything is launched
     B, T, D = 4, 2048, 4096
-    assert pr.pararnn_workspace_size(pr.PARARNN_LSTM, B, T, D, 0, 1) > (8 << 20)
+    assert pr.pararnn_workspace_size(pr.PARARNN_LSTM, B, T, D, 0, 1) > (16 << 20)
     lib = pr.load_library()
     rc = lib.pararnn_adjoint_noalloc(pr.PARARNN_LSTM, 16, pr.PARARNN_BF16, 16, None, None,
                                      None, 16, 16, 16, 16, 16, None, None, None, B, T, D,
