@@ -30,6 +30,7 @@ __all__ = [
 PARARNN_F32, PARARNN_BF16 = 0, 1
 PARARNN_GRU, PARARNN_LSTM = 0, 1
 PARARNN_FLAG_INJECT_WITHHOLD = 1
+PARARNN_FLAG_FORCE_CHUNKED = 2
 STATUS_NAMES = {0: "converged", 1: "not_converged", 2: "nonfinite", 3: "timeout"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -236,7 +237,7 @@ def _new_stats(device):
 
 def gru_solve(u, a, bias=None, h0=None, *, tol=1e-6, max_iters=64, hist=False,
               workspace=None, h=None, stats=None, stream=None, opts=None,
-              max_cluster=0):
+              max_cluster=0, flags=0):
     B, T, G, D = u.shape
     dev = u.device
     h = torch.empty((B, T, D), dtype=torch.float32, device=dev) if h is None else h
@@ -244,7 +245,8 @@ def gru_solve(u, a, bias=None, h0=None, *, tol=1e-6, max_iters=64, hist=False,
     ih = torch.empty(max_iters + 2, dtype=torch.int32, device=dev) if hist else None
     ws = workspace if workspace is not None else Workspace(dev)
     buf = ws.get(pararnn_workspace_size(PARARNN_GRU, B, T, D, max_iters, 0), stream)
-    o = opts if opts is not None else _opts(tol, max_iters, max_cluster=max_cluster)
+    o = opts if opts is not None else _opts(tol, max_iters, flags=flags,
+                                            max_cluster=max_cluster)
     pararnn_gru_solve(u, a, bias, h0, h, o, stats, ih, buf, stream)
     return h, stats, ih
 

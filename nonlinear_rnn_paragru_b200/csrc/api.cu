@@ -13,6 +13,10 @@ int launch_gru_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int n
                    cudaStream_t stream);
 int gru_chunk_steps();
 int gru_max_cluster(bool bf16);
+int gru_seq_wpc(int T);
+int gru_row_box_steps();
+int gru_row_channels();
+int launch_gru_seq(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
 int lstm_chunk_steps();
@@ -58,14 +62,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Tensor map over u [B][T][G][D] with a box of 32 channels x G gates x tc steps.
-int make_u_map(CUtensorMap* map, const void* u, bool bf16, int B, int T, int G, int D, int tc) {
+// Tensor map over u [B][T][G][D] with a box of `ch` channels x G gates x tc steps.
+int make_u_map(CUtensorMap* map, const void* u, bool bf16, int B, int T, int G, int D, int tc,
+               int ch = kChan) {
   auto fn = encode_fn();
   if (fn == nullptr) return PARARNN_ERR_CUDA;
   const cuuint64_t es = bf16 ? 2 : 4;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {D * es, (cuuint64_t)G * D * es, (cuuint64_t)T * G * D * es};
-  cuuint32_t box[4] = {(cuuint32_t)kChan, (cuuint32_t)G, (cuuint32_t)tc, 1};
+  cuuint32_t box[4] = {(cuuint32_t)ch, (cuuint32_t)G, (cuuint32_t)tc, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
                   const_cast<void*>(u), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -219,9 +224,21 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const unsigned igrid = iter_hist ? (unsigned)std::min<size_t>((nch + 255) / 256, 1024) : 1u;
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
-  const int e = cell == PARARNN_GRU
-                    ? launch_gru_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream)
-                    : launch_lstm_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream);
+  // ParaGRU, bf16 projections, sequences of up to 4096 steps: whole sequences
+  // per CTA (no cross-CTA scan); otherwise, or on request, the chunked
+  // cluster solve
+  const bool seq = cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && gru_seq_wpc(T) > 0 &&
+                   !(opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED));
+  int e;
+  if (seq) {
+    CUtensorMap rmap;
+    rc = make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels());
+    if (rc) return rc;
+    e = launch_gru_seq(rmap, p, stream);
+  } else
+    e = cell == PARARNN_GRU
+            ? launch_gru_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream)
+            : launch_lstm_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream);
   if (e != 0) return PARARNN_ERR_CUDA;
   if (iter_hist) {
     hist_kernel<<<(unsigned)((nch + 255) / 256), 256, 0, stream>>>(p.chan_k, nch, iter_hist,

@@ -156,3 +156,24 @@ def test_binding_rejects_wrong_dtype(cuda_ok):
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=64, D=32))
     with pytest.raises(TypeError):
         pr.gru_solve(x["u"].cuda(), x["a"].double().cuda(), None, None)
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 1000, 96), (1, 2049, 128), (1, 4096, 64),
+                                   (3, 37, 24)])
+def test_both_solvers_match_oracle(cuda_ok, B, T, D):
+    # T <= 4096 runs whole sequences per CTA by default; the chunked cluster
+    # solve is forced here so both stay covered on short sequences
+    x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        h, st, hist = _solve(x, flags=flags, hist=True)
+        err = np.abs(h - ref).max()
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == B * D
+
+
+def test_whole_sequence_fp32_inputs(cuda_ok):
+    x = make_inputs(WORKLOADS[4].scaled(B=2, T=3000, D=40))
+    h, st, _ = _solve(x)
+    assert np.abs(h - _ref(x)).max() < TOL_STATE
