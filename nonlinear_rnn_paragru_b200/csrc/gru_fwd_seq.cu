@@ -20,24 +20,29 @@
 // its scalar form); the second half is composed after the first when the
 // chunk's map is formed and in the fix-up.  The chunk maps (P, ds) are
 // scanned: over the four chunks of a warp by shuffles; over the 8 warps of the
-// CTA by one scan warp per channel, after one CTA barrier; over the CTAs of
-// the cluster through distributed shared memory (the scan warp pushes the
-// CTA's map and last state into the mailboxes of the CTAs after it, one
-// cluster barrier).  The fix-up adds P_t ds_in.  Mailboxes and per-warp data
-// are double-buffered by the parity of a phase counter that runs on across
-// tiles.  The cluster stops after the update of the first iteration whose
+// CTA after one CTA barrier, each thread composing the maps of the warps
+// before its own from shared memory; over the CTAs of the cluster by remote
+// asynchronous stores into the peers' mailboxes (the CTA's map and last state
+// to the CTAs after it, its residual maximum to all), each completing on the
+// receiver's mbarrier, so a CTA waits only for the bytes it needs and no
+// cluster-wide barrier is taken per iteration.  The fix-up adds P_t ds_in.
+// Mailboxes and per-warp data are double-buffered by the parity of a phase
+// counter that runs on across tiles.  The cluster stops after the update of the first iteration whose
 // residual over the tile is below tol, or after a residual-only evaluation at
 // the cap; the state before each chunk is re-anchored every iteration to its
 // predecessor's pre-update last state plus the incoming delta.
 //
 // Data: the tile's u arrives bf16 by four TMA boxes of 256 steps into the top
-// of the CTA's 98 KB buffer and is expanded in place, once per tile, into the
+// of the CTA's 98 KB buffer (with a, bias and h0 of its channels as 32-byte
+// bulk copies on the same mbarrier; the boxes of the tile after it are
+// prefetched into L2 meanwhile) and is expanded in place, once per tile, into the
 // fp32 arguments -log2e u_z + b'_z, -log2e u_r + b'_r, 2 log2e u_c + b'_c
 // (b' the bias scaled alike), stored per chunk as [gate][pair i][channel]
 // {step i, step i + 16}: one 8-byte load per gate and pair, channel c at slot
 // c ^ ((i >> 1) & 7) of its pair row so that the expansion's stores are free
 // of bank conflicts.  Chunk slots are 3136 bytes, so the four chunks a warp
-// reads fall in alternate 64-byte bank halves.  Steps past T get a z argument of 3e30 (clamped to 63), so z -> 0 and f(h) = h.
+// reads fall in alternate 64-byte bank halves.  Steps past T get a z argument
+// of 3e30 (clamped to 31), so z < 5e-10 and f(h) = h.
 // Clusters are persistent over tiles; the next tile's boxes are issued as
 // soon as the last pass of the current tile is done.  States are stored
 // straight from registers (the 8 lanes of a chunk write a 32-byte run).
@@ -72,30 +77,56 @@ constexpr int kRowMaxCluster = 4;
 constexpr float kRowLn2 = 0.693147180559945309f;
 constexpr int kRowTmax = kRowSteps * kRowMaxCluster;  // 4096
 static_assert(kRowStage % 128 == 0 && kRowBoxBytes % 128 == 0, "TMA destinations");
-// expansion block j writes chunk slots below the staging bytes of blocks > j
-static_assert((kRowBox / kRowL) * kRowS * (kRowNBox - 1) <=
-                  kRowStage + kRowBoxBytes * (kRowNBox - 1), "in-place expansion order");
-static_assert(kRowThreads == kRowBox, "the expansion takes one step of a box per thread");
+static_assert(kRowThreads == (kRowChunks / 2) * kRowH, "the expansion: one (chunk, pair) per thread");
+// expansion block 0 (chunks below kRowChunks / 2) writes below every staged byte
+static_assert((kRowChunks / 2) * kRowS <= kRowStage, "in-place expansion order");
 
-struct RowMailbox {  // written by the cluster peers (push model)
-  float2 agg[kRowMaxCluster][kRowC];   // CTA map (P, ds) per channel, by rank
-  float last[kRowMaxCluster][kRowC];   // CTA's last state before the update
-  float cmax[kRowMaxCluster];          // CTA's max|r|
+struct RowMailbox {  // written by the cluster peers with remote async stores
+  float4 map[kRowMaxCluster][kRowC];   // (P, ds, last state before the update, -) by rank
+  float cmax[kRowMaxCluster];          // CTA max|r| by rank
 };
 
 struct RowShared {
-  float2 wagg[2][kRowWarps][kRowC];  // per (warp, channel) map, then its exclusive prefix
+  float2 wagg[2][kRowWarps][kRowC];  // per (warp, channel) inclusive map of the warp
   float wlast[2][kRowWarps][kRowC];  // per (warp, channel): last state before the update
   float wmax[2][kRowWarps];
-  RowMailbox mbox[2];
-  float bias[3][kRowC];              // scaled bias of the tile's channels
+  __align__(16) RowMailbox mbox[2];
+  __align__(16) float par[7][kRowC];  // a (3 rows), bias (3 rows), h0 of the tile's channels
   uint64_t bar;                      // the staging buffer's mbarrier
+  uint64_t mbar[2];                  // mailbox mbarriers, by parity
 };
 
 __device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// shared::cluster address of the same variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_u32(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// remote asynchronous stores that complete on the receiver's mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, float4 v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(raddr), "r"(__float_as_uint(v.x)), "r"(__float_as_uint(v.y)),
+      "r"(__float_as_uint(v.z)), "r"(__float_as_uint(v.w)), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t raddr, unsigned v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               ::"r"(raddr), "r"(v), "r"(rbar)
+               : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 // channel slot of channel c in pair row i is c ^ row_swizzle(i)
 __host__ __device__ constexpr int row_swizzle(int i) { return (i >> 1) & 7; }
 
@@ -124,19 +155,24 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
     const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kRowH * kRowC * 8);
     const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kRowH * kRowC * 8);
     const float2 HT = H[i];
-    // z, r = 1/(1+e) with e = 2^(argument); one shared reciprocal per step
+    // z, r = 1/(1+e) with e = 2^(argument).  One reciprocal serves the four
+    // sigmoids of the pair and one the two tanh: every argument is clamped
+    // at 31, so the product of four (1+e) stays below 2^124 (the clamp moves
+    // a sigmoid or tanh by under 1e-9).
     const float2 TZ = ffma2(AZ2, HP, UZ), TR = ffma2(AR2, HP, UR);
-    const float2 EZ = f2(ex2(fminf(TZ.x, 63.f)), ex2(fminf(TZ.y, 63.f)));
-    const float2 ER = f2(ex2(fminf(TR.x, 63.f)), ex2(fminf(TR.y, 63.f)));
+    const float2 EZ = f2(ex2(fminf(TZ.x, 31.f)), ex2(fminf(TZ.y, 31.f)));
+    const float2 ER = f2(ex2(fminf(TR.x, 31.f)), ex2(fminf(TR.y, 31.f)));
     const float2 PZ = fadd2(ONE, EZ), PR = fadd2(ONE, ER);
     const float2 PP = fmul2(PZ, PR);
-    const float2 INV = f2(rcp(PP.x), rcp(PP.y));
+    const float inv = rcp(PP.x * PP.y);
+    const float2 INV = f2(PP.y * inv, PP.x * inv);          // 1/(pz pr) per step
     const float2 Z = fmul2(PR, INV), R = fmul2(PZ, INV);
     const float2 RH = fmul2(R, HP);
     const float2 TC = ffma2(AC2, RH, UC);
-    const float2 EC = f2(ex2(TC.x), ex2(TC.y));             // e^{2y}
+    const float2 EC = f2(ex2(fminf(TC.x, 31.f)), ex2(fminf(TC.y, 31.f)));  // e^{2y}
     const float2 PC = fadd2(ONE, EC);
-    const float2 TT = f2(rcp(PC.x), rcp(PC.y));             // t = 1/(1+e^{2y})
+    const float ic = rcp(PC.x * PC.y);
+    const float2 TT = f2(PC.y * ic, PC.x * ic);             // t = 1/(1+e^{2y})
     const float2 C = ffma2(M2, TT, ONE);                    // tanh(y) = 1 - 2t
     const float2 CMH = ffma2(HP, M1, C);
     const float2 F = ffma2(Z, CMH, HP);
@@ -167,13 +203,34 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
 }
 
 // Thread 0: load the tile's four 256-step boxes for CTA `rank` into the
-// staging area.
-__device__ __forceinline__ void row_issue(unsigned char* smem, uint64_t* bar,
-                                          const CUtensorMap* map, int b, int d0, int t0) {
+// staging area, and the tile's a, bias and h0 into `par`, all on `bar`.
+__device__ __forceinline__ void row_issue(unsigned char* smem, RowShared& sh,
+                                          const CUtensorMap* map, const FwdParams& p, int b,
+                                          int d0, int t0) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  mbar_arrive_expect_tx(bar, (unsigned)(kRowNBox * kRowBoxBytes));
+  const unsigned pb = kRowC * 4;
+  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kRowNBox * kRowBoxBytes) + 3 * pb +
+                                     (p.bias ? 3 * pb : 0) + (p.h0 ? pb : 0));
   for (int j = 0; j < kRowNBox; ++j)
-    tma_load_4d(smem + kRowStage + j * kRowBoxBytes, map, bar, d0, 0, t0 + j * kRowBox, b);
+    tma_load_4d(smem + kRowStage + j * kRowBoxBytes, map, &sh.bar, d0, 0, t0 + j * kRowBox, b);
+  for (int g = 0; g < 3; ++g) {
+    bulk_load(&sh.par[g][0], p.a + (size_t)g * p.D + d0, pb, &sh.bar);
+    if (p.bias) bulk_load(&sh.par[3 + g][0], p.bias + (size_t)g * p.D + d0, pb, &sh.bar);
+  }
+  if (p.h0) bulk_load(&sh.par[6][0], p.h0 + (size_t)b * p.D + d0, pb, &sh.bar);
+}
+// L2 prefetch of a tile's boxes (no shared memory touched).
+__device__ __forceinline__ void row_prefetch(const CUtensorMap* map, int b, int d0, int t0) {
+  for (int j = 0; j < kRowNBox; ++j)
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(d0), "r"(0), "r"(t0 + j * kRowBox), "r"(b)
+                 : "memory");
+}
+// Bytes a CTA of rank `rank` receives per exchange phase: the maps of the CTAs
+// before it and the residual maximum of every other CTA.
+__host__ __device__ constexpr unsigned row_rx_bytes(int rank, int cls) {
+  return (unsigned)(rank * kRowC * 16 + (cls - 1) * 4);
 }
 
 template <int CLS>
@@ -190,12 +247,24 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   const int ntiles = p.B * nDTc;
   const int nclus = gridDim.x / CLS, clus = blockIdx.x / CLS;
   const int t0 = rank * kRowSteps;           // first step of this CTA
+  const unsigned rx = row_rx_bytes(rank, CLS);
 
-  if (tid == 0) mbar_init(&sh.bar, 1);
+  if (tid < 7 * kRowC) (&sh.par[0][0])[tid] = 0.f;  // bias and h0 stay 0 when absent
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    if (CLS > 1) {
+      mbar_init(&sh.mbar[0], 1);
+      mbar_init(&sh.mbar[1], 1);
+      mbar_arrive_expect_tx(&sh.mbar[0], rx);
+      mbar_arrive_expect_tx(&sh.mbar[1], rx);
+    }
+  }
   __syncthreads();
+  // the peers' mailbox barriers are armed before anyone sends
+  if (CLS > 1) cluster.sync();
   if (tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    row_issue(smem, &sh.bar, &map, b, (clus - b * nDTc) * kRowC, t0);
+    row_issue(smem, sh, &map, p, b, (clus - b * nDTc) * kRowC, t0);
   }
   const unsigned char* base = smem + q * kRowS;
   int status = 0;
@@ -205,53 +274,61 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kRowC;
     const int d = d0 + c;
     const bool dval = d < p.D;
-    if (tid < 3 * kRowC) {
-      const int g = tid / kRowC, cc = tid - g * kRowC;
-      const float v = (p.bias && d0 + cc < p.D) ? p.bias[g * p.D + d0 + cc] : 0.f;
-      sh.bias[g][cc] = (g == 2 ? 2.f * kLog2e : -kLog2e) * v;
+    const int next = tile + nclus;
+    if (tid == 0 && next < ntiles) {
+      const int b2 = next / nDTc;
+      row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, t0);
     }
     if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
-    __syncthreads();
-    // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32 arguments,
-    // box by box (each box's rows are read before any of its slots is
-    // written).  Thread j takes step j of the box: a warp writes one chunk,
-    // and the swizzle spreads its 32 stores over the 32 banks.
-#pragma unroll 1
-    for (int j = 0; j < kRowNBox; ++j) {
-      uint4 v[3];
-#pragma unroll
-      for (int g = 0; g < 3; ++g)
-        v[g] = *reinterpret_cast<const uint4*>(smem + kRowStage + j * kRowBoxBytes +
-                                               (tid * 3 + g) * 16);
-      __syncthreads();
-      const int t = j * kRowBox + tid;  // step within the CTA
-      const int qq = t / kRowL, s = t % kRowL, i = s % kRowH;
-      float* dst = reinterpret_cast<float*>(smem + qq * kRowS + i * kRowC * 8 + (s / kRowH) * 4);
+    // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32 arguments
+    // in two blocks of 512 steps (each block's rows are read before any of
+    // its slots is written; block 0 writes below all staging bytes).  Thread
+    // (qb, i) takes steps i and i + 16 of chunk qb of the block.
+    {
+      const int qb = tid / kRowH, i = tid % kRowH;
       const int sw = row_swizzle(i);
-      const bool pad = (t0 + t >= p.T);
+#pragma unroll 1
+      for (int blk = 0; blk < 2; ++blk) {
+        const int qq = blk * (kRowChunks / 2) + qb;
+        const int ta = qq * kRowL + i, tb = ta + kRowH;  // steps within the CTA
+        uint4 va[3], vb[3];
 #pragma unroll
-      for (int g = 0; g < 3; ++g) {
-        const float sc = (g == 2) ? 2.f * kLog2e : -kLog2e;
-        const unsigned w[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
-#pragma unroll
-        for (int cc = 0; cc < kRowC; ++cc) {
-          const unsigned bits = (cc & 1) ? (w[cc >> 1] & 0xffff0000u) : (w[cc >> 1] << 16);
-          float o = fmaf(sc, __uint_as_float(bits), sh.bias[g][cc]);
-          if (g == 0 && pad) o = 3e30f;  // clamps to 2^63 whatever a_z h is
-          dst[g * kRowH * kRowC * 2 + (cc ^ sw) * 2] = o;
+        for (int g = 0; g < 3; ++g) {
+          va[g] = *reinterpret_cast<const uint4*>(
+              smem + kRowStage + (ta / kRowBox) * kRowBoxBytes + ((ta % kRowBox) * 3 + g) * 16);
+          vb[g] = *reinterpret_cast<const uint4*>(
+              smem + kRowStage + (tb / kRowBox) * kRowBoxBytes + ((tb % kRowBox) * 3 + g) * 16);
         }
+        __syncthreads();
+        const bool pa = t0 + ta >= p.T, pbd = t0 + tb >= p.T;
+        unsigned char* dst = smem + qq * kRowS + i * kRowC * 8;
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+          const float sc = (g == 2) ? 2.f * kLog2e : -kLog2e;
+          const unsigned wa[4] = {va[g].x, va[g].y, va[g].z, va[g].w};
+          const unsigned wb[4] = {vb[g].x, vb[g].y, vb[g].z, vb[g].w};
+#pragma unroll
+          for (int cc = 0; cc < kRowC; ++cc) {
+            const int sh16 = (cc & 1) ? 0 : 16;
+            const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
+            const float xa = __uint_as_float((wa[cc >> 1] << sh16) & mk);
+            const float xb = __uint_as_float((wb[cc >> 1] << sh16) & mk);
+            const float bs = sc * sh.par[3 + g][cc];
+            float2 o = ffma2(f2(sc, sc), f2(xa, xb), f2(bs, bs));
+            if (g == 0) {  // steps past T: z < 5e-10 whatever a_z h is
+              if (pa) o.x = 3e30f;
+              if (pbd) o.y = 3e30f;
+            }
+            *reinterpret_cast<float2*>(dst + g * kRowH * kRowC * 8 + (cc ^ sw) * 8) = o;
+          }
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
-    float az = 0.f, ar = 0.f, ac = 0.f;
-    if (dval) {
-      az = p.a[d];
-      ar = p.a[p.D + d];
-      ac = p.a[2 * p.D + d];
-    }
+    const float az = sh.par[0][c], ar = sh.par[1][c], ac = sh.par[2][c];
     const float az2 = -kLog2e * az, ar2 = -kLog2e * ar, ac2 = 2.f * kLog2e * ac;
     const float2 AZ2 = f2(az2, az2), AR2 = f2(ar2, ar2), AC2 = f2(ac2, ac2), AZ = f2(az, az);
-    const float h0v = (dval && p.h0) ? p.h0[(size_t)b * p.D + d] : 0.f;
+    const float h0v = sh.par[6][c];
     const bool first = (rank == 0 && q == 0);  // chunk holding step 0
 
     float2 H[kRowH], P[kRowH];
@@ -266,6 +343,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     for (;; ++k) {
       const bool cap = (k >= p.max_iters);
       const int par = phase & 1;
+      const unsigned mpar = (phase >> 1) & 1;  // phase parity of mbar[par]
       ++phase;
       const float last_pre = H[kRowH - 1].y;
       float2 DL, PA;
@@ -301,63 +379,55 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       }
       if (lane == 0) sh.wmax[par][warp] = __uint_as_float(wm);
       __syncthreads();
-      {
-        // scan warp for channel `warp` (one per channel): lane l < 8 holds
-        // warp l's map; inclusive scan by shuffles, written back in place as
-        // the exclusive prefix (CTA incoming delta -> delta entering warp l)
-        static_assert(kRowWarps == kRowC, "one scan warp per channel");
-        const int cs = warp;
-        float2 e = make_float2(1.f, 0.f);
-        if (lane < kRowWarps) e = sh.wagg[par][lane][cs];
+      // maps of the warps before this one: CTA incoming delta -> delta
+      // entering this warp; and the CTA's residual maximum
+      float cP = 1.f, cd = 0.f;
 #pragma unroll
-        for (int o = 1; o < kRowWarps; o <<= 1) {
-          const float pP = __shfl_up_sync(kFull, e.x, o), pd = __shfl_up_sync(kFull, e.y, o);
-          if (lane >= o) {
-            e.y = fmaf(e.x, pd, e.y);
-            e.x *= pP;
-          }
-        }
-        float sP = __shfl_up_sync(kFull, e.x, 1), sd = __shfl_up_sync(kFull, e.y, 1);
-        if (lane == 0) {
-          sP = 1.f;
-          sd = 0.f;
-        }
-        // the CTA's residual maximum (warp 0 publishes it)
-        const float wv = (lane < kRowWarps) ? sh.wmax[par][lane] : 0.f;
-        const unsigned cm = __reduce_max_sync(kFull, __float_as_uint(wv));
-        if (lane < kRowWarps) sh.wagg[par][lane][cs] = make_float2(sP, sd);
-        if (CLS > 1 && lane == kRowWarps - 1) {
-          // this CTA's map and last state, to every CTA from this one on
-          const float lastc = sh.wlast[par][kRowWarps - 1][cs];
-          for (int r = rank; r < CLS; ++r) {
-            RowMailbox* mb = (r == rank) ? &sh.mbox[par] : cluster.map_shared_rank(&sh.mbox[par], r);
-            mb->agg[rank][cs] = e;
-            mb->last[rank][cs] = lastc;
-          }
-        }
-        if (warp == 0 && lane < CLS) {
-          RowMailbox* mb =
-              (lane == rank) ? &sh.mbox[par] : cluster.map_shared_rank(&sh.mbox[par], lane);
-          mb->cmax[rank] = __uint_as_float(cm);
+      for (int w = 0; w < kRowWarps - 1; ++w) {
+        if (w < warp) {
+          const float2 a2 = sh.wagg[par][w][c];
+          cd = fmaf(a2.x, cd, a2.y);
+          cP *= a2.x;
         }
       }
-      if (CLS > 1)
-        cluster.sync();
-      else
-        __syncthreads();
-      const float2 pre = sh.wagg[par][warp][c];
-      float tmax = 0.f;
+      const float4 wm0 = *reinterpret_cast<const float4*>(&sh.wmax[par][0]);
+      const float4 wm1 = *reinterpret_cast<const float4*>(&sh.wmax[par][4]);
+      float tmax = fmax_nan(fmax_nan(fmax_nan(wm0.x, wm0.y), fmax_nan(wm0.z, wm0.w)),
+                            fmax_nan(fmax_nan(wm1.x, wm1.y), fmax_nan(wm1.z, wm1.w)));
       float din_cta = 0.f;          // delta entering this CTA
       float prev_cta_last = h0v;    // state before this CTA's first step
-#pragma unroll
-      for (int r = 0; r < CLS; ++r) {
-        tmax = fmax_nan(tmax, sh.mbox[par].cmax[r]);
-        if (r < rank) {
-          const float2 a2 = sh.mbox[par].agg[r][c];
-          din_cta = fmaf(a2.x, din_cta, a2.y);
+      if (CLS > 1) {
+        if (warp == kRowWarps - 1) {
+          // the CTA map of channel c: last warp's inclusive map after the
+          // warps before it; to every CTA after this one.  Lanes r < CLS
+          // send the residual maximum to CTA r.
+          const float cmax = tmax;
+          if (kk == kRowK - 1) {
+            const float4 v = make_float4(IP * cP, fmaf(IP, cd, Id), last_pre, 0.f);
+            for (int r = rank + 1; r < CLS; ++r)
+              st_async_v4(mapa_u32(smem_u32(&sh.mbox[par].map[rank][c]), r), v,
+                          mapa_u32(smem_u32(&sh.mbar[par]), r));
+          }
+          if (lane < CLS && lane != rank)
+            st_async_b32(mapa_u32(smem_u32(&sh.mbox[par].cmax[rank]), lane),
+                         __float_as_uint(cmax), mapa_u32(smem_u32(&sh.mbar[par]), lane));
         }
+        if (!mbar_wait_bounded(&sh.mbar[par], mpar, p.timeout_ns) && status == 0)
+          status = PARARNN_STATUS_TIMEOUT;
+#pragma unroll
+        for (int r = 0; r < CLS; ++r) {
+          if (r != rank) tmax = fmax_nan(tmax, sh.mbox[par].cmax[r]);
+          if (r < rank) {
+            const float4 a4 = sh.mbox[par].map[r][c];
+            din_cta = fmaf(a4.x, din_cta, a4.y);
+            if (r == rank - 1) prev_cta_last = a4.z;
+          }
+        }
+        // re-arm this mailbox for its next phase; every thread of the CTA
+        // has passed the wait before any peer can send that phase's bytes
+        __syncwarp();
+        if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
-      if (CLS > 1 && rank > 0) prev_cta_last = sh.mbox[par].last[rank - 1][c];
       // the histogram input uses the tile's maximum, an upper bound of the
       // channel's own residual
       if (!(tmax < p.tol)) last_bad = k;
@@ -368,7 +438,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
         break;
       }
-      const float cin = fmaf(pre.x, din_cta, pre.y);  // delta entering this warp
+      const float cin = fmaf(cP, din_cta, cd);  // delta entering this warp
       const float din = first ? 0.f : fmaf(xP, cin, xd);
       float prev_last = __shfl_up_sync(kFull, last_pre, kRowC);
       if (kk == 0) prev_last = (warp == 0) ? prev_cta_last : sh.wlast[par][warp - 1][c];
@@ -382,10 +452,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     }
     // every thread of the CTA is past its last pass of this tile (the
     // barrier of the last exchange): the staging area takes the next tile
-    const int next = tile + nclus;
     if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_issue(smem, &sh.bar, &map, b2, (next - b2 * nDTc) * kRowC, t0);
+      row_issue(smem, sh, &map, p, b2, (next - b2 * nDTc) * kRowC, t0);
     }
 
     // ---- states straight from registers
@@ -416,6 +485,8 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   }
   const int st = __reduce_max_sync(kFull, status);
   if (lane == 0 && st) atomicMax(&p.stats->status, st);
+  // no CTA leaves while a peer may still store into its mailboxes
+  if (CLS > 1) cluster.sync();
 }
 
 // ------------------------------------------------------------- launcher --
