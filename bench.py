@@ -38,10 +38,22 @@ UNIT = "tokch/s"
 # Counters of the dominant kernel taken with ncu on this build (one launch of
 # the default workload; see profiles/).  None when not captured for the
 # kernel as it stands.
-NCU_TRAFFIC_BYTES = {}
-# special-function (MUFU) operations per element and cell evaluation, as the
-# kernels issue them: ParaGRU 3 ex2 + 2 rcp; ParaLSTM 5 ex2 + 3 rcp
-MUFU_PER_EVAL = {"gru": 5, "lstm": 8}
+NCU_TRAFFIC_BYTES = {
+    # profiles/gru_newton_row_b8_t4096_d1024.md: dram read + write of one launch
+    ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 212_082_944 + 108_779_520,
+}
+# The forward kernel a workload runs and its special-function (MUFU)
+# operations per element and cell evaluation, as the kernel issues them:
+#   gru_newton_row (ParaGRU, bf16 u, T <= 4096): 3 ex2 + 1 rcp (one reciprocal
+#     serves the four sigmoids of a step pair, one the pair's two tanh);
+#   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
+#   lstm_newton_fused: 5 ex2 + 3 rcp.
+def fwd_kernel(w):
+    if w.cell == "lstm":
+        return "lstm_newton_fused", 8
+    if w.u_dtype == "bf16" and w.T <= 4096:
+        return "gru_newton_row", 4
+    return "gru_newton_fused", 5
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
 def fwd_bytes(w):
     ue = 2 if w.u_dtype == "bf16" else 4
@@ -296,15 +308,15 @@ def run_ours(args, world, rank):
     peaks, src = measured_peaks()
     f_mhz = clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
     mufu_peak = 148 * 16 * f_mhz * 1e6 / 1e12          # Tops/s
-    mufu_done = w.tokch * st["evals"] * MUFU_PER_EVAL[w.cell] / (fwd_ms * 1e-3) / 1e12
+    kern, mufu_per_eval = fwd_kernel(w)
+    mufu_done = w.tokch * st["evals"] * mufu_per_eval / (fwd_ms * 1e-3) / 1e12
     hbm_ach = w.tokch * fwd_bytes(w) / (fwd_ms * 1e-3) / 1e9
-    kern = ("lstm_newton_fused" if w.cell == "lstm" else "gru_newton_fused")
     traffic = NCU_TRAFFIC_BYTES.get((kern, w.name))
     roofline = {"bound": "alu", "kernel": kern, "achieved": round(mufu_done, 3),
                 "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
                 "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
                 "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
-                "ops_per_launch": w.tokch * st["evals"] * MUFU_PER_EVAL[w.cell]}
+                "ops_per_launch": w.tokch * st["evals"] * mufu_per_eval}
     hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
            "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,
            "fwd_bytes_per_tokch": fwd_bytes(w)}
