@@ -88,9 +88,9 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
 /* opts.flags */
 #define PARARNN_FLAG_INJECT_WITHHOLD 1u /* testing: chunk `inject_chunk` never
                                            publishes its look-back record */
-#define PARARNN_FLAG_FORCE_CHUNKED 2u   /* ParaGRU, bf16 u, T <= 4096: use the
-                                           chunked (cluster + look-back) solve
-                                           instead of whole sequences per CTA */
+#define PARARNN_FLAG_FORCE_CHUNKED 2u   /* bf16 u, T <= 4096: use the chunked
+                                           (cluster + look-back) solve instead
+                                           of the whole-sequence row kernels */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */

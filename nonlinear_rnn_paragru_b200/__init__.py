@@ -253,7 +253,7 @@ def gru_solve(u, a, bias=None, h0=None, *, tol=1e-6, max_iters=64, hist=False,
 
 def lstm_solve(u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
                hist=False, workspace=None, c=None, h=None, stats=None,
-               stream=None, opts=None, max_cluster=0):
+               stream=None, opts=None, max_cluster=0, flags=0):
     B, T, G, D = u.shape
     dev = u.device
     c = torch.empty((B, T, D), dtype=torch.float32, device=dev) if c is None else c
@@ -262,7 +262,8 @@ def lstm_solve(u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
     ih = torch.empty(max_iters + 2, dtype=torch.int32, device=dev) if hist else None
     ws = workspace if workspace is not None else Workspace(dev)
     buf = ws.get(pararnn_workspace_size(PARARNN_LSTM, B, T, D, max_iters, 0), stream)
-    o = opts if opts is not None else _opts(tol, max_iters, max_cluster=max_cluster)
+    o = opts if opts is not None else _opts(tol, max_iters, flags=flags,
+                                            max_cluster=max_cluster)
     pararnn_lstm_solve(u, a, bias, c0, h0, c, h, o, stats, ih, buf, stream)
     return c, h, stats, ih
 

@@ -21,6 +21,10 @@ int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int 
                     cudaStream_t stream);
 int lstm_chunk_steps();
 int lstm_max_cluster(bool bf16);
+int lstm_row_cluster(int T);
+int lstm_row_box_steps();
+int lstm_row_channels();
+int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
 int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, const float* bias,
                         const float* c0, const float* h0, float* c, float* h, int B, int T,
                         int D, cudaStream_t stream);
@@ -224,21 +228,24 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const unsigned igrid = iter_hist ? (unsigned)std::min<size_t>((nch + 255) / 256, 1024) : 1u;
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
-  // ParaGRU, bf16 projections, sequences of up to 4096 steps: whole sequences
-  // per CTA (no cross-CTA scan); otherwise, or on request, the chunked
-  // cluster solve
-  const bool seq = cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && gru_seq_wpc(T) > 0 &&
-                   !(opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED));
+  // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
+  // 8-channel tile holds the whole sequence (row kernels); otherwise, or on
+  // request, the chunked cluster + look-back solve
+  const bool force = opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED);
+  const bool bf16 = u_dtype == PARARNN_BF16;
+  const bool row_gru = cell == PARARNN_GRU && bf16 && gru_seq_wpc(T) > 0 && !force;
+  const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
   int e;
-  if (seq) {
+  if (row_gru || row_lstm) {
     CUtensorMap rmap;
-    rc = make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels());
+    rc = row_gru ? make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels())
+                 : make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(),
+                              lstm_row_channels());
     if (rc) return rc;
-    e = launch_gru_seq(rmap, p, stream);
+    e = row_gru ? launch_gru_seq(rmap, p, stream) : launch_lstm_row(rmap, p, stream);
   } else
-    e = cell == PARARNN_GRU
-            ? launch_gru_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream)
-            : launch_lstm_fwd(map, u_dtype == PARARNN_BF16, p, (int)nctas, stream);
+    e = cell == PARARNN_GRU ? launch_gru_fwd(map, bf16, p, (int)nctas, stream)
+                            : launch_lstm_fwd(map, bf16, p, (int)nctas, stream);
   if (e != 0) return PARARNN_ERR_CUDA;
   if (iter_hist) {
     hist_kernel<<<(unsigned)((nch + 255) / 256), 256, 0, stream>>>(p.chan_k, nch, iter_hist,

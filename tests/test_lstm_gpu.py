@@ -81,6 +81,22 @@ def test_capped_iterates_match_oracle_newton(cuda_ok, n):
     assert max(np.abs(c - r["c"]).max(), np.abs(h - r["h"]).max()) < TOL_STATE
 
 
+@pytest.mark.parametrize("B,T,D", [(2, 500, 96), (1, 1000, 64), (1, 2049, 32), (1, 4096, 40),
+                                   (3, 37, 24)])
+def test_both_solvers_match_oracle(cuda_ok, B, T, D):
+    # bf16 u with T <= 4096 runs the whole-sequence row kernel (clusters of
+    # 1, 2, 4 and 8 CTAs above); the chunked solve is forced here so both stay
+    # covered on short sequences
+    x = make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D))
+    rc, rh = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        c, h, st, hist = _solve(x, flags=flags, hist=True)
+        err = max(np.abs(c - rc).max(), np.abs(h - rh).max())
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == B * D
+
+
 def test_seq_baseline_matches_oracle(cuda_ok):
     x = make_inputs(WORKLOADS[3].scaled(B=2, T=300, D=64))
     c, h = pr.seq_baseline(pr.PARARNN_LSTM, x["u"].cuda(), x["a"].cuda(),
