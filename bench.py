@@ -47,11 +47,15 @@ NCU_TRAFFIC_BYTES = {
 #   gru_newton_row (ParaGRU, bf16 u, T <= 4096): 3 ex2 + 1 rcp (one reciprocal
 #     serves the four sigmoids of a step pair, one the pair's two tanh);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
-#   lstm_newton_fused: 5 ex2 + 3 rcp.
+#   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096): 5 ex2 + 1.5 rcp (one
+#     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
+#     one for the two tanh(c'));
+#   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
 def fwd_kernel(w):
+    row = w.u_dtype == "bf16" and w.T <= 4096
     if w.cell == "lstm":
-        return "lstm_newton_fused", 8
-    if w.u_dtype == "bf16" and w.T <= 4096:
+        return ("lstm_newton_row", 6.5) if row else ("lstm_newton_fused", 8)
+    if row:
         return "gru_newton_row", 4
     return "gru_newton_fused", 5
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
@@ -227,6 +231,28 @@ class Path:
             pr.pararnn_gru_solve(x["u"], x["a"], x["bias"], x["h0"], self.h, self.opts,
                                  self.stats, self.hist, self.fbuf)
 
+    def element_evaluations(self, x=None):
+        """Cell evaluations performed by one solve, summed over (b, t, d).
+
+        Every tile stops on its own, so this is counted from the per-channel
+        convergence histogram: a channel whose tile first passed the test at
+        iteration k was evaluated k + 1 times.  Exact for the row kernels
+        (a tile is a whole sequence); for the chunked kernels a channel
+        reports its slowest chunk, so this is an upper bound there.  Runs one
+        untimed solve.
+        """
+        x = x or self.x
+        pr = self.pr
+        hb = torch.zeros(66, dtype=torch.int32, device="cuda")
+        if self.lstm:
+            pr.pararnn_lstm_solve(x["u"], x["a"], x["bias"], x["c0"], x["h0"], self.c,
+                                  self.h, self.opts, self.stats, hb, self.fbuf)
+        else:
+            pr.pararnn_gru_solve(x["u"], x["a"], x["bias"], x["h0"], self.h, self.opts,
+                                 self.stats, hb, self.fbuf)
+        hist = hb.cpu().tolist()
+        return self.w.T * sum(n * (k + 1) for k, n in enumerate(hist))
+
     def backward(self, x=None):
         x = x or self.x
         pr = self.pr
@@ -309,14 +335,16 @@ def run_ours(args, world, rank):
     f_mhz = clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
     mufu_peak = 148 * 16 * f_mhz * 1e6 / 1e12          # Tops/s
     kern, mufu_per_eval = fwd_kernel(w)
-    mufu_done = w.tokch * st["evals"] * mufu_per_eval / (fwd_ms * 1e-3) / 1e12
+    elem_evals = path.element_evaluations()
+    mufu_done = elem_evals * mufu_per_eval / (fwd_ms * 1e-3) / 1e12
     hbm_ach = w.tokch * fwd_bytes(w) / (fwd_ms * 1e-3) / 1e9
     traffic = NCU_TRAFFIC_BYTES.get((kern, w.name))
     roofline = {"bound": "alu", "kernel": kern, "achieved": round(mufu_done, 3),
                 "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
                 "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
                 "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
-                "ops_per_launch": w.tokch * st["evals"] * mufu_per_eval}
+                "ops_per_launch": elem_evals * mufu_per_eval,
+                "mean_evals": round(elem_evals / w.tokch, 3)}
     hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
            "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,
            "fwd_bytes_per_tokch": fwd_bytes(w)}

@@ -94,6 +94,7 @@ struct RowShared {
   __align__(16) float par[7][kRowC];  // a (3 rows), bias (3 rows), h0 of the tile's channels
   uint64_t bar;                      // the staging buffer's mbarrier
   uint64_t mbar[2];                  // mailbox mbarriers, by parity
+  int ntile[4];                      // tile indices published by cluster rank 0
 };
 
 __device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
@@ -270,11 +271,25 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   int status = 0;
   int n = 0;
   unsigned phase = 0;  // exchange phases so far, over all tiles
-  for (int tile = clus; tile < ntiles; tile += nclus, ++n) {
+  // Tiles: the first two of a cluster are clus and clus + nclus; after that
+  // each cluster takes the next ticket of a counter (reset per launch), so
+  // clusters that meet slowly converging tiles take fewer.  Cluster rank 0
+  // draws the ticket for tile n + 2 at the start of tile n and publishes it
+  // into every CTA's ring at the end of tile n; the barrier opening each tile
+  // makes it visible.  Tickets rise monotonically, so no tile is skipped.
+  const bool drawer = rank == 0 && tid == kRowThreads - 32;
+  unsigned ticket = 0;
+  int tile = clus, next = clus + nclus;
+  for (; tile < ntiles; tile = next, ++n) {
+    if (CLS > 1)
+      cluster.sync();
+    else
+      __syncthreads();
+    if (n >= 1) next = sh.ntile[(n + 1) & 3];
+    if (drawer) ticket = atomicAdd(&p.hdr->ticket, 1u);
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kRowC;
     const int d = d0 + c;
     const bool dval = d < p.D;
-    const int next = tile + nclus;
     if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
       row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, t0);
@@ -457,6 +472,13 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       row_issue(smem, sh, &map, p, b2, (next - b2 * nDTc) * kRowC, t0);
     }
 
+    if (drawer) {
+      const int nt = 2 * nclus + (int)ticket;
+      for (int r = 0; r < CLS; ++r) {
+        int* dst = (r == rank) ? &sh.ntile[(n + 2) & 3] : cluster.map_shared_rank(&sh.ntile[(n + 2) & 3], r);
+        *dst = nt;
+      }
+    }
     // ---- states straight from registers
     bool bad = false;
     if (dval) {
