@@ -25,6 +25,13 @@ int lstm_row_cluster(int T);
 int lstm_row_box_steps();
 int lstm_row_channels();
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
+int adjoint_row_cluster(int T);
+int adjoint_row_channels();
+int adjoint_row_box_steps(int which);
+size_t adjoint_row_part_bytes(int B, int T, int D);
+int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bias,
+                       const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
+                       int T, int D, int* status, void* ws, cudaStream_t stream);
 int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, const float* bias,
                         const float* c0, const float* h0, float* c, float* h, int B, int T,
                         int D, cudaStream_t stream);
@@ -83,13 +90,13 @@ int make_u_map(CUtensorMap* map, const void* u, bool bf16, int B, int T, int G, 
   return r == CUDA_SUCCESS ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 
-// Tensor map over an fp32 [B][T][D] array with a box of 32 channels x tc steps.
-int make_s_map(CUtensorMap* map, const float* x, int B, int T, int D, int tc) {
+// Tensor map over an fp32 [B][T][D] array with a box of `ch` channels x tc steps.
+int make_s_map(CUtensorMap* map, const float* x, int B, int T, int D, int tc, int ch = kChan) {
   auto fn = encode_fn();
   if (fn == nullptr) return PARARNN_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)T * D * 4};
-  cuuint32_t box[3] = {(cuuint32_t)kChan, (cuuint32_t)tc, 1};
+  cuuint32_t box[3] = {(cuuint32_t)ch, (cuuint32_t)tc, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(x), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -310,6 +317,20 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
     return PARARNN_ERR_MISALIGNED;
   if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const int G = cell == PARARNN_GRU ? 3 : 4;
+  // ParaGRU, bf16 projections, sequences of up to 4096 steps: a cluster of
+  // CTAs per 8-channel tile holds the whole sequence (no look-back)
+  if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&
+      adjoint_row_part_bytes(B, T, D) <= ws_bytes) {
+    const int ch = adjoint_row_channels();
+    CUtensorMap rmaps[3];  // u, h (states before each step), dL/dh
+    rc = make_u_map(&rmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
+    if (!rc) rc = make_s_map(&rmaps[1], h, B, T, D, adjoint_row_box_steps(1), ch);
+    if (!rc) rc = make_s_map(&rmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+    if (rc) return rc;
+    const int e = launch_adjoint_row(rmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status,
+                                     workspace, (cudaStream_t)stream);
+    return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
   const int tc = adjoint_chunk_steps(cell);
   CUtensorMap maps[4];  // u, h, c (ParaLSTM; h again for ParaGRU), dL/dh
   rc = make_u_map(&maps[0], u, u_dtype == PARARNN_BF16, B, T, G, D, tc);

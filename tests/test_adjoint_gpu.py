@@ -61,6 +61,15 @@ def test_gru_adjoint_shapes(cuda_ok, B, T, D):
     _check_gru(x, h)
 
 
+def test_gru_adjoint_lookback_path(cuda_ok):
+    # fp32 projections and T > 4096 take the chunked look-back adjoint; bf16
+    # with T <= 4096 (the shapes above) the whole-sequence one
+    x = make_inputs(WORKLOADS[4].scaled(B=2, T=700, D=24), with_grad=True)
+    _check_gru(x, oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"]))
+    y = make_inputs(WORKLOADS[2].scaled(B=1, T=5000, D=16))
+    _check_gru(y, oracle.gru_seq(y["u"], y["a"], y["bias"], y["h0"]))
+
+
 @pytest.mark.parametrize("B,T,D", [(2, 700, 64), (1, 128, 32), (1, 3, 8), (1, 2500, 40)])
 def test_lstm_adjoint_shapes(cuda_ok, B, T, D):
     x = make_inputs(WORKLOADS[5].scaled(B=B, T=T, D=D))
