@@ -111,3 +111,34 @@ def test_adjoint_is_bitwise_reproducible(cuda_ok):
     b = _gpu_adjoint(pr.PARARNN_GRU, x, h)
     for k in ("du", "da", "dbias", "dh0"):
         assert np.array_equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("T", [1500, 4500])
+def test_gru_adjoint_nonzero_h0_without_bias(cuda_ok, T):
+    # the state before the first step is h0, not the zero fill of a load that
+    # starts before the sequence; an absent bias reads as zero.  T = 1500
+    # takes the whole-sequence adjoint, T = 4500 the look-back one.
+    x = make_inputs(WORKLOADS[2].scaled(B=2, T=T, D=24))
+    x["h0"] = torch.randn((2, 24), generator=torch.Generator().manual_seed(7)) * 0.5
+    x["bias"] = torch.zeros_like(x["bias"])
+    h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+    d = "cuda"
+    out = pr.adjoint(pr.PARARNN_GRU, x["u"].to(d), x["a"].to(d), None, x["h0"].to(d),
+                     torch.as_tensor(h, dtype=torch.float32).to(d).contiguous(),
+                     x["dLdh"].to(d))
+    torch.cuda.synchronize()
+    g = {k: (v.cpu().numpy() if v is not None else None) for k, v in out.items()}
+    assert int(g["status"][0]) == 0
+    ref = oracle.gru_bptt(x["u"], x["a"], x["bias"], x["h0"],
+                          h.astype(np.float32).astype(np.float64), x["dLdh"])
+    for k in ("du", "da", "dbias", "dh0"):
+        assert _rel(g[k], ref[k]) <= TOL_GRAD, (k, _rel(g[k], ref[k]))
+
+
+def test_lstm_adjoint_nonzero_initial_state(cuda_ok):
+    x = make_inputs(WORKLOADS[5].scaled(B=2, T=700, D=32))
+    gen = torch.Generator().manual_seed(9)
+    x["c0"] = torch.randn((2, 32), generator=gen) * 0.5
+    x["h0"] = torch.randn((2, 32), generator=gen) * 0.5
+    c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    _check_lstm(x, c, h)

@@ -177,3 +177,15 @@ def test_whole_sequence_fp32_inputs(cuda_ok):
     x = make_inputs(WORKLOADS[4].scaled(B=2, T=3000, D=40))
     h, st, _ = _solve(x)
     assert np.abs(h - _ref(x)).max() < TOL_STATE
+
+
+def test_absent_bias_and_h0_read_as_zero(cuda_ok):
+    # null bias and h0 on both solvers equal explicit zeros
+    x = make_inputs(WORKLOADS[2].scaled(B=2, T=1500, D=40))
+    x["bias"] = torch.zeros_like(x["bias"])
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        h, st, _ = pr.gru_solve(x["u"].cuda(), x["a"].cuda(), None, None, flags=flags)
+        torch.cuda.synchronize()
+        assert np.abs(h.cpu().numpy() - ref).max() < TOL_STATE, flags
+        assert pr.read_stats(st)["status"] == "converged"

@@ -104,3 +104,19 @@ def test_seq_baseline_matches_oracle(cuda_ok):
     torch.cuda.synchronize()
     rc, rh = _ref(x)
     assert max(np.abs(c.cpu().numpy() - rc).max(), np.abs(h.cpu().numpy() - rh).max()) < TOL_STATE
+
+
+def test_absent_bias_with_nonzero_state_both_solvers(cuda_ok):
+    x = make_inputs(WORKLOADS[3].scaled(B=2, T=1100, D=32))
+    x["bias"] = torch.zeros_like(x["bias"])
+    gen = torch.Generator().manual_seed(11)
+    x["c0"] = torch.randn((2, 32), generator=gen) * 0.5
+    x["h0"] = torch.randn((2, 32), generator=gen) * 0.5
+    rc, rh = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        c, h, st, _ = pr.lstm_solve(x["u"].cuda(), x["a"].cuda(), None, x["c0"].cuda(),
+                                    x["h0"].cuda(), flags=flags)
+        torch.cuda.synchronize()
+        err = max(np.abs(c.cpu().numpy() - rc).max(), np.abs(h.cpu().numpy() - rh).max())
+        assert err < TOL_STATE, (flags, err)
+        assert pr.read_stats(st)["status"] == "converged"
