@@ -91,7 +91,8 @@ struct RowShared {
   float wlast[2][kRowWarps][kRowC];  // per (warp, channel): last state before the update
   float wmax[2][kRowWarps];
   __align__(16) RowMailbox mbox[2];
-  __align__(16) float par[7][kRowC];  // a (3 rows), bias (3 rows), h0 of the tile's channels
+  // a (3 rows), bias (3 rows), h0 of a tile's channels, by tile parity
+  __align__(16) float par[2][7][kRowC];
   uint64_t bar;                      // the staging buffer's mbarrier
   uint64_t mbar[2];                  // mailbox mbarriers, by parity
   int ntile[4];                      // tile indices published by cluster rank 0
@@ -204,21 +205,21 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
 }
 
 // Thread 0: load the tile's four 256-step boxes for CTA `rank` into the
-// staging area, and the tile's a, bias and h0 into `par`, all on `bar`.
+// staging area, on `bar`.
 __device__ __forceinline__ void row_issue(unsigned char* smem, RowShared& sh,
-                                          const CUtensorMap* map, const FwdParams& p, int b,
-                                          int d0, int t0) {
+                                          const CUtensorMap* map, int b, int d0, int t0) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  const unsigned pb = kRowC * 4;
-  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kRowNBox * kRowBoxBytes) + 3 * pb +
-                                     (p.bias ? 3 * pb : 0) + (p.h0 ? pb : 0));
+  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kRowNBox * kRowBoxBytes));
   for (int j = 0; j < kRowNBox; ++j)
     tma_load_4d(smem + kRowStage + j * kRowBoxBytes, map, &sh.bar, d0, 0, t0 + j * kRowBox, b);
-  for (int g = 0; g < 3; ++g) {
-    bulk_load(&sh.par[g][0], p.a + (size_t)g * p.D + d0, pb, &sh.bar);
-    if (p.bias) bulk_load(&sh.par[3 + g][0], p.bias + (size_t)g * p.D + d0, pb, &sh.bar);
-  }
-  if (p.h0) bulk_load(&sh.par[6][0], p.h0 + (size_t)b * p.D + d0, pb, &sh.bar);
+}
+// Parameter j (0..55) of the tile at (b, d0): a[g][c] (j < 24), bias[g][c]
+// (j < 48, 0 when absent), h0[c] (0 when absent).
+__device__ __forceinline__ float row_param(const FwdParams& p, int j, int b, int d0) {
+  const int row = j / kRowC, c = j % kRowC;
+  if (row < 3) return p.a[(size_t)row * p.D + d0 + c];
+  if (row < 6) return p.bias ? p.bias[(size_t)(row - 3) * p.D + d0 + c] : 0.f;
+  return p.h0 ? p.h0[(size_t)b * p.D + d0 + c] : 0.f;
 }
 // L2 prefetch of a tile's boxes (no shared memory touched).
 __device__ __forceinline__ void row_prefetch(const CUtensorMap* map, int b, int d0, int t0) {
@@ -250,7 +251,11 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   const int t0 = rank * kRowSteps;           // first step of this CTA
   const unsigned rx = row_rx_bytes(rank, CLS);
 
-  if (tid < 7 * kRowC) (&sh.par[0][0])[tid] = 0.f;  // bias and h0 stay 0 when absent
+  // the first tile's parameters; later tiles' are loaded a tile ahead
+  if (tid < 7 * kRowC && clus < ntiles) {
+    const int b = clus / nDTc;
+    (&sh.par[0][0][0])[tid] = row_param(p, tid, b, (clus - b * nDTc) * kRowC);
+  }
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
     if (CLS > 1) {
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   if (CLS > 1) cluster.sync();
   if (tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    row_issue(smem, sh, &map, p, b, (clus - b * nDTc) * kRowC, t0);
+    row_issue(smem, sh, &map, b, (clus - b * nDTc) * kRowC, t0);
   }
   const unsigned char* base = smem + q * kRowS;
   int status = 0;
@@ -287,6 +292,14 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       __syncthreads();
     if (n >= 1) next = sh.ntile[(n + 1) & 3];
     if (drawer) ticket = atomicAdd(&p.hdr->ticket, 1u);
+    // the next tile's parameters: loaded now, stored at the end of this tile
+    const int pj = tid - 32;
+    float pnext = 0.f;
+    if (pj >= 0 && pj < 7 * kRowC && next < ntiles) {
+      const int b2 = next / nDTc;
+      pnext = row_param(p, pj, b2, (next - b2 * nDTc) * kRowC);
+    }
+    const int pb = n & 1;
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kRowC;
     const int d = d0 + c;
     const bool dval = d < p.D;
@@ -328,7 +341,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
             const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
             const float xa = __uint_as_float((wa[cc >> 1] << sh16) & mk);
             const float xb = __uint_as_float((wb[cc >> 1] << sh16) & mk);
-            const float bs = sc * sh.par[3 + g][cc];
+            const float bs = sc * sh.par[pb][3 + g][cc];
             float2 o = ffma2(f2(sc, sc), f2(xa, xb), f2(bs, bs));
             if (g == 0) {  // steps past T: z < 5e-10 whatever a_z h is
               if (pa) o.x = 3e30f;
@@ -340,10 +353,10 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         __syncthreads();
       }
     }
-    const float az = sh.par[0][c], ar = sh.par[1][c], ac = sh.par[2][c];
+    const float az = sh.par[pb][0][c], ar = sh.par[pb][1][c], ac = sh.par[pb][2][c];
     const float az2 = -kLog2e * az, ar2 = -kLog2e * ar, ac2 = 2.f * kLog2e * ac;
     const float2 AZ2 = f2(az2, az2), AR2 = f2(ar2, ar2), AC2 = f2(ac2, ac2), AZ = f2(az, az);
-    const float h0v = sh.par[6][c];
+    const float h0v = sh.par[pb][6][c];
     const bool first = (rank == 0 && q == 0);  // chunk holding step 0
 
     float2 H[kRowH], P[kRowH];
@@ -469,8 +482,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     // barrier of the last exchange): the staging area takes the next tile
     if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_issue(smem, sh, &map, p, b2, (next - b2 * nDTc) * kRowC, t0);
+      row_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kRowC, t0);
     }
+    if (pj >= 0 && pj < 7 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
 
     if (drawer) {
       const int nt = 2 * nclus + (int)ticket;

@@ -88,7 +88,8 @@ struct LrShared {
   float4 wagg[2][kLrWarps][kLrC][2];
   float wmax[2][kLrWarps];
   __align__(16) LrMailbox mbox[2];
-  __align__(16) float par[10][kLrC];  // a (4 rows), bias (4 rows), c0, h0
+  // a (4 rows), bias (4 rows), c0, h0 of a tile's channels, by tile parity
+  __align__(16) float par[2][10][kLrC];
   uint64_t bar;                       // the staging area's mbarrier
   uint64_t mbar[2];                   // mailbox mbarriers, by parity
 };
@@ -231,23 +232,22 @@ __device__ __forceinline__ float lr_pass(const unsigned char* __restrict__ base,
   return m;
 }
 
-// Thread 0: the tile's two 256-step boxes and its a, bias, c0, h0 rows, all
-// on `bar`.
+// Thread 0: the tile's two 256-step boxes, on `bar`.
 __device__ __forceinline__ void lr_issue(unsigned char* smem, LrShared& sh, const CUtensorMap* map,
-                                         const FwdParams& p, int b, int d0, int t0) {
+                                         int b, int d0, int t0) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  const unsigned pb = kLrC * 4;
-  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kLrNBox * kLrBoxBytes) + kLrG * pb +
-                                     (p.bias ? kLrG * pb : 0) + (p.c0 ? pb : 0) +
-                                     (p.h0 ? pb : 0));
+  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kLrNBox * kLrBoxBytes));
   for (int j = 0; j < kLrNBox; ++j)
     tma_load_4d(smem + kLrStage + j * kLrBoxBytes, map, &sh.bar, d0, 0, t0 + j * kLrBox, b);
-  for (int g = 0; g < kLrG; ++g) {
-    lr_bulk_load(&sh.par[g][0], p.a + (size_t)g * p.D + d0, pb, &sh.bar);
-    if (p.bias) lr_bulk_load(&sh.par[kLrG + g][0], p.bias + (size_t)g * p.D + d0, pb, &sh.bar);
-  }
-  if (p.c0) lr_bulk_load(&sh.par[8][0], p.c0 + (size_t)b * p.D + d0, pb, &sh.bar);
-  if (p.h0) lr_bulk_load(&sh.par[9][0], p.h0 + (size_t)b * p.D + d0, pb, &sh.bar);
+}
+// Parameter j (0..79) of the tile at (b, d0): a[g][c] (j < 32), bias[g][c]
+// (j < 64, 0 when absent), c0[c], h0[c] (0 when absent).
+__device__ __forceinline__ float lr_param(const FwdParams& p, int j, int b, int d0) {
+  const int row = j / kLrC, c = j % kLrC;
+  if (row < kLrG) return p.a[(size_t)row * p.D + d0 + c];
+  if (row < 2 * kLrG) return p.bias ? p.bias[(size_t)(row - kLrG) * p.D + d0 + c] : 0.f;
+  if (row == 8) return p.c0 ? p.c0[(size_t)b * p.D + d0 + c] : 0.f;
+  return p.h0 ? p.h0[(size_t)b * p.D + d0 + c] : 0.f;
 }
 
 // Bytes a CTA of rank `rank` receives per exchange phase.
@@ -271,7 +271,11 @@ __global__ void __launch_bounds__(kLrThreads, 1)
   const int t0 = rank * kLrSteps;            // first step of this CTA
   const unsigned rx = lr_rx_bytes(rank, CLS);
 
-  if (tid < 10 * kLrC) (&sh.par[0][0])[tid] = 0.f;  // bias, c0, h0 stay 0 when absent
+  // the first tile's parameters; later tiles' are loaded a tile ahead
+  if (tid < 10 * kLrC && clus < ntiles) {
+    const int b = clus / nDTc;
+    (&sh.par[0][0][0])[tid] = lr_param(p, tid, b, (clus - b * nDTc) * kLrC);
+  }
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
     if (CLS > 1) {
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
   if (CLS > 1) cluster.sync();  // the peers' mailbox barriers are armed before anyone sends
   if (tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    lr_issue(smem, sh, &map, p, b, (clus - b * nDTc) * kLrC, t0);
+    lr_issue(smem, sh, &map, b, (clus - b * nDTc) * kLrC, t0);
   }
   const unsigned char* base = smem + q * kLrS;
   int status = 0;
@@ -296,6 +300,14 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     const int d = d0 + c;
     const bool dval = d < p.D;
     const int next = tile + nclus;
+    // the next tile's parameters: loaded now, stored at the end of this tile
+    const int pj = tid - 32;
+    float pnext = 0.f;
+    if (pj >= 0 && pj < 10 * kLrC && next < ntiles) {
+      const int b2 = next / nDTc;
+      pnext = lr_param(p, pj, b2, (next - b2 * nDTc) * kLrC);
+    }
+    const int pb = n & 1;
     if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
     // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32
     // arguments.  Thread (qq, i) takes steps i and i + 8 of chunk qq.
@@ -322,7 +334,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
           const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
           const float xa = __uint_as_float((wa[cc >> 1] << sh16) & mk);
           const float xb = __uint_as_float((wb[cc >> 1] << sh16) & mk);
-          const float bs = sc * sh.par[kLrG + g][cc];
+          const float bs = sc * sh.par[pb][kLrG + g][cc];
           float2 o = lfma(lf2(sc, sc), lf2(xa, xb), lf2(bs, bs));
           if (pa) o.x = padv;
           if (pbd) o.y = padv;
@@ -332,7 +344,8 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     }
     LrPar k;
     {
-      const float ai = sh.par[0][c], af = sh.par[1][c], ag = sh.par[2][c], ao = sh.par[3][c];
+      const float ai = sh.par[pb][0][c], af = sh.par[pb][1][c], ag = sh.par[pb][2][c],
+                  ao = sh.par[pb][3][c];
       k.ai = lf2(ai, ai);
       k.af = lf2(af, af);
       k.ag = lf2(ag, ag);
@@ -344,12 +357,12 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       k.ag2 = lf2(ag2, ag2);
       k.ao2 = lf2(ao2, ao2);
     }
-    const float c0v = sh.par[8][c], h0v = sh.par[9][c];
+    const float c0v = sh.par[pb][8][c], h0v = sh.par[pb][9][c];
     __syncthreads();
     // the staging area and the parameter rows are free: the next tile's
     if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      lr_issue(smem, sh, &map, p, b2, (next - b2 * nDTc) * kLrC, t0);
+      lr_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kLrC, t0);
     }
     const bool first = (rank == 0 && q == 0);  // chunk holding step 0
 
@@ -472,6 +485,9 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       updates = kit + 1;
       if (own_ok) break;
     }
+
+    if (pj >= 0 && pj < 10 * kLrC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
+    __syncthreads();  // the next tile reads them
 
     // ---- states straight from registers
     bool bad = false;
