@@ -13,10 +13,10 @@ int launch_gru_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int n
                    cudaStream_t stream);
 int gru_chunk_steps();
 int gru_max_cluster(bool bf16);
-int gru_seq_wpc(int T);
+int gru_row_cluster(int T);
 int gru_row_box_steps();
 int gru_row_channels();
-int launch_gru_seq(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
+int launch_gru_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
 int lstm_chunk_steps();
@@ -240,7 +240,7 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   // request, the chunked cluster + look-back solve
   const bool force = opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED);
   const bool bf16 = u_dtype == PARARNN_BF16;
-  const bool row_gru = cell == PARARNN_GRU && bf16 && gru_seq_wpc(T) > 0 && !force;
+  const bool row_gru = cell == PARARNN_GRU && bf16 && gru_row_cluster(T) > 0 && !force;
   const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
   int e;
   if (row_gru || row_lstm) {
@@ -249,7 +249,7 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
                  : make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(),
                               lstm_row_channels());
     if (rc) return rc;
-    e = row_gru ? launch_gru_seq(rmap, p, stream) : launch_lstm_row(rmap, p, stream);
+    e = row_gru ? launch_gru_row(rmap, p, stream) : launch_lstm_row(rmap, p, stream);
   } else
     e = cell == PARARNN_GRU ? launch_gru_fwd(map, bf16, p, (int)nctas, stream)
                             : launch_lstm_fwd(map, bf16, p, (int)nctas, stream);

@@ -1,4 +1,4 @@
-// gru_fwd_seq.cu -- fused Newton-scan ParaGRU solve for sequences of up to
+// gru_fwd_row.cu -- fused Newton-scan ParaGRU solve for sequences of up to
 // 4096 steps with bf16 input projections: 8 channels per CTA, a cluster of
 // CLS = ceil(T / 1024) CTAs per tile, two CTAs per SM, the cell evaluated on
 // packed fp32 pairs.
@@ -526,11 +526,10 @@ __global__ void __launch_bounds__(kRowThreads, 2)
 }
 
 // ------------------------------------------------------------- launcher --
+// CTAs per cluster for sequences of length T; 0 when this solve does not apply
 int gru_row_cluster(int T) {
   return T <= 1024 ? 1 : (T <= 2048 ? 2 : (T <= kRowTmax ? 4 : 0));
 }
-// non-zero when this solve applies to sequences of length T
-int gru_seq_wpc(int T) { return gru_row_cluster(T); }
 int gru_row_box_steps() { return kRowBox; }
 int gru_row_channels() { return kRowC; }
 
@@ -568,7 +567,7 @@ static int launch_row_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t
   return (int)cudaLaunchKernelEx(&cfg, kern, map, p);
 }
 
-int launch_gru_seq(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
+int launch_gru_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
   switch (gru_row_cluster(p.T)) {
     case 1: return launch_row_t<1>(map, p, stream);
     case 2: return launch_row_t<2>(map, p, stream);
