@@ -44,18 +44,21 @@ NCU_TRAFFIC_BYTES = {
 }
 # The forward kernel a workload runs and its special-function (MUFU)
 # operations per element and cell evaluation, as the kernel issues them:
-#   gru_newton_row (ParaGRU, bf16 u, T <= 4096): 3 ex2 + 1 rcp (one reciprocal
-#     serves the four sigmoids of a step pair, one the pair's two tanh);
+#   gru_newton_row (ParaGRU with T <= 4096, or longer with at least one
+#     8-channel tile per SM, then in 4096-step segments): 3 ex2 + 1 rcp (one
+#     reciprocal serves the four sigmoids of a step pair, one the pair's two
+#     tanh);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
 #   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096): 5 ex2 + 1.5 rcp (one
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
 def fwd_kernel(w):
-    row = w.u_dtype == "bf16" and w.T <= 4096
     if w.cell == "lstm":
+        row = w.u_dtype == "bf16" and w.T <= 4096
         return ("lstm_newton_row", 6.5) if row else ("lstm_newton_fused", 8)
-    if row:
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if w.T <= 4096 or w.B * ((w.D + 7) // 8) >= sms:
         return "gru_newton_row", 4
     return "gru_newton_fused", 5
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
@@ -236,10 +239,11 @@ class Path:
 
         Every tile stops on its own, so this is counted from the per-channel
         convergence histogram: a channel whose tile first passed the test at
-        iteration k was evaluated k + 1 times.  Exact for the row kernels
-        (a tile is a whole sequence); for the chunked kernels a channel
-        reports its slowest chunk, so this is an upper bound there.  Runs one
-        untimed solve.
+        iteration k was evaluated k + 1 times.  Exact for the row kernels on
+        sequences of up to 4096 steps (a tile is a whole sequence); for the
+        chunked kernels, and for longer sequences solved segment by segment,
+        a channel reports its slowest chunk or segment, so this is an upper
+        bound there.  Runs one untimed solve.
         """
         x = x or self.x
         pr = self.pr

@@ -16,7 +16,8 @@ int gru_max_cluster(bool bf16);
 int gru_row_cluster(int T);
 int gru_row_box_steps();
 int gru_row_channels();
-int launch_gru_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
+int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStream_t stream);
+int gru_row_max_steps();
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
 int lstm_chunk_steps();
@@ -170,6 +171,17 @@ __global__ void hist_kernel(const int* __restrict__ chan_k, size_t n, int* hist,
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA; }
 
+// between the segments of a long sequence: the row kernel's tile counter
+__global__ void ticket_reset_kernel(WsHeader* hdr) { hdr->ticket = 0u; }
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
+  return sms;
+}
+
 int forward(int cell, const void* u, int u_dtype, const float* a, const float* bias,
             const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
             const pararnn_opts* opts, pararnn_stats* stats, int* iter_hist, void* workspace,
@@ -229,30 +241,56 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.rec_vals = reinterpret_cast<float*>(ws + L.vals);
   p.chan_k = iter_hist ? reinterpret_cast<int*>(ws + L.chan_k) : nullptr;
   p.stats = stats;
+  p.u = u;
+  p.t_base = 0;
+  p.t_len = T;
+  p.ld_h0 = D;
 
   const size_t nch = (size_t)B * D;
   const int nhist = max_iters + 2;
   const unsigned igrid = iter_hist ? (unsigned)std::min<size_t>((nch + 255) / 256, 1024) : 1u;
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
-  // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
-  // 8-channel tile holds the whole sequence (row kernels); otherwise, or on
-  // request, the chunked cluster + look-back solve
+  // Row kernels: a cluster of CTAs per 8-channel tile holds a whole sequence
+  // of up to 4096 steps (ParaGRU: bf16 or fp32 u; ParaLSTM: bf16 u).  A
+  // longer ParaGRU sequence with at least one 8-channel tile per SM is solved
+  // 4096-step segment by segment, each segment starting from the state the
+  // one before it converged to: the same work as one solve over the whole
+  // sequence, and each segment still fills the GPU.  Otherwise, or on
+  // request, the chunked cluster + look-back solve.
   const bool force = opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED);
   const bool bf16 = u_dtype == PARARNN_BF16;
-  const bool row_gru = cell == PARARNN_GRU && bf16 && gru_row_cluster(T) > 0 && !force;
+  const long long tiles8 = (long long)B * ((D + 7) / 8);
+  const bool row_gru = cell == PARARNN_GRU && !force &&
+                       (gru_row_cluster(T) > 0 || tiles8 >= sm_count());
   const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
-  int e;
-  if (row_gru || row_lstm) {
+  int e = 0;
+  if (row_gru) {
     CUtensorMap rmap;
-    rc = row_gru ? make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels())
-                 : make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(),
-                              lstm_row_channels());
+    rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());
     if (rc) return rc;
-    e = row_gru ? launch_gru_row(rmap, p, stream) : launch_lstm_row(rmap, p, stream);
-  } else
+    const int seg = gru_row_max_steps();
+    for (int s0 = 0; s0 < T && e == 0; s0 += seg) {
+      FwdParams ps = p;
+      ps.t_base = s0;
+      ps.t_len = std::min(seg, T - s0);
+      if (s0 > 0) {
+        ps.h0 = h + (size_t)(s0 - 1) * D;  // the last state of the segment before
+        ps.ld_h0 = (long long)T * D;
+        ticket_reset_kernel<<<1, 1, 0, stream>>>(p.hdr);
+        if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
+      }
+      e = launch_gru_row(rmap, ps, !bf16, stream);
+    }
+  } else if (row_lstm) {
+    CUtensorMap rmap;
+    rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(), lstm_row_channels());
+    if (rc) return rc;
+    e = launch_lstm_row(rmap, p, stream);
+  } else {
     e = cell == PARARNN_GRU ? launch_gru_fwd(map, bf16, p, (int)nctas, stream)
                             : launch_lstm_fwd(map, bf16, p, (int)nctas, stream);
+  }
   if (e != 0) return PARARNN_ERR_CUDA;
   if (iter_hist) {
     hist_kernel<<<(unsigned)((nch + 255) / 256), 256, 0, stream>>>(p.chan_k, nch, iter_hist,

@@ -171,6 +171,13 @@ struct FwdParams {
   float* rec_vals;
   int* chan_k;        // [B*D] or null
   pararnn_stats* stats;
+  // whole-sequence (row) kernel only: the projections (fp32 read directly),
+  // the first step and the length of the segment this launch solves, and the
+  // batch stride of h0 in floats (a segment starts from the state the one
+  // before it ended with)
+  const void* u;
+  int t_base, t_len;
+  long long ld_h0;
 };
 
 }  // namespace pararnn

@@ -219,7 +219,7 @@ __device__ __forceinline__ float row_param(const FwdParams& p, int j, int b, int
   const int row = j / kRowC, c = j % kRowC;
   if (row < 3) return p.a[(size_t)row * p.D + d0 + c];
   if (row < 6) return p.bias ? p.bias[(size_t)(row - 3) * p.D + d0 + c] : 0.f;
-  return p.h0 ? p.h0[(size_t)b * p.D + d0 + c] : 0.f;
+  return p.h0 ? p.h0[(size_t)b * p.ld_h0 + d0 + c] : 0.f;
 }
 // L2 prefetch of a tile's boxes (no shared memory touched).
 __device__ __forceinline__ void row_prefetch(const CUtensorMap* map, int b, int d0, int t0) {
@@ -235,7 +235,7 @@ __host__ __device__ constexpr unsigned row_rx_bytes(int rank, int cls) {
   return (unsigned)(rank * kRowC * 16 + (cls - 1) * 4);
 }
 
-template <int CLS>
+template <int CLS, bool kF32>
 __global__ void __launch_bounds__(kRowThreads, 2)
     gru_newton_row(const __grid_constant__ CUtensorMap map, const FwdParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -248,7 +248,8 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   const int nDTc = (p.D + kRowC - 1) / kRowC;
   const int ntiles = p.B * nDTc;
   const int nclus = gridDim.x / CLS, clus = blockIdx.x / CLS;
-  const int t0 = rank * kRowSteps;           // first step of this CTA
+  const int t0 = rank * kRowSteps;           // first step of this CTA in the segment
+  const int tg0 = p.t_base + t0;             // ... in the sequence
   const unsigned rx = row_rx_bytes(rank, CLS);
 
   // the first tile's parameters; later tiles' are loaded a tile ahead
@@ -268,9 +269,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   __syncthreads();
   // the peers' mailbox barriers are armed before anyone sends
   if (CLS > 1) cluster.sync();
-  if (tid == 0 && clus < ntiles) {
+  if (!kF32 && tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    row_issue(smem, sh, &map, b, (clus - b * nDTc) * kRowC, t0);
+    row_issue(smem, sh, &map, b, (clus - b * nDTc) * kRowC, tg0);
   }
   const unsigned char* base = smem + q * kRowS;
   int status = 0;
@@ -303,11 +304,12 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kRowC;
     const int d = d0 + c;
     const bool dval = d < p.D;
-    if (tid == 0 && next < ntiles) {
+    if (!kF32 && tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, t0);
+      row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, tg0);
     }
-    if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
+    if (!kF32 && !mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns))
+      status = PARARNN_STATUS_TIMEOUT;
     // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32 arguments
     // in two blocks of 512 steps (each block's rows are read before any of
     // its slots is written; block 0 writes below all staging bytes).  Thread
@@ -319,30 +321,62 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       for (int blk = 0; blk < 2; ++blk) {
         const int qq = blk * (kRowChunks / 2) + qb;
         const int ta = qq * kRowL + i, tb = ta + kRowH;  // steps within the CTA
-        uint4 va[3], vb[3];
+        const bool pa = t0 + ta >= p.t_len, pbd = t0 + tb >= p.t_len;
+        // the 8 channels of gate g at steps ta (xa) and tb (xb): bf16 from
+        // the staging area, fp32 straight from global memory
+        float xa[3][kRowC], xb[3][kRowC];
+        if (kF32) {
+          const float* ug = static_cast<const float*>(p.u);
 #pragma unroll
-        for (int g = 0; g < 3; ++g) {
-          va[g] = *reinterpret_cast<const uint4*>(
-              smem + kRowStage + (ta / kRowBox) * kRowBoxBytes + ((ta % kRowBox) * 3 + g) * 16);
-          vb[g] = *reinterpret_cast<const uint4*>(
-              smem + kRowStage + (tb / kRowBox) * kRowBoxBytes + ((tb % kRowBox) * 3 + g) * 16);
+          for (int g = 0; g < 3; ++g) {
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+            if (!pa) {
+              const float4* ra = reinterpret_cast<const float4*>(
+                  ug + (((size_t)b * p.T + tg0 + ta) * 3 + g) * p.D + d0);
+              a0 = __ldg(ra);
+              a1 = __ldg(ra + 1);
+            }
+            if (!pbd) {
+              const float4* rb = reinterpret_cast<const float4*>(
+                  ug + (((size_t)b * p.T + tg0 + tb) * 3 + g) * p.D + d0);
+              b0 = __ldg(rb);
+              b1 = __ldg(rb + 1);
+            }
+            const float fa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float fb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int cc = 0; cc < kRowC; ++cc) {
+              xa[g][cc] = fa[cc];
+              xb[g][cc] = fb[cc];
+            }
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < 3; ++g) {
+            const uint4 va = *reinterpret_cast<const uint4*>(
+                smem + kRowStage + (ta / kRowBox) * kRowBoxBytes + ((ta % kRowBox) * 3 + g) * 16);
+            const uint4 vb = *reinterpret_cast<const uint4*>(
+                smem + kRowStage + (tb / kRowBox) * kRowBoxBytes + ((tb % kRowBox) * 3 + g) * 16);
+            const unsigned wa[4] = {va.x, va.y, va.z, va.w};
+            const unsigned wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+            for (int cc = 0; cc < kRowC; ++cc) {
+              const int sh16 = (cc & 1) ? 0 : 16;
+              const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
+              xa[g][cc] = __uint_as_float((wa[cc >> 1] << sh16) & mk);
+              xb[g][cc] = __uint_as_float((wb[cc >> 1] << sh16) & mk);
+            }
+          }
         }
         __syncthreads();
-        const bool pa = t0 + ta >= p.T, pbd = t0 + tb >= p.T;
         unsigned char* dst = smem + qq * kRowS + i * kRowC * 8;
 #pragma unroll
         for (int g = 0; g < 3; ++g) {
           const float sc = (g == 2) ? 2.f * kLog2e : -kLog2e;
-          const unsigned wa[4] = {va[g].x, va[g].y, va[g].z, va[g].w};
-          const unsigned wb[4] = {vb[g].x, vb[g].y, vb[g].z, vb[g].w};
 #pragma unroll
           for (int cc = 0; cc < kRowC; ++cc) {
-            const int sh16 = (cc & 1) ? 0 : 16;
-            const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
-            const float xa = __uint_as_float((wa[cc >> 1] << sh16) & mk);
-            const float xb = __uint_as_float((wb[cc >> 1] << sh16) & mk);
             const float bs = sc * sh.par[pb][3 + g][cc];
-            float2 o = ffma2(f2(sc, sc), f2(xa, xb), f2(bs, bs));
+            float2 o = ffma2(f2(sc, sc), f2(xa[g][cc], xb[g][cc]), f2(bs, bs));
             if (g == 0) {  // steps past T: z < 5e-10 whatever a_z h is
               if (pa) o.x = 3e30f;
               if (pbd) o.y = 3e30f;
@@ -480,9 +514,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     }
     // every thread of the CTA is past its last pass of this tile (the
     // barrier of the last exchange): the staging area takes the next tile
-    if (tid == 0 && next < ntiles) {
+    if (!kF32 && tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kRowC, t0);
+      row_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kRowC, tg0);
     }
     if (pj >= 0 && pj < 7 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
 
@@ -497,14 +531,14 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     bool bad = false;
     if (dval) {
       const int tq = t0 + q * kRowL;
-      float* out = p.h + ((size_t)b * p.T + tq) * p.D + d;
+      float* out = p.h + ((size_t)b * p.T + p.t_base + tq) * p.D + d;
 #pragma unroll
       for (int i = 0; i < kRowH; ++i) {
-        if (tq + i < p.T) {
+        if (tq + i < p.t_len) {
           out[(size_t)i * p.D] = H[i].x;
           bad |= !isfinite(H[i].x);
         }
-        if (tq + kRowH + i < p.T) {
+        if (tq + kRowH + i < p.t_len) {
           out[(size_t)(kRowH + i) * p.D] = H[i].y;
           bad |= !isfinite(H[i].y);
         }
@@ -533,13 +567,13 @@ int gru_row_cluster(int T) {
 int gru_row_box_steps() { return kRowBox; }
 int gru_row_channels() { return kRowC; }
 
-template <int CLS>
+template <int CLS, bool kF32>
 static int launch_row_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
   const long long ntiles = (long long)p.B * ((p.D + kRowC - 1) / kRowC);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  auto kern = gru_newton_row<CLS>;
+  auto kern = gru_newton_row<CLS, kF32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmem);
   if (e != cudaSuccess) return (int)e;
   // persistent clusters: as many as can be resident (two CTAs per SM), at
@@ -567,13 +601,16 @@ static int launch_row_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t
   return (int)cudaLaunchKernelEx(&cfg, kern, map, p);
 }
 
-int launch_gru_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
-  switch (gru_row_cluster(p.T)) {
-    case 1: return launch_row_t<1>(map, p, stream);
-    case 2: return launch_row_t<2>(map, p, stream);
-    case 4: return launch_row_t<4>(map, p, stream);
+// One launch solves steps [p.t_base, p.t_base + p.t_len) (t_len <= 4096) of
+// every tile; u is bf16 through `map` or, with f32, read from p.u.
+int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStream_t stream) {
+  switch (gru_row_cluster(p.t_len)) {
+    case 1: return f32 ? launch_row_t<1, true>(map, p, stream) : launch_row_t<1, false>(map, p, stream);
+    case 2: return f32 ? launch_row_t<2, true>(map, p, stream) : launch_row_t<2, false>(map, p, stream);
+    case 4: return f32 ? launch_row_t<4, true>(map, p, stream) : launch_row_t<4, false>(map, p, stream);
     default: return 1;
   }
 }
+int gru_row_max_steps() { return kRowTmax; }
 
 }  // namespace pararnn

@@ -189,3 +189,28 @@ def test_absent_bias_and_h0_read_as_zero(cuda_ok):
         torch.cuda.synchronize()
         assert np.abs(h.cpu().numpy() - ref).max() < TOL_STATE, flags
         assert pr.read_stats(st)["status"] == "converged"
+
+
+def test_long_sequence_segments_match_oracle(cuda_ok):
+    # T > 4096 with at least one 8-channel tile per SM (B * D / 8 = 150):
+    # the sequence is solved 4096-step segment by segment, each starting from
+    # the state the one before ended with; the look-back solve is forced for
+    # comparison.  A nonzero h0 checks the first segment's start.
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=9000, D=1200))
+    x["h0"] = torch.randn((1, 1200), generator=torch.Generator().manual_seed(13)) * 0.5
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        h, st, hist = _solve(x, flags=flags, hist=True)
+        err = np.abs(h - ref).max()
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == 1200
+
+
+def test_fp32_inputs_both_solvers(cuda_ok):
+    x = make_inputs(WORKLOADS[4].scaled(B=3, T=2500, D=48))
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        h, st, _ = _solve(x, flags=flags)
+        assert np.abs(h - ref).max() < TOL_STATE, flags
+        assert st["status"] == "converged", (flags, st)
