@@ -308,6 +308,18 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       const int b2 = next / nDTc;
       row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, tg0);
     }
+    if (kF32 && next < ntiles) {
+      // the next tile's fp32 rows into L2, 12 (step, gate) rows per thread
+      const int b2 = next / nDTc, d2 = (next - b2 * nDTc) * kRowC;
+      const float* ug = static_cast<const float*>(p.u);
+#pragma unroll 4
+      for (int r = tid; r < kRowSteps * 3; r += kRowThreads) {
+        const int t = r / 3, g = r - t * 3;
+        if (t0 + t < p.t_len)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(
+              ug + (((size_t)b2 * p.T + tg0 + t) * 3 + g) * p.D + d2));
+      }
+    }
     if (!kF32 && !mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns))
       status = PARARNN_STATUS_TIMEOUT;
     // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32 arguments
