@@ -29,10 +29,14 @@ int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t str
 int adjoint_row_cluster(int T);
 int adjoint_row_channels();
 int adjoint_row_box_steps(int which);
-size_t adjoint_row_part_bytes(int B, int T, int D);
+size_t adjoint_row_part_bytes(int G, int B, int T, int D);
 int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bias,
                        const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
                        int T, int D, int* status, void* ws, cudaStream_t stream);
+int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float* bias,
+                            const float* c0, const float* h0, float* du, float* da,
+                            float* dbias, float* dc0, float* dh0, int B, int T, int D,
+                            int* status, void* ws, cudaStream_t stream);
 int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, const float* bias,
                         const float* c0, const float* h0, float* c, float* h, int B, int T,
                         int D, cudaStream_t stream);
@@ -355,18 +359,29 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
     return PARARNN_ERR_MISALIGNED;
   if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const int G = cell == PARARNN_GRU ? 3 : 4;
-  // ParaGRU, bf16 projections, sequences of up to 4096 steps: a cluster of
-  // CTAs per 8-channel tile holds the whole sequence (no look-back)
-  if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&
-      adjoint_row_part_bytes(B, T, D) <= ws_bytes) {
+  // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
+  // 8-channel tile holds the whole sequence (no look-back)
+  if (u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&
+      adjoint_row_part_bytes(G, B, T, D) <= ws_bytes) {
     const int ch = adjoint_row_channels();
-    CUtensorMap rmaps[3];  // u, h (states before each step), dL/dh
-    rc = make_u_map(&rmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
-    if (!rc) rc = make_s_map(&rmaps[1], h, B, T, D, adjoint_row_box_steps(1), ch);
-    if (!rc) rc = make_s_map(&rmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
-    if (rc) return rc;
-    const int e = launch_adjoint_row(rmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status,
-                                     workspace, (cudaStream_t)stream);
+    CUtensorMap rmaps[4];
+    int e;
+    if (cell == PARARNN_GRU) {  // u, h (states before each step), dL/dh
+      rc = make_u_map(&rmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
+      if (!rc) rc = make_s_map(&rmaps[1], h, B, T, D, adjoint_row_box_steps(1), ch);
+      if (!rc) rc = make_s_map(&rmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+      if (rc) return rc;
+      e = launch_adjoint_row(rmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status, workspace,
+                             (cudaStream_t)stream);
+    } else {  // u, c and h (states before each step), dL/dh
+      rc = make_u_map(&rmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
+      if (!rc) rc = make_s_map(&rmaps[1], c, B, T, D, adjoint_row_box_steps(1), ch);
+      if (!rc) rc = make_s_map(&rmaps[2], h, B, T, D, adjoint_row_box_steps(1), ch);
+      if (!rc) rc = make_s_map(&rmaps[3], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+      if (rc) return rc;
+      e = launch_adjoint_row_lstm(rmaps, a, bias, c0, h0, du, da, dbias, dc0, dh0, B, T, D,
+                                  status, workspace, (cudaStream_t)stream);
+    }
     return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
   }
   const int tc = adjoint_chunk_steps(cell);

@@ -142,3 +142,24 @@ def test_lstm_adjoint_nonzero_initial_state(cuda_ok):
     x["h0"] = torch.randn((2, 32), generator=gen) * 0.5
     c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
     _check_lstm(x, c, h)
+
+
+def test_lstm_adjoint_lookback_path(cuda_ok):
+    # fp32 projections and T > 4096 take the chunked look-back adjoint; bf16
+    # with T <= 4096 (the shapes above) the whole-sequence one
+    x = make_inputs(WORKLOADS[5].scaled(B=2, T=500, D=24))
+    x["u"] = x["u"].float()  # the same values, read as fp32
+    c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    _check_lstm(x, c, h)
+    y = make_inputs(WORKLOADS[5].scaled(B=1, T=4500, D=16))
+    c, h = oracle.lstm_seq(y["u"], y["a"], y["bias"], y["c0"], y["h0"])
+    _check_lstm(y, c, h)
+
+
+def test_lstm_adjoint_is_bitwise_reproducible(cuda_ok):
+    x = make_inputs(WORKLOADS[5].scaled(B=2, T=1500, D=32))
+    c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    g1 = _gpu_adjoint(pr.PARARNN_LSTM, x, h, c)
+    g2 = _gpu_adjoint(pr.PARARNN_LSTM, x, h, c)
+    for k in ("du", "da", "dbias", "dh0", "dc0"):
+        assert np.array_equal(g1[k], g2[k]), k
