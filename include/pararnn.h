@@ -88,9 +88,14 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
 /* opts.flags */
 #define PARARNN_FLAG_INJECT_WITHHOLD 1u /* testing: chunk `inject_chunk` never
                                            publishes its look-back record */
-#define PARARNN_FLAG_FORCE_CHUNKED 2u   /* bf16 u, T <= 4096: use the chunked
-                                           (cluster + look-back) solve instead
-                                           of the whole-sequence row kernels */
+#define PARARNN_FLAG_FORCE_CHUNKED 2u   /* use the chunked (cluster + decoupled
+                                           look-back) solve where the
+                                           whole-sequence row kernels would
+                                           run: ParaGRU with T <= 4096 (bf16 or
+                                           fp32 u) or longer with at least one
+                                           8-channel tile per SM (solved in
+                                           4096-step segments), ParaLSTM with
+                                           bf16 u and T <= 4096 */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
@@ -133,7 +138,13 @@ int pararnn_workspace_init(void* workspace, size_t ws_bytes,
  *      never got there within the cap.
  * Newton starts from h = 0 at every t, applies the page's update until the
  * residual of an iterate is below tol everywhere upstream (and then applies
- * that last update), or until max_iters updates have been applied. */
+ * that last update), or until max_iters updates have been applied.  Channels
+ * are independent; each 8-channel tile stops on its own.  A sequence longer
+ * than 4096 steps with at least one 8-channel tile (B * D / 8) per SM is
+ * solved 4096-step segment by segment, each segment starting from the state
+ * the one before it converged to; stats and iter_hist then take the maximum
+ * over the segments.  Shorter-tiled long sequences use one solve over the
+ * whole sequence (cluster chunks joined by decoupled look-back). */
 int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
                       const float* bias, const float* h0, float* h, int B,
                       int T, int D, const pararnn_opts* opts,
