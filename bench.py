@@ -35,12 +35,14 @@ from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs  # noqa: E4
 
 METRIC = "Newton-solved token*channels/s (fwd+bwd)"
 UNIT = "tokch/s"
-# Counters of the dominant kernel taken with ncu on this build (one launch of
-# the default workload; see profiles/).  None when not captured for the
+# Counters of the dominant kernel taken with ncu on this build (one launch on
+# the workload in the key; see profiles/).  None when not captured for the
 # kernel as it stands.
 NCU_TRAFFIC_BYTES = {
     # profiles/gru_newton_row_b8_t4096_d1024.md: dram read + write of one launch
     ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 201_523_456 + 107_096_576,
+    # profiles/lstm_newton_row_b8_t4096_d1024.md: one 512-step segment's launch
+    ("lstm_newton_row", "lstm_b8_t4096_d1024_bf16"): 33_703_168 + 5_925_120,
 }
 # The forward kernel a workload runs and its special-function (MUFU)
 # operations per element and cell evaluation, as the kernel issues them:
@@ -49,18 +51,44 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal serves the four sigmoids of a step pair, one the pair's two
 #     tanh);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
-#   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096): 5 ex2 + 1.5 rcp (one
+#   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096, in segments where
+#     smaller clusters fill the SMs): 5 ex2 + 1.5 rcp (one
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
-def fwd_kernel(w):
-    if w.cell == "lstm":
-        row = w.u_dtype == "bf16" and w.T <= 4096
-        return ("lstm_newton_row", 6.5) if row else ("lstm_newton_fused", 8)
+def fwd_plan(w):
+    """(kernel, MUFU ops per evaluation, segment length) of the forward solve
+    as the library dispatches it: the row kernels solve a ParaGRU sequence
+    longer than 4096 steps in 4096-step segments, and a ParaLSTM sequence
+    in segments of k x 512 steps, k the smallest cluster size below the one
+    the whole sequence needs at which its 8-channel tiles fill the SMs."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    if w.T <= 4096 or w.B * ((w.D + 7) // 8) >= sms:
-        return "gru_newton_row", 4
-    return "gru_newton_fused", 5
+    tiles8 = w.B * ((w.D + 7) // 8)
+    if w.cell == "lstm":
+        if w.u_dtype == "bf16" and w.T <= 4096:
+            cls, seg = 1, w.T
+            while cls * 512 < w.T:
+                cls *= 2
+            k = 1
+            while k < cls:
+                if k * tiles8 >= sms:
+                    seg = k * 512
+                    break
+                k *= 2
+            return "lstm_newton_row", 6.5, seg
+        return "lstm_newton_fused", 8, w.T
+    if w.T <= 4096 or tiles8 >= sms:
+        return "gru_newton_row", 4, min(w.T, 4096)
+    return "gru_newton_fused", 5, w.T
+
+
+def fwd_kernel(w):
+    return fwd_plan(w)[:2]
+
+
+def fwd_segments(w):
+    seg = fwd_plan(w)[2]
+    return [(s0, min(seg, w.T - s0)) for s0 in range(0, w.T, seg)]
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
 def fwd_bytes(w):
     ue = 2 if w.u_dtype == "bf16" else 4
@@ -221,7 +249,9 @@ class Path:
             self.abuf = self.wsa.get(pr.pararnn_workspace_size(cell, B, T, D, 0, 1))
 
     def launches_per_step(self):
-        n = 2 + (1 if self.hist is not None else 0)        # init, solve, [hist]
+        nseg = len(fwd_segments(self.w))
+        resets = nseg - 1 if fwd_kernel(self.w)[0] == "gru_newton_row" else 0
+        n = 1 + nseg + resets + (1 if self.hist is not None else 0)  # init, solves, [hist]
         return n + (3 if self.w.adjoint else 0)            # init, adjoint, reduce
 
     def forward(self, x=None):
@@ -239,23 +269,32 @@ class Path:
 
         Every tile stops on its own, so this is counted from the per-channel
         convergence histogram: a channel whose tile first passed the test at
-        iteration k was evaluated k + 1 times.  Exact for the row kernels on
-        sequences of up to 4096 steps (a tile is a whole sequence); for the
-        chunked kernels, and for longer sequences solved segment by segment,
-        a channel reports its slowest chunk or segment, so this is an upper
-        bound there.  Runs one untimed solve.
+        iteration k was evaluated k + 1 times.  Exact for the row kernels (a
+        tile is a whole sequence or segment): a sequence the library solves
+        segment by segment is solved here one segment per call, each from the
+        state the one before ended in, which is the arithmetic the segmented
+        solve does.  For the chunked kernels a channel reports its slowest
+        chunk, so this is an upper bound there.  Untimed.
         """
         x = x or self.x
         pr = self.pr
-        hb = torch.zeros(66, dtype=torch.int32, device="cuda")
-        if self.lstm:
-            pr.pararnn_lstm_solve(x["u"], x["a"], x["bias"], x["c0"], x["h0"], self.c,
-                                  self.h, self.opts, self.stats, hb, self.fbuf)
-        else:
-            pr.pararnn_gru_solve(x["u"], x["a"], x["bias"], x["h0"], self.h, self.opts,
-                                 self.stats, hb, self.fbuf)
-        hist = hb.cpu().tolist()
-        return self.w.T * sum(n * (k + 1) for k, n in enumerate(hist))
+        evals = 0
+        c_in, h_in = x.get("c0"), x["h0"]
+        for s0, n in fwd_segments(self.w):
+            hb = torch.zeros(66, dtype=torch.int32, device="cuda")
+            u = x["u"][:, s0:s0 + n].contiguous()
+            h = torch.empty((self.w.B, n, self.w.D), dtype=torch.float32, device="cuda")
+            if self.lstm:
+                c = torch.empty_like(h)
+                pr.pararnn_lstm_solve(u, x["a"], x["bias"], c_in, h_in, c, h, self.opts,
+                                      self.stats, hb, self.fbuf)
+                c_in = c[:, -1].contiguous()
+            else:
+                pr.pararnn_gru_solve(u, x["a"], x["bias"], h_in, h, self.opts, self.stats,
+                                     hb, self.fbuf)
+            h_in = h[:, -1].contiguous()
+            evals += n * sum(m * (k + 1) for k, m in enumerate(hb.cpu().tolist()))
+        return evals
 
     def backward(self, x=None):
         x = x or self.x
@@ -347,7 +386,8 @@ def run_ours(args, world, rank):
                 "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
                 "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
                 "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
-                "ops_per_launch": elem_evals * mufu_per_eval,
+                "ops_per_launch": elem_evals * mufu_per_eval / len(fwd_segments(w)),
+                "launches_per_solve": len(fwd_segments(w)),
                 "mean_evals": round(elem_evals / w.tokch, 3)}
     hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
            "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,

@@ -95,7 +95,8 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            fp32 u) or longer with at least one
                                            8-channel tile per SM (solved in
                                            4096-step segments), ParaLSTM with
-                                           bf16 u and T <= 4096 */
+                                           bf16 u and T <= 4096 (segmented as
+                                           pararnn_lstm_solve says) */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
@@ -154,7 +155,12 @@ int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
 /* ParaLSTM forward solve.  As pararnn_gru_solve with u [B][T][4][D]
  * (i, f, g, o), a/bias [4][D], initial cell state c0 (NULL = zeros) and both
  * state trajectories out: c [B][T][D], h [B][T][D].  The residual norm is the
- * max over both components. */
+ * max over both components.  With bf16 u and T <= 4096 a tile's sequence is
+ * held by a cluster of k CTAs of 512 steps each; when a smaller cluster of
+ * k' CTAs already puts one CTA on every SM (k' * B * D / 8 >= SMs), the
+ * sequence is solved in segments of k' * 512 steps instead, each starting
+ * from the (c, h) the one before it converged to; stats and iter_hist then
+ * take the maximum over the segments. */
 int pararnn_lstm_solve(const void* u, int u_dtype, const float* a,
                        const float* bias, const float* c0, const float* h0,
                        float* c, float* h, int B, int T, int D,

@@ -23,6 +23,7 @@ int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int 
 int lstm_chunk_steps();
 int lstm_max_cluster(bool bf16);
 int lstm_row_cluster(int T);
+int lstm_row_cta_steps();
 int lstm_row_box_steps();
 int lstm_row_channels();
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
@@ -260,7 +261,11 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   // longer ParaGRU sequence with at least one 8-channel tile per SM is solved
   // 4096-step segment by segment, each segment starting from the state the
   // one before it converged to: the same work as one solve over the whole
-  // sequence, and each segment still fills the GPU.  Otherwise, or on
+  // sequence, and each segment still fills the GPU.  A ParaLSTM sequence is
+  // solved the same way in segments of k x 512 steps, k the smallest cluster
+  // size below the one the whole sequence needs at which the 8-channel tiles
+  // put a CTA on every SM: smaller clusters fit the SMs without gaps, and
+  // shorter segments converge in fewer iterations.  Otherwise, or on
   // request, the chunked cluster + look-back solve.
   const bool force = opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED);
   const bool bf16 = u_dtype == PARARNN_BF16;
@@ -290,7 +295,23 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(), lstm_row_channels());
     if (rc) return rc;
-    e = launch_lstm_row(rmap, p, stream);
+    int seg = T;
+    for (int k = 1; k < lstm_row_cluster(T); k *= 2)
+      if (k * tiles8 >= sm_count()) {
+        seg = k * lstm_row_cta_steps();
+        break;
+      }
+    for (int s0 = 0; s0 < T && e == 0; s0 += seg) {
+      FwdParams ps = p;
+      ps.t_base = s0;
+      ps.t_len = std::min(seg, T - s0);
+      if (s0 > 0) {  // the last (c, h) of the segment before
+        ps.c0 = c + (size_t)(s0 - 1) * D;
+        ps.h0 = h + (size_t)(s0 - 1) * D;
+        ps.ld_h0 = (long long)T * D;
+      }
+      e = launch_lstm_row(rmap, ps, stream);
+    }
   } else {
     e = cell == PARARNN_GRU ? launch_gru_fwd(map, bf16, p, (int)nctas, stream)
                             : launch_lstm_fwd(map, bf16, p, (int)nctas, stream);

@@ -246,8 +246,8 @@ __device__ __forceinline__ float lr_param(const FwdParams& p, int j, int b, int 
   const int row = j / kLrC, c = j % kLrC;
   if (row < kLrG) return p.a[(size_t)row * p.D + d0 + c];
   if (row < 2 * kLrG) return p.bias ? p.bias[(size_t)(row - kLrG) * p.D + d0 + c] : 0.f;
-  if (row == 8) return p.c0 ? p.c0[(size_t)b * p.D + d0 + c] : 0.f;
-  return p.h0 ? p.h0[(size_t)b * p.D + d0 + c] : 0.f;
+  if (row == 8) return p.c0 ? p.c0[(size_t)b * p.ld_h0 + d0 + c] : 0.f;
+  return p.h0 ? p.h0[(size_t)b * p.ld_h0 + d0 + c] : 0.f;
 }
 
 // Bytes a CTA of rank `rank` receives per exchange phase.
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
   if (CLS > 1) cluster.sync();  // the peers' mailbox barriers are armed before anyone sends
   if (tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    lr_issue(smem, sh, &map, b, (clus - b * nDTc) * kLrC, t0);
+    lr_issue(smem, sh, &map, b, (clus - b * nDTc) * kLrC, p.t_base + t0);
   }
   const unsigned char* base = smem + q * kLrS;
   int status = 0;
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       const int qq = tid / kLrH, i = tid % kLrH;
       const int sw = lr_swizzle(i);
       const int ta = qq * kLrL + i, tb = ta + kLrH;  // steps within the CTA
-      const bool pa = t0 + ta >= p.T, pbd = t0 + tb >= p.T;
+      const bool pa = t0 + ta >= p.t_len, pbd = t0 + tb >= p.t_len;
       unsigned char* dst = smem + qq * kLrS + i * kLrC * 8;
 #pragma unroll
       for (int g = 0; g < kLrG; ++g) {
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     // the staging area and the parameter rows are free: the next tile's
     if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      lr_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kLrC, t0);
+      lr_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kLrC, p.t_base + t0);
     }
     const bool first = (rank == 0 && q == 0);  // chunk holding step 0
 
@@ -493,15 +493,15 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     bool bad = false;
     if (dval) {
       const int tq = t0 + q * kLrL;
-      const size_t o0 = ((size_t)b * p.T + tq) * p.D + d;
+      const size_t o0 = ((size_t)b * p.T + p.t_base + tq) * p.D + d;
 #pragma unroll
       for (int i = 0; i < kLrH; ++i) {
-        if (tq + i < p.T) {
+        if (tq + i < p.t_len) {
           p.c[o0 + (size_t)i * p.D] = C[i].x;
           p.h[o0 + (size_t)i * p.D] = H[i].x;
           bad |= !isfinite(C[i].x) || !isfinite(H[i].x);
         }
-        if (tq + kLrH + i < p.T) {
+        if (tq + kLrH + i < p.t_len) {
           p.c[o0 + (size_t)(kLrH + i) * p.D] = C[i].y;
           p.h[o0 + (size_t)(kLrH + i) * p.D] = H[i].y;
           bad |= !isfinite(C[i].y) || !isfinite(H[i].y);
@@ -531,6 +531,8 @@ int lstm_row_cluster(int T) {
   return cls;
 }
 int lstm_row_box_steps() { return kLrBox; }
+// steps one CTA holds: a cluster of k CTAs solves up to k times this many
+int lstm_row_cta_steps() { return kLrSteps; }
 int lstm_row_channels() { return kLrC; }
 
 template <int CLS>
@@ -566,7 +568,7 @@ static int launch_lr_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t 
 }
 
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
-  switch (lstm_row_cluster(p.T)) {
+  switch (lstm_row_cluster(p.t_len)) {
     case 1: return launch_lr_t<1>(map, p, stream);
     case 2: return launch_lr_t<2>(map, p, stream);
     case 4: return launch_lr_t<4>(map, p, stream);

@@ -120,3 +120,24 @@ def test_absent_bias_with_nonzero_state_both_solvers(cuda_ok):
         err = max(np.abs(c.cpu().numpy() - rc).max(), np.abs(h.cpu().numpy() - rh).max())
         assert err < TOL_STATE, (flags, err)
         assert pr.read_stats(st)["status"] == "converged"
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 3000, 160), (1, 4095, 320), (1, 2500, 640),
+                                   (2, 3000, 600)])
+def test_segmented_long_sequence_matches_oracle(cuda_ok, B, T, D):
+    # with 40, 80 and 150 8-channel tiles, clusters of 4, 2 and 1 CTAs put a
+    # CTA on each of 148 SMs: the row solve then runs in segments of 2048,
+    # 1024 and 512 steps (ragged last segments here), each starting from the
+    # (c, h) the one before converged to; a nonzero initial state checks the
+    # first
+    x = make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D))
+    gen = torch.Generator().manual_seed(13)
+    x["c0"] = torch.randn((B, D), generator=gen) * 0.5
+    x["h0"] = torch.randn((B, D), generator=gen) * 0.5
+    rc, rh = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        c, h, st, hist = _solve(x, flags=flags, hist=True)
+        err = max(np.abs(c - rc).max(), np.abs(h - rh).max())
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == B * D
