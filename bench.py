@@ -39,8 +39,8 @@ UNIT = "tokch/s"
 # the workload in the key; see profiles/).  None when not captured for the
 # kernel as it stands.
 NCU_TRAFFIC_BYTES = {
-    # profiles/gru_newton_row_b8_t4096_d1024.md: dram read + write of one launch
-    ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 201_523_456 + 107_096_576,
+    # profiles/gru_newton_row_b8_t4096_d1024.md: one 1024-step segment's launch
+    ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 50_585_600 + 7_483_392,
     # profiles/lstm_newton_row_b8_t4096_d1024.md: one 512-step segment's launch
     ("lstm_newton_row", "lstm_b8_t4096_d1024_bf16"): 33_703_168 + 5_925_120,
 }
@@ -58,10 +58,11 @@ NCU_TRAFFIC_BYTES = {
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
 def fwd_plan(w):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
-    as the library dispatches it: the row kernels solve a ParaGRU sequence
-    longer than 4096 steps in 4096-step segments, and a ParaLSTM sequence
-    in segments of k x 512 steps, k the smallest cluster size below the one
-    the whole sequence needs at which its 8-channel tiles fill the SMs."""
+    as the library dispatches it: the row kernels solve a sequence in
+    segments of k x 1024 (ParaGRU, two CTAs per SM) or k x 512 steps
+    (ParaLSTM, one CTA per SM), k the smallest cluster size below the one
+    the whole sequence needs at which its 8-channel tiles fill the SMs, and
+    a ParaGRU sequence longer than 4096 steps in 4096-step segments."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles8 = w.B * ((w.D + 7) // 8)
     if w.cell == "lstm":
@@ -77,8 +78,19 @@ def fwd_plan(w):
                 k *= 2
             return "lstm_newton_row", 6.5, seg
         return "lstm_newton_fused", 8, w.T
-    if w.T <= 4096 or tiles8 >= sms:
-        return "gru_newton_row", 4, min(w.T, 4096)
+    if w.T <= 4096:
+        cls, seg = 1, w.T
+        while cls * 1024 < w.T:
+            cls *= 2
+        k = 1
+        while k < cls:
+            if k * tiles8 >= 2 * sms:
+                seg = k * 1024
+                break
+            k *= 2
+        return "gru_newton_row", 4, seg
+    if tiles8 >= sms:
+        return "gru_newton_row", 4, 4096
     return "gru_newton_fused", 5, w.T
 
 
@@ -250,8 +262,7 @@ class Path:
 
     def launches_per_step(self):
         nseg = len(fwd_segments(self.w))
-        resets = nseg - 1 if fwd_kernel(self.w)[0] == "gru_newton_row" else 0
-        n = 1 + nseg + resets + (1 if self.hist is not None else 0)  # init, solves, [hist]
+        n = 1 + nseg + (1 if self.hist is not None else 0)  # init, solves, [hist]
         return n + (3 if self.w.adjoint else 0)            # init, adjoint, reduce
 
     def forward(self, x=None):

@@ -93,10 +93,9 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            whole-sequence row kernels would
                                            run: ParaGRU with T <= 4096 (bf16 or
                                            fp32 u) or longer with at least one
-                                           8-channel tile per SM (solved in
-                                           4096-step segments), ParaLSTM with
+                                           8-channel tile per SM, ParaLSTM with
                                            bf16 u and T <= 4096 (segmented as
-                                           pararnn_lstm_solve says) */
+                                           the solves' comments say) */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
@@ -140,12 +139,15 @@ int pararnn_workspace_init(void* workspace, size_t ws_bytes,
  * Newton starts from h = 0 at every t, applies the page's update until the
  * residual of an iterate is below tol everywhere upstream (and then applies
  * that last update), or until max_iters updates have been applied.  Channels
- * are independent; each 8-channel tile stops on its own.  A sequence longer
- * than 4096 steps with at least one 8-channel tile (B * D / 8) per SM is
- * solved 4096-step segment by segment, each segment starting from the state
- * the one before it converged to; stats and iter_hist then take the maximum
- * over the segments.  Shorter-tiled long sequences use one solve over the
- * whole sequence (cluster chunks joined by decoupled look-back). */
+ * are independent; each 8-channel tile stops on its own.  A sequence of up
+ * to 4096 steps is held by a cluster of k CTAs of 1024 steps per tile; when a
+ * smaller cluster of k' CTAs already gives two CTAs per SM
+ * (k' * B * D / 8 >= 2 * SMs), it is solved in segments of k' * 1024 steps.
+ * A longer sequence with at least one 8-channel tile (B * D / 8) per SM is
+ * solved in 4096-step segments.  Each segment starts from the state the one
+ * before it converged to; stats and iter_hist then take the maximum over the
+ * segments.  Shorter-tiled long sequences use one solve over the whole
+ * sequence (cluster chunks joined by decoupled look-back). */
 int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
                       const float* bias, const float* h0, float* h, int B,
                       int T, int D, const pararnn_opts* opts,

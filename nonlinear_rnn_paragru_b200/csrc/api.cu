@@ -18,6 +18,7 @@ int gru_row_box_steps();
 int gru_row_channels();
 int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStream_t stream);
 int gru_row_max_steps();
+int gru_row_cta_steps();
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
 int lstm_chunk_steps();
@@ -177,7 +178,6 @@ __global__ void hist_kernel(const int* __restrict__ chan_k, size_t n, int* hist,
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PARARNN_OK : PARARNN_ERR_CUDA; }
 
 // between the segments of a long sequence: the row kernel's tile counter
-__global__ void ticket_reset_kernel(WsHeader* hdr) { hdr->ticket = 0u; }
 
 int sm_count() {
   int dev = 0, sms = 148;
@@ -249,6 +249,7 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.u = u;
   p.t_base = 0;
   p.t_len = T;
+  p.seg = 0;
   p.ld_h0 = D;
 
   const size_t nch = (size_t)B * D;
@@ -257,16 +258,16 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   // Row kernels: a cluster of CTAs per 8-channel tile holds a whole sequence
-  // of up to 4096 steps (ParaGRU: bf16 or fp32 u; ParaLSTM: bf16 u).  A
-  // longer ParaGRU sequence with at least one 8-channel tile per SM is solved
-  // 4096-step segment by segment, each segment starting from the state the
-  // one before it converged to: the same work as one solve over the whole
-  // sequence, and each segment still fills the GPU.  A ParaLSTM sequence is
-  // solved the same way in segments of k x 512 steps, k the smallest cluster
-  // size below the one the whole sequence needs at which the 8-channel tiles
-  // put a CTA on every SM: smaller clusters fit the SMs without gaps, and
-  // shorter segments converge in fewer iterations.  Otherwise, or on
-  // request, the chunked cluster + look-back solve.
+  // of up to 4096 steps (ParaGRU: bf16 or fp32 u; ParaLSTM: bf16 u).  Where a
+  // smaller cluster of k CTAs already fills the SMs with the tiles (ParaGRU:
+  // two CTAs per SM, 1024 steps per CTA; ParaLSTM: one, 512 steps), the
+  // sequence is solved in segments of k CTAs' steps, in order, each segment
+  // starting from the state the one before it converged to: the same work as
+  // one solve over the whole sequence, with smaller clusters that fit the SMs
+  // without gaps and shorter segments that converge in fewer iterations.  A
+  // ParaGRU sequence longer than 4096 steps with at least one 8-channel tile
+  // per SM is solved in 4096-step segments.  Otherwise, or on request, the
+  // chunked cluster + look-back solve.
   const bool force = opts && (opts->flags & PARARNN_FLAG_FORCE_CHUNKED);
   const bool bf16 = u_dtype == PARARNN_BF16;
   const long long tiles8 = (long long)B * ((D + 7) / 8);
@@ -278,16 +279,23 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());
     if (rc) return rc;
-    const int seg = gru_row_max_steps();
+    int seg = gru_row_max_steps();
+    if (T <= seg) {
+      seg = T;
+      for (int k = 1; k < gru_row_cluster(T); k *= 2)
+        if (k * tiles8 >= 2 * sm_count()) {  // two CTAs per SM
+          seg = k * gru_row_cta_steps();
+          break;
+        }
+    }
     for (int s0 = 0; s0 < T && e == 0; s0 += seg) {
       FwdParams ps = p;
       ps.t_base = s0;
       ps.t_len = std::min(seg, T - s0);
+      ps.seg = s0 / seg;
       if (s0 > 0) {
         ps.h0 = h + (size_t)(s0 - 1) * D;  // the last state of the segment before
         ps.ld_h0 = (long long)T * D;
-        ticket_reset_kernel<<<1, 1, 0, stream>>>(p.hdr);
-        if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
       }
       e = launch_gru_row(rmap, ps, !bf16, stream);
     }

@@ -128,7 +128,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 struct WsHeader {
   unsigned epoch;
   unsigned ticket;
-  unsigned pad[62];
+  unsigned ticket_odd;  // tile counter of the odd-numbered segments of a row solve
+  unsigned pad[61];
 };
 enum : unsigned { kRecAgg = 1, kRecIncl = 2 };
 
@@ -172,11 +173,11 @@ struct FwdParams {
   int* chan_k;        // [B*D] or null
   pararnn_stats* stats;
   // whole-sequence (row) kernel only: the projections (fp32 read directly),
-  // the first step and the length of the segment this launch solves, and the
-  // batch stride of h0 in floats (a segment starts from the state the one
-  // before it ended with)
+  // the first step, the length and the index of the segment this launch
+  // solves, and the batch stride of h0 in floats (a segment starts from the
+  // state the one before it ended with)
   const void* u;
-  int t_base, t_len;
+  int t_base, t_len, seg;
   long long ld_h0;
 };
 

@@ -278,12 +278,16 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   int n = 0;
   unsigned phase = 0;  // exchange phases so far, over all tiles
   // Tiles: the first two of a cluster are clus and clus + nclus; after that
-  // each cluster takes the next ticket of a counter (reset per launch), so
+  // each cluster takes the next ticket of a counter (zero at launch), so
   // clusters that meet slowly converging tiles take fewer.  Cluster rank 0
   // draws the ticket for tile n + 2 at the start of tile n and publishes it
   // into every CTA's ring at the end of tile n; the barrier opening each tile
   // makes it visible.  Tickets rise monotonically, so no tile is skipped.
   const bool drawer = rank == 0 && tid == kRowThreads - 32;
+  // even and odd segments draw from two counters; each launch zeroes the one
+  // the next segment's launch will draw from (the solve's first counter is
+  // zeroed before the first launch)
+  if (blockIdx.x == 0 && tid == 0) *((p.seg & 1) ? &p.hdr->ticket : &p.hdr->ticket_odd) = 0u;
   unsigned ticket = 0;
   int tile = clus, next = clus + nclus;
   for (; tile < ntiles; tile = next, ++n) {
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     else
       __syncthreads();
     if (n >= 1) next = sh.ntile[(n + 1) & 3];
-    if (drawer) ticket = atomicAdd(&p.hdr->ticket, 1u);
+    if (drawer) ticket = atomicAdd((p.seg & 1) ? &p.hdr->ticket_odd : &p.hdr->ticket, 1u);
     // the next tile's parameters: loaded now, stored at the end of this tile
     const int pj = tid - 32;
     float pnext = 0.f;
@@ -624,5 +628,7 @@ int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStr
   }
 }
 int gru_row_max_steps() { return kRowTmax; }
+// steps one CTA holds: a cluster of k CTAs solves up to k times this many
+int gru_row_cta_steps() { return kRowSteps; }
 
 }  // namespace pararnn

@@ -214,3 +214,21 @@ def test_fp32_inputs_both_solvers(cuda_ok):
         h, st, _ = _solve(x, flags=flags)
         assert np.abs(h - ref).max() < TOL_STATE, flags
         assert st["status"] == "converged", (flags, st)
+
+
+@pytest.mark.parametrize("B,T,D,wl", [(1, 3000, 2400, 2), (2, 4000, 1200, 2),
+                                      (1, 3500, 1600, 2), (1, 2500, 2400, 4)])
+def test_short_segments_match_oracle(cuda_ok, B, T, D, wl):
+    # 300 and 200 8-channel tiles: clusters of 1 and 2 CTAs already give two
+    # CTAs per SM on 148 SMs, so sequences of up to 4096 steps are solved in
+    # 1024- and 2048-step segments (ragged last segments here; the last case
+    # has fp32 u), each from the state the one before converged to
+    x = make_inputs(WORKLOADS[wl].scaled(B=B, T=T, D=D))
+    x["h0"] = torch.randn((B, D), generator=torch.Generator().manual_seed(17)) * 0.5
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_CHUNKED):
+        h, st, hist = _solve(x, flags=flags, hist=True)
+        err = np.abs(h - ref).max()
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == B * D
