@@ -316,7 +316,11 @@ __global__ void __launch_bounds__(kArThreads, 2)
           ar_st_async_v2(ar_mapa(smem_u32(&sh.mbox[ms][rank][c]), r), m,
                          ar_mapa(smem_u32(&sh.mbar[ms]), r));
       }
-      if (!mbar_wait_bounded(&sh.mbar[ms], (n / kArSlots) & 1, p.timeout_ns) && status == 0)
+      // The last rank receives nothing, so it neither waits nor re-arms: a
+      // zero-byte re-arm completes the next phase at once, and a warp yet to
+      // wait would then wait for the phase after that one.
+      if (rank < CLS - 1 &&
+          !mbar_wait_bounded(&sh.mbar[ms], (n / kArSlots) & 1, p.timeout_ns) && status == 0)
         status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
       for (int r = CLS - 1; r > 0; --r) {
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kArThreads, 2)
         }
       }
       __syncwarp();
-      if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
+      if (tid == 0 && rank < CLS - 1) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
     }
     const float cwarp = fmaf(cw.x, cin_cta, cw.y);
     const float cchunk = fmaf(xm.x, cwarp, xm.y);
@@ -686,7 +690,9 @@ __global__ void __launch_bounds__(kArThreads, 2)
           ar_st_async_v4(ar_mapa(smem_u32(&sh.mbox[ms][rank][c][1]), r), m1, rb);
         }
       }
-      if (!mbar_wait_bounded(&sh.mbar[ms], (n / kAlSlots) & 1, p.timeout_ns) && status == 0)
+      // the last rank receives nothing: no wait, no re-arm (as for ParaGRU)
+      if (rank < CLS - 1 &&
+          !mbar_wait_bounded(&sh.mbar[ms], (n / kAlSlots) & 1, p.timeout_ns) && status == 0)
         status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
       for (int r = CLS - 1; r > 0; --r) {
@@ -696,7 +702,7 @@ __global__ void __launch_bounds__(kArThreads, 2)
         }
       }
       __syncwarp();
-      if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
+      if (tid == 0 && rank < CLS - 1) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
     }
     const float2 cchunk = xm.apply(cw.apply(cin_cta));
     const float2 cx = My.apply(cchunk);  // entering step 7 from step 8

@@ -163,3 +163,18 @@ def test_lstm_adjoint_is_bitwise_reproducible(cuda_ok):
     g2 = _gpu_adjoint(pr.PARARNN_LSTM, x, h, c)
     for k in ("du", "da", "dbias", "dh0", "dc0"):
         assert np.array_equal(g1[k], g2[k]), k
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+def test_adjoint_clusters_with_many_tiles(cuda_ok, cell):
+    # T = 1000 takes clusters of 2 CTAs; 1024 tiles of 8 channels give each
+    # cluster about seven, so the mailbox ring turns over many times while the
+    # last rank (which receives nothing) runs ahead of the first
+    w = WORKLOADS[2 if cell == "gru" else 5].scaled(B=8, T=1000, D=1024)
+    x = make_inputs(w)
+    if cell == "gru":
+        h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+        _check_gru(x, h)
+    else:
+        c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+        _check_lstm(x, c, h)
