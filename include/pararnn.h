@@ -222,6 +222,31 @@ int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a,
                          float* c, float* h, int B, int T, int D,
                          pararnn_stream_t stream);
 
+/* One recurrence step, for autoregressive decoding.  Generating a token
+ * costs one update of the hidden state whatever the context length
+ * ("Apple научила классические RNN масштабироваться...", "Инференс быстрее и
+ * стабильнее по длине контекста", Figure 8); this applies the cell of
+ * pararnn_gru_solve once to a batch of states.
+ * In:  u_t [B][3][D] (the step's z, r, c projections; dtype u_dtype), a [3][D],
+ *      bias [3][D] or NULL (zeros), h_prev [B][D] or NULL (zeros).
+ * Out: h_next [B][D].  h_next may be h_prev itself (in-place update: every
+ *      element is read before it is written); other overlaps are not allowed.
+ * D must be a multiple of 8, as for the solves.  Stream-ordered, no
+ * workspace, no synchronisation.  Returns PARARNN_ERR_INVALID_ARG /
+ * _UNSUPPORTED_DTYPE / _MISALIGNED (4 B for float arrays, 2 B for bf16 u_t)
+ * without launching, PARARNN_ERR_CUDA if the launch fails. */
+int pararnn_gru_step(const void* u_t, int u_dtype, const float* a,
+                     const float* bias, const float* h_prev, float* h_next,
+                     int B, int D, pararnn_stream_t stream);
+
+/* ParaLSTM step: u_t [B][4][D] (i, f, g, o), a/bias [4][D], c_prev/h_prev
+ * [B][D] or NULL (zeros) -> c_next, h_next [B][D].  c_next and h_next must
+ * be distinct; each may be the matching *_prev array (in-place update). */
+int pararnn_lstm_step(const void* u_t, int u_dtype, const float* a,
+                      const float* bias, const float* c_prev,
+                      const float* h_prev, float* c_next, float* h_next,
+                      int B, int D, pararnn_stream_t stream);
+
 /* Human-readable text for a return code. */
 const char* pararnn_strerror(int code);
 

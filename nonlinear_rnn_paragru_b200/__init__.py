@@ -22,8 +22,9 @@ __all__ = [
     "PararnnOpts", "PararnnError", "library_path", "load_library",
     "pararnn_workspace_size", "pararnn_workspace_init", "pararnn_gru_solve",
     "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_noalloc",
-    "pararnn_seq_baseline",
+    "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
+    "gru_step", "lstm_step",
     "Workspace", "read_stats",
 ]
 
@@ -81,6 +82,8 @@ def load_library():
                                      i, vp]),
         "pararnn_adjoint_noalloc": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, fp,
                                         fp, fp, fp, fp, fp, i, i, i, ip, vp]),
+        "pararnn_gru_step": (i, [vp, i, fp, fp, fp, fp, i, i, vp]),
+        "pararnn_lstm_step": (i, [vp, i, fp, fp, fp, fp, fp, fp, i, i, vp]),
         "pararnn_strerror": (ctypes.c_char_p, [i]),
     }
     for name, (res, args) in sigs.items():
@@ -205,6 +208,20 @@ def pararnn_seq_baseline(cell, u, a, bias, c0, h0, c, h, stream=None):
         _stream(stream)), "pararnn_seq_baseline")
 
 
+def pararnn_gru_step(u_t, a, bias, h_prev, h_next, stream=None):
+    _check(load_library().pararnn_gru_step(
+        _uptr(u_t), _dtype_code(u_t), _ptr(a), _ptr(bias), _ptr(h_prev),
+        _ptr(h_next), u_t.shape[0], u_t.shape[2], _stream(stream)),
+        "pararnn_gru_step")
+
+
+def pararnn_lstm_step(u_t, a, bias, c_prev, h_prev, c_next, h_next, stream=None):
+    _check(load_library().pararnn_lstm_step(
+        _uptr(u_t), _dtype_code(u_t), _ptr(a), _ptr(bias), _ptr(c_prev),
+        _ptr(h_prev), _ptr(c_next), _ptr(h_next), u_t.shape[0], u_t.shape[2],
+        _stream(stream)), "pararnn_lstm_step")
+
+
 def pararnn_strerror(code) -> str:
     return load_library().pararnn_strerror(int(code)).decode()
 
@@ -287,6 +304,26 @@ def adjoint(cell, u, a, bias, h0, h, dLdh, c0=None, c=None, *, workspace=None,
                     status, buf, stream)
     return {"du": du, "da": da, "dbias": db, "dh0": dh0, "dc0": dc0,
             "status": status}
+
+
+def gru_step(u_t, a, bias=None, h_prev=None, *, out=None, stream=None):
+    """One ParaGRU decode step: u_t [B, 3, D] -> the next state [B, D].
+    `out` may be `h_prev` (in-place update)."""
+    B, G, D = u_t.shape
+    h = torch.empty((B, D), dtype=torch.float32, device=u_t.device) if out is None else out
+    pararnn_gru_step(u_t, a, bias, h_prev, h, stream)
+    return h
+
+
+def lstm_step(u_t, a, bias=None, c_prev=None, h_prev=None, *, out=None, stream=None):
+    """One ParaLSTM decode step: u_t [B, 4, D] -> (c, h) [B, D] each.
+    `out` = (c, h) may be (c_prev, h_prev) (in-place update)."""
+    B, G, D = u_t.shape
+    if out is None:
+        out = (torch.empty((B, D), dtype=torch.float32, device=u_t.device),
+               torch.empty((B, D), dtype=torch.float32, device=u_t.device))
+    pararnn_lstm_step(u_t, a, bias, c_prev, h_prev, out[0], out[1], stream)
+    return out
 
 
 def seq_baseline(cell, u, a, bias=None, c0=None, h0=None, stream=None):

@@ -39,6 +39,9 @@ int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float
                             const float* c0, const float* h0, float* du, float* da,
                             float* dbias, float* dc0, float* dh0, int B, int T, int D,
                             int* status, void* ws, cudaStream_t stream);
+int launch_decode_step(int cell, bool bf16, const void* u, const float* a, const float* bias,
+                       const float* c_prev, const float* h_prev, float* c_next, float* h_next,
+                       int B, int D, cudaStream_t stream);
 int launch_seq_baseline(int cell, bool bf16, const void* u, const float* a, const float* bias,
                         const float* c0, const float* h0, float* c, float* h, int B, int T,
                         int D, cudaStream_t stream);
@@ -437,6 +440,42 @@ int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a, c
   if (cell == PARARNN_GRU && (c || c0)) return PARARNN_ERR_INVALID_ARG;
   const int e = launch_seq_baseline(cell, u_dtype == PARARNN_BF16, u, a, bias, c0, h0, c, h, B, T,
                                     D, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+// Shared checks of the two single-step entry points.
+static int step_args(const void* u_t, int u_dtype, const float* a, const float* bias, int B, int D) {
+  const int rc = check_sizes(B, 1, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  if (!u_t || !a) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(u_t, u_dtype == PARARNN_BF16 ? 2 : 4) || !aligned(a, 4) || (bias && !aligned(bias, 4)))
+    return PARARNN_ERR_MISALIGNED;
+  return PARARNN_OK;
+}
+
+int pararnn_gru_step(const void* u_t, int u_dtype, const float* a, const float* bias,
+                     const float* h_prev, float* h_next, int B, int D, pararnn_stream_t stream) {
+  int rc = step_args(u_t, u_dtype, a, bias, B, D);
+  if (rc) return rc;
+  if (!h_next) return PARARNN_ERR_INVALID_ARG;
+  if ((h_prev && !aligned(h_prev, 4)) || !aligned(h_next, 4)) return PARARNN_ERR_MISALIGNED;
+  const int e = launch_decode_step(PARARNN_GRU, u_dtype == PARARNN_BF16, u_t, a, bias, nullptr,
+                                   h_prev, nullptr, h_next, B, D, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+int pararnn_lstm_step(const void* u_t, int u_dtype, const float* a, const float* bias,
+                      const float* c_prev, const float* h_prev, float* c_next, float* h_next,
+                      int B, int D, pararnn_stream_t stream) {
+  int rc = step_args(u_t, u_dtype, a, bias, B, D);
+  if (rc) return rc;
+  if (!c_next || !h_next || c_next == h_next) return PARARNN_ERR_INVALID_ARG;
+  if ((c_prev && !aligned(c_prev, 4)) || (h_prev && !aligned(h_prev, 4)) ||
+      !aligned(c_next, 4) || !aligned(h_next, 4))
+    return PARARNN_ERR_MISALIGNED;
+  const int e = launch_decode_step(PARARNN_LSTM, u_dtype == PARARNN_BF16, u_t, a, bias, c_prev,
+                                   h_prev, c_next, h_next, B, D, (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 

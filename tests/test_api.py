@@ -32,7 +32,8 @@ def test_header_declares_the_boundary_calls():
     names = _declared()
     for n in ("pararnn_gru_solve", "pararnn_lstm_solve", "pararnn_adjoint",
               "pararnn_workspace_size", "pararnn_workspace_init",
-              "pararnn_seq_baseline", "pararnn_strerror"):
+              "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
+              "pararnn_strerror"):
         assert n in names
 
 
@@ -108,3 +109,28 @@ def test_binding_rejects_host_tensors():
         pr._ptr(a)
     with pytest.raises(ValueError):
         pr._uptr(u)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(u=None), -1), (dict(a=None), -1), (dict(hn=None), -1), (dict(D=12), -1),
+    (dict(B=0), -1), (dict(dt=5), -2), (dict(u=0x1001), -5), (dict(hn=0x3002), -5),
+    (dict(hp=0x5002), -5), (dict(bias=0x6001), -5),
+])
+def test_step_rejects_bad_arguments_on_host(over, code):
+    lib = pr.load_library()
+    g = dict(u=0x1000, dt=pr.PARARNN_BF16, a=0x2000, bias=None, hp=None, hn=0x3000,
+             B=2, D=32)
+    g.update(over)
+    assert lib.pararnn_gru_step(g["u"], g["dt"], g["a"], g["bias"], g["hp"], g["hn"],
+                                g["B"], g["D"], None) == code
+
+
+def test_lstm_step_needs_distinct_outputs():
+    lib = pr.load_library()
+    ok = [0x1000, pr.PARARNN_F32, 0x2000, None, None, None, 0x3000, 0x4000, 2, 32, None]
+    a = list(ok); a[6] = None
+    assert lib.pararnn_lstm_step(*a) == -1         # no c output
+    a = list(ok); a[7] = 0x3000
+    assert lib.pararnn_lstm_step(*a) == -1         # c and h the same array
+    a = list(ok); a[0] = 0x1002
+    assert lib.pararnn_lstm_step(*a) == -5         # fp32 u_t needs 4-byte alignment
