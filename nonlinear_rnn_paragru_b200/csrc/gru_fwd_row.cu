@@ -1,10 +1,12 @@
-// gru_fwd_row.cu -- fused Newton-scan ParaGRU solve for sequences of up to
-// 4096 steps with bf16 input projections: 8 channels per CTA, a cluster of
-// CLS = ceil(T / 1024) CTAs per tile, two CTAs per SM, the cell evaluated on
-// packed fp32 pairs.
+// gru_fwd_row.cu -- fused Newton-scan ParaGRU solve for sequences (or
+// segments of sequences) of up to 4096 steps with bf16 or fp32 input
+// projections: 8 channels per CTA, a cluster of CLS = ceil(T / 1024) CTAs per
+// tile, two CTAs per SM, the cell evaluated on packed fp32 pairs.
 //
-// A tile is 8 consecutive channels of one batch row over the whole sequence.
-// CTA rank r of the cluster owns steps [1024 r, 1024 (r+1)): 8 warps x 32
+// A tile is 8 consecutive channels of one batch row over the steps this launch
+// solves: the whole sequence, or one segment of it that starts from the state
+// the segment before ended with (the host launches the segments in order).  CTA
+// rank r of the cluster owns steps [1024 r, 1024 (r+1)) of them: 8 warps x 32
 // lanes, lane = (k, c) with the channel c = lane % 8 fastest and k = lane / 8
 // one of four 32-step chunks; warp w covers steps [128 w, 128 w + 128) of the
 // CTA's range.  A thread keeps its chunk's iterate h and running Jacobian
@@ -27,15 +29,16 @@
 // receiver's mbarrier, so a CTA waits only for the bytes it needs and no
 // cluster-wide barrier is taken per iteration.  The fix-up adds P_t ds_in.
 // Mailboxes and per-warp data are double-buffered by the parity of a phase
-// counter that runs on across tiles.  The cluster stops after the update of the first iteration whose
-// residual over the tile is below tol, or after a residual-only evaluation at
-// the cap; the state before each chunk is re-anchored every iteration to its
+// counter that runs on across tiles.  The cluster stops after the update of
+// the first iteration whose residual over the tile is below tol, or after a
+// residual-only evaluation at the cap; the state before each chunk is re-anchored every iteration to its
 // predecessor's pre-update last state plus the incoming delta.
 //
-// Data: the tile's u arrives bf16 by four TMA boxes of 256 steps into the top
-// of the CTA's 98 KB buffer (with a, bias and h0 of its channels as 32-byte
-// bulk copies on the same mbarrier; the boxes of the tile after it are
-// prefetched into L2 meanwhile) and is expanded in place, once per tile, into the
+// Data: bf16 u arrives by four TMA boxes of 256 steps into the top of the
+// CTA's 98 KB buffer (fp32 u is read straight from global memory by the
+// expansion, the next tile's rows prefetched into L2 meanwhile); a, bias and
+// h0 of the next tile's channels are read with plain loads a tile ahead into
+// a double-buffered block.  Once per tile u is expanded in place into the
 // fp32 arguments -log2e u_z + b'_z, -log2e u_r + b'_r, 2 log2e u_c + b'_c
 // (b' the bias scaled alike), stored per chunk as [gate][pair i][channel]
 // {step i, step i + 16}: one 8-byte load per gate and pair, channel c at slot

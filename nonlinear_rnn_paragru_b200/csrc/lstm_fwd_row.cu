@@ -1,9 +1,12 @@
-// lstm_fwd_row.cu -- fused Newton-scan ParaLSTM solve for sequences of up to
-// 4096 steps with bf16 input projections: 8 channels per CTA, a cluster of
-// CLS = ceil(T / 512) CTAs per tile, the cell evaluated on packed fp32 pairs.
+// lstm_fwd_row.cu -- fused Newton-scan ParaLSTM solve for sequences (or
+// segments of sequences) of up to 4096 steps with bf16 input projections: 8
+// channels per CTA, a cluster of CLS = ceil(T / 512) CTAs per tile, the cell
+// evaluated on packed fp32 pairs.
 //
-// A tile is 8 consecutive channels of one batch row over the whole sequence.
-// CTA rank r of the cluster owns steps [512 r, 512 (r+1)): 8 warps x 32
+// A tile is 8 consecutive channels of one batch row over the steps this launch
+// solves: the whole sequence, or one segment of it that starts from the (c, h)
+// the segment before ended with (the host launches the segments in order).  CTA
+// rank r of the cluster owns steps [512 r, 512 (r+1)) of them: 8 warps x 32
 // lanes, lane = (k, c) with the channel c = lane % 8 fastest and k = lane / 8
 // one of four 16-step chunks; warp w covers steps [64 w, 64 w + 64) of the
 // CTA's range.  A thread keeps its chunk's iterate (c, h) and the running
@@ -34,8 +37,9 @@
 // last state plus the incoming delta.
 //
 // Data: the tile's u arrives bf16 by two TMA boxes of 256 steps into a
-// staging area (with a, bias, c0 and h0 of its channels as 32-byte bulk
-// copies on the same mbarrier) and is expanded, once per tile, into the fp32
+// staging area (a, bias, c0 and h0 of the next tile's channels are read with
+// plain loads a tile ahead into a double-buffered block) and is expanded,
+// once per tile, into the fp32
 // arguments -log2e u + b' (i, f, o) and 2 log2e u + b' (g), stored per chunk
 // as [gate][pair i][channel] {step i, step i + 8}, channel c at slot
 // c ^ (i >> 1): one 8-byte load per gate and pair.  The next tile's boxes are
