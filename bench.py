@@ -35,13 +35,13 @@ from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs  # noqa: E4
 
 METRIC = "Newton-solved token*channels/s (fwd+bwd)"
 UNIT = "tokch/s"
-# Counters of the dominant kernel taken with ncu on this build (one launch on
-# the workload in the key; see profiles/).  None when not captured for the
-# kernel as it stands.
+# DRAM bytes (read + write) of one launch of the dominant kernel, taken with
+# ncu on this build for the workload in the key.  None when not captured for
+# the kernel as it stands.
 NCU_TRAFFIC_BYTES = {
-    # profiles/gru_newton_row_b8_t4096_d1024.md: one 1024-step segment's launch
+    # one 1024-step segment's launch (the solve is four of them)
     ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 50_585_600 + 7_483_392,
-    # profiles/lstm_newton_row_b8_t4096_d1024.md: one 512-step segment's launch
+    # one 512-step segment's launch (the solve is eight of them)
     ("lstm_newton_row", "lstm_b8_t4096_d1024_bf16"): 33_703_168 + 5_925_120,
 }
 # The forward kernel a workload runs and its special-function (MUFU)
