@@ -222,6 +222,34 @@ int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a,
                          float* c, float* h, int B, int T, int D,
                          pararnn_stream_t stream);
 
+/* Unfused Newton solve: the "CUDA-accelerated" tier of the pages' three
+ * ("Apple научила классические RNN масштабироваться...", "Три уровня
+ * производительности"), kept as an ablation against the fused solves.  Each
+ * iteration ("Параллельность RNN?", §1.2-§1.3) runs one kernel that writes
+ * the Jacobian blocks A_t and the right-hand sides -r_t of every element to
+ * the workspace, three kernels that solve ds_t = A_t ds_{t-1} - r_t by a
+ * chunked scan and add ds to the iterate, and a host check of the residual.
+ * cell: PARARNN_GRU (c0 and c NULL) or PARARNN_LSTM; u, a, bias, c0, h0, c, h
+ * as for pararnn_gru_solve / pararnn_lstm_solve.  Stopping is global: the
+ * update of the first iteration whose max|r| over the whole problem is below
+ * opts->tol is applied and the solve ends; the cap ends with a residual-only
+ * evaluation and NOT_CONVERGED.  *stats as for the fused solves; there is no
+ * iteration histogram.
+ * Blocking: the host reads the residual after every iteration, so the call
+ * synchronises `stream` and returns when the solve is done.
+ * Workspace: pararnn_unfused_workspace_size(cell, B, T, D) bytes, 256-byte
+ * aligned, no initialisation (4 B per element for each Jacobian entry and
+ * right-hand side: 8 B per element for ParaGRU, 24 B for ParaLSTM, plus the
+ * scan's chunk maps).  Alignment: u 2 B (bf16) or 4 B (fp32), the float
+ * arrays 4 B.  Errors as for the fused solves. */
+size_t pararnn_unfused_workspace_size(int cell, int B, int T, int D);
+int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a,
+                          const float* bias, const float* c0,
+                          const float* h0, float* c, float* h, int B, int T,
+                          int D, const pararnn_opts* opts,
+                          pararnn_stats* stats, void* workspace,
+                          size_t ws_bytes, pararnn_stream_t stream);
+
 /* One recurrence step, for autoregressive decoding.  Generating a token
  * costs one update of the hidden state whatever the context length
  * ("Apple научила классические RNN масштабироваться...", "Инференс быстрее и

@@ -23,6 +23,7 @@ __all__ = [
     "pararnn_workspace_size", "pararnn_workspace_init", "pararnn_gru_solve",
     "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_noalloc",
     "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
+    "pararnn_unfused_workspace_size", "pararnn_solve_unfused", "solve_unfused",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
     "gru_step", "lstm_step",
     "Workspace", "read_stats",
@@ -82,6 +83,9 @@ def load_library():
                                      i, vp]),
         "pararnn_adjoint_noalloc": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, fp,
                                         fp, fp, fp, fp, fp, i, i, i, ip, vp]),
+        "pararnn_unfused_workspace_size": (sz, [i, i, i, i]),
+        "pararnn_solve_unfused": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i, i,
+                                      op, vp, vp, sz, vp]),
         "pararnn_gru_step": (i, [vp, i, fp, fp, fp, fp, i, i, vp]),
         "pararnn_lstm_step": (i, [vp, i, fp, fp, fp, fp, fp, fp, i, i, vp]),
         "pararnn_strerror": (ctypes.c_char_p, [i]),
@@ -208,6 +212,20 @@ def pararnn_seq_baseline(cell, u, a, bias, c0, h0, c, h, stream=None):
         _stream(stream)), "pararnn_seq_baseline")
 
 
+def pararnn_unfused_workspace_size(cell, B, T, D) -> int:
+    return int(load_library().pararnn_unfused_workspace_size(cell, B, T, D))
+
+
+def pararnn_solve_unfused(cell, u, a, bias, c0, h0, c, h, opts, stats, workspace,
+                          stream=None):
+    _check(load_library().pararnn_solve_unfused(
+        cell, _uptr(u), _dtype_code(u), _ptr(a), _ptr(bias), _ptr(c0), _ptr(h0),
+        _ptr(c), _ptr(h), u.shape[0], u.shape[1], u.shape[3], ctypes.byref(opts),
+        _iptr(stats), _wptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "pararnn_solve_unfused")
+
+
 def pararnn_gru_step(u_t, a, bias, h_prev, h_next, stream=None):
     _check(load_library().pararnn_gru_step(
         _uptr(u_t), _dtype_code(u_t), _ptr(a), _ptr(bias), _ptr(h_prev),
@@ -304,6 +322,22 @@ def adjoint(cell, u, a, bias, h0, h, dLdh, c0=None, c=None, *, workspace=None,
                     status, buf, stream)
     return {"du": du, "da": da, "dbias": db, "dh0": dh0, "dc0": dc0,
             "status": status}
+
+
+def solve_unfused(cell, u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
+                  workspace=None, stream=None):
+    """The unfused tier: returns (c, h, stats) with c None for ParaGRU.
+    Synchronises the stream (the host checks the residual each iteration)."""
+    B, T, G, D = u.shape
+    dev = u.device
+    h = torch.empty((B, T, D), dtype=torch.float32, device=dev)
+    c = torch.empty((B, T, D), dtype=torch.float32, device=dev) if cell == PARARNN_LSTM else None
+    stats = _new_stats(dev)
+    ws = workspace if workspace is not None else Workspace(dev)
+    buf = ws.get(pararnn_unfused_workspace_size(cell, B, T, D), stream)
+    pararnn_solve_unfused(cell, u, a, bias, c0, h0, c, h, _opts(tol, max_iters), stats,
+                          buf, stream)
+    return c, h, stats
 
 
 def gru_step(u_t, a, bias=None, h_prev=None, *, out=None, stream=None):

@@ -39,6 +39,11 @@ int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float
                             const float* c0, const float* h0, float* du, float* da,
                             float* dbias, float* dc0, float* dh0, int B, int T, int D,
                             int* status, void* ws, cudaStream_t stream);
+size_t unfused_ws_bytes(int cell, int B, int T, int D);
+int unfused_solve(int cell, bool bf16, const void* u, const float* a, const float* bias,
+                  const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
+                  float tol, int max_iters, pararnn_stats* stats, void* workspace,
+                  cudaStream_t stream);
 int launch_decode_step(int cell, bool bf16, const void* u, const float* a, const float* bias,
                        const float* c_prev, const float* h_prev, float* c_next, float* h_next,
                        int B, int D, cudaStream_t stream);
@@ -440,6 +445,36 @@ int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a, c
   if (cell == PARARNN_GRU && (c || c0)) return PARARNN_ERR_INVALID_ARG;
   const int e = launch_seq_baseline(cell, u_dtype == PARARNN_BF16, u, a, bias, c0, h0, c, h, B, T,
                                     D, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+size_t pararnn_unfused_workspace_size(int cell, int B, int T, int D) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return 0;
+  if (check_sizes(B, T, D)) return 0;
+  return unfused_ws_bytes(cell, B, T, D);
+}
+
+int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+                          const float* c0, const float* h0, float* c, float* h, int B, int T,
+                          int D, const pararnn_opts* opts, pararnn_stats* stats, void* workspace,
+                          size_t ws_bytes, pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, T, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  if (!u || !a || !h || !stats || !workspace) return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_LSTM && !c) return PARARNN_ERR_INVALID_ARG;
+  if (cell == PARARNN_GRU && (c || c0)) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(u, u_dtype == PARARNN_BF16 ? 2 : 4) || !aligned(h, 4) || (c && !aligned(c, 4)) ||
+      !aligned(a, 4) || (bias && !aligned(bias, 4)) || (h0 && !aligned(h0, 4)) ||
+      (c0 && !aligned(c0, 4)) || !aligned(stats, 4) || !aligned(workspace, 256))
+    return PARARNN_ERR_MISALIGNED;
+  if (ws_bytes < unfused_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
+  const float tol = (opts && opts->tol > 0.f) ? opts->tol : kDefaultTol;
+  const int max_iters = resolve_max_iters(opts ? opts->max_iters : 0);
+  if (max_iters > kMaxItersLimit) return PARARNN_ERR_INVALID_ARG;
+  const int e = unfused_solve(cell, u_dtype == PARARNN_BF16, u, a, bias, c0, h0, c, h, B, T, D,
+                              tol, max_iters, stats, workspace, (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 

@@ -134,3 +134,30 @@ def test_lstm_step_needs_distinct_outputs():
     assert lib.pararnn_lstm_step(*a) == -1         # c and h the same array
     a = list(ok); a[0] = 0x1002
     assert lib.pararnn_lstm_step(*a) == -5         # fp32 u_t needs 4-byte alignment
+
+
+def test_unfused_workspace_and_argument_checks():
+    lib = pr.load_library()
+    g = pr.pararnn_unfused_workspace_size(pr.PARARNN_GRU, 8, 4096, 1024)
+    l = pr.pararnn_unfused_workspace_size(pr.PARARNN_LSTM, 8, 4096, 1024)
+    n = 8 * 4096 * 1024
+    assert g >= 8 * n and l >= 24 * n and g % 256 == 0 and l % 256 == 0
+    assert pr.pararnn_unfused_workspace_size(pr.PARARNN_GRU, 1, 16, 12) == 0   # D % 8
+    assert pr.pararnn_unfused_workspace_size(5, 1, 16, 16) == 0                # cell
+    o = pr._opts()
+    base = [pr.PARARNN_GRU, 0x1000, pr.PARARNN_BF16, 0x2000, None, None, None, None,
+            0x3000, 1, 8, 16, ctypes.byref(o), 0x4000, 0x10000, 1 << 20, None]
+    a = list(base); a[0] = 7
+    assert lib.pararnn_solve_unfused(*a) == -1      # bad cell
+    a = list(base); a[7] = 0x5000
+    assert lib.pararnn_solve_unfused(*a) == -1      # c given for ParaGRU
+    a = list(base); a[8] = None
+    assert lib.pararnn_solve_unfused(*a) == -1      # no h
+    a = list(base); a[2] = 4
+    assert lib.pararnn_solve_unfused(*a) == -2      # dtype
+    a = list(base); a[14] = 0x10010
+    assert lib.pararnn_solve_unfused(*a) == -5      # workspace alignment
+    a = list(base); a[15] = 64
+    assert lib.pararnn_solve_unfused(*a) == -3      # workspace too small
+    a = list(base); a[0] = pr.PARARNN_LSTM
+    assert lib.pararnn_solve_unfused(*a) == -1      # ParaLSTM without c

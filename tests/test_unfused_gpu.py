@@ -1,0 +1,76 @@
+"""GPU parity of the unfused Newton solve (Jacobians and right-hand sides
+written to HBM, a separate chunked scan, the host checking the residual)
+against the fp64 oracle: its capped iterates against the oracle's Newton, its
+converged states against the sequential recurrence (max-abs 1e-4)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nonlinear_rnn_paragru_b200 as pr
+from nonlinear_rnn_paragru_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_STATE = 1e-4
+
+
+def _inputs(cell, B, T, D, f32=False, seed=2):
+    x = make_inputs(WORKLOADS[2 if cell == "gru" else 3].scaled(B=B, T=T, D=D))
+    g = torch.Generator().manual_seed(seed)
+    x["h0"] = torch.randn((B, D), generator=g) * 0.5
+    if cell == "lstm":
+        x["c0"] = torch.randn((B, D), generator=g) * 0.5
+    if f32:
+        x["u"] = x["u"].float()  # the same values, read as fp32
+    return x
+
+
+def _run(cell, x, **kw):
+    d = "cuda"
+    cid = pr.PARARNN_GRU if cell == "gru" else pr.PARARNN_LSTM
+    c, h, st = pr.solve_unfused(cid, x["u"].to(d), x["a"].to(d), x["bias"].to(d),
+                                x["c0"].to(d) if cell == "lstm" else None, x["h0"].to(d),
+                                **kw)
+    torch.cuda.synchronize()
+    return (c.cpu().numpy() if c is not None else None), h.cpu().numpy(), pr.read_stats(st)
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("n", [1, 2])
+def test_capped_iterates_match_oracle_newton(cuda_ok, cell, n):
+    x = _inputs(cell, 2, 150, 16)   # 150 steps: three scan chunks, the last ragged
+    c, h, st = _run(cell, x, tol=1e-30, max_iters=n)
+    assert st["status"] == "not_converged" and st["iters"] == n and st["evals"] == n + 1
+    if cell == "gru":
+        r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=n)
+        err = np.abs(h - r["h"]).max()
+    else:
+        r = oracle.lstm_newton(x["u"], x["a"], x["bias"], x["c0"], x["h0"], tol=0.0,
+                               max_iters=n)
+        err = max(np.abs(h - r["h"]).max(), np.abs(c - r["c"]).max())
+    assert err < TOL_STATE, err
+
+
+@pytest.mark.parametrize("cell", ["gru", "lstm"])
+@pytest.mark.parametrize("f32", [False, True])
+def test_converges_to_the_sequential_recurrence(cuda_ok, cell, f32):
+    x = _inputs(cell, 2, 1000, 40, f32=f32)
+    c, h, st = _run(cell, x)
+    assert st["status"] == "converged", st
+    if cell == "gru":
+        err = np.abs(h - oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])).max()
+    else:
+        rc, rh = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+        err = max(np.abs(h - rh).max(), np.abs(c - rc).max())
+    assert err < TOL_STATE, (err, st)
+
+
+def test_agrees_with_the_fused_solve(cuda_ok):
+    x = _inputs("gru", 4, 2048, 64)
+    _, h_u, st_u = _run("gru", x)
+    d = "cuda"
+    h_f, st_f, _ = pr.gru_solve(x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d))
+    torch.cuda.synchronize()
+    assert st_u["status"] == "converged" and pr.read_stats(st_f)["status"] == "converged"
+    assert np.abs(h_u - h_f.cpu().numpy()).max() < TOL_STATE
