@@ -14,6 +14,9 @@ Pins of each function (tests/test_oracle.py):
   gru_newton / lstm_newton prefix exactness, affine one/two-step convergence,
                            convergence to the sequential root
   linrec                   closed form and tree-order scans
+  dense_gru_*              the general cell: ParaGRU when W is diagonal, torch's
+                           GRU cell and autograd Jacobian, prefix exactness and
+                           convergence of its Newton to the sequential root
 """
 import ctypes
 import os
@@ -53,6 +56,10 @@ def _L():
                                         dp, dp, dp, i, i, i]),
             "oracle_lstm_newton": (None, [dp, dp, dp, dp, dp, dp, dp, i, i, i,
                                           d, i, dp, ip, ip]),
+            "oracle_dense_gru_step": (None, [i, i, dp, dp, dp, dp, dp, dp]),
+            "oracle_dense_gru_seq": (None, [dp, dp, dp, dp, dp, i, i, i]),
+            "oracle_dense_gru_newton": (None, [dp, dp, dp, dp, dp, i, i, i, d, i,
+                                               dp, ip]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(_lib, name)
@@ -216,3 +223,38 @@ def lstm_newton(u, a, bias=None, c0=None, h0=None, tol=1e-6, max_iters=None,
                             ck.ctypes.data_as(ctypes.POINTER(ctypes.c_int)))
     n = it.value
     return {"c": c, "h": h, "iters": n, "trace": trace[: n + 1], "chan_k": ck}
+
+
+# ------------------------------------------- general cell (dense Jacobian) --
+def dense_gru_step(h, u, W, bias=None):
+    """GRU with full recurrent matrices, one step over n rows: h [n,D],
+    u [n,3,D], W [3,D,D], bias [3,D] -> (h' [n,D], J [n,D,D])."""
+    h, u, W, bias = map(_f64, (h, u, W, bias))
+    n, D = h.shape
+    hn, J = np.empty((n, D)), np.empty((n, D, D))
+    _L().oracle_dense_gru_step(n, D, _p(h), _p(u), _p(W), _p(bias), _p(hn), _p(J))
+    return hn, J
+
+
+def dense_gru_seq(u, W, bias=None, h0=None):
+    u, W, bias, h0 = map(_f64, (u, W, bias, h0))
+    B, T, G, D = u.shape
+    assert G == 3 and W.shape == (3, D, D)
+    h = np.empty((B, T, D))
+    _L().oracle_dense_gru_seq(_p(u), _p(W), _p(bias), _p(h0), _p(h), B, T, D)
+    return h
+
+
+def dense_gru_newton(u, W, bias=None, h0=None, tol=1e-6, max_iters=None, h_init=None):
+    """-> dict(h, iters, trace (max|r| per iterate))"""
+    u, W, bias, h0 = map(_f64, (u, W, bias, h0))
+    B, T, _, D = u.shape
+    if max_iters is None:
+        max_iters = T
+    h = np.zeros((B, T, D)) if h_init is None else _f64(h_init).copy()
+    trace = np.full(max_iters + 1, np.nan)
+    it = ctypes.c_int(0)
+    _L().oracle_dense_gru_newton(_p(u), _p(W), _p(bias), _p(h0), _p(h), B, T, D,
+                                 float(tol), int(max_iters), _p(trace), ctypes.byref(it))
+    n = it.value
+    return {"h": h, "iters": n, "trace": trace[: n + 1]}

@@ -23,6 +23,8 @@
  *      substitution equations].  It is used for iteration counts and for the
  *      invariants the page fixes (prefix exactness, one-step convergence of an
  *      affine map); the states oracle is (1).
+ *   4. The same three for a general cell with a dense D x D Jacobian (the GRU
+ *      with full recurrent matrices), at the end of the file.
  *
  * Cells.  Both cells have diagonal recurrent weights, so every channel is an
  * independent scalar (ParaGRU) or 2-state (ParaLSTM) recurrence and the
@@ -545,3 +547,167 @@ void oracle_lstm_newton(const double* u, const double* a, const double* bias,
   free(J);
   free(last_bad);
 }
+
+/* ------------------------------------------------------------------------- */
+/* A general cell: the GRU with full recurrent matrices (dense Jacobian)     */
+/* ------------------------------------------------------------------------- */
+/*
+ * The Newton step of the pages holds for any Markov cell: the Jacobian of the
+ * residual is block-bidiagonal, identity blocks on the diagonal and
+ * -df/ds(s_{t-1}) below it, a full D x D matrix for a general cell
+ * [Параллельность RNN?, §1.3, the block-bidiagonal J and "Сколько нам реально
+ * нужно памяти"].  The general cell here is the standard GRU with full
+ * recurrent matrices W [3][D][D] (row i of W_g feeds h into gate g of unit i),
+ * the reset gate applied to the recurrent term of the candidate, as in
+ * PyTorch's GRU cell:
+ *
+ *   z = sig(W_z h + u_z + b_z)        r = sig(W_r h + u_r + b_r)
+ *   q = W_c h                         c = tanh(u_c + b_c + r q)
+ *   h' = (1 - z) h + z c              (products of vectors elementwise)
+ *
+ * With W_g = diag(a_g), r q = a_c (r h) and this is the ParaGRU cell above.
+ * Its Jacobian, by the chain rule on each line:
+ *
+ *   dh'/dh = diag(1 - z) + diag((c - h) z (1 - z)) W_z
+ *            + diag(z (1 - c^2)) [diag(r) W_c + diag(q r (1 - r)) W_r]
+ *
+ * Layouts: u [B][T][3][D] as for ParaGRU, W [3][D][D] row-major, bias [3][D],
+ * h0 [B][D], h [B][T][D], J [D][D] row-major (J[i][j] = dh'_i / dh_j).
+ */
+#define DW(g, i, j) W[((size_t)(g) * D + (i)) * D + (j)]
+
+/* One step for one batch row: h [D], u [3][D] (gate stride D) -> hn [D] and,
+ * if J is not NULL, the Jacobian [D][D].  work holds 4 D doubles. */
+static void dense_gru_cell(int D, const double* W, const double* bias, const double* h,
+                           const double* u, double* hn, double* J, double* work) {
+  double* z = work;
+  double* r = work + D;
+  double* q = work + 2 * D;
+  double* c = work + 3 * D;
+  for (int i = 0; i < D; ++i) {
+    double pz = u[i] + (bias ? bias[i] : 0.0), pr = u[D + i] + (bias ? bias[D + i] : 0.0);
+    double qi = 0.0;
+    for (int j = 0; j < D; ++j) {
+      pz += DW(0, i, j) * h[j];
+      pr += DW(1, i, j) * h[j];
+      qi += DW(2, i, j) * h[j];
+    }
+    z[i] = sigm(pz);
+    r[i] = sigm(pr);
+    q[i] = qi;
+  }
+  for (int i = 0; i < D; ++i) {
+    c[i] = tanh(u[2 * D + i] + (bias ? bias[2 * D + i] : 0.0) + r[i] * q[i]);
+    hn[i] = (1.0 - z[i]) * h[i] + z[i] * c[i];
+  }
+  if (!J) return;
+  for (int i = 0; i < D; ++i) {
+    const double gz = (c[i] - h[i]) * z[i] * (1.0 - z[i]);
+    const double gc = z[i] * (1.0 - c[i] * c[i]);
+    const double gr = q[i] * r[i] * (1.0 - r[i]);
+    for (int j = 0; j < D; ++j)
+      J[(size_t)i * D + j] = (i == j ? 1.0 - z[i] : 0.0) + gz * DW(0, i, j) +
+                             gc * (r[i] * DW(2, i, j) + gr * DW(1, i, j));
+  }
+}
+
+/* Single step over a batch: h [n][D], u [n][3][D] -> hn [n][D], J [n][D][D]
+ * (J may be NULL). */
+void oracle_dense_gru_step(int n, int D, const double* h, const double* u, const double* W,
+                           const double* bias, double* hn, double* J) {
+#pragma omp parallel for schedule(static)
+  for (int b = 0; b < n; ++b) {
+    double* work = (double*)malloc(4 * (size_t)D * sizeof(double));
+    dense_gru_cell(D, W, bias, h + (size_t)b * D, u + (size_t)b * 3 * D, hn + (size_t)b * D,
+                   J ? J + (size_t)b * D * D : NULL, work);
+    free(work);
+  }
+}
+
+/* The sequential recurrence h_t = f(h_{t-1}, u_t) with the general cell. */
+void oracle_dense_gru_seq(const double* u, const double* W, const double* bias,
+                          const double* h0, double* h, int B, int T, int D) {
+#pragma omp parallel for schedule(static)
+  for (int b = 0; b < B; ++b) {
+    double* work = (double*)malloc(5 * (size_t)D * sizeof(double));
+    double* hp = work + 4 * D;
+    for (int d = 0; d < D; ++d) hp[d] = h0 ? h0[(size_t)b * D + d] : 0.0;
+    for (int t = 0; t < T; ++t) {
+      double* ht = h + ((size_t)b * T + t) * D;
+      dense_gru_cell(D, W, bias, hp, u + ((size_t)b * T + t) * 3 * D, ht, NULL, work);
+      memcpy(hp, ht, (size_t)D * sizeof(double));
+    }
+    free(work);
+  }
+}
+
+/* Reference DEER/Newton with dense Jacobian blocks, in the pages' order:
+ * evaluate r_t = h_t - f(h_{t-1}) and J_t = df/dh(h_{t-1}) at the iterate,
+ * record max|r| in trace[k], stop if it is below tol or k == max_iters, else
+ * forward-substitute ds_t = J_t ds_{t-1} - r_t (ds_0 = 0: h0 is given) and
+ * update h += ds.  h (in/out) [B][T][D] holds the initial guess and the final
+ * iterate; iters_out = updates applied; trace has max_iters + 1 entries.  The
+ * whole [B, T, D] system is one Newton system (global stopping). */
+void oracle_dense_gru_newton(const double* u, const double* W, const double* bias,
+                             const double* h0, double* h, int B, int T, int D, double tol,
+                             int max_iters, double* trace, int* iters_out) {
+  const size_t n = (size_t)B * T * D;
+  double* res = (double*)malloc(n * sizeof(double));
+  double* J = (double*)malloc(n * (size_t)D * sizeof(double));
+  int k = 0;
+  for (;; ++k) {
+    double m = 0.0;
+    int nonfinite = 0;
+#pragma omp parallel for schedule(static) reduction(max : m) reduction(| : nonfinite)
+    for (int b = 0; b < B; ++b) {
+      double* work = (double*)malloc(5 * (size_t)D * sizeof(double));
+      double* f = work + 4 * D;
+      for (int t = 0; t < T; ++t) {
+        const double* hp = t > 0 ? h + ((size_t)b * T + t - 1) * D : NULL;
+        double* zero = NULL;
+        if (!hp) { /* the state before step 1 is h0 (zeros when absent) */
+          zero = (double*)calloc((size_t)D, sizeof(double));
+          if (h0) memcpy(zero, h0 + (size_t)b * D, (size_t)D * sizeof(double));
+          hp = zero;
+        }
+        const size_t o = ((size_t)b * T + t) * D;
+        dense_gru_cell(D, W, bias, hp, u + o * 3, f, J + o * D, work);
+        for (int d = 0; d < D; ++d) {
+          const double rt = h[o + d] - f[d];
+          res[o + d] = rt;
+          if (!isfinite(rt)) nonfinite = 1;
+          if (fabs(rt) > m) m = fabs(rt);
+        }
+        free(zero);
+      }
+      free(work);
+    }
+    if (nonfinite) m = INFINITY;
+    if (trace) trace[k] = m;
+    if (m < tol || k >= max_iters) break;
+#pragma omp parallel for schedule(static)
+    for (int b = 0; b < B; ++b) {
+      double* ds = (double*)calloc((size_t)D, sizeof(double));
+      double* nx = (double*)malloc((size_t)D * sizeof(double));
+      for (int t = 0; t < T; ++t) {
+        const size_t o = ((size_t)b * T + t) * D;
+        for (int i = 0; i < D; ++i) {
+          double v = -res[o + i];
+          if (t > 0)
+            for (int j = 0; j < D; ++j) v += J[(o + i) * D + j] * ds[j];
+          nx[i] = v;
+        }
+        for (int i = 0; i < D; ++i) {
+          ds[i] = nx[i];
+          h[o + i] += nx[i];
+        }
+      }
+      free(ds);
+      free(nx);
+    }
+  }
+  if (iters_out) *iters_out = k;
+  free(res);
+  free(J);
+}
+#undef DW

@@ -424,3 +424,100 @@ def test_linrec_equals_closed_form_and_tree_order():
         PA, Pb = nA, nb
         step *= 2
     np.testing.assert_allclose(xs, Pb, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------- general cell (dense Jacobian) --
+def _rand_dense(B, T, D, seed, w_scale=1.0):
+    g = np.random.default_rng(seed)
+    return dict(u=g.standard_normal((B, T, 3, D)),
+                W=g.uniform(-1, 1, (3, D, D)) * w_scale / np.sqrt(D),
+                bias=g.standard_normal((3, D)) * 0.3,
+                h0=g.standard_normal((B, D)) * 0.5)
+
+
+def _torch_dense_gru_cell(W, D):
+    """nn.GRUCell with full recurrent matrices; our z is torch's 1 - z."""
+    cell = torch.nn.GRUCell(3 * D, D, bias=False, dtype=torch.float64)
+    W = torch.as_tensor(W)
+    with torch.no_grad():
+        cell.weight_ih.copy_(torch.eye(3 * D, dtype=torch.float64))     # gate rows r, z, n
+        cell.weight_hh.copy_(torch.cat([W[1], -W[0], W[2]], 0))
+    return cell
+
+
+def test_dense_gru_seq_matches_torch_grucell():
+    x = _rand_dense(2, 23, 7, seed=11)
+    h = oracle.dense_gru_seq(**x)
+    cell = _torch_dense_gru_cell(x["W"], 7)
+    hh = torch.as_tensor(x["h0"]).clone()
+    out = []
+    with torch.no_grad():
+        for t in range(23):
+            hh = cell(_torch_gru_x(x["u"][:, t], x["bias"]), hh)
+            out.append(hh)
+    np.testing.assert_allclose(h, torch.stack(out, 1).numpy(), rtol=0, atol=1e-13)
+
+
+def test_dense_gru_with_diagonal_matrices_is_paragru():
+    x = _rand_gru(3, 40, 6, seed=12)
+    W = np.stack([np.diag(x["a"][g]) for g in range(3)])
+    hd = oracle.dense_gru_seq(x["u"], W, x["bias"], x["h0"])
+    np.testing.assert_allclose(hd, oracle.gru_seq(**x), rtol=0, atol=1e-14)
+    # one step: the dense Jacobian is diagonal with ParaGRU's A on it
+    hp = x["h0"]
+    f, J = oracle.dense_gru_step(hp, x["u"][:, 0], W, x["bias"])
+    for b in range(3):
+        f1, A1, _, _ = oracle.gru_step(hp[b], x["u"][b, 0].T, x["a"].T, x["bias"].T)
+        np.testing.assert_allclose(f[b], f1, rtol=0, atol=1e-14)
+        np.testing.assert_allclose(J[b], np.diag(A1), rtol=0, atol=1e-14)
+
+
+def test_dense_gru_jacobian_vs_torch_autograd():
+    D = 6
+    x = _rand_dense(2, 1, D, seed=13, w_scale=2.0)
+    _, J = oracle.dense_gru_step(x["h0"], x["u"][:, 0], x["W"], x["bias"])
+    cell = _torch_dense_gru_cell(x["W"], D)
+    for b in range(2):
+        xt = _torch_gru_x(x["u"][b:b + 1, 0], x["bias"])
+        Jt = torch.autograd.functional.jacobian(
+            lambda h: cell(xt, h.unsqueeze(0))[0], torch.as_tensor(x["h0"][b]))
+        np.testing.assert_allclose(J[b], Jt.numpy(), rtol=0, atol=1e-12)
+
+
+def test_dense_gru_jacobian_vs_central_differences():
+    D = 5
+    x = _rand_dense(1, 1, D, seed=14, w_scale=2.0)
+    h, u = x["h0"], x["u"][:, 0]
+    _, J = oracle.dense_gru_step(h, u, x["W"], x["bias"])
+    eps = 1e-6
+    for j in range(D):
+        e = np.zeros((1, D))
+        e[0, j] = eps
+        fp, _ = oracle.dense_gru_step(h + e, u, x["W"], x["bias"])
+        fm, _ = oracle.dense_gru_step(h - e, u, x["W"], x["bias"])
+        np.testing.assert_allclose(J[0][:, j], ((fp - fm) / (2 * eps))[0], rtol=0, atol=1e-8)
+
+
+def test_dense_newton_prefix_exactness_and_root():
+    # after k updates the first k states are exact [P4 §1.3: the first block
+    # row of J ds = -r involves ds_1 alone, and so on down the bidiagonal]
+    x = _rand_dense(2, 12, 5, seed=15, w_scale=1.5)
+    ref = oracle.dense_gru_seq(**x)
+    for k in range(1, 6):
+        r = oracle.dense_gru_newton(**x, tol=0.0, max_iters=k)
+        assert r["iters"] == k
+        np.testing.assert_allclose(r["h"][:, :k], ref[:, :k], rtol=0, atol=1e-12)
+        if k <= 2:   # (Newton converges quadratically, so only early on)
+            assert np.abs(r["h"][:, k:] - ref[:, k:]).max() > 1e-6   # not exact further on
+    r = oracle.dense_gru_newton(**x, tol=1e-12, max_iters=40)
+    assert r["trace"][-1] < 1e-12
+    np.testing.assert_allclose(r["h"], ref, rtol=0, atol=1e-12)
+
+
+def test_dense_newton_with_diagonal_matrices_follows_paragru_newton():
+    x = _rand_gru(2, 30, 4, seed=16)
+    W = np.stack([np.diag(x["a"][g]) for g in range(3)])
+    for n in (1, 2, 3):
+        rd = oracle.dense_gru_newton(x["u"], W, x["bias"], x["h0"], tol=0.0, max_iters=n)
+        rg = oracle.gru_newton(**x, tol=0.0, max_iters=n)
+        np.testing.assert_allclose(rd["h"], rg["h"], rtol=0, atol=1e-13)
