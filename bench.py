@@ -121,6 +121,8 @@ def parse():
     ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the unfused-tier and decode-step measurements")
     ap.add_argument("--e2e-steps", type=int, default=3)
     return ap.parse_args()
 
@@ -332,6 +334,67 @@ def time_events(fn, n):
     return e0.elapsed_time(e1) / n  # ms
 
 
+def extra_measurements(w, x, pr, fwd_ms):
+    """Measurements outside the timed step, each guarded so that a failure is
+    reported in the JSON line instead of ending the run:
+      unfused: the same forward solve by the unfused tier (Jacobians and
+        residuals through HBM, a separate scan, the host checking the
+        residual each iteration), against the fused solve's fwd_ms;
+      decode: one decode step for the workload's batch of states, replayed
+        from a captured CUDA graph of 64 steps (kernel time, not the
+        Python call rate), with its algorithmic bytes per step."""
+    lstm = w.cell == "lstm"
+    cell = pr.PARARNN_LSTM if lstm else pr.PARARNN_GRU
+    res = {}
+    try:
+        ws = pr.Workspace("cuda")
+
+        def unfused():
+            return pr.solve_unfused(cell, x["u"], x["a"], x["bias"],
+                                    x["c0"] if lstm else None, x["h0"], workspace=ws)
+        _, _, st = unfused()
+        ms = time_events(unfused, 3)
+        s = pr.read_stats(st)
+        res["unfused"] = {"fwd_ms": round(ms, 4), "fused_fwd_ms": round(fwd_ms, 4),
+                          "unfused_over_fused": round(ms / fwd_ms, 2),
+                          "status": s["status"], "iters": s["iters"]}
+    except Exception as e:  # reported, not fatal
+        res["unfused"] = {"error": str(e)[:300]}
+    try:
+        G = w.G
+        u_t = x["u"][:, 0].contiguous()
+        h = x["h0"].clone()
+        c = x["c0"].clone() if lstm else None
+
+        def step():
+            if lstm:
+                pr.lstm_step(u_t, x["a"], x["bias"], c, h, out=(c, h))
+            else:
+                pr.gru_step(u_t, x["a"], x["bias"], h, out=h)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        n = 64
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(n):
+                step()
+        graph.replay()
+        ms = time_events(graph.replay, 10) / n
+        ue = 2 if w.u_dtype == "bf16" else 4
+        nbytes = w.B * w.D * (G * ue + (16 if lstm else 8))
+        res["decode"] = {"us_per_step": round(ms * 1e3, 3), "B": w.B, "D": w.D,
+                         "bytes_per_step": nbytes,
+                         "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+    except Exception as e:
+        res["decode"] = {"error": str(e)[:300]}
+    return res
+
+
 def cpu_baseline(w, seconds_hint=10.0):
     """The fp64 oracle (sequential recurrence + BPTT) on a bounded sample of
     the workload: all of T, a slice of the channels."""
@@ -460,6 +523,8 @@ def run_ours(args, world, rank):
         "clocks": clk,
         "gpu_launches": path.launches_per_step() * args.steps,
     }
+    if rank == 0 and not args.no_extra:
+        out.update(extra_measurements(w, x, pr, fwd_ms))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w)
     return out
