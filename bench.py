@@ -56,14 +56,15 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
-def fwd_plan(w):
+def fwd_plan(w, sms=None):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
     as the library dispatches it: the row kernels solve a sequence in
     segments of k x 1024 (ParaGRU, two CTAs per SM) or k x 512 steps
     (ParaLSTM, one CTA per SM), k the smallest cluster size below the one
     the whole sequence needs at which its 8-channel tiles fill the SMs, and
     a ParaGRU sequence longer than 4096 steps in 4096-step segments."""
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if sms is None:
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles8 = w.B * ((w.D + 7) // 8)
     if w.cell == "lstm":
         if w.u_dtype == "bf16" and w.T <= 4096:
@@ -94,12 +95,12 @@ def fwd_plan(w):
     return "gru_newton_fused", 5, w.T
 
 
-def fwd_kernel(w):
-    return fwd_plan(w)[:2]
+def fwd_kernel(w, sms=None):
+    return fwd_plan(w, sms)[:2]
 
 
-def fwd_segments(w):
-    seg = fwd_plan(w)[2]
+def fwd_segments(w, sms=None):
+    seg = fwd_plan(w, sms)[2]
     return [(s0, min(seg, w.T - s0)) for s0 in range(0, w.T, seg)]
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
 def fwd_bytes(w):

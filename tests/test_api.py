@@ -161,3 +161,25 @@ def test_unfused_workspace_and_argument_checks():
     assert lib.pararnn_solve_unfused(*a) == -3      # workspace too small
     a = list(base); a[0] = pr.PARARNN_LSTM
     assert lib.pararnn_solve_unfused(*a) == -1      # ParaLSTM without c
+
+
+def test_bench_plan_follows_the_library_dispatch_rules():
+    # bench.py counts launches and cell evaluations per segment from its own
+    # statement of the library's dispatch (csrc/api.cu); on 148 SMs:
+    import bench
+    from nonlinear_rnn_paragru_b200.inputs import WORKLOADS
+    plan = {k: bench.fwd_plan(w, sms=148) for k, w in WORKLOADS.items()}
+    assert plan[1] == ("gru_newton_row", 4, 256)      # 8 tiles: one launch
+    assert plan[2] == ("gru_newton_row", 4, 1024)     # 1024 tiles: 2 CTAs/SM at k = 1
+    assert plan[3] == ("lstm_newton_row", 6.5, 512)   # 1024 tiles: 1 CTA/SM at k = 1
+    assert plan[4] == ("gru_newton_row", 4, 4096)     # T > 4096, 256 tiles >= 148
+    assert plan[5] == ("lstm_newton_row", 6.5, 512)   # 2048 tiles
+    assert len(bench.fwd_segments(WORKLOADS[4], sms=148)) == 16
+    # few tiles keep one launch over the whole sequence
+    assert bench.fwd_plan(WORKLOADS[2].scaled(B=1, D=64), sms=148)[2] == 4096
+    assert bench.fwd_plan(WORKLOADS[3].scaled(B=1, D=64), sms=148)[2] == 4096
+    # fp32 ParaLSTM and long sequences with few tiles take the chunked kernels
+    import dataclasses
+    lstm_f32 = dataclasses.replace(WORKLOADS[3], u_dtype="f32")
+    assert bench.fwd_plan(lstm_f32, sms=148)[0] == "lstm_newton_fused"
+    assert bench.fwd_plan(WORKLOADS[2].scaled(B=1, T=9000, D=64), sms=148)[0] == "gru_newton_fused"
