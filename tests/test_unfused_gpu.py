@@ -52,11 +52,18 @@ def test_capped_iterates_match_oracle_newton(cuda_ok, cell, n):
     assert err < TOL_STATE, err
 
 
+# The stopping test here is global (every element of the problem at once), so
+# it runs at tol = 1e-5, a decade above fp32 rounding of states of magnitude a
+# few units; the update applied after the test leaves the states far inside the
+# 1e-4 bound (Newton converges quadratically).
+TOL_SOLVE = 1e-5
+
+
 @pytest.mark.parametrize("cell", ["gru", "lstm"])
 @pytest.mark.parametrize("f32", [False, True])
 def test_converges_to_the_sequential_recurrence(cuda_ok, cell, f32):
     x = _inputs(cell, 2, 1000, 40, f32=f32)
-    c, h, st = _run(cell, x)
+    c, h, st = _run(cell, x, tol=TOL_SOLVE)
     assert st["status"] == "converged", st
     if cell == "gru":
         err = np.abs(h - oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])).max()
@@ -68,7 +75,7 @@ def test_converges_to_the_sequential_recurrence(cuda_ok, cell, f32):
 
 def test_agrees_with_the_fused_solve(cuda_ok):
     x = _inputs("gru", 4, 2048, 64)
-    _, h_u, st_u = _run("gru", x)
+    _, h_u, st_u = _run("gru", x, tol=TOL_SOLVE)
     d = "cuda"
     h_f, st_f, _ = pr.gru_solve(x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d))
     torch.cuda.synchronize()
