@@ -420,11 +420,23 @@ def cpu_baseline(w, seconds_hint=10.0):
         reps += 1
         if time.perf_counter() - t0 > seconds_hint or reps >= 2000:
             break
-    return {"value": n / t_total, "unit": UNIT, "cores": oracle.get_threads(),
-            "kind": "oracle",
-            "sample": f"B=1, T={w.T}, D={Dk} slice of {w.name}, fp64 sequential "
-                      f"{'recurrence + BPTT' if w.adjoint else 'recurrence'}, "
-                      f"{reps} repetition(s), {t_total:.1f} s"}
+    res = {"value": n / t_total, "unit": UNIT, "cores": oracle.get_threads(),
+           "kind": "oracle",
+           "sample": f"B=1, T={w.T}, D={Dk} slice of {w.name}, fp64 sequential "
+                     f"{'recurrence + BPTT' if w.adjoint else 'recurrence'}, "
+                     f"{reps} repetition(s), {t_total:.1f} s"}
+    # the fp64 reference Newton on the same slice (global stopping at the
+    # same tol): updates it applies before its residual is below tol
+    try:
+        if w.cell == "gru":
+            r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=64)
+        else:
+            r = oracle.lstm_newton(x["u"], x["a"], x["bias"], x["c0"], x["h0"], tol=1e-6,
+                                   max_iters=64)
+        res["oracle_newton_updates"] = int(r["iters"])
+    except Exception as e:  # reported, not fatal
+        res["oracle_newton_updates"] = f"error: {str(e)[:120]}"
+    return res
 
 
 def run_ours(args, world, rank):
