@@ -250,6 +250,28 @@ int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a,
                           pararnn_stats* stats, void* workspace,
                           size_t ws_bytes, pararnn_stream_t stream);
 
+/* Newton solve for a general cell with a dense D x D Jacobian: the GRU with
+ * full recurrent matrices ("Параллельность RNN?", §1.3: the block-bidiagonal
+ * Jacobian with full blocks -df/ds below the identities):
+ *   z = sig(W_z h + u_z + b_z), r = sig(W_r h + u_r + b_r),
+ *   c = tanh(u_c + b_c + r (W_c h)), h' = (1 - z) h + z c.
+ * With diagonal W_g it is the ParaGRU cell.  In: u [B][T][3][D] (dtype
+ * u_dtype), W [3][D][D] row-major (row i of W_g feeds unit i), bias [3][D]
+ * or NULL, h0 [B][D] or NULL.  Out: h [B][T][D], *stats (device).  Each
+ * iteration writes the blocks J_t and -r_t to the workspace, solves
+ * ds_t = J_t ds_{t-1} - r_t by a chunked scan of D x D maps and checks the
+ * residual on the host: stopping is global, as for pararnn_solve_unfused,
+ * and the call synchronises `stream`.  D a multiple of 8, at most 128.
+ * Workspace: pararnn_dense_workspace_size(B, T, D) bytes (4 D^2 + 16 D bytes
+ * per (b, t), and the chunk maps), 256-byte aligned, no initialisation; 0
+ * means the shape is not supported.  Errors as for the other solves. */
+size_t pararnn_dense_workspace_size(int B, int T, int D);
+int pararnn_dense_gru_solve(const void* u, int u_dtype, const float* W,
+                            const float* bias, const float* h0, float* h,
+                            int B, int T, int D, const pararnn_opts* opts,
+                            pararnn_stats* stats, void* workspace,
+                            size_t ws_bytes, pararnn_stream_t stream);
+
 /* One recurrence step, for autoregressive decoding.  Generating a token
  * costs one update of the hidden state whatever the context length
  * ("Apple научила классические RNN масштабироваться...", "Инференс быстрее и

@@ -24,6 +24,7 @@ __all__ = [
     "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_noalloc",
     "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
     "pararnn_unfused_workspace_size", "pararnn_solve_unfused", "solve_unfused",
+    "pararnn_dense_workspace_size", "pararnn_dense_gru_solve", "dense_gru_solve",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
     "gru_step", "lstm_step",
     "Workspace", "read_stats",
@@ -86,6 +87,9 @@ def load_library():
         "pararnn_unfused_workspace_size": (sz, [i, i, i, i]),
         "pararnn_solve_unfused": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i, i,
                                       op, vp, vp, sz, vp]),
+        "pararnn_dense_workspace_size": (sz, [i, i, i]),
+        "pararnn_dense_gru_solve": (i, [vp, i, fp, fp, fp, fp, i, i, i, op, vp, vp,
+                                        sz, vp]),
         "pararnn_gru_step": (i, [vp, i, fp, fp, fp, fp, i, i, vp]),
         "pararnn_lstm_step": (i, [vp, i, fp, fp, fp, fp, fp, fp, i, i, vp]),
         "pararnn_strerror": (ctypes.c_char_p, [i]),
@@ -226,6 +230,18 @@ def pararnn_solve_unfused(cell, u, a, bias, c0, h0, c, h, opts, stats, workspace
         "pararnn_solve_unfused")
 
 
+def pararnn_dense_workspace_size(B, T, D) -> int:
+    return int(load_library().pararnn_dense_workspace_size(B, T, D))
+
+
+def pararnn_dense_gru_solve(u, W, bias, h0, h, opts, stats, workspace, stream=None):
+    _check(load_library().pararnn_dense_gru_solve(
+        _uptr(u), _dtype_code(u), _ptr(W), _ptr(bias), _ptr(h0), _ptr(h), u.shape[0],
+        u.shape[1], u.shape[3], ctypes.byref(opts), _iptr(stats), _wptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "pararnn_dense_gru_solve")
+
+
 def pararnn_gru_step(u_t, a, bias, h_prev, h_next, stream=None):
     _check(load_library().pararnn_gru_step(
         _uptr(u_t), _dtype_code(u_t), _ptr(a), _ptr(bias), _ptr(h_prev),
@@ -338,6 +354,22 @@ def solve_unfused(cell, u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iter
     pararnn_solve_unfused(cell, u, a, bias, c0, h0, c, h, _opts(tol, max_iters), stats,
                           buf, stream)
     return c, h, stats
+
+
+def dense_gru_solve(u, W, bias=None, h0=None, *, tol=1e-6, max_iters=64, workspace=None,
+                    stream=None):
+    """Newton solve of the GRU with full recurrent matrices W [3, D, D]:
+    returns (h, stats).  Synchronises the stream."""
+    B, T, G, D = u.shape
+    h = torch.empty((B, T, D), dtype=torch.float32, device=u.device)
+    stats = _new_stats(u.device)
+    ws = workspace if workspace is not None else Workspace(u.device)
+    nbytes = pararnn_dense_workspace_size(B, T, D)
+    if nbytes == 0:
+        raise PararnnError(-1, "pararnn_dense_workspace_size (unsupported shape)")
+    buf = ws.get(nbytes, stream)
+    pararnn_dense_gru_solve(u, W, bias, h0, h, _opts(tol, max_iters), stats, buf, stream)
+    return h, stats
 
 
 def gru_step(u_t, a, bias=None, h_prev=None, *, out=None, stream=None):

@@ -1,0 +1,379 @@
+// dense.cu -- Newton solve for a general cell whose Jacobian is a full D x D
+// matrix: the GRU with full recurrent matrices W_z, W_r, W_c.
+//
+// The pages derive the Newton step for any Markov cell: the Jacobian of the
+// residual is block-bidiagonal, identities on the diagonal and -df/ds below
+// it, a dense D x D block for a general cell ("Параллельность RNN?", §1.3),
+// and the fully general solver of the pages works with such blocks ("Apple
+// научила классические RNN масштабироваться...", "Три уровня
+// производительности").  Cell (the reset gate on the recurrent term of the
+// candidate):  z = sig(W_z h + u_z + b_z),  r = sig(W_r h + u_r + b_r),
+// c = tanh(u_c + b_c + r (W_c h)),  h' = (1 - z) h + z c,  and
+//   dh'/dh = diag(1 - z) + diag((c - h) z (1 - z)) W_z
+//            + diag(z (1 - c^2)) [diag(r) W_c + diag((W_c h) r (1 - r)) W_r].
+// Each Newton iteration, as in the unfused tier but with matrix blocks:
+//   dn_pre       Q = [W_z; W_r; W_c] h_{t-1} for every (b, t): a tiled fp32
+//                GEMM of the shifted states [B*T, D] by W^T [D, 3D];
+//   dn_assemble  one CTA per (b, t): gates, residual, -r_t and the block
+//                J_t = df/dh (h_{t-1}) [D][D] to HBM, and the residual maximum;
+//   dn_chunk_maps, dn_carry, dn_apply: ds_t = J_t ds_{t-1} - r_t by 16-step
+//                chunks: each chunk's map (P = J_{t1-1} ... J_{t0}, d) from a
+//                zero delta in shared memory (a D x D x D product per step),
+//                the carries chunk by chunk, then every chunk re-run from its
+//                carry, adding ds to the iterate;
+// and the host reads the residual maximum to stop (the first iteration below
+// tol has its update applied; the cap ends with a residual-only evaluation).
+// These are CUDA-core kernels: the products of D x D maps are where tensor
+// cores would apply.  Layouts: u [B][T][3][D], W [3][D][D] row-major (row i
+// of W_g feeds unit i), bias [3][D], h0 [B][D], h [B][T][D].  D <= 128.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace pararnn {
+
+namespace {
+
+constexpr int kDnThreads = 256;
+constexpr int kDnChunk = 16;   // steps per scan chunk
+constexpr int kDnMaxD = 128;   // three (D x (D+1)) fp32 tiles fit in shared memory
+
+template <bool kBF16>
+__device__ __forceinline__ float dn_u(const void* u, size_t i) {
+  if constexpr (kBF16)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(u)[i]);
+  else
+    return reinterpret_cast<const float*>(u)[i];
+}
+
+__device__ __forceinline__ float dn_sig(float x) { return 1.f / (1.f + expf(-x)); }
+
+__device__ __forceinline__ unsigned dn_abs_bits(float v) {
+  return isnan(v) ? 0x7fc00000u : __float_as_uint(fabsf(v));
+}
+
+struct DnParams {
+  const void* u;
+  const float *W, *bias, *h0;
+  float* h;        // the iterate [B][T][D]
+  float* Q;        // recurrent pre-activations [B][T][3][D]
+  float* J;        // Jacobian blocks [B][T][D][D]
+  float* rhs;      // -r [B][T][D]
+  float* P;        // chunk maps [B][nC][D][D]
+  float* d;        // chunk offsets [B][nC][D]
+  float* carry;    // delta entering each chunk [B][nC][D]
+  unsigned* rmax;  // residual maximum (ordered bits)
+  int B, T, D, nC;
+};
+
+// ---------------------------------------------------------- pre-activations --
+// Q[m][n] = sum_k S[m][k] W[n][k], m = b*T + t over the shifted states
+// S[m] = h_{t-1} (h0 at t = 0), n over the 3D rows of W.  64 x 64 tiles, K in
+// steps of 16, each thread a 4 x 4 block of outputs.
+__global__ void __launch_bounds__(kDnThreads) dn_pre(const DnParams p) {
+  __shared__ float As[16][64];
+  __shared__ float Bs[16][64];
+  const int M = p.B * p.T, N = 3 * p.D, K = p.D;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int e = tid + r * kDnThreads;  // 0 .. 1023: 64 rows x 16 columns
+      const int row = e / 16, col = e % 16;
+      const int m = m0 + row, k = k0 + col;
+      float a = 0.f;
+      if (m < M && k < K) {
+        const int b = m / p.T, t = m - b * p.T;
+        a = t > 0 ? p.h[(size_t)(m - 1) * K + k] : (p.h0 ? p.h0[(size_t)b * K + k] : 0.f);
+      }
+      As[col][row] = a;
+      const int n = n0 + row;
+      Bs[col][row] = (n < N && k < K) ? p.W[(size_t)n * K + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[kk][ty * 4 + i];
+        w[i] = Bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], w[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) p.Q[(size_t)m * N + n] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- assemble --
+template <bool kBF16>
+__global__ void __launch_bounds__(kDnThreads) dn_assemble(const DnParams p) {
+  __shared__ float co[4][kDnMaxD];  // per row i: 1 - z, (c - h) z (1 - z), z (1 - c^2) r, z (1 - c^2) q r (1 - r)
+  __shared__ unsigned wmax[kDnThreads / 32];
+  const int D = p.D;
+  const size_t bt = blockIdx.x;  // b * T + t
+  const int b = (int)(bt / p.T), t = (int)(bt - (size_t)b * p.T);
+  unsigned m = 0;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    const float hp = t > 0 ? p.h[(bt - 1) * D + i] : (p.h0 ? p.h0[(size_t)b * D + i] : 0.f);
+    const size_t iu = bt * 3 * D + i;
+    const float* q3 = p.Q + bt * 3 * D;
+    const float z = dn_sig(q3[i] + dn_u<kBF16>(p.u, iu) + (p.bias ? p.bias[i] : 0.f));
+    const float r = dn_sig(q3[D + i] + dn_u<kBF16>(p.u, iu + D) + (p.bias ? p.bias[D + i] : 0.f));
+    const float q = q3[2 * D + i];
+    const float c =
+        tanhf(dn_u<kBF16>(p.u, iu + 2 * (size_t)D) + (p.bias ? p.bias[2 * D + i] : 0.f) + r * q);
+    const float f = fmaf(z, c - hp, hp);
+    const float res = p.h[bt * D + i] - f;
+    p.rhs[bt * D + i] = -res;
+    m = max(m, dn_abs_bits(res));
+    const float gc = z * (1.f - c * c);
+    co[0][i] = 1.f - z;
+    co[1][i] = (c - hp) * z * (1.f - z);
+    co[2][i] = gc * r;
+    co[3][i] = gc * q * r * (1.f - r);
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned mm = 0;
+    for (int w = 0; w < kDnThreads / 32; ++w) mm = max(mm, wmax[w]);
+    atomicMax(p.rmax, mm);
+  }
+  const size_t DD = (size_t)D * D;
+  float* Jt = p.J + bt * DD;
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+    const int i = e / D, j = e - i * D;
+    Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.W[e] + co[2][i] * p.W[2 * DD + e] +
+            co[3][i] * p.W[DD + e];
+  }
+}
+
+// -------------------------------------------------------------------- scan --
+// Shared memory of dn_chunk_maps: three D x (D + 1) tiles (J_t, P, the next
+// P; the padding keeps column walks free of bank conflicts) and two D-vectors.
+size_t dn_maps_smem(int D) { return ((size_t)3 * D * (D + 1) + 2 * (size_t)D) * 4; }
+size_t dn_apply_smem(int D) { return ((size_t)D * (D + 1) + 2 * (size_t)D) * 4; }
+
+// Loads J_t [D][D] into a padded shared tile.
+__device__ __forceinline__ void dn_load_tile(float* dst, const float* src, int D) {
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+    const int i = e / D, j = e - i * D;
+    dst[i * (D + 1) + j] = src[e];
+  }
+}
+
+// One CTA per (b, chunk): the chunk's map x_out = P x_in + d.
+__global__ void __launch_bounds__(kDnThreads) dn_chunk_maps(const DnParams p) {
+  extern __shared__ float sm[];
+  const int D = p.D, ld = D + 1;
+  float* Js = sm;
+  float* Pa = Js + (size_t)D * ld;
+  float* Pb = Pa + (size_t)D * ld;
+  float* xa = Pb + (size_t)D * ld;
+  float* xb = xa + D;
+  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
+  const int t0 = k * kDnChunk, t1 = min(p.T, t0 + kDnChunk);
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+    const int i = e / D, j = e - i * D;
+    Pa[i * ld + j] = (i == j) ? 1.f : 0.f;
+  }
+  for (int i = threadIdx.x; i < D; i += blockDim.x) xa[i] = 0.f;
+  for (int t = t0; t < t1; ++t) {
+    const size_t bt = (size_t)b * p.T + t;
+    dn_load_tile(Js, p.J + bt * D * D, D);
+    __syncthreads();
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+      const int i = e / D, j = e - i * D;
+      float s = 0.f;
+      for (int q = 0; q < D; ++q) s = fmaf(Js[i * ld + q], Pa[q * ld + j], s);
+      Pb[i * ld + j] = s;
+    }
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      float s = p.rhs[bt * D + i];
+      for (int q = 0; q < D; ++q) s = fmaf(Js[i * ld + q], xa[q], s);
+      xb[i] = s;
+    }
+    __syncthreads();
+    float* tp = Pa;
+    Pa = Pb;
+    Pb = tp;
+    float* tx = xa;
+    xa = xb;
+    xb = tx;
+  }
+  const size_t o = (size_t)blockIdx.x * D;  // (b * nC + k) * D
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+    const int i = e / D, j = e - i * D;
+    p.P[o * D + e] = Pa[i * ld + j];
+  }
+  for (int i = threadIdx.x; i < D; i += blockDim.x) p.d[o + i] = xa[i];
+}
+
+// One CTA per b: the delta entering each chunk, chunk by chunk.
+__global__ void __launch_bounds__(kDnThreads) dn_carry(const DnParams p) {
+  __shared__ float x[2][kDnMaxD];
+  const int D = p.D, b = blockIdx.x;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) x[0][i] = 0.f;
+  __syncthreads();
+  int cur = 0;
+  for (int k = 0; k < p.nC; ++k) {
+    const size_t o = ((size_t)b * p.nC + k) * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      p.carry[o + i] = x[cur][i];
+      float s = p.d[o + i];
+      const float* Pi = p.P + (o + i) * D;
+      for (int q = 0; q < D; ++q) s = fmaf(Pi[q], x[cur][q], s);
+      x[cur ^ 1][i] = s;
+    }
+    __syncthreads();
+    cur ^= 1;
+  }
+}
+
+// One CTA per (b, chunk): the chunk re-run from its carry; ds added to h.
+__global__ void __launch_bounds__(kDnThreads) dn_apply(const DnParams p) {
+  extern __shared__ float sm[];
+  const int D = p.D, ld = D + 1;
+  float* Js = sm;
+  float* xa = Js + (size_t)D * ld;
+  float* xb = xa + D;
+  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
+  const int t0 = k * kDnChunk, t1 = min(p.T, t0 + kDnChunk);
+  const size_t o = (size_t)blockIdx.x * D;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) xa[i] = p.carry[o + i];
+  for (int t = t0; t < t1; ++t) {
+    const size_t bt = (size_t)b * p.T + t;
+    dn_load_tile(Js, p.J + bt * D * D, D);
+    __syncthreads();
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      float s = p.rhs[bt * D + i];
+      for (int q = 0; q < D; ++q) s = fmaf(Js[i * ld + q], xa[q], s);
+      xb[i] = s;
+      p.h[bt * D + i] += s;
+    }
+    __syncthreads();
+    float* tx = xa;
+    xa = xb;
+    xb = tx;
+  }
+}
+
+struct DnLayout {
+  size_t rmax, Q, J, rhs, P, d, carry, total;
+};
+
+DnLayout dn_layout(int B, int T, int D) {
+  const size_t BT = (size_t)B * T, nC = (size_t)(T + kDnChunk - 1) / kDnChunk;
+  const size_t BC = (size_t)B * nC;
+  DnLayout L;
+  L.rmax = 0;
+  L.Q = 256;
+  L.J = L.Q + align256(BT * 3 * D * 4);
+  L.rhs = L.J + align256(BT * D * D * 4);
+  L.P = L.rhs + align256(BT * D * 4);
+  L.d = L.P + align256(BC * D * D * 4);
+  L.carry = L.d + align256(BC * D * 4);
+  L.total = L.carry + align256(BC * D * 4);
+  return L;
+}
+
+}  // namespace
+
+int dense_max_d() { return kDnMaxD; }
+size_t dense_ws_bytes(int B, int T, int D) { return dn_layout(B, T, D).total; }
+
+// The host-driven loop; arguments are validated by the caller.  Writes
+// *stats (device) at the end.  Returns 0 or a CUDA error.
+int dense_gru_solve(bool bf16, const void* u, const float* W, const float* bias, const float* h0,
+                    float* h, int B, int T, int D, float tol, int max_iters, pararnn_stats* stats,
+                    void* workspace, cudaStream_t stream) {
+  const DnLayout L = dn_layout(B, T, D);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  DnParams p;
+  p.u = u;
+  p.W = W;
+  p.bias = bias;
+  p.h0 = h0;
+  p.h = h;
+  p.Q = reinterpret_cast<float*>(ws + L.Q);
+  p.J = reinterpret_cast<float*>(ws + L.J);
+  p.rhs = reinterpret_cast<float*>(ws + L.rhs);
+  p.P = reinterpret_cast<float*>(ws + L.P);
+  p.d = reinterpret_cast<float*>(ws + L.d);
+  p.carry = reinterpret_cast<float*>(ws + L.carry);
+  p.rmax = reinterpret_cast<unsigned*>(ws + L.rmax);
+  p.B = B;
+  p.T = T;
+  p.D = D;
+  p.nC = (T + kDnChunk - 1) / kDnChunk;
+  const size_t BT = (size_t)B * T;
+  const unsigned nmaps = (unsigned)((size_t)B * p.nC);
+  const size_t sm_maps = dn_maps_smem(D), sm_apply = dn_apply_smem(D);
+  cudaError_t e = cudaFuncSetAttribute(dn_chunk_maps, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sm_maps);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(dn_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_apply);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h, 0, BT * D * 4, stream);  // initial guess: zero
+  if (e != cudaSuccess) return (int)e;
+  const dim3 pre_grid((unsigned)((3 * D + 63) / 64), (unsigned)((BT + 63) / 64));
+  pararnn_stats st = {0, 0.f, PARARNN_STATUS_CONVERGED, 0};
+  for (int k = 0;; ++k) {
+    e = cudaMemsetAsync(p.rmax, 0, sizeof(unsigned), stream);
+    if (e != cudaSuccess) return (int)e;
+    dn_pre<<<pre_grid, kDnThreads, 0, stream>>>(p);
+    if (bf16)
+      dn_assemble<true><<<(unsigned)BT, kDnThreads, 0, stream>>>(p);
+    else
+      dn_assemble<false><<<(unsigned)BT, kDnThreads, 0, stream>>>(p);
+    unsigned bits = 0;
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(&bits, p.rmax, sizeof(unsigned), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return (int)e;
+    float r;
+    std::memcpy(&r, &bits, sizeof r);  // the ordered bits are the float's own
+    st.evals = k + 1;
+    st.max_residual = r;
+    if (!(r == r) || bits >= 0x7f800000u) {  // NaN or inf
+      st.status = PARARNN_STATUS_NONFINITE;
+      break;
+    }
+    if (k == max_iters) {  // residual-only evaluation at the cap
+      if (!(r < tol)) st.status = PARARNN_STATUS_NOT_CONVERGED;
+      break;
+    }
+    dn_chunk_maps<<<nmaps, kDnThreads, sm_maps, stream>>>(p);
+    dn_carry<<<(unsigned)B, kDnThreads, 0, stream>>>(p);
+    dn_apply<<<nmaps, kDnThreads, sm_apply, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+    st.iters = k + 1;
+    if (r < tol) break;  // the update of the first certified iteration is applied
+  }
+  e = cudaMemcpyAsync(stats, &st, sizeof(st), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // st lives on this stack
+  return (int)e;
+}
+
+}  // namespace pararnn

@@ -183,3 +183,23 @@ def test_bench_plan_follows_the_library_dispatch_rules():
     lstm_f32 = dataclasses.replace(WORKLOADS[3], u_dtype="f32")
     assert bench.fwd_plan(lstm_f32, sms=148)[0] == "lstm_newton_fused"
     assert bench.fwd_plan(WORKLOADS[2].scaled(B=1, T=9000, D=64), sms=148)[0] == "gru_newton_fused"
+
+
+def test_dense_workspace_and_argument_checks():
+    lib = pr.load_library()
+    assert pr.pararnn_dense_workspace_size(2, 300, 64) >= 2 * 300 * 64 * 64 * 4
+    assert pr.pararnn_dense_workspace_size(2, 300, 136) == 0     # D above 128
+    assert pr.pararnn_dense_workspace_size(2, 300, 60) == 0      # D % 8
+    o = pr._opts()
+    base = [0x1000, pr.PARARNN_BF16, 0x2000, None, None, 0x3000, 2, 16, 64,
+            ctypes.byref(o), 0x4000, 0x10000, 1 << 30, None]
+    a = list(base); a[8] = 136
+    assert lib.pararnn_dense_gru_solve(*a) == -1    # D above 128
+    a = list(base); a[2] = None
+    assert lib.pararnn_dense_gru_solve(*a) == -1    # no W
+    a = list(base); a[1] = 9
+    assert lib.pararnn_dense_gru_solve(*a) == -2    # dtype
+    a = list(base); a[2] = 0x2002
+    assert lib.pararnn_dense_gru_solve(*a) == -5    # W alignment
+    a = list(base); a[12] = 1024
+    assert lib.pararnn_dense_gru_solve(*a) == -3    # workspace too small
