@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kDnThreads) dn_pre(const DnParams p) {
   __shared__ float As[16][64];
   __shared__ float Bs[16][64];
   const int M = p.B * p.T, N = 3 * p.D, K = p.D;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int m0 = blockIdx.x * 64, n0 = blockIdx.y * 64;  // rows on x: B*T may be large
   const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
   float acc[4][4] = {};
   for (int k0 = 0; k0 < K; k0 += 16) {
@@ -335,7 +335,7 @@ int dense_gru_solve(bool bf16, const void* u, const float* W, const float* bias,
     e = cudaFuncSetAttribute(dn_apply, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_apply);
   if (e == cudaSuccess) e = cudaMemsetAsync(h, 0, BT * D * 4, stream);  // initial guess: zero
   if (e != cudaSuccess) return (int)e;
-  const dim3 pre_grid((unsigned)((3 * D + 63) / 64), (unsigned)((BT + 63) / 64));
+  const dim3 pre_grid((unsigned)((BT + 63) / 64), (unsigned)((3 * D + 63) / 64));
   pararnn_stats st = {0, 0.f, PARARNN_STATUS_CONVERGED, 0};
   for (int k = 0;; ++k) {
     e = cudaMemsetAsync(p.rmax, 0, sizeof(unsigned), stream);
