@@ -521,3 +521,46 @@ def test_dense_newton_with_diagonal_matrices_follows_paragru_newton():
         rd = oracle.dense_gru_newton(x["u"], W, x["bias"], x["h0"], tol=0.0, max_iters=n)
         rg = oracle.gru_newton(**x, tol=0.0, max_iters=n)
         np.testing.assert_allclose(rd["h"], rg["h"], rtol=0, atol=1e-13)
+
+
+def test_dense_affine_maps_compose_in_any_grouping():
+    # ds_t = J_t ds_{t-1} + b_t with full D x D blocks [P4 §1.3]: forward
+    # substitution, 16-step chunks (chunk maps, carries, re-run) and a
+    # Hillis-Steele tree of (J, b) maps give the same trajectory
+    g = np.random.default_rng(17)
+    T, D = 53, 6
+    J = g.uniform(-1, 1, (T, D, D)) / np.sqrt(D)
+    b = g.standard_normal((T, D))
+    x, fs = np.zeros(D), []
+    for t in range(T):
+        x = J[t] @ x + b[t]
+        fs.append(x)
+    fs = np.array(fs)
+    L = 16
+    chunks = [(J[k:k + L], b[k:k + L]) for k in range(0, T, L)]
+    maps = []
+    for Jc, bc in chunks:
+        P, dv = np.eye(D), np.zeros(D)
+        for Jt, bt in zip(Jc, bc):
+            P, dv = Jt @ P, Jt @ dv + bt
+        maps.append((P, dv))
+    carry, cs = np.zeros(D), []
+    for P, dv in maps:
+        cs.append(carry)
+        carry = P @ carry + dv
+    out = []
+    for (Jc, bc), c0 in zip(chunks, cs):
+        x = c0
+        for Jt, bt in zip(Jc, bc):
+            x = Jt @ x + bt
+            out.append(x)
+    np.testing.assert_allclose(np.array(out), fs, rtol=0, atol=1e-12)
+    A, B_ = J.copy(), b.copy()          # inclusive prefix maps by doubling
+    s = 1
+    while s < T:
+        A2, B2 = A.copy(), B_.copy()
+        for t in range(s, T):
+            A2[t] = A[t] @ A[t - s]
+            B2[t] = A[t] @ B_[t - s] + B_[t]
+        A, B_, s = A2, B2, 2 * s
+    np.testing.assert_allclose(B_, fs, rtol=0, atol=1e-12)   # applied to x_0 = 0
