@@ -12,7 +12,8 @@ Pins of each function (tests/test_oracle.py):
   gru_step / lstm_step     Jacobians and gate derivatives vs central differences
   gru_bptt / lstm_bptt     vs finite differences of L = sum(g * h)
   gru_newton / lstm_newton prefix exactness, affine one/two-step convergence,
-                           convergence to the sequential root
+                           convergence to the sequential root; chan_k equal to
+                           each channel's update count when solved alone
   linrec                   closed form and tree-order scans
   dense_gru_*              the general cell: ParaGRU when W is diagonal, torch's
                            GRU cell and autograd Jacobian, prefix exactness and
