@@ -106,6 +106,14 @@ typedef struct {
   unsigned timeout_us;/* bound on any cross-block wait; 0 -> 2,000,000 */
   int max_cluster;    /* cap on CTAs per thread-block cluster (2..16);
                          0 -> the largest the device can keep resident */
+  int* chan_iters;    /* fused forward solves only: device int [B][D] or NULL.
+                         Receives each (b, d) channel's iteration index, the
+                         input of iter_hist: the number of updates applied
+                         before the first evaluation from which the channel's
+                         own max_t |r_t| stays below tol (max_iters + 1 if it
+                         never got there).  Where the sequence is solved in
+                         segments, the largest index over the segments.
+                         4-byte aligned; the call overwrites every entry. */
 } pararnn_opts;
 
 /* Device-resident solve statistics (written by the solve; zeroed by it at
@@ -197,10 +205,12 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * results as pararnn_adjoint minus the workspace: the scratch is a fixed
  * PARARNN_NOALLOC_SCRATCH_BYTES array inside the library, held in device
  * memory by every GPU that loads the library until the process exits.  The
- * call allocates nothing.  The first call on a device looks the array up and
- * clears it (a synchronous step), so make that first call before any stream
- * capture.  All calls on a device share the array: calls that overlap on the
- * GPU race and must not be made.  Problems that need more scratch than the
+ * call allocates nothing.  The first call on a device looks the array's
+ * address up (cudaGetSymbolAddress) and clears the array with a memset on
+ * `stream`, ordered before that call's kernels; make that first call before
+ * any stream capture.  All calls on a device share the array, which keeps
+ * what the last call left in it (nothing that can mislead the next call):
+ * calls that overlap on the GPU race and must not be made.  Problems that need more scratch than the
  * array holds (pararnn_workspace_size(cell, B, T, D, 0, 1) above the limit:
  * about 13000 ParaGRU chunks of 32 channels x 128 steps, i.e.
  * B*ceil(D/32)*ceil(T/128), or about 6500 ParaLSTM chunks of 32 x 64) return

@@ -50,7 +50,8 @@ class PararnnError(RuntimeError):
 class PararnnOpts(ctypes.Structure):
     _fields_ = [("tol", ctypes.c_float), ("max_iters", ctypes.c_int),
                 ("flags", ctypes.c_uint), ("inject_chunk", ctypes.c_int),
-                ("timeout_us", ctypes.c_uint), ("max_cluster", ctypes.c_int)]
+                ("timeout_us", ctypes.c_uint), ("max_cluster", ctypes.c_int),
+                ("chan_iters", ctypes.c_void_p)]
 
 
 def library_path() -> str:
@@ -150,9 +151,9 @@ def _check(rc, what):
 
 
 def _opts(tol=1e-6, max_iters=0, flags=0, inject_chunk=-1, timeout_us=0,
-          max_cluster=0):
+          max_cluster=0, chan_iters=None):
     return PararnnOpts(float(tol), int(max_iters), int(flags), int(inject_chunk),
-                       int(timeout_us), int(max_cluster))
+                       int(timeout_us), int(max_cluster), _iptr(chan_iters))
 
 
 # ------------------------------------------------------------ C entry points --
@@ -288,7 +289,9 @@ def _new_stats(device):
 
 def gru_solve(u, a, bias=None, h0=None, *, tol=1e-6, max_iters=64, hist=False,
               workspace=None, h=None, stats=None, stream=None, opts=None,
-              max_cluster=0, flags=0):
+              max_cluster=0, flags=0, chan_iters=None):
+    """ParaGRU solve -> (h, stats, iter_hist or None).  `chan_iters`: an
+    int32 [B, D] CUDA tensor that receives each channel's iteration index."""
     B, T, G, D = u.shape
     dev = u.device
     h = torch.empty((B, T, D), dtype=torch.float32, device=dev) if h is None else h
@@ -297,14 +300,17 @@ def gru_solve(u, a, bias=None, h0=None, *, tol=1e-6, max_iters=64, hist=False,
     ws = workspace if workspace is not None else Workspace(dev)
     buf = ws.get(pararnn_workspace_size(PARARNN_GRU, B, T, D, max_iters, 0), stream)
     o = opts if opts is not None else _opts(tol, max_iters, flags=flags,
-                                            max_cluster=max_cluster)
+                                            max_cluster=max_cluster,
+                                            chan_iters=chan_iters)
     pararnn_gru_solve(u, a, bias, h0, h, o, stats, ih, buf, stream)
     return h, stats, ih
 
 
 def lstm_solve(u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
                hist=False, workspace=None, c=None, h=None, stats=None,
-               stream=None, opts=None, max_cluster=0, flags=0):
+               stream=None, opts=None, max_cluster=0, flags=0, chan_iters=None):
+    """ParaLSTM solve -> (c, h, stats, iter_hist or None); `chan_iters` as
+    for gru_solve."""
     B, T, G, D = u.shape
     dev = u.device
     c = torch.empty((B, T, D), dtype=torch.float32, device=dev) if c is None else c
@@ -314,7 +320,8 @@ def lstm_solve(u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
     ws = workspace if workspace is not None else Workspace(dev)
     buf = ws.get(pararnn_workspace_size(PARARNN_LSTM, B, T, D, max_iters, 0), stream)
     o = opts if opts is not None else _opts(tol, max_iters, flags=flags,
-                                            max_cluster=max_cluster)
+                                            max_cluster=max_cluster,
+                                            chan_iters=chan_iters)
     pararnn_lstm_solve(u, a, bias, c0, h0, c, h, o, stats, ih, buf, stream)
     return c, h, stats, ih
 

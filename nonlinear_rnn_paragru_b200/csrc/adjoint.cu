@@ -24,6 +24,8 @@
 // order (reproducible).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "lookback.cuh"
 
@@ -429,12 +431,19 @@ __global__ void adjoint_reduce(const float* __restrict__ part, float* da, float*
   }
 }
 
-__global__ void adjoint_init(WsHeader* hdr, int* status) {
-  unsigned e = (hdr->epoch + 1u) & 0x1fffffffu;
-  if (e == 0u) e = 1u;
-  hdr->epoch = e;
-  hdr->ticket = 0u;
-  *status = 0;
+// New epoch, ticket counter and status; and the look-back flags cleared, so
+// no flag another call left in the workspace can pass for one of this call.
+__global__ void adjoint_init(WsHeader* hdr, int* status, unsigned* flags, size_t nflags) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    unsigned e = (hdr->epoch + 1u) & 0x1fffffffu;
+    if (e == 0u) e = 1u;
+    hdr->epoch = e;
+    hdr->ticket = 0u;
+    *status = 0;
+  }
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nflags;
+       i += (size_t)gridDim.x * blockDim.x)
+    flags[i] = 0u;
 }
 
 // ---------------------------------------------------------------- host --
@@ -450,7 +459,7 @@ static AdjLayout adj_layout(int cell, int B, int T, int D) {
   const int G = cell == PARARNN_GRU ? 3 : 4, RF = cell == PARARNN_GRU ? 4 : 12;
   const size_t nch = (size_t)B * ((D + kChan - 1) / kChan) * ((T + tc - 1) / tc);
   AdjLayout L;
-  L.flags = 256;
+  L.flags = kWsHeaderBytes;
   L.vals = L.flags + align256(nch * 4);
   L.part = L.vals + align256(nch * kChan * RF * 4);
   L.total = L.part + align256(nch * 2 * G * kChan * 4);
@@ -506,7 +515,8 @@ int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, 
   p.status = status;
   const long long nch = (long long)B * p.nDT * p.nC;
   if (nch >= (1LL << 31)) return 1;
-  adjoint_init<<<1, 1, 0, stream>>>(p.hdr, status);
+  adjoint_init<<<(unsigned)std::min<long long>((nch + 255) / 256, 256), 256, 0, stream>>>(
+      p.hdr, status, p.rec_flags, (size_t)nch);
   if (cudaGetLastError() != cudaSuccess) return 1;
   int e;
   if (cell == PARARNN_GRU)

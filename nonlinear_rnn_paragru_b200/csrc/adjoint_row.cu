@@ -875,7 +875,7 @@ int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bia
   p.h0 = h0;
   p.du = du;
   p.dh0 = dh0;
-  p.part = static_cast<float*>(ws);
+  p.part = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
   p.B = B;
   p.T = T;
   p.D = D;
@@ -942,7 +942,7 @@ int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float
   p.du = du;
   p.dc0 = dc0;
   p.dh0 = dh0;
-  p.part = static_cast<float*>(ws);
+  p.part = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
   p.B = B;
   p.T = T;
   p.D = D;

@@ -160,8 +160,11 @@ int max_cluster(int cell, bool bf16) {
   return c;
 }
 
+// New epoch, ticket counter and stats; the per-channel indices and the
+// histogram zeroed; and, for the look-back solve, its record flags cleared so
+// that nothing another call left in the workspace can pass for a record.
 __global__ void fwd_init_kernel(WsHeader* hdr, pararnn_stats* stats, int* chan_k, size_t nch,
-                                int* hist, int nhist) {
+                                int* hist, int nhist, unsigned* flags, size_t nflags) {
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     unsigned e = (hdr->epoch + 1u) & 0x1fffffffu;
     if (e == 0u) e = 1u;
@@ -178,6 +181,7 @@ __global__ void fwd_init_kernel(WsHeader* hdr, pararnn_stats* stats, int* chan_k
     for (size_t i = i0; i < nch; i += stride) chan_k[i] = 0;
   if (hist)
     for (size_t i = i0; i < (size_t)nhist; i += stride) hist[i] = 0;
+  for (size_t i = i0; i < nflags; i += stride) flags[i] = 0u;
 }
 
 __global__ void hist_kernel(const int* __restrict__ chan_k, size_t n, int* hist, int max_iters) {
@@ -213,6 +217,8 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
       (bias && !aligned(bias, 4)) || (h0 && !aligned(h0, 4)) || (c0 && !aligned(c0, 4)) ||
       !aligned(stats, 4) || !aligned(workspace, 256) || (iter_hist && !aligned(iter_hist, 4)))
     return PARARNN_ERR_MISALIGNED;
+  int* const chan_iters = opts ? opts->chan_iters : nullptr;
+  if (chan_iters && !aligned(chan_iters, 4)) return PARARNN_ERR_MISALIGNED;
   const float tol = (opts && opts->tol > 0.f) ? opts->tol : kDefaultTol;
   const int max_iters = resolve_max_iters(opts ? opts->max_iters : 0);
   if (max_iters > kMaxItersLimit) return PARARNN_ERR_INVALID_ARG;
@@ -257,7 +263,8 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.hdr = reinterpret_cast<WsHeader*>(ws);
   p.rec_flags = reinterpret_cast<unsigned*>(ws + L.flags);
   p.rec_vals = reinterpret_cast<float*>(ws + L.vals);
-  p.chan_k = iter_hist ? reinterpret_cast<int*>(ws + L.chan_k) : nullptr;
+  p.chan_k = chan_iters ? chan_iters
+                        : (iter_hist ? reinterpret_cast<int*>(ws + L.chan_k) : nullptr);
   p.stats = stats;
   p.u = u;
   p.t_base = 0;
@@ -265,11 +272,6 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.seg = 0;
   p.ld_h0 = D;
 
-  const size_t nch = (size_t)B * D;
-  const int nhist = max_iters + 2;
-  const unsigned igrid = iter_hist ? (unsigned)std::min<size_t>((nch + 255) / 256, 1024) : 1u;
-  fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist);
-  if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   // Row kernels: a cluster of CTAs per 8-channel tile holds a whole sequence
   // of up to 4096 steps (ParaGRU: bf16 or fp32 u; ParaLSTM: bf16 u).  Where a
   // smaller cluster of k CTAs already fills the SMs with the tiles (ParaGRU:
@@ -287,6 +289,14 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const bool row_gru = cell == PARARNN_GRU && !force &&
                        (gru_row_cluster(T) > 0 || tiles8 >= sm_count());
   const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
+  const size_t nch = (size_t)B * D;
+  const int nhist = max_iters + 2;
+  const size_t nflags = (row_gru || row_lstm) ? 0 : (size_t)ncc * (size_t)(max_iters + 1);
+  const size_t ninit = std::max(p.chan_k ? nch : (size_t)1, nflags);
+  const unsigned igrid = (unsigned)std::min<size_t>((ninit + 255) / 256, 1024);
+  fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist,
+                                             p.rec_flags, nflags);
+  if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   int e = 0;
   if (row_gru) {
     CUtensorMap rmap;
@@ -404,7 +414,7 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
   // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
   // 8-channel tile holds the whole sequence (no look-back)
   if (u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&
-      adjoint_row_part_bytes(G, B, T, D) <= ws_bytes) {
+      kWsHeaderBytes + adjoint_row_part_bytes(G, B, T, D) <= ws_bytes) {
     const int ch = adjoint_row_channels();
     CUtensorMap rmaps[4];
     int e;

@@ -124,7 +124,11 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 //   flags  u32 [nrec]  look-back record flags, nrec = cluster chunks * (max_iters+1)
 //   vals   f32 [nrec][kChan][RW]  record payload (RW floats per channel)
 //   chan_k int [B*D]   per-channel convergence iterate (histogram input)
-// A record flag is (epoch << 3) | (kind << 1) | ok.
+// A record flag is (epoch << 3) | (kind << 1) | ok.  The look-back paths
+// clear their flag slice at the start of every call (the epoch alone cannot
+// tell a stale flag from another path's leftovers in a shared workspace); the
+// paths without look-back keep their scratch after the header.
+constexpr size_t kWsHeaderBytes = 256;
 struct WsHeader {
   unsigned epoch;
   unsigned ticket;
@@ -142,7 +146,7 @@ __host__ __device__ inline FwdWsLayout fwd_ws_layout(size_t nchunks, int max_ite
                                                      size_t BD) {
   FwdWsLayout L;
   size_t nrec = nchunks * (size_t)(max_iters + 1);
-  L.flags = 256;
+  L.flags = kWsHeaderBytes;
   L.vals = L.flags + align256(nrec * 4);
   L.chan_k = L.vals + align256(nrec * kChan * rec_floats * 4);
   L.total = L.chan_k + align256(BD * 4);

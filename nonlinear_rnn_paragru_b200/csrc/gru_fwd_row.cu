@@ -93,6 +93,7 @@ struct RowShared {
   float2 wagg[2][kRowWarps][kRowC];  // per (warp, channel) inclusive map of the warp
   float wlast[2][kRowWarps][kRowC];  // per (warp, channel): last state before the update
   float wmax[2][kRowWarps];
+  float wcm[2][kRowWarps][kRowC];    // per (warp, channel) max|r| (histogram)
   __align__(16) RowMailbox mbox[2];
   // a (3 rows), bias (3 rows), h0 of a tile's channels, by tile parity
   __align__(16) float par[2][7][kRowC];
@@ -454,12 +455,26 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       // residuals are >= 0 (or NaN with the sign cleared): their bit patterns
       // order like unsigned integers, NaN above +inf
       const unsigned wm = __reduce_max_sync(kFull, __float_as_uint(m));
+      // the channel's maximum over the warp's four chunks (lanes c + 8k)
+      unsigned cmu = __float_as_uint(m);
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 8));
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 16));
       if (kk == kRowK - 1) {
         sh.wagg[par][warp][c] = make_float2(IP, Id);
         sh.wlast[par][warp][c] = last_pre;
       }
+      if (kk == 0) sh.wcm[par][warp][c] = __uint_as_float(cmu);
       if (lane == 0) sh.wmax[par][warp] = __uint_as_float(wm);
       __syncthreads();
+      // the histogram input: the channel's own maximum over this CTA's steps
+      // (warp 0, lanes 0..7 track it; the other CTAs of the cluster track
+      // theirs and the per-channel index is the maximum over them)
+      if (q == 0) {
+        float chm = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRowWarps; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
+        if (!(chm < p.tol)) last_bad = k;
+      }
       // maps of the warps before this one: CTA incoming delta -> delta
       // entering this warp; and the CTA's residual maximum
       float cP = 1.f, cd = 0.f;
@@ -509,9 +524,6 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         __syncwarp();
         if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
-      // the histogram input uses the tile's maximum, an upper bound of the
-      // channel's own residual
-      if (!(tmax < p.tol)) last_bad = k;
       final_m = tmax;
       const bool own_ok = tmax < p.tol;
       if (cap) {
@@ -564,7 +576,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       }
     }
     if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
-    if (p.chan_k != nullptr && q == 0 && rank == 0 && dval)
+    if (p.chan_k != nullptr && q == 0 && dval)
       atomicMax(&p.chan_k[(size_t)b * p.D + d], last_bad + 1);
     if (tid == 0) {
       atomicMax(&p.stats->iters, updates);

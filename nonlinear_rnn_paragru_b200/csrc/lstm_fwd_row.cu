@@ -91,6 +91,7 @@ struct LrShared {
   // the update, laid out like a mailbox entry
   float4 wagg[2][kLrWarps][kLrC][2];
   float wmax[2][kLrWarps];
+  float wcm[2][kLrWarps][kLrC];       // per (warp, channel) max|r| (histogram)
   __align__(16) LrMailbox mbox[2];
   // a (4 rows), bias (4 rows), c0, h0 of a tile's channels, by tile parity
   __align__(16) float par[2][10][kLrC];
@@ -406,12 +407,25 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       Aff2 xm = lr_shfl_up(inc, kLrC);
       if (kk == 0) xm = Aff2::id();
       const unsigned wm = __reduce_max_sync(kFull, __float_as_uint(m));
+      // the channel's maximum over the warp's four chunks (lanes c + 8k)
+      unsigned cmu = __float_as_uint(m);
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 8));
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 16));
       if (kk == kLrK - 1) {
         sh.wagg[par][warp][c][0] = make_float4(inc.m00, inc.m01, inc.m10, inc.m11);
         sh.wagg[par][warp][c][1] = make_float4(inc.d0, inc.d1, lastc, lasth);
       }
+      if (kk == 0) sh.wcm[par][warp][c] = __uint_as_float(cmu);
       if (lane == 0) sh.wmax[par][warp] = __uint_as_float(wm);
       __syncthreads();
+      // the histogram input: the channel's own maximum over this CTA's steps
+      // (warp 0, lanes 0..7; every CTA of the cluster records its own)
+      if (q == 0) {
+        float chm = 0.f;
+#pragma unroll
+        for (int w = 0; w < kLrWarps; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
+        if (!(chm < p.tol)) last_bad = kit;
+      }
       // maps of the warps before this one: CTA incoming delta -> delta
       // entering this warp; and the CTA's residual maximum
       Aff2 cw = Aff2::id();
@@ -457,7 +471,6 @@ __global__ void __launch_bounds__(kLrThreads, 1)
         __syncwarp();
         if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
-      if (!(tmax < p.tol)) last_bad = kit;
       final_m = tmax;
       const bool own_ok = tmax < p.tol;
       if (cap) {
@@ -513,7 +526,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       }
     }
     if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
-    if (p.chan_k != nullptr && q == 0 && rank == 0 && dval)
+    if (p.chan_k != nullptr && q == 0 && dval)
       atomicMax(&p.chan_k[(size_t)b * p.D + d], last_bad + 1);
     if (tid == 0) {
       atomicMax(&p.stats->iters, updates);

@@ -11,12 +11,14 @@
 //
 // The array lives in device memory of every GPU that loads the library and
 // stays there until the process exits.  It is shared by all calls on that
-// device and keeps what the last call left in it; the adjoint only needs its
-// header and look-back flags to start in a known state, which the array's
-// zero initialisation plus the per-call epoch bump of the adjoint guarantee
-// (the set-up below clears it once more explicitly).  Calls that overlap on
-// the GPU (different streams, or different host threads, without ordering)
-// race on the array and must not be made.
+// device and keeps what the last call left in it.  Nothing a call leaves
+// behind can mislead the next one: the look-back adjoint clears its flags on
+// the stream at the start of every call, and the whole-sequence adjoint keeps
+// its partial sums after the 256-byte header, which it does not touch.  The
+// first call on a device also clears the whole array, on the caller's stream
+// ahead of that call's kernels.  Calls that overlap on the GPU (different
+// streams, or different host threads, without ordering) race on the array and
+// must not be made.
 #include <mutex>
 
 #include "common.cuh"
@@ -33,9 +35,10 @@ static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_ptr[kMaxDevices] = {};
 
-// Once per device, with that device current: look up the array's address
-// and clear it.  Returns null on failure.
-void* scratch_for_current_device() {
+// Once per device, with that device current: look up the array's address and
+// clear it on `stream` (ordered before the kernels the caller enqueues next on
+// that stream).  Returns null on failure.
+void* scratch_for_current_device(cudaStream_t stream) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
@@ -45,7 +48,7 @@ void* scratch_for_current_device() {
       cudaGetLastError();
       return nullptr;
     }
-    if (cudaMemset(p, 0, kScratchBytes) != cudaSuccess) {
+    if (cudaMemsetAsync(p, 0, kScratchBytes, stream) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
@@ -62,10 +65,12 @@ extern "C" int pararnn_adjoint_noalloc(int cell, const void* u, int u_dtype, con
                                        float* du, float* da, float* dbias, float* dc0,
                                        float* dh0, int B, int T, int D, int* status,
                                        pararnn_stream_t stream) {
-  // sizes beyond the built-in scratch are refused before anything else runs
+  // an invalid cell or size (no workspace size) and sizes beyond the built-in
+  // scratch are refused before anything else runs
   const size_t need = pararnn_workspace_size(cell, B, T, D, 0, 1);
+  if (need == 0) return PARARNN_ERR_INVALID_ARG;
   if (need > kScratchBytes) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
-  void* ws = scratch_for_current_device();
+  void* ws = scratch_for_current_device((cudaStream_t)stream);
   if (ws == nullptr) return PARARNN_ERR_CUDA;
   return pararnn_adjoint(cell, u, u_dtype, a, bias, c0, h0, c, h, dLdh, du, da, dbias, dc0, dh0,
                          B, T, D, status, ws, kScratchBytes, stream);

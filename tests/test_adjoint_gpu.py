@@ -178,3 +178,18 @@ def test_adjoint_clusters_with_many_tiles(cuda_ok, cell):
     else:
         c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
         _check_lstm(x, c, h)
+
+
+@pytest.mark.parametrize("cell,wl", [(pr.PARARNN_GRU, 2), (pr.PARARNN_GRU, 4),
+                                     (pr.PARARNN_LSTM, 5)])
+def test_nan_input_reports_nonfinite(cuda_ok, cell, wl):
+    # bf16 u: the whole-sequence adjoint; fp32 u (workload 4): the look-back one
+    x = make_inputs(WORKLOADS[wl].scaled(B=1, T=600, D=32), with_grad=True)
+    if cell == pr.PARARNN_GRU:
+        h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+        c = None
+    else:
+        c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    x["u"][0, 200, 0, 3] = float("nan")
+    g = _gpu_adjoint(cell, x, h, c)
+    assert int(g["status"][0]) == 2          # PARARNN_STATUS_NONFINITE

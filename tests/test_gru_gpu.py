@@ -232,3 +232,54 @@ def test_short_segments_match_oracle(cuda_ok, B, T, D, wl):
         assert err < TOL_STATE, (flags, err, st)
         assert st["status"] == "converged", (flags, st)
         assert hist.sum() == B * D
+
+
+@pytest.mark.parametrize("B,T,D,wl,flags", [
+    (1, 2048, 64, 2, 0),                          # clusters of 2 over the whole sequence
+    (2, 4000, 32, 4, 0),                          # fp32 u, clusters of 4
+    (3, 900, 40, 2, 0),                           # one CTA per tile
+    (1, 2048, 64, 2, pr.PARARNN_FLAG_FORCE_CHUNKED)])
+def test_channel_iteration_index_matches_oracle(cuda_ok, B, T, D, wl, flags):
+    # Per (b, d) channel: the updates applied before the first evaluation from
+    # which the channel's own max_t |r_t| stays below tol.  Channels are
+    # independent, so this is the oracle's per-channel chan_k of the joint
+    # Newton solve, within one for fp32 against fp64 near the threshold.  The
+    # sequences here are solved in one launch (no segments).
+    x = make_inputs(WORKLOADS[wl].scaled(B=B, T=T, D=D))
+    ci = torch.full((B, D), -5, dtype=torch.int32, device="cuda")
+    h, st, hist = _solve(x, hist=True, chan_iters=ci, flags=flags)
+    k_gpu = ci.cpu().numpy()
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=64)
+    diff = np.abs(k_gpu - r["chan_k"])
+    assert diff.max() <= 1, (diff.max(), np.argwhere(diff > 1)[:5])
+    assert (diff == 0).mean() > 0.9
+    assert len(np.unique(r["chan_k"])) >= 2        # the index varies by channel
+    np.testing.assert_array_equal(hist, np.bincount(k_gpu.ravel(), minlength=66))
+    assert k_gpu.max() + 1 <= st["evals"]
+
+
+def test_config4_full_size_with_histogram(cuda_ok):
+    # B=1, T=65536, D=2048, fp32 u: 4096-step segments, each from the state the
+    # one before converged to; states against the fp64 sequential recurrence
+    w = WORKLOADS[4]
+    x = make_inputs(w)
+    ci = torch.empty((w.B, w.D), dtype=torch.int32, device="cuda")
+    h, st, hist = _solve(x, hist=True, chan_iters=ci)
+    err = np.abs(h - _ref(x)).max()
+    assert err < TOL_STATE, (err, st)
+    assert st["status"] == "converged" and st["max_residual"] < 1e-6
+    assert hist.sum() == w.D and hist[-1] == 0
+    np.testing.assert_array_equal(hist, np.bincount(ci.cpu().numpy().ravel(), minlength=66))
+
+
+@pytest.mark.parametrize("flags", [0, pr.PARARNN_FLAG_FORCE_CHUNKED])
+def test_nan_input_reports_nonfinite(cuda_ok, flags):
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=1500, D=32))
+    x["u"][0, 700, 1, 5] = float("nan")
+    _, st, _ = _solve(x, flags=flags, max_iters=8)
+    assert st["status"] == "nonfinite", st
+    # the context stays usable
+    y = make_inputs(WORKLOADS[2].scaled(B=1, T=1500, D=32))
+    h, st2, _ = _solve(y, flags=flags)
+    assert st2["status"] == "converged"
+    assert np.abs(h - _ref(y)).max() < TOL_STATE

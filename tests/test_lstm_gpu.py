@@ -141,3 +141,59 @@ def test_segmented_long_sequence_matches_oracle(cuda_ok, B, T, D):
         assert err < TOL_STATE, (flags, err, st)
         assert st["status"] == "converged", (flags, st)
         assert hist.sum() == B * D
+
+
+@pytest.mark.parametrize("B,T,D,flags", [
+    (1, 1500, 64, 0),                            # clusters of 4 over the whole sequence
+    (2, 400, 48, 0),                             # one CTA per tile
+    (1, 1500, 64, pr.PARARNN_FLAG_FORCE_CHUNKED)])
+def test_channel_iteration_index_matches_oracle(cuda_ok, B, T, D, flags):
+    # the per-channel index against the oracle's chan_k (within one; see the
+    # ParaGRU test), for sequences solved in one launch
+    x = make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D))
+    ci = torch.full((B, D), -5, dtype=torch.int32, device="cuda")
+    c, h, st, hist = _solve(x, hist=True, chan_iters=ci, flags=flags)
+    k_gpu = ci.cpu().numpy()
+    r = oracle.lstm_newton(x["u"], x["a"], x["bias"], x["c0"], x["h0"], tol=1e-6,
+                           max_iters=64)
+    diff = np.abs(k_gpu - r["chan_k"])
+    assert diff.max() <= 1, (diff.max(), np.argwhere(diff > 1)[:5])
+    assert (diff == 0).mean() > 0.9
+    np.testing.assert_array_equal(hist, np.bincount(k_gpu.ravel(), minlength=66))
+
+
+def test_config5_full_size(cuda_ok):
+    # B=4, T=2048, D=4096, u ~ N(0, 4/sqrt(D)): 512-step segments on all SMs
+    st, hist = _check(make_inputs(WORKLOADS[5]), hist=True)
+    assert hist.sum() == 4 * 4096 and hist[-1] == 0
+    assert st["max_residual"] < 1e-6
+
+
+def test_config5_fwd_then_adjoint_end_to_end(cuda_ok):
+    # the GPU trajectory feeds the GPU adjoint; compared with BPTT on the exact
+    # sequential trajectory (per-tensor relative error 1e-3)
+    w = WORKLOADS[5]
+    x = make_inputs(w)
+    d = "cuda"
+    xd = {k: v.to(d) for k, v in x.items()}
+    c, h, st, _ = pr.lstm_solve(xd["u"], xd["a"], xd["bias"], xd["c0"], xd["h0"])
+    g = pr.adjoint(pr.PARARNN_LSTM, xd["u"], xd["a"], xd["bias"], xd["h0"], h, xd["dLdh"],
+                   c0=xd["c0"], c=c)
+    torch.cuda.synchronize()
+    assert pr.read_stats(st)["status"] == "converged"
+    assert int(g["status"][0]) == 0
+    rc, rh = _ref(x)
+    ref = oracle.lstm_bptt(x["u"], x["a"], x["bias"], x["c0"], x["h0"], rc, rh, x["dLdh"])
+    for k in ("du", "da", "dbias", "dh0", "dc0"):
+        gk = g[k].cpu().numpy()
+        rel = float(np.abs(gk - ref[k]).max() / max(np.abs(ref[k]).max(), 1e-30))
+        assert rel <= 1e-3, (k, rel)
+
+
+@pytest.mark.parametrize("flags", [0, pr.PARARNN_FLAG_FORCE_CHUNKED])
+def test_nan_input_reports_nonfinite(cuda_ok, flags):
+    x = make_inputs(WORKLOADS[3].scaled(B=1, T=900, D=32))
+    x["u"][0, 300, 2, 9] = float("nan")
+    _, _, st, _ = _solve(x, flags=flags, max_iters=8)
+    assert st["status"] == "nonfinite", st
+    _check(make_inputs(WORKLOADS[3].scaled(B=1, T=900, D=32)), flags=flags)
