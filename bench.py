@@ -46,6 +46,9 @@ NCU_TRAFFIC_BYTES = {
 }
 # The forward kernel a workload runs and its special-function (MUFU)
 # operations per element and cell evaluation, as the kernel issues them:
+#   gru_newton_queue (ParaGRU with bf16 u and at least one 8-channel tile per
+#     resident CTA, four CTAs per SM: every 512-step segment of every tile in
+#     one launch): the cell pass of gru_newton_row, 3 ex2 + 1 rcp;
 #   gru_newton_row (ParaGRU with T <= 4096, or longer with at least one
 #     8-channel tile per SM, then in 4096-step segments): 3 ex2 + 1 rcp (one
 #     reciprocal serves the four sigmoids of a step pair, one the pair's two
@@ -56,16 +59,24 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
+QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue (128 registers, 53 KB smem)
+
+
 def fwd_plan(w, sms=None):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
-    as the library dispatches it: the row kernels solve a sequence in
-    segments of k x 1024 (ParaGRU, two CTAs per SM) or k x 512 steps
-    (ParaLSTM, one CTA per SM), k the smallest cluster size below the one
-    the whole sequence needs at which its 8-channel tiles fill the SMs, and
-    a ParaGRU sequence longer than 4096 steps in 4096-step segments."""
+    as the library dispatches it: the segment-queue kernel solves every
+    512-step segment of a ParaGRU problem with bf16 u and at least one
+    8-channel tile per resident CTA in one launch; otherwise the row kernels
+    solve a sequence in segments of k x 1024 (ParaGRU, two CTAs per SM) or
+    k x 512 steps (ParaLSTM, one CTA per SM), one launch each, k the smallest
+    cluster size below the one the whole sequence needs at which its
+    8-channel tiles fill the SMs, and a ParaGRU sequence longer than 4096
+    steps in 4096-step segments."""
     if sms is None:
         sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles8 = w.B * ((w.D + 7) // 8)
+    if w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms:
+        return "gru_newton_queue", 4, 512
     if w.cell == "lstm":
         if w.u_dtype == "bf16" and w.T <= 4096:
             cls, seg = 1, w.T
@@ -102,6 +113,11 @@ def fwd_kernel(w, sms=None):
 def fwd_segments(w, sms=None):
     seg = fwd_plan(w, sms)[2]
     return [(s0, min(seg, w.T - s0)) for s0 in range(0, w.T, seg)]
+
+
+def fwd_launches(w, sms=None):
+    """Launches of the forward kernel per solve."""
+    return 1 if fwd_plan(w, sms)[0] == "gru_newton_queue" else len(fwd_segments(w, sms))
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
 def fwd_bytes(w):
     ue = 2 if w.u_dtype == "bf16" else 4
@@ -264,8 +280,7 @@ class Path:
             self.abuf = self.wsa.get(pr.pararnn_workspace_size(cell, B, T, D, 0, 1))
 
     def launches_per_step(self):
-        nseg = len(fwd_segments(self.w))
-        n = 1 + nseg + (1 if self.hist is not None else 0)  # init, solves, [hist]
+        n = 1 + fwd_launches(self.w) + (1 if self.hist is not None else 0)  # init, solves, [hist]
         return n + (3 if self.w.adjoint else 0)            # init, adjoint, reduce
 
     def forward(self, x=None):
@@ -283,10 +298,10 @@ class Path:
 
         Every tile stops on its own, so this is counted from the per-channel
         convergence histogram: a channel whose tile first passed the test at
-        iteration k was evaluated k + 1 times.  Exact for the row kernels (a
-        tile is a whole sequence or segment): a sequence the library solves
-        segment by segment is solved here one segment per call, each from the
-        state the one before ended in, which is the arithmetic the segmented
+        iteration k was evaluated k + 1 times.  Exact for the row and queue
+        kernels (a tile is a whole sequence or segment): a sequence the library
+        solves segment by segment is solved here one segment per call, each from
+        the state the one before ended in, which is the arithmetic the segmented
         solve does.  For the chunked kernels a channel reports its slowest
         chunk, so this is an upper bound there.  Untimed.
         """
@@ -473,8 +488,8 @@ def run_ours(args, world, rank):
                 "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
                 "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
                 "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
-                "ops_per_launch": elem_evals * mufu_per_eval / len(fwd_segments(w)),
-                "launches_per_solve": len(fwd_segments(w)),
+                "ops_per_launch": elem_evals * mufu_per_eval / fwd_launches(w),
+                "launches_per_solve": fwd_launches(w),
                 "mean_evals": round(elem_evals / w.tokch, 3)}
     hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
            "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,

@@ -96,6 +96,11 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            8-channel tile per SM, ParaLSTM with
                                            bf16 u and T <= 4096 (segmented as
                                            the solves' comments say) */
+#define PARARNN_FLAG_FORCE_ROW 4u       /* ParaGRU with bf16 u: launch the
+                                           row kernel segment by segment
+                                           instead of the one-launch
+                                           segment-queue solve (kept for
+                                           comparison) */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
@@ -281,6 +286,65 @@ int pararnn_dense_gru_solve(const void* u, int u_dtype, const float* W,
                             int B, int T, int D, const pararnn_opts* opts,
                             pararnn_stats* stats, void* workspace,
                             size_t ws_bytes, pararnn_stream_t stream);
+
+/* Sequence sharding: the time axis split over processes (GPUs).  Shard r of
+ * W holds steps [T_r, T_{r+1}) of every (b, d) channel: its slice of u
+ * ([B][Ts][G][D], Ts = T_{r+1} - T_r) and of the iterate.  The page's linear
+ * system of a Newton iteration ("Параллельность RNN?", §1.3) couples a shard
+ * to the shards before it only through the delta entering its first step,
+ * and the scan's operator is associative ("Уровень 2"), so long sequences
+ * can be cut into chunks solved apart and joined ("ParaRNN：解锁非线性RNN并行
+ * 训练的革命性框架", on long sequences).  One Newton iteration of the
+ * sharded solve is
+ *   1. pararnn_shard_eval on every shard: residual and Jacobians at the
+ *      iterate, the shard's system solved from a zero incoming delta, its map
+ *      ds_out = P ds_in + d and its last state(s) before the update, max|r|;
+ *   2. an exchange of every shard's map, last states and max|r| (all-gather
+ *      and all-reduce over the processes: NCCL between GPUs);
+ *   3. pararnn_shard_combine on every shard: the delta entering it (the maps
+ *      of the shards before it, composed in order) and its new initial state
+ *      for the next iteration (the previous shard's last state plus that
+ *      delta; shard 0 keeps the true initial state);
+ *   4. pararnn_shard_apply: the local solution plus P_t ds_in added to the
+ *      iterate.
+ * These are the Newton iterates of the whole sequence (with the stopping
+ * rule of pararnn_solve_unfused applied to the global max|r|), so the result
+ * does not depend on how T is split.  The loop and the exchange run on the
+ * host (nonlinear_rnn_paragru_b200.shard).  cell PARARNN_GRU or PARARNN_LSTM;
+ * for ParaGRU the c arguments are NULL.
+ *
+ * Workspace: pararnn_shard_workspace_size(cell, B, Ts, D) bytes, 256-byte
+ * aligned, no initialisation; it carries the Jacobians and chunk maps from
+ * pararnn_shard_eval to pararnn_shard_apply of the same iteration. */
+size_t pararnn_shard_workspace_size(int cell, int B, int Ts, int D);
+/* In:  u, a, bias as for the solves (u a shard's slice); c_bound, h_bound
+ *      [B][D] the states before the shard's first step (NULL = zeros); c, h
+ *      [B][Ts][D] the shard's iterate (not changed).
+ * Out: agg [NA][B][D] the shard's map, NA = 2 (ParaGRU: P, d) or 6
+ *      (ParaLSTM: P00, P01, P10, P11, d0, d1 for the state order c, h);
+ *      last [S][B][D] the iterate's last state(s), S = 1 (h) or 2 (c, h);
+ *      *rmax (device float) max|r| over the shard (NaN if any is NaN).
+ * Alignment 4 bytes (u: 2 for bf16), workspace 256. */
+int pararnn_shard_eval(int cell, const void* u, int u_dtype, const float* a,
+                       const float* bias, const float* c_bound,
+                       const float* h_bound, const float* c, const float* h,
+                       int B, int Ts, int D, float* agg, float* last,
+                       float* rmax, void* workspace, size_t ws_bytes,
+                       pararnn_stream_t stream);
+/* In:  aggs [W][NA][B][D] and lasts [W][S][B][D], every shard's agg and last
+ *      in shard order; r this shard's index.
+ * Out: din [S][B][D] the delta entering shard r; for r > 0, bound [S][B][D]
+ *      its initial state for the next iteration (bound may be NULL for r = 0,
+ *      whose initial state is the true one). */
+int pararnn_shard_combine(int cell, const float* aggs, const float* lasts,
+                          int W, int r, int B, int D, float* din, float* bound,
+                          pararnn_stream_t stream);
+/* Adds the Newton update to the shard's iterate c, h [B][Ts][D] (c NULL for
+ * ParaGRU), given din from pararnn_shard_combine and the workspace of this
+ * iteration's pararnn_shard_eval. */
+int pararnn_shard_apply(int cell, const float* din, float* c, float* h, int B,
+                        int Ts, int D, void* workspace, size_t ws_bytes,
+                        pararnn_stream_t stream);
 
 /* One recurrence step, for autoregressive decoding.  Generating a token
  * costs one update of the hidden state whatever the context length

@@ -25,6 +25,8 @@ __all__ = [
     "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
     "pararnn_unfused_workspace_size", "pararnn_solve_unfused", "solve_unfused",
     "pararnn_dense_workspace_size", "pararnn_dense_gru_solve", "dense_gru_solve",
+    "pararnn_shard_workspace_size", "pararnn_shard_eval", "pararnn_shard_combine",
+    "pararnn_shard_apply",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
     "gru_step", "lstm_step",
     "Workspace", "read_stats",
@@ -91,6 +93,11 @@ def load_library():
         "pararnn_dense_workspace_size": (sz, [i, i, i]),
         "pararnn_dense_gru_solve": (i, [vp, i, fp, fp, fp, fp, i, i, i, op, vp, vp,
                                         sz, vp]),
+        "pararnn_shard_workspace_size": (sz, [i, i, i, i]),
+        "pararnn_shard_eval": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i, i, fp, fp, fp,
+                                   vp, sz, vp]),
+        "pararnn_shard_combine": (i, [i, fp, fp, i, i, i, i, fp, fp, vp]),
+        "pararnn_shard_apply": (i, [i, fp, fp, fp, i, i, i, vp, sz, vp]),
         "pararnn_gru_step": (i, [vp, i, fp, fp, fp, fp, i, i, vp]),
         "pararnn_lstm_step": (i, [vp, i, fp, fp, fp, fp, fp, fp, i, i, vp]),
         "pararnn_strerror": (ctypes.c_char_p, [i]),
@@ -241,6 +248,33 @@ def pararnn_dense_gru_solve(u, W, bias, h0, h, opts, stats, workspace, stream=No
         u.shape[1], u.shape[3], ctypes.byref(opts), _iptr(stats), _wptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)),
         "pararnn_dense_gru_solve")
+
+
+def pararnn_shard_workspace_size(cell, B, Ts, D) -> int:
+    return int(load_library().pararnn_shard_workspace_size(cell, B, Ts, D))
+
+
+def pararnn_shard_eval(cell, u, a, bias, c_bound, h_bound, c, h, agg, last, rmax, workspace,
+                       stream=None):
+    _check(load_library().pararnn_shard_eval(
+        cell, _uptr(u), _dtype_code(u), _ptr(a), _ptr(bias), _ptr(c_bound), _ptr(h_bound),
+        _ptr(c), _ptr(h), u.shape[0], u.shape[1], u.shape[3], _ptr(agg), _ptr(last),
+        _ptr(rmax), _wptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)), "pararnn_shard_eval")
+
+
+def pararnn_shard_combine(cell, aggs, lasts, r, din, bound, stream=None):
+    W, _, B, D = aggs.shape
+    _check(load_library().pararnn_shard_combine(
+        cell, _ptr(aggs), _ptr(lasts), W, r, B, D, _ptr(din), _ptr(bound), _stream(stream)),
+        "pararnn_shard_combine")
+
+
+def pararnn_shard_apply(cell, din, c, h, workspace, stream=None):
+    B, Ts, D = h.shape
+    _check(load_library().pararnn_shard_apply(
+        cell, _ptr(din), _ptr(c), _ptr(h), B, Ts, D, _wptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)), "pararnn_shard_apply")
 
 
 def pararnn_gru_step(u_t, a, bias, h_prev, h_next, stream=None):

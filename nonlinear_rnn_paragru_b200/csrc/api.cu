@@ -19,6 +19,9 @@ int gru_row_channels();
 int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStream_t stream);
 int gru_row_max_steps();
 int gru_row_cta_steps();
+int gru_queue_resident();
+int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+                     unsigned* seg_done, cudaStream_t stream);
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
 int lstm_chunk_steps();
@@ -49,6 +52,14 @@ int unfused_solve(int cell, bool bf16, const void* u, const float* a, const floa
                   const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
                   float tol, int max_iters, pararnn_stats* stats, void* workspace,
                   cudaStream_t stream);
+int shard_eval(int cell, bool bf16, const void* u, const float* a, const float* bias,
+               const float* c_bound, const float* h_bound, const float* c, const float* h, int B,
+               int Ts, int D, float* agg, float* last, float* rmax, void* workspace,
+               cudaStream_t stream);
+int shard_combine(int cell, const float* aggs, const float* lasts, int r, int B, int D,
+                  float* din, float* bound, cudaStream_t stream);
+int shard_apply(int cell, const float* din, float* c, float* h, int B, int Ts, int D,
+                void* workspace, cudaStream_t stream);
 int launch_decode_step(int cell, bool bf16, const void* u, const float* a, const float* bias,
                        const float* c_prev, const float* h_prev, float* c_next, float* h_next,
                        int B, int D, cudaStream_t stream);
@@ -163,6 +174,8 @@ int max_cluster(int cell, bool bf16) {
 // New epoch, ticket counter and stats; the per-channel indices and the
 // histogram zeroed; and, for the look-back solve, its record flags cleared so
 // that nothing another call left in the workspace can pass for a record.
+// (`flags` is the segment-queue solve's per-tile segment counts when that
+// solve runs.)
 __global__ void fwd_init_kernel(WsHeader* hdr, pararnn_stats* stats, int* chan_k, size_t nch,
                                 int* hist, int nhist, unsigned* flags, size_t nflags) {
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -289,16 +302,27 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const bool row_gru = cell == PARARNN_GRU && !force &&
                        (gru_row_cluster(T) > 0 || tiles8 >= sm_count());
   const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
+  // ParaGRU with bf16 u and at least one 8-channel tile per resident CTA of
+  // the segment-queue solve: all segments of all tiles in one launch
+  const bool queue_gru = row_gru && bf16 && !(opts && (opts->flags & PARARNN_FLAG_FORCE_ROW)) &&
+                         tiles8 >= (long long)std::max(1, gru_queue_resident());
   const size_t nch = (size_t)B * D;
   const int nhist = max_iters + 2;
-  const size_t nflags = (row_gru || row_lstm) ? 0 : (size_t)ncc * (size_t)(max_iters + 1);
+  unsigned* const seg_done = reinterpret_cast<unsigned*>(ws + L.seg);
+  const size_t nflags = queue_gru ? (size_t)tiles8
+                                  : ((row_gru || row_lstm) ? 0 : (size_t)ncc * (size_t)(max_iters + 1));
   const size_t ninit = std::max(p.chan_k ? nch : (size_t)1, nflags);
   const unsigned igrid = (unsigned)std::min<size_t>((ninit + 255) / 256, 1024);
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist,
-                                             p.rec_flags, nflags);
+                                             queue_gru ? seg_done : p.rec_flags, nflags);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   int e = 0;
-  if (row_gru) {
+  if (queue_gru) {
+    CUtensorMap rmap;
+    rc = make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels());
+    if (rc) return rc;
+    e = launch_gru_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
+  } else if (row_gru) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());
     if (rc) return rc;
@@ -460,6 +484,60 @@ int pararnn_seq_baseline(int cell, const void* u, int u_dtype, const float* a, c
   if (cell == PARARNN_GRU && (c || c0)) return PARARNN_ERR_INVALID_ARG;
   const int e = launch_seq_baseline(cell, u_dtype == PARARNN_BF16, u, a, bias, c0, h0, c, h, B, T,
                                     D, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+size_t pararnn_shard_workspace_size(int cell, int B, int Ts, int D) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return 0;
+  if (check_sizes(B, Ts, D)) return 0;
+  return unfused_ws_bytes(cell, B, Ts, D);
+}
+
+int pararnn_shard_eval(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+                       const float* c_bound, const float* h_bound, const float* c,
+                       const float* h, int B, int Ts, int D, float* agg, float* last,
+                       float* rmax, void* workspace, size_t ws_bytes, pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Ts, D);
+  if (rc) return rc;
+  if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
+  const bool lstm = cell == PARARNN_LSTM;
+  if (!u || !a || !h || !agg || !last || !rmax || !workspace || (lstm && !c))
+    return PARARNN_ERR_INVALID_ARG;
+  if (!lstm && (c || c_bound)) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(u, u_dtype == PARARNN_BF16 ? 2 : 4) || !aligned(a, 4) ||
+      (bias && !aligned(bias, 4)) || (c_bound && !aligned(c_bound, 4)) ||
+      (h_bound && !aligned(h_bound, 4)) || (c && !aligned(c, 4)) || !aligned(h, 4) ||
+      !aligned(agg, 4) || !aligned(last, 4) || !aligned(rmax, 4) || !aligned(workspace, 256))
+    return PARARNN_ERR_MISALIGNED;
+  if (ws_bytes < unfused_ws_bytes(cell, B, Ts, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
+  const int e = shard_eval(cell, u_dtype == PARARNN_BF16, u, a, bias, c_bound, h_bound, c, h, B,
+                           Ts, D, agg, last, rmax, workspace, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+int pararnn_shard_combine(int cell, const float* aggs, const float* lasts, int W, int r, int B,
+                          int D, float* din, float* bound, pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  if (W < 1 || r < 0 || r >= W || B < 1 || D < 1) return PARARNN_ERR_INVALID_ARG;
+  if (!aggs || !lasts || !din || (r > 0 && !bound)) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(aggs, 4) || !aligned(lasts, 4) || !aligned(din, 4) || (bound && !aligned(bound, 4)))
+    return PARARNN_ERR_MISALIGNED;
+  const int e = shard_combine(cell, aggs, lasts, r, B, D, din, bound, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
+int pararnn_shard_apply(int cell, const float* din, float* c, float* h, int B, int Ts, int D,
+                        void* workspace, size_t ws_bytes, pararnn_stream_t stream) {
+  if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Ts, D);
+  if (rc) return rc;
+  const bool lstm = cell == PARARNN_LSTM;
+  if (!din || !h || !workspace || (lstm && !c) || (!lstm && c)) return PARARNN_ERR_INVALID_ARG;
+  if (!aligned(din, 4) || !aligned(h, 4) || (c && !aligned(c, 4)) || !aligned(workspace, 256))
+    return PARARNN_ERR_MISALIGNED;
+  if (ws_bytes < unfused_ws_bytes(cell, B, Ts, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
+  const int e = shard_apply(cell, din, c, h, B, Ts, D, workspace, (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 

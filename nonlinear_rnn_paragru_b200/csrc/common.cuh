@@ -124,6 +124,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 //   flags  u32 [nrec]  look-back record flags, nrec = cluster chunks * (max_iters+1)
 //   vals   f32 [nrec][kChan][RW]  record payload (RW floats per channel)
 //   chan_k int [B*D]   per-channel convergence iterate (histogram input)
+//   seg    u32 [B*D/8] segments stored per 8-channel tile (segment-queue solve)
 // A record flag is (epoch << 3) | (kind << 1) | ok.  The look-back paths
 // clear their flag slice at the start of every call (the epoch alone cannot
 // tell a stale flag from another path's leftovers in a shared workspace); the
@@ -140,7 +141,7 @@ enum : unsigned { kRecAgg = 1, kRecIncl = 2 };
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct FwdWsLayout {
-  size_t flags, vals, chan_k, total;
+  size_t flags, vals, chan_k, seg, total;
 };
 __host__ __device__ inline FwdWsLayout fwd_ws_layout(size_t nchunks, int max_iters, int rec_floats,
                                                      size_t BD) {
@@ -149,7 +150,8 @@ __host__ __device__ inline FwdWsLayout fwd_ws_layout(size_t nchunks, int max_ite
   L.flags = kWsHeaderBytes;
   L.vals = L.flags + align256(nrec * 4);
   L.chan_k = L.vals + align256(nrec * kChan * rec_floats * 4);
-  L.total = L.chan_k + align256(BD * 4);
+  L.seg = L.chan_k + align256(BD * 4);
+  L.total = L.seg + align256((BD + 7) / 8 * 4);
   return L;
 }
 

@@ -1,0 +1,465 @@
+// gru_fwd_queue.cu -- fused Newton-scan ParaGRU solve of many 8-channel
+// tiles with bf16 input projections: every sequence is cut into segments of
+// NW * 128 steps, and all (tile, segment) items of the solve are worked off
+// by one persistent launch from a queue.
+//
+// An item is 8 consecutive channels of one batch row over one segment.  Its
+// Newton solve ("Параллельность RNN?", §1.2-§1.3) starts from the state the
+// tile's previous segment converged to, exactly as a solve of the whole
+// sequence would see it at convergence: the fixed point of the segment given
+// its true initial state is the true trajectory over the segment.  A CTA of
+// NW warps holds a segment: lane = (chunk k = lane / 8, channel c = lane % 8),
+// a thread keeps its 32-step chunk's iterate and running Jacobian product in
+// registers, and each iteration runs the cell pass of gru_row_pass.cuh, a
+// shuffle scan over the warp's four chunks, one CTA barrier and a scan over
+// the warps from shared memory, and the fix-up.  The item stops after the
+// update of the first iteration whose residual over the item is below tol
+// (or after a residual-only evaluation at the cap).
+//
+// Queue.  Items are numbered segment-major (item = s * ntiles + tile) and
+// CTAs draw them from a counter one item ahead, so a CTA's items increase.
+// Segment s of a tile may start only once segment s - 1 has stored its
+// states: that CTA publishes the segment count of the tile with a release
+// store after its stores, and the first chunk's threads of the successor
+// wait for it with a bounded acquire poll before reading their initial state.
+// The item with the lowest number that is not done is always being worked on
+// and never waits (its predecessor has a lower number), so the queue cannot
+// deadlock while all CTAs are resident; a wait that runs out sets TIMEOUT.
+// With at least as many tiles as resident CTAs the predecessor of an item was
+// drawn about a wave earlier and has normally finished.
+//
+// Data.  u arrives by NW / 2 TMA boxes of 256 steps into the top of the
+// CTA's argument buffer and is expanded in place into fp32 gate arguments
+// (the layout of gru_row_pass.cuh); the next item's boxes are issued as soon
+// as the last pass of the current item is done, and prefetched into L2 when
+// the item is drawn.  a and bias of the next item's channels are loaded
+// while the current item runs.  Compared with one launch per segment, the
+// queue leaves no SM idle at a segment boundary, and with four CTAs of four
+// warps per SM the CTAs' barrier and load phases overlap other CTAs' passes.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "gru_row_pass.cuh"
+
+namespace pararnn {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+struct QParams {
+  const float* a;       // [3][D]
+  const float* bias;    // [3][D] or null
+  const float* h0;      // [B][D] or null
+  float* h;             // [B][T][D]
+  int B, T, D;
+  int nDTc;             // 8-channel tiles per batch row
+  int ntiles;           // B * nDTc
+  int nseg;             // segments per sequence
+  int nitems;           // ntiles * nseg (below 2^31: B*T*D <= 2^40)
+  int max_iters;
+  float tol;
+  uint64_t timeout_ns;
+  unsigned* counter;    // item tickets (zero at launch)
+  unsigned* seg_done;   // [ntiles] segments of each tile stored (zero at launch)
+  int* chan_k;          // [B * D] or null
+  pararnn_stats* stats;
+};
+
+template <int NW>
+struct QCfg {
+  static constexpr int kThreads = NW * 32;
+  static constexpr int kSteps = NW * kRowK * kRowL;        // steps per item
+  static constexpr int kChunks = kSteps / kRowL;
+  static constexpr int kU = kChunks * kRowS;               // fp32 argument bytes
+  static constexpr int kNBox = kSteps / kRowBox;
+  static constexpr int kStage = kU - kNBox * kRowBoxBytes;  // bf16 staging at the top
+  static_assert(kStage % 128 == 0 && kRowBoxBytes % 128 == 0, "TMA destinations");
+  static_assert(kThreads == (kChunks / 2) * kRowH, "the expansion: one (chunk, pair) per thread");
+  static_assert((kChunks / 2) * kRowS <= kStage, "in-place expansion order");
+  static_assert(NW == 4 || NW == 8, "the CTA's residual maximum is read as float4s");
+};
+
+template <int NW>
+struct QShared {
+  float2 wagg[2][NW][kRowC];   // per (warp, channel) inclusive map of the warp
+  float wlast[2][NW][kRowC];   // per (warp, channel) last state before the update
+  float wcm[2][NW][kRowC];     // per (warp, channel) max|r| (histogram)
+  __align__(16) float wmax[2][NW];
+  __align__(16) float par[2][6][kRowC];  // a (3 rows), bias (3 rows), by item parity
+  uint64_t bar;                // the staging area's mbarrier
+  int nx[2];                   // this and the next item, by item parity
+};
+
+__device__ __forceinline__ void q_issue(unsigned char* smem, int stage, int nbox, uint64_t* bar,
+                                        const CUtensorMap* map, int b, int d0, int t0) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  mbar_arrive_expect_tx(bar, (unsigned)(nbox * kRowBoxBytes));
+  for (int j = 0; j < nbox; ++j)
+    tma_load_4d(smem + stage + j * kRowBoxBytes, map, bar, d0, 0, t0 + j * kRowBox, b);
+}
+__device__ __forceinline__ void q_prefetch(const CUtensorMap* map, int nbox, int b, int d0,
+                                           int t0) {
+  for (int j = 0; j < nbox; ++j)
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(d0), "r"(0), "r"(t0 + j * kRowBox), "r"(b)
+                 : "memory");
+}
+// a[g][c] (j < 24) or bias[g][c] (j < 48, 0 when absent) of the tile at d0
+__device__ __forceinline__ float q_param(const QParams& p, int j, int d0) {
+  const int row = j / kRowC, c = j % kRowC;
+  if (row < 3) return p.a[(size_t)row * p.D + d0 + c];
+  return p.bias ? p.bias[(size_t)(row - 3) * p.D + d0 + c] : 0.f;
+}
+__device__ __forceinline__ int q_draw(unsigned* counter) {
+  return (int)min(atomicAdd(counter, 1u), 0x7fffffffu);
+}
+
+template <int NW>
+__global__ void __launch_bounds__(NW * 32, 16 / NW)
+    gru_newton_queue(const __grid_constant__ CUtensorMap map, const QParams p) {
+  using Cfg = QCfg<NW>;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ QShared<NW> sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = lane % kRowC, kk = lane / kRowC;
+  const int q = warp * kRowK + kk;  // chunk index within the item
+  const unsigned char* base = smem + q * kRowS;
+
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    sh.nx[0] = q_draw(p.counter);
+  }
+  __syncthreads();
+  int item = sh.nx[0];
+  if (item < p.nitems) {
+    const int tile = item % p.ntiles;
+    const int d0 = (tile % p.nDTc) * kRowC;
+    if (tid < 6 * kRowC) (&sh.par[0][0][0])[tid] = q_param(p, tid, d0);
+    if (tid == 0)
+      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, tile / p.nDTc, d0,
+              (item / p.ntiles) * Cfg::kSteps);
+  }
+  int status = 0;
+  unsigned phase = 0;  // exchange phases so far, over all items
+  int prev_item = -1;
+  for (int n = 0; item < p.nitems; ++n) {
+    __syncthreads();
+    // publish the previous item: every thread's state stores precede the
+    // barrier above; the fence and release order them before the count
+    if (tid == 0 && prev_item >= 0) {
+      __threadfence();
+      st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+    }
+    if (tid == 0) sh.nx[(n + 1) & 1] = q_draw(p.counter);
+    const int pb = n & 1;
+    const int tile = item % p.ntiles, seg = item / p.ntiles;
+    const int b = tile / p.nDTc, d0 = (tile % p.nDTc) * kRowC;
+    const int d = d0 + c;
+    const bool dval = d < p.D;
+    const int t_base = seg * Cfg::kSteps;
+    const int t_len = min(Cfg::kSteps, p.T - t_base);
+    if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
+    // ---- expand the staged bf16 rows [t][gate][8 ch] into fp32 arguments in
+    // two blocks (each block's rows are read before any of its slots is
+    // written; block 0 writes below all staging bytes)
+    {
+      const int qb = tid / kRowH, i = tid % kRowH;
+      const int sw = row_swizzle(i);
+#pragma unroll 1
+      for (int blk = 0; blk < 2; ++blk) {
+        const int qq = blk * (Cfg::kChunks / 2) + qb;
+        const int ta = qq * kRowL + i, tb = ta + kRowH;
+        const bool pa = ta >= t_len, pbd = tb >= t_len;
+        float xa[3][kRowC], xb[3][kRowC];
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+          const uint4 va = *reinterpret_cast<const uint4*>(
+              smem + Cfg::kStage + (ta / kRowBox) * kRowBoxBytes + ((ta % kRowBox) * 3 + g) * 16);
+          const uint4 vb = *reinterpret_cast<const uint4*>(
+              smem + Cfg::kStage + (tb / kRowBox) * kRowBoxBytes + ((tb % kRowBox) * 3 + g) * 16);
+          const unsigned wa[4] = {va.x, va.y, va.z, va.w};
+          const unsigned wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+          for (int cc = 0; cc < kRowC; ++cc) {
+            const int sh16 = (cc & 1) ? 0 : 16;
+            const unsigned mk = (cc & 1) ? 0xffff0000u : 0xffffffffu;
+            xa[g][cc] = __uint_as_float((wa[cc >> 1] << sh16) & mk);
+            xb[g][cc] = __uint_as_float((wb[cc >> 1] << sh16) & mk);
+          }
+        }
+        __syncthreads();
+        unsigned char* dst = smem + qq * kRowS + i * kRowC * 8;
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+          const float sc = (g == 2) ? 2.f * kLog2e : -kLog2e;
+#pragma unroll
+          for (int cc = 0; cc < kRowC; ++cc) {
+            const float bs = sc * sh.par[pb][3 + g][cc];
+            float2 o = ffma2(f2(sc, sc), f2(xa[g][cc], xb[g][cc]), f2(bs, bs));
+            if (g == 0) {  // steps past the segment: z < 5e-10 whatever a_z h is
+              if (pa) o.x = 3e30f;
+              if (pbd) o.y = 3e30f;
+            }
+            *reinterpret_cast<float2*>(dst + g * kRowH * kRowC * 8 + (cc ^ sw) * 8) = o;
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // the next item: its boxes prefetched into L2 and its parameters loaded
+    // now, the parameters stored after the last pass
+    const int pj = tid - 32;
+    float pnext = 0.f;
+    {
+      const int next = sh.nx[(n + 1) & 1];
+      if (next < p.nitems) {
+        const int ntile = next % p.ntiles;
+        const int nd0 = (ntile % p.nDTc) * kRowC;
+        if (tid == 0)
+          q_prefetch(&map, Cfg::kNBox, ntile / p.nDTc, nd0, (next / p.ntiles) * Cfg::kSteps);
+        if (pj >= 0 && pj < 6 * kRowC) pnext = q_param(p, pj, nd0);
+      }
+    }
+
+    const float az = sh.par[pb][0][c], ar = sh.par[pb][1][c], ac = sh.par[pb][2][c];
+    const float az2 = -kLog2e * az, ar2 = -kLog2e * ar, ac2 = 2.f * kLog2e * ac;
+    const float2 AZ2 = f2(az2, az2), AR2 = f2(ar2, ar2), AC2 = f2(ac2, ac2), AZ = f2(az, az);
+    const bool first = (q == 0);  // the chunk holding the segment's first step
+    // the segment's initial state: h0, or the last state of the previous
+    // segment once that segment's CTA has published it
+    float h0v = 0.f;
+    if (first) {
+      if (seg == 0) {
+        h0v = (p.h0 && dval) ? p.h0[(size_t)b * p.D + d] : 0.f;
+      } else {
+        const unsigned* f = &p.seg_done[tile];
+        if (ld_acquire(f) < (unsigned)seg) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire(f) < (unsigned)seg) {
+            if (globaltimer_ns() - t0 > p.timeout_ns) {
+              status = PARARNN_STATUS_TIMEOUT;
+              break;
+            }
+          }
+        }
+        if (dval) h0v = __ldcg(p.h + ((size_t)b * p.T + t_base - 1) * p.D + d);
+      }
+    }
+
+    float2 H[kRowH], P[kRowH];
+#pragma unroll
+    for (int i = 0; i < kRowH; ++i) {
+      H[i] = f2(0.f, 0.f);
+      P[i] = f2(1.f, 1.f);
+    }
+    float hb = first ? h0v : 0.f;  // state before this chunk
+    int last_bad = -1, updates = 0, k = 0;
+    float final_m = 0.f;
+    for (;; ++k) {
+      const bool cap = (k >= p.max_iters);
+      const int par = phase & 1;
+      ++phase;
+      const float last_pre = H[kRowH - 1].y;
+      float2 DL, PA;
+      float m;
+      if (cap)
+        m = row_pass<false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+      else
+        m = row_pass<true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+      if (!dval) m = 0.f;
+      // the chunk's map: second half after the first
+      float IP = PA.y * PA.x, Id = fmaf(PA.y, DL.x, DL.y);
+      // inclusive scan over the warp's four chunks of channel c (lanes c + 8k)
+#pragma unroll
+      for (int o = kRowC; o < 32; o <<= 1) {
+        const float oP = __shfl_up_sync(kFull, IP, o), od = __shfl_up_sync(kFull, Id, o);
+        if (lane >= o) {
+          Id = fmaf(IP, od, Id);
+          IP *= oP;
+        }
+      }
+      float xP = __shfl_up_sync(kFull, IP, kRowC), xd = __shfl_up_sync(kFull, Id, kRowC);
+      if (kk == 0) {
+        xP = 1.f;
+        xd = 0.f;
+      }
+      // residuals are >= 0 (or NaN with the sign cleared): their bit patterns
+      // order like unsigned integers, NaN above +inf
+      const unsigned wm = __reduce_max_sync(kFull, __float_as_uint(m));
+      unsigned cmu = __float_as_uint(m);
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 8));
+      cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 16));
+      if (kk == kRowK - 1) {
+        sh.wagg[par][warp][c] = make_float2(IP, Id);
+        sh.wlast[par][warp][c] = last_pre;
+      }
+      if (kk == 0) sh.wcm[par][warp][c] = __uint_as_float(cmu);
+      if (lane == 0) sh.wmax[par][warp] = __uint_as_float(wm);
+      __syncthreads();
+      if (q == 0) {  // the channel's own maximum over the item (histogram)
+        float chm = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
+        if (!(chm < p.tol)) last_bad = k;
+      }
+      // the delta entering this warp: the maps of the warps before it applied
+      // to the zero delta entering the item; and the item's residual maximum
+      float cd = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW - 1; ++w) {
+        if (w < warp) {
+          const float2 a2 = sh.wagg[par][w][c];
+          cd = fmaf(a2.x, cd, a2.y);
+        }
+      }
+      float tmax = 0.f;
+#pragma unroll
+      for (int w4 = 0; w4 < NW; w4 += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(&sh.wmax[par][w4]);
+        tmax = fmax_nan(tmax, fmax_nan(fmax_nan(v.x, v.y), fmax_nan(v.z, v.w)));
+      }
+      final_m = tmax;
+      const bool own_ok = tmax < p.tol;
+      if (cap) {
+        updates = k;
+        if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
+        break;
+      }
+      const float din = first ? 0.f : fmaf(xP, cd, xd);  // delta entering this chunk
+      float prev_last = __shfl_up_sync(kFull, last_pre, kRowC);
+      if (kk == 0) prev_last = (warp == 0) ? h0v : sh.wlast[par][warp - 1][c];
+      hb = first ? h0v : prev_last + din;
+      const float2 DIN = f2(din, fmaf(PA.x, din, DL.x));
+#pragma unroll
+      for (int i = 0; i < kRowH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
+      updates = k + 1;
+      if (own_ok) break;
+    }
+    // every thread is past its last pass of this item (the barrier of the last
+    // exchange): the staging area takes the next item
+    const int next = sh.nx[(n + 1) & 1];
+    if (tid == 0 && next < p.nitems) {
+      const int ntile = next % p.ntiles;
+      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, ntile / p.nDTc,
+              (ntile % p.nDTc) * kRowC, (next / p.ntiles) * Cfg::kSteps);
+    }
+    if (pj >= 0 && pj < 6 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
+    // ---- states straight from registers (indices re-derived from the item)
+    item = sh.nx[n & 1];
+    const int itile = item % p.ntiles, it_base = (item / p.ntiles) * Cfg::kSteps;
+    const int ib = itile / p.nDTc, id = (itile % p.nDTc) * kRowC + c;
+    const int it_len = min(Cfg::kSteps, p.T - it_base);
+    bool bad = false;
+    if (id < p.D) {
+      const int tq = q * kRowL;
+      float* out = p.h + ((size_t)ib * p.T + it_base + tq) * p.D + id;
+#pragma unroll
+      for (int i = 0; i < kRowH; ++i) {
+        if (tq + i < it_len) {
+          out[(size_t)i * p.D] = H[i].x;
+          bad |= !isfinite(H[i].x);
+        }
+        if (tq + kRowH + i < it_len) {
+          out[(size_t)(kRowH + i) * p.D] = H[i].y;
+          bad |= !isfinite(H[i].y);
+        }
+      }
+    }
+    if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
+    if (p.chan_k != nullptr && q == 0 && id < p.D)
+      atomicMax(&p.chan_k[(size_t)ib * p.D + id], last_bad + 1);
+    if (tid == 0) {
+      atomicMax(&p.stats->iters, updates);
+      atomicMax(&p.stats->evals, k + 1);
+      atomicMax(reinterpret_cast<int*>(&p.stats->max_residual), __float_as_int(final_m));
+    }
+    prev_item = item;
+    item = next;
+  }
+  __syncthreads();
+  if (tid == 0 && prev_item >= 0) {
+    __threadfence();
+    st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+  }
+  const int st = __reduce_max_sync(kFull, status);
+  if (lane == 0 && st) atomicMax(&p.stats->status, st);
+}
+
+template <int NW>
+int launch_queue_t(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
+  using Cfg = QCfg<NW>;
+  auto kern = gru_newton_queue<NW>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kU);
+  if (e != cudaSuccess) return (int)e;
+  int dev = 0, sms = 148, per_sm = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, Cfg::kU) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  cudaGetLastError();
+  // persistent: every CTA resident at once (the queue's progress argument)
+  const long long grid = std::min<long long>((long long)sms * per_sm, p.nitems);
+  kern<<<(unsigned)std::max<long long>(grid, 1), Cfg::kThreads, Cfg::kU, stream>>>(map, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+// Warps per CTA of the segment-queue solve (segments of 128 * this steps).
+int gru_queue_warps() { return 4; }
+int gru_queue_steps() { return QCfg<4>::kSteps; }
+int gru_queue_channels() { return kRowC; }
+int gru_queue_box_steps() { return kRowBox; }
+
+// Resident CTAs of the segment-queue solve on the current device (0 if it
+// cannot run).
+int gru_queue_resident() {
+  int dev = 0, sms = 148, per_sm = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  auto kern = gru_newton_queue<4>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<4>::kU) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QCfg<4>::kThreads,
+                                                    QCfg<4>::kU) != cudaSuccess)
+    per_sm = 0;
+  cudaGetLastError();
+  return sms * per_sm;
+}
+
+// One launch solves every segment of every tile; u is bf16 through `map`
+// (boxes of 8 channels x 3 gates x 256 steps).  counter and seg_done must be
+// zero at launch (ntiles entries of seg_done).
+int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+                     unsigned* seg_done, cudaStream_t stream) {
+  QParams p;
+  p.a = f.a;
+  p.bias = f.bias;
+  p.h0 = f.h0;
+  p.h = f.h;
+  p.B = f.B;
+  p.T = f.T;
+  p.D = f.D;
+  p.nDTc = (f.D + kRowC - 1) / kRowC;
+  p.ntiles = f.B * p.nDTc;
+  p.nseg = (f.T + QCfg<4>::kSteps - 1) / QCfg<4>::kSteps;
+  if ((long long)p.ntiles * p.nseg >= (1LL << 31)) return 1;
+  p.nitems = p.ntiles * p.nseg;
+  p.max_iters = f.max_iters;
+  p.tol = f.tol;
+  p.timeout_ns = f.timeout_ns;
+  p.counter = counter;
+  p.seg_done = seg_done;
+  p.chan_k = f.chan_k;
+  p.stats = f.stats;
+  return launch_queue_t<4>(map, p, stream);
+}
+
+}  // namespace pararnn

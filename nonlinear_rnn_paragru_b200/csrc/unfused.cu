@@ -73,6 +73,7 @@ struct UfParams {
   float* agg;        // chunk maps: [B][nC][D] per entry (P then d)
   float* carry;      // carry entering each chunk: [B][nC][D] per state entry
   unsigned* rmax;    // residual maximum (ordered bits)
+  const float* cin;  // delta entering the sequence [S][B][D] (a shard's), or null = 0
   int B, T, D, nC;
 };
 
@@ -208,13 +209,13 @@ __global__ void __launch_bounds__(kUfThreads) uf_scan_carry(const UfParams p) {
     const int b = (int)(j / p.D), d = (int)(j - (size_t)b * p.D);
     size_t g = (size_t)b * p.nC * p.D + d;
     if constexpr (!kLSTM) {
-      float x = 0.f;
+      float x = p.cin ? p.cin[j] : 0.f;
       for (int k = 0; k < p.nC; ++k, g += p.D) {
         p.carry[g] = x;
         x = fmaf(p.agg[g], x, p.agg[M + g]);
       }
     } else {
-      float x0 = 0.f, x1 = 0.f;
+      float x0 = p.cin ? p.cin[j] : 0.f, x1 = p.cin ? p.cin[BD + j] : 0.f;
       for (int k = 0; k < p.nC; ++k, g += p.D) {
         p.carry[g] = x0;
         p.carry[M + g] = x1;
@@ -256,6 +257,99 @@ __global__ void __launch_bounds__(kUfThreads) uf_scan_apply(const UfParams p) {
         p.c[i] += x0;
         p.h[i] += x1;
       }
+    }
+  }
+}
+
+// ---------------------------------------------------------- sequence shards --
+// A shard is a contiguous range of steps of every (b, d) channel, solved by
+// one process (GPU).  Its part of the page's linear system couples to the
+// shards before it only through the delta entering its first step, so a
+// Newton iteration is: each shard solves its range from a zero incoming
+// delta and composes its range's map ds_out = P ds_in + d; the maps of all
+// shards are exchanged; each shard composes the maps of the shards before it
+// into its incoming delta, and adds P_t ds_in to its local solution.
+
+// One thread per (b, d): the shard's map (the chunk maps composed in order,
+// first chunk innermost) and the shard's last states before the update.
+// agg planes: ParaGRU P, d; ParaLSTM P00 P01 P10 P11 d0 d1 (state order c, h).
+template <bool kLSTM>
+__global__ void __launch_bounds__(kUfThreads) uf_shard_total(const UfParams p, float* agg,
+                                                            float* last) {
+  const size_t M = (size_t)p.B * p.nC * p.D;
+  const size_t BD = (size_t)p.B * p.D;
+  for (size_t j = (size_t)blockIdx.x * blockDim.x + threadIdx.x; j < BD;
+       j += (size_t)gridDim.x * blockDim.x) {
+    const int b = (int)(j / p.D), d = (int)(j - (size_t)b * p.D);
+    size_t g = (size_t)b * p.nC * p.D + d;
+    const size_t il = ((size_t)b * p.T + p.T - 1) * p.D + d;
+    if constexpr (!kLSTM) {
+      float P = 1.f, x = 0.f;
+      for (int k = 0; k < p.nC; ++k, g += p.D) {
+        x = fmaf(p.agg[g], x, p.agg[M + g]);
+        P *= p.agg[g];
+      }
+      agg[j] = P;
+      agg[BD + j] = x;
+      last[j] = p.h[il];
+    } else {
+      float p00 = 1.f, p01 = 0.f, p10 = 0.f, p11 = 1.f, x0 = 0.f, x1 = 0.f;
+      for (int k = 0; k < p.nC; ++k, g += p.D) {
+        const float a00 = p.agg[g], a01 = p.agg[M + g], a10 = p.agg[2 * M + g],
+                    a11 = p.agg[3 * M + g];
+        const float y0 = fmaf(a00, x0, fmaf(a01, x1, p.agg[4 * M + g]));
+        const float y1 = fmaf(a10, x0, fmaf(a11, x1, p.agg[5 * M + g]));
+        x0 = y0;
+        x1 = y1;
+        const float q00 = fmaf(a00, p00, a01 * p10), q01 = fmaf(a00, p01, a01 * p11);
+        const float q10 = fmaf(a10, p00, a11 * p10), q11 = fmaf(a10, p01, a11 * p11);
+        p00 = q00;
+        p01 = q01;
+        p10 = q10;
+        p11 = q11;
+      }
+      agg[j] = p00;
+      agg[BD + j] = p01;
+      agg[2 * BD + j] = p10;
+      agg[3 * BD + j] = p11;
+      agg[4 * BD + j] = x0;
+      agg[5 * BD + j] = x1;
+      last[j] = p.c[il];
+      last[BD + j] = p.h[il];
+    }
+  }
+}
+
+// One thread per (b, d): the delta entering shard r (the maps of shards
+// 0 .. r-1 applied in order to the zero delta entering shard 0) and, for
+// r > 0, shard r's new initial state: shard r-1's last state before the
+// update plus that delta.
+template <bool kLSTM>
+__global__ void __launch_bounds__(kUfThreads) uf_shard_combine(const float* aggs,
+                                                              const float* lasts, int r, int B,
+                                                              int D, float* din, float* bound) {
+  const size_t BD = (size_t)B * D;
+  const int NA = kLSTM ? 6 : 2, S = kLSTM ? 2 : 1;
+  for (size_t j = (size_t)blockIdx.x * blockDim.x + threadIdx.x; j < BD;
+       j += (size_t)gridDim.x * blockDim.x) {
+    float x0 = 0.f, x1 = 0.f;
+    for (int q = 0; q < r; ++q) {
+      const float* A = aggs + (size_t)q * NA * BD + j;
+      if constexpr (!kLSTM) {
+        x0 = fmaf(A[0], x0, A[BD]);
+      } else {
+        const float y0 = fmaf(A[0], x0, fmaf(A[BD], x1, A[4 * BD]));
+        const float y1 = fmaf(A[2 * BD], x0, fmaf(A[3 * BD], x1, A[5 * BD]));
+        x0 = y0;
+        x1 = y1;
+      }
+    }
+    din[j] = x0;
+    if (kLSTM) din[BD + j] = x1;
+    if (r > 0) {
+      const float* L = lasts + (size_t)(r - 1) * S * BD + j;
+      bound[j] = L[0] + x0;
+      if (kLSTM) bound[BD + j] = L[BD] + x1;
     }
   }
 }
@@ -313,6 +407,7 @@ int unfused_solve(int cell, bool bf16, const void* u, const float* a, const floa
   p.agg = reinterpret_cast<float*>(ws + L.agg);
   p.carry = reinterpret_cast<float*>(ws + L.carry);
   p.rmax = reinterpret_cast<unsigned*>(ws + L.rmax);
+  p.cin = nullptr;
   p.B = B;
   p.T = T;
   p.D = D;
@@ -367,6 +462,93 @@ int unfused_solve(int cell, bool bf16, const void* u, const float* a, const floa
   e = cudaMemcpyAsync(stats, &st, sizeof(st), cudaMemcpyHostToDevice, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // st lives on this stack
   return (int)e;
+}
+
+namespace {
+UfParams uf_shard_params(int cell, const void* u, const float* a, const float* bias,
+                         const float* c_bound, const float* h_bound, float* c, float* h, int B,
+                         int Ts, int D, void* workspace) {
+  const UfLayout L = uf_layout(cell, B, Ts, D);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  UfParams p;
+  p.u = u;
+  p.a = a;
+  p.bias = bias;
+  p.c0 = c_bound;
+  p.h0 = h_bound;
+  p.c = c;
+  p.h = h;
+  p.jac = reinterpret_cast<float*>(ws + L.jac);
+  p.rhs = reinterpret_cast<float*>(ws + L.rhs);
+  p.agg = reinterpret_cast<float*>(ws + L.agg);
+  p.carry = reinterpret_cast<float*>(ws + L.carry);
+  p.rmax = nullptr;
+  p.cin = nullptr;
+  p.B = B;
+  p.T = Ts;
+  p.D = D;
+  p.nC = (Ts + kUfChunk - 1) / kUfChunk;
+  return p;
+}
+}  // namespace
+
+// First half of a shard's Newton iteration: residual and Jacobians at the
+// iterate (c, h) given the state before the shard (c_bound, h_bound), the
+// shard's system solved from a zero incoming delta (chunk maps in the
+// workspace), its map and last states to agg / last, and max|r| to *rmax.
+// The iterate is not changed.  Arguments are validated by the caller.
+int shard_eval(int cell, bool bf16, const void* u, const float* a, const float* bias,
+               const float* c_bound, const float* h_bound, const float* c, const float* h, int B,
+               int Ts, int D, float* agg, float* last, float* rmax, void* workspace,
+               cudaStream_t stream) {
+  const bool lstm = cell == PARARNN_LSTM;
+  UfParams p = uf_shard_params(cell, u, a, bias, c_bound, h_bound, const_cast<float*>(c),
+                               const_cast<float*>(h), B, Ts, D, workspace);
+  p.rmax = reinterpret_cast<unsigned*>(rmax);  // ordered bits of |r| are the float's own
+  const size_t N = (size_t)B * Ts * D, M = (size_t)B * p.nC * D, BD = (size_t)B * D;
+  cudaError_t e = cudaMemsetAsync(rmax, 0, sizeof(float), stream);
+  if (e != cudaSuccess) return (int)e;
+  if (lstm) {
+    if (bf16) uf_assemble_lstm<true><<<uf_grid(N), kUfThreads, 0, stream>>>(p);
+    else uf_assemble_lstm<false><<<uf_grid(N), kUfThreads, 0, stream>>>(p);
+    uf_scan_chunks<true><<<uf_grid(M), kUfThreads, 0, stream>>>(p);
+    uf_shard_total<true><<<uf_grid(BD), kUfThreads, 0, stream>>>(p, agg, last);
+  } else {
+    if (bf16) uf_assemble_gru<true><<<uf_grid(N), kUfThreads, 0, stream>>>(p);
+    else uf_assemble_gru<false><<<uf_grid(N), kUfThreads, 0, stream>>>(p);
+    uf_scan_chunks<false><<<uf_grid(M), kUfThreads, 0, stream>>>(p);
+    uf_shard_total<false><<<uf_grid(BD), kUfThreads, 0, stream>>>(p, agg, last);
+  }
+  return (int)cudaGetLastError();
+}
+
+int shard_combine(int cell, const float* aggs, const float* lasts, int r, int B, int D,
+                  float* din, float* bound, cudaStream_t stream) {
+  const size_t BD = (size_t)B * D;
+  if (cell == PARARNN_LSTM)
+    uf_shard_combine<true><<<uf_grid(BD), kUfThreads, 0, stream>>>(aggs, lasts, r, B, D, din, bound);
+  else
+    uf_shard_combine<false><<<uf_grid(BD), kUfThreads, 0, stream>>>(aggs, lasts, r, B, D, din,
+                                                                     bound);
+  return (int)cudaGetLastError();
+}
+
+// Second half: the chunks re-run from their true carries, starting from the
+// delta entering the shard, and the deltas added to the iterate.
+int shard_apply(int cell, const float* din, float* c, float* h, int B, int Ts, int D,
+                void* workspace, cudaStream_t stream) {
+  UfParams p = uf_shard_params(cell, nullptr, nullptr, nullptr, nullptr, nullptr, c, h, B, Ts, D,
+                               workspace);
+  p.cin = din;
+  const size_t M = (size_t)B * p.nC * D, BD = (size_t)B * D;
+  if (cell == PARARNN_LSTM) {
+    uf_scan_carry<true><<<uf_grid(BD), kUfThreads, 0, stream>>>(p);
+    uf_scan_apply<true><<<uf_grid(M), kUfThreads, 0, stream>>>(p);
+  } else {
+    uf_scan_carry<false><<<uf_grid(BD), kUfThreads, 0, stream>>>(p);
+    uf_scan_apply<false><<<uf_grid(M), kUfThreads, 0, stream>>>(p);
+  }
+  return (int)cudaGetLastError();
 }
 
 }  // namespace pararnn

@@ -122,6 +122,25 @@ def _cases(pr):
             ("dtype", dict(a1=9), -2), ("W_misaligned", dict(a2=0x2002), -5),
             ("ws_too_small", dict(a12=1024), -3)]:
         C["dense_" + name] = ((lambda o: lambda lib: _dense(lib, pr, **o))(over), code)
+    # sequence sharding: ParaGRU shard B=1, Ts=8, D=32
+    def _seval(lib, **over):
+        a = [pr.PARARNN_GRU, 0x1000, pr.PARARNN_BF16, 0x2000, None, None, None, None, 0x3000,
+             1, 8, 32, 0x4000, 0x5000, 0x6000, 0x10000, 1 << 20, None]
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return lib.pararnn_shard_eval(*a)
+    for name, over, code in [("bad_cell", dict(a0=5), -1), ("c_for_gru", dict(a7=0x7000), -1),
+                             ("no_h", dict(a8=None), -1), ("no_agg", dict(a12=None), -1),
+                             ("dtype", dict(a2=3), -2), ("D12", dict(a11=12), -1),
+                             ("agg_misaligned", dict(a12=0x4002), -5),
+                             ("ws_too_small", dict(a16=64), -3)]:
+        C["shard_eval_" + name] = ((lambda o: lambda lib: _seval(lib, **o))(over), code)
+    C["shard_combine_rank_out_of_range"] = (lambda lib: lib.pararnn_shard_combine(
+        pr.PARARNN_GRU, 0x1000, 0x2000, 2, 2, 1, 32, 0x3000, 0x4000, None), -1)
+    C["shard_combine_needs_bound"] = (lambda lib: lib.pararnn_shard_combine(
+        pr.PARARNN_GRU, 0x1000, 0x2000, 2, 1, 1, 32, 0x3000, None, None), -1)
+    C["shard_apply_lstm_needs_c"] = (lambda lib: lib.pararnn_shard_apply(
+        pr.PARARNN_LSTM, 0x1000, None, 0x3000, 1, 8, 32, 0x10000, 1 << 20, None), -1)
     return C
 
 

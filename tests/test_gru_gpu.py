@@ -283,3 +283,42 @@ def test_nan_input_reports_nonfinite(cuda_ok, flags):
     h, st2, _ = _solve(y, flags=flags)
     assert st2["status"] == "converged"
     assert np.abs(h - _ref(y)).max() < TOL_STATE
+
+
+# ---- the segment-queue solve (bf16 u, at least one 8-channel tile per
+# resident CTA: 4 x 148 = 592 on a B200): every 512-step segment of every tile
+# in one launch, each segment from the state its predecessor converged to
+@pytest.mark.parametrize("B,T,D", [(1, 1300, 4800), (2, 2100, 2400), (3, 513, 1600)])
+def test_segment_queue_matches_oracle(cuda_ok, B, T, D):
+    x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
+    x["h0"] = torch.randn((B, D), generator=torch.Generator().manual_seed(29)) * 0.5
+    ref = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_ROW):
+        h, st, hist = _solve(x, flags=flags, hist=True)
+        err = np.abs(h - ref).max()
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged" and st["max_residual"] < 1e-6, (flags, st)
+        assert hist.sum() == B * D and hist[-1] == 0
+
+
+def test_segment_queue_channel_index_one_segment(cuda_ok):
+    # T <= 512: one item per tile, so the per-channel index is the oracle's
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=500, D=4800))
+    ci = torch.full((1, 4800), -5, dtype=torch.int32, device="cuda")
+    h, st, hist = _solve(x, hist=True, chan_iters=ci)
+    k_gpu = ci.cpu().numpy()
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=64)
+    diff = np.abs(k_gpu - r["chan_k"])
+    assert diff.max() <= 1 and (diff == 0).mean() > 0.9, diff.max()
+    np.testing.assert_array_equal(hist, np.bincount(k_gpu.ravel(), minlength=66))
+    assert np.abs(h - _ref(x)).max() < TOL_STATE
+
+
+def test_segment_queue_capped_iterates(cuda_ok):
+    # with the cap at one update, every segment returns the first Newton
+    # iterate from the state its predecessor ended with
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=512, D=4800))
+    h, st, _ = _solve(x, max_iters=1)
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=1)
+    assert st["status"] == "not_converged" and st["iters"] == 1 and st["evals"] == 2
+    assert np.abs(h - r["h"]).max() < TOL_STATE
