@@ -96,6 +96,10 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            8-channel tile per SM, ParaLSTM with
                                            bf16 u and T <= 4096 (segmented as
                                            the solves' comments say) */
+#define PARARNN_FLAG_DENSE_SIMT 8u      /* pararnn_dense_gru_solve: fp32
+                                           products on CUDA cores (exact
+                                           Newton steps, D <= 128) instead of
+                                           tf32 tensor-core products */
 #define PARARNN_FLAG_FORCE_ROW 4u       /* ParaGRU with bf16 u: launch the
                                            row kernel segment by segment
                                            instead of the one-launch
@@ -276,11 +280,31 @@ int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a,
  * iteration writes the blocks J_t and -r_t to the workspace, solves
  * ds_t = J_t ds_{t-1} - r_t by a chunked scan of D x D maps and checks the
  * residual on the host: stopping is global, as for pararnn_solve_unfused,
- * and the call synchronises `stream`.  D a multiple of 8, at most 128.
- * Workspace: pararnn_dense_workspace_size(B, T, D) bytes (4 D^2 + 16 D bytes
- * per (b, t), and the chunk maps), 256-byte aligned, no initialisation; 0
- * means the shape is not supported.  Errors as for the other solves. */
+ * and the call synchronises `stream`.  The contractions (the recurrent
+ * pre-activations, and the products of blocks that compose 16-step chunk
+ * maps, a tree of four levels) run on the tensor cores with tf32 inputs and
+ * fp32 accumulation: each Newton step is then inexact (about 1e-3 relative
+ * in the chunk maps) while the residual, evaluated in fp32, still defines the
+ * fixed point.  opts->flags PARARNN_FLAG_DENSE_SIMT takes fp32 products on
+ * CUDA cores instead (exact steps).  D a multiple of 8, at most 512 (128 with
+ * PARARNN_FLAG_DENSE_SIMT).  W, h and h0 16-byte aligned.  Status TIMEOUT if
+ * a tensor-core product's bounded wait ran out.
+ * Workspace: pararnn_dense_workspace_size(B, T, D) bytes (about 8 D^2 + 32 D
+ * bytes per (b, t) with T rounded up to 16, plus 12 D^2 for W^T), 256-byte
+ * aligned, no initialisation; 0 means the shape is not supported.  Errors as
+ * for the other solves. */
 size_t pararnn_dense_workspace_size(int B, int T, int D);
+/* The tensor-core contraction of pararnn_dense_gru_solve, exposed so that it
+ * can be checked on its own: C[z] = A[z] B[z]^T for z < Z, with A[z] M x K
+ * and B[z] N x K row-major fp32 (A[z] at A + z M K, B[z] at Bm + z N K),
+ * tf32 products (tcgen05.mma kind::tf32) accumulated in fp32.  C[z] at
+ * C + z M N: row-major M x N (store_mode 0), transposed N x M (1), or
+ * row-major for odd z and transposed for even z (2).  K a multiple of 4; A,
+ * Bm, C 16-byte aligned.  *err (device int) is set to 1 if a bounded wait ran
+ * out (the affected tiles are not written); it is not cleared. */
+int pararnn_dense_matmul(const float* A, const float* Bm, float* C, int M,
+                         int N, int K, int Z, int store_mode, int* err,
+                         pararnn_stream_t stream);
 int pararnn_dense_gru_solve(const void* u, int u_dtype, const float* W,
                             const float* bias, const float* h0, float* h,
                             int B, int T, int D, const pararnn_opts* opts,

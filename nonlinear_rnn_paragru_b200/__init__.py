@@ -25,6 +25,7 @@ __all__ = [
     "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
     "pararnn_unfused_workspace_size", "pararnn_solve_unfused", "solve_unfused",
     "pararnn_dense_workspace_size", "pararnn_dense_gru_solve", "dense_gru_solve",
+    "pararnn_dense_matmul",
     "pararnn_shard_workspace_size", "pararnn_shard_eval", "pararnn_shard_combine",
     "pararnn_shard_apply",
     "pararnn_strerror", "gru_solve", "lstm_solve", "adjoint", "seq_baseline",
@@ -36,6 +37,8 @@ PARARNN_F32, PARARNN_BF16 = 0, 1
 PARARNN_GRU, PARARNN_LSTM = 0, 1
 PARARNN_FLAG_INJECT_WITHHOLD = 1
 PARARNN_FLAG_FORCE_CHUNKED = 2
+PARARNN_FLAG_FORCE_ROW = 4
+PARARNN_FLAG_DENSE_SIMT = 8
 STATUS_NAMES = {0: "converged", 1: "not_converged", 2: "nonfinite", 3: "timeout"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +94,7 @@ def load_library():
         "pararnn_solve_unfused": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i, i,
                                       op, vp, vp, sz, vp]),
         "pararnn_dense_workspace_size": (sz, [i, i, i]),
+        "pararnn_dense_matmul": (i, [fp, fp, fp, i, i, i, i, i, ip, vp]),
         "pararnn_dense_gru_solve": (i, [vp, i, fp, fp, fp, fp, i, i, i, op, vp, vp,
                                         sz, vp]),
         "pararnn_shard_workspace_size": (sz, [i, i, i, i]),
@@ -236,6 +240,17 @@ def pararnn_solve_unfused(cell, u, a, bias, c0, h0, c, h, opts, stats, workspace
         _iptr(stats), _wptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)),
         "pararnn_solve_unfused")
+
+
+def pararnn_dense_matmul(A, Bm, C, store_mode, err, stream=None):
+    """C[z] = A[z] @ Bm[z].T on the tensor cores (tf32 products, fp32 sums):
+    A [Z, M, K], Bm [Z, N, K], C [Z, M, N] (or [Z, N, M] transposed per
+    store_mode), err int32 [1]."""
+    Z, M, K = A.shape
+    N = Bm.shape[1]
+    _check(load_library().pararnn_dense_matmul(
+        _ptr(A), _ptr(Bm), _ptr(C), M, N, K, Z, int(store_mode), _iptr(err), _stream(stream)),
+        "pararnn_dense_matmul")
 
 
 def pararnn_dense_workspace_size(B, T, D) -> int:
@@ -398,7 +413,7 @@ def solve_unfused(cell, u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iter
 
 
 def dense_gru_solve(u, W, bias=None, h0=None, *, tol=1e-6, max_iters=64, workspace=None,
-                    stream=None):
+                    stream=None, flags=0):
     """Newton solve of the GRU with full recurrent matrices W [3, D, D]:
     returns (h, stats).  Synchronises the stream."""
     B, T, G, D = u.shape
@@ -409,7 +424,8 @@ def dense_gru_solve(u, W, bias=None, h0=None, *, tol=1e-6, max_iters=64, workspa
     if nbytes == 0:
         raise PararnnError(-1, "pararnn_dense_workspace_size (unsupported shape)")
     buf = ws.get(nbytes, stream)
-    pararnn_dense_gru_solve(u, W, bias, h0, h, _opts(tol, max_iters), stats, buf, stream)
+    pararnn_dense_gru_solve(u, W, bias, h0, h, _opts(tol, max_iters, flags=flags), stats, buf,
+                            stream)
     return h, stats
 
 

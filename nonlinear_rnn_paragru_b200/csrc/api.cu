@@ -43,11 +43,14 @@ int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float
                             float* dbias, float* dc0, float* dh0, int B, int T, int D,
                             int* status, void* ws, cudaStream_t stream);
 size_t unfused_ws_bytes(int cell, int B, int T, int D);
-int dense_max_d();
+int dense_max_d(bool simt);
+int tc_operand_map(CUtensorMap* map, const float* base, int K, int rows, int Z, long long zstride);
+int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, float* C, int M, int N, int K,
+                   int Z, int store_mode, int* err, cudaStream_t stream);
 size_t dense_ws_bytes(int B, int T, int D);
-int dense_gru_solve(bool bf16, const void* u, const float* W, const float* bias, const float* h0,
-                    float* h, int B, int T, int D, float tol, int max_iters, pararnn_stats* stats,
-                    void* workspace, cudaStream_t stream);
+int dense_gru_solve(bool bf16, bool simt, const void* u, const float* W, const float* bias,
+                    const float* h0, float* h, int B, int T, int D, float tol, int max_iters,
+                    pararnn_stats* stats, void* workspace, cudaStream_t stream);
 int unfused_solve(int cell, bool bf16, const void* u, const float* a, const float* bias,
                   const float* c0, const float* h0, float* c, float* h, int B, int T, int D,
                   float tol, int max_iters, pararnn_stats* stats, void* workspace,
@@ -571,8 +574,25 @@ int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a, 
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 
+int pararnn_dense_matmul(const float* A, const float* Bm, float* C, int M, int N, int K, int Z,
+                         int store_mode, int* err, pararnn_stream_t stream) {
+  if (!A || !Bm || !C || !err || M < 1 || N < 1 || K < 1 || Z < 1 || (K % 4) != 0 ||
+      store_mode < 0 || store_mode > 2)
+    return PARARNN_ERR_INVALID_ARG;
+  if ((long long)M * N * Z >= (1LL << 40) || M >= (1 << 30) || N >= (1 << 30))
+    return PARARNN_ERR_TOO_LARGE;
+  if (!aligned(A, 16) || !aligned(Bm, 16) || !aligned(C, 16) || !aligned(err, 4))
+    return PARARNN_ERR_MISALIGNED;
+  CUtensorMap ma, mb;
+  if (tc_operand_map(&ma, A, K, M, Z, (long long)M * K) ||
+      tc_operand_map(&mb, Bm, K, N, Z, (long long)N * K))
+    return PARARNN_ERR_CUDA;
+  const int e = launch_tc_gemm(ma, mb, C, M, N, K, Z, store_mode, err, (cudaStream_t)stream);
+  return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+}
+
 size_t pararnn_dense_workspace_size(int B, int T, int D) {
-  if (check_sizes(B, T, D) || D > dense_max_d()) return 0;
+  if (check_sizes(B, T, D) || D > dense_max_d(false)) return 0;
   return dense_ws_bytes(B, T, D);
 }
 
@@ -582,19 +602,20 @@ int pararnn_dense_gru_solve(const void* u, int u_dtype, const float* W, const fl
                             size_t ws_bytes, pararnn_stream_t stream) {
   int rc = check_sizes(B, T, D);
   if (rc) return rc;
-  if (D > dense_max_d()) return PARARNN_ERR_INVALID_ARG;
+  const bool simt = opts && (opts->flags & PARARNN_FLAG_DENSE_SIMT);
+  if (D > dense_max_d(simt)) return PARARNN_ERR_INVALID_ARG;
   if ((long long)B * T >= (1LL << 31)) return PARARNN_ERR_TOO_LARGE;
   if (u_dtype != PARARNN_F32 && u_dtype != PARARNN_BF16) return PARARNN_ERR_UNSUPPORTED_DTYPE;
   if (!u || !W || !h || !stats || !workspace) return PARARNN_ERR_INVALID_ARG;
-  if (!aligned(u, u_dtype == PARARNN_BF16 ? 2 : 4) || !aligned(W, 4) || !aligned(h, 4) ||
-      (bias && !aligned(bias, 4)) || (h0 && !aligned(h0, 4)) || !aligned(stats, 4) ||
+  if (!aligned(u, u_dtype == PARARNN_BF16 ? 2 : 4) || !aligned(W, 16) || !aligned(h, 16) ||
+      (bias && !aligned(bias, 4)) || (h0 && !aligned(h0, 16)) || !aligned(stats, 4) ||
       !aligned(workspace, 256))
     return PARARNN_ERR_MISALIGNED;
   if (ws_bytes < dense_ws_bytes(B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const float tol = (opts && opts->tol > 0.f) ? opts->tol : kDefaultTol;
   const int max_iters = resolve_max_iters(opts ? opts->max_iters : 0);
   if (max_iters > kMaxItersLimit) return PARARNN_ERR_INVALID_ARG;
-  const int e = dense_gru_solve(u_dtype == PARARNN_BF16, u, W, bias, h0, h, B, T, D, tol,
+  const int e = dense_gru_solve(u_dtype == PARARNN_BF16, simt, u, W, bias, h0, h, B, T, D, tol,
                                 max_iters, stats, workspace, (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }

@@ -11,21 +11,32 @@
 // c = tanh(u_c + b_c + r (W_c h)),  h' = (1 - z) h + z c,  and
 //   dh'/dh = diag(1 - z) + diag((c - h) z (1 - z)) W_z
 //            + diag(z (1 - c^2)) [diag(r) W_c + diag((W_c h) r (1 - r)) W_r].
-// Each Newton iteration, as in the unfused tier but with matrix blocks:
-//   dn_pre       Q = [W_z; W_r; W_c] h_{t-1} for every (b, t): a tiled fp32
-//                GEMM of the shifted states [B*T, D] by W^T [D, 3D];
-//   dn_assemble  one CTA per (b, t): gates, residual, -r_t and the block
-//                J_t = df/dh (h_{t-1}) [D][D] to HBM, and the residual maximum;
-//   dn_chunk_maps, dn_carry, dn_apply: ds_t = J_t ds_{t-1} - r_t by 16-step
-//                chunks: each chunk's map (P = J_{t1-1} ... J_{t0}, d) from a
-//                zero delta in shared memory (a D x D x D product per step),
-//                the carries chunk by chunk, then every chunk re-run from its
-//                carry, adding ds to the iterate;
-// and the host reads the residual maximum to stop (the first iteration below
-// tol has its update applied; the cap ends with a residual-only evaluation).
-// These are CUDA-core kernels: the products of D x D maps are where tensor
-// cores would apply.  Layouts: u [B][T][3][D], W [3][D][D] row-major (row i
-// of W_g feeds unit i), bias [3][D], h0 [B][D], h [B][T][D].  D <= 128.
+// Each Newton iteration, with the host checking the residual as in the
+// unfused tier, runs (tensor-core path, the default):
+//   pre-activations  Q = h W^T for every step: a tcgen05 tf32 GEMM of the
+//                    states [B*T, D] by the stacked matrices [3D, D]
+//                    (tc_gemm.cu), W h0 once per solve;
+//   dn_assemble2     one CTA per (b, step): gates, residual, -r_t and the
+//                    block J_t to HBM, row-major at odd positions of its
+//                    16-step chunk and transposed at even ones;
+//   chunk maps       each chunk's product J_15 ... J_0 as a tree of pairwise
+//                    products, four levels of batched D x D tcgen05 GEMMs (left
+//                    factor row-major, right factor transposed: both operands
+//                    K-major; each level stores its products in the layout the
+//                    next level reads them in);
+//   dn_offsets, dn_carry2, dn_apply2
+//                    the chunk offsets (the chunk's recurrence from a zero
+//                    delta), the delta entering each chunk chunk by chunk,
+//                    and every chunk re-run from its delta, ds added to h
+//                    (matrix-vector products, coalesced in either layout).
+// tf32 products make each Newton step inexact (about 1e-3 relative in the
+// chunk maps); the residual is evaluated in fp32, so the fixed point is that
+// of the cell and the iteration still converges, in a step or two more.  The
+// CUDA-core path (fp32 products, exact steps, D <= 128) is kept for
+// comparison (PARARNN_FLAG_DENSE_SIMT): dn_pre, dn_assemble, dn_chunk_maps
+// (a D x D x D product per step in shared memory), dn_carry, dn_apply.
+// Layouts: u [B][T][3][D], W [3][D][D] row-major (row i of W_g feeds unit i),
+// bias [3][D], h0 [B][D], h [B][T][D].  D <= 512.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -38,8 +49,10 @@ namespace pararnn {
 namespace {
 
 constexpr int kDnThreads = 256;
-constexpr int kDnChunk = 16;   // steps per scan chunk
-constexpr int kDnMaxD = 128;   // three (D x (D+1)) fp32 tiles fit in shared memory
+constexpr int kDnChunk = 16;       // steps per scan chunk (four levels of pairwise products)
+constexpr int kDnLevels = 4;
+constexpr int kDnMaxDSimt = 128;   // three (D x (D+1)) fp32 tiles fit in shared memory
+constexpr int kDnMaxD = 512;
 
 template <bool kBF16>
 __device__ __forceinline__ float dn_u(const void* u, size_t i) {
@@ -278,9 +291,204 @@ __global__ void __launch_bounds__(kDnThreads) dn_apply(const DnParams p) {
   }
 }
 
+// ------------------------------------------------------ tensor-core path --
+struct Dn2Params {
+  const void* u;
+  const float *W, *Wt, *bias, *h0;
+  float* h;        // the iterate [B][T][D]
+  const float* Q;  // row b*T + t: W h_t, [B][T][3D]
+  const float* Q0; // W h0 [B][3D] (zeros when h0 is absent)
+  float* J;        // [B][Tp][D][D]: odd positions of a chunk row-major, even transposed
+  const float* P;  // chunk maps [B][nC][D][D] row-major (the last tree level)
+  float* rhs;      // -r [B][Tp][D], zero on padded steps
+  float* d;        // chunk offsets [B][nC][D]
+  float* carry;    // delta entering each chunk [B][nC][D]
+  unsigned* rmax;
+  int B, T, D, nC, Tp;
+};
+
+// W_g^T for each gate: Wt[g][j][i] = W[g][i][j]
+__global__ void dn_transpose_w(const float* __restrict__ W, float* __restrict__ Wt, int D) {
+  __shared__ float tile[32][33];
+  const int g = blockIdx.z, i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  const size_t off = (size_t)g * D * D;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int i = i0 + r, j = j0 + threadIdx.x;
+    if (i < D && j < D) tile[r][threadIdx.x] = W[off + (size_t)i * D + j];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    const int j = j0 + r, i = i0 + threadIdx.x;
+    if (i < D && j < D) Wt[off + (size_t)j * D + i] = tile[threadIdx.x][r];
+  }
+}
+
+// One CTA per (b, padded step t): gates from the pre-activations of h_{t-1},
+// residual, -r_t and J_t; padded steps (t >= T) get J = I and -r = 0.
+template <bool kBF16>
+__global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
+  __shared__ float co[4][kDnMaxD];
+  __shared__ unsigned wmax[kDnThreads / 32];
+  const int D = p.D;
+  const size_t bt = blockIdx.x;  // b * Tp + t
+  const int b = (int)(bt / p.Tp), t = (int)(bt - (size_t)b * p.Tp);
+  const size_t DD = (size_t)D * D;
+  float* Jt = p.J + bt * DD;
+  if (t >= p.T) {
+    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) Jt[e] = (e / D == e % D) ? 1.f : 0.f;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) p.rhs[bt * D + i] = 0.f;
+    return;
+  }
+  const size_t bs = (size_t)b * p.T + t;  // (b, t) in the unpadded arrays
+  const float* q3 = t > 0 ? p.Q + (bs - 1) * 3 * D : p.Q0 + (size_t)b * 3 * D;
+  unsigned m = 0;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    const float hp = t > 0 ? p.h[(bs - 1) * D + i] : (p.h0 ? p.h0[(size_t)b * D + i] : 0.f);
+    const size_t iu = bs * 3 * D + i;
+    const float z = dn_sig(q3[i] + dn_u<kBF16>(p.u, iu) + (p.bias ? p.bias[i] : 0.f));
+    const float r = dn_sig(q3[D + i] + dn_u<kBF16>(p.u, iu + D) + (p.bias ? p.bias[D + i] : 0.f));
+    const float q = q3[2 * D + i];
+    const float c =
+        tanhf(dn_u<kBF16>(p.u, iu + 2 * (size_t)D) + (p.bias ? p.bias[2 * D + i] : 0.f) + r * q);
+    const float f = fmaf(z, c - hp, hp);
+    const float res = p.h[bs * D + i] - f;
+    p.rhs[bt * D + i] = -res;
+    m = max(m, dn_abs_bits(res));
+    const float gc = z * (1.f - c * c);
+    co[0][i] = 1.f - z;
+    co[1][i] = (c - hp) * z * (1.f - z);
+    co[2][i] = gc * r;
+    co[3][i] = gc * q * r * (1.f - r);
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned mm = 0;
+    for (int w = 0; w < kDnThreads / 32; ++w) mm = max(mm, wmax[w]);
+    atomicMax(p.rmax, mm);
+  }
+  // J[i][j] = [i == j] (1 - z_i) + co1_i Wz[i][j] + co2_i Wc[i][j] + co3_i Wr[i][j]
+  if (t & 1) {  // row-major, element e = i * D + j
+    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) {
+      const int i = (int)(e / D), j = (int)(e - (size_t)i * D);
+      Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.W[e] + co[2][i] * p.W[2 * DD + e] +
+              co[3][i] * p.W[DD + e];
+    }
+  } else {      // transposed, element e = j * D + i (W^T read contiguously)
+    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) {
+      const int j = (int)(e / D), i = (int)(e - (size_t)j * D);
+      Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.Wt[e] + co[2][i] * p.Wt[2 * DD + e] +
+              co[3][i] * p.Wt[DD + e];
+    }
+  }
+}
+
+// y = M x + add over a CTA (M D x D in global memory, row-major or
+// transposed; x, y in shared memory); ends with a CTA barrier.
+__device__ __forceinline__ void dn_matvec(const float* __restrict__ M, bool rowmajor,
+                                          const float* x, const float* __restrict__ add, float* y,
+                                          int D) {
+  if (rowmajor) {  // a warp per row: coalesced along the row
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = warp; i < D; i += kDnThreads / 32) {
+      const float* Mi = M + (size_t)i * D;
+      float s = 0.f;
+      for (int q = lane; q < D; q += 32) s = fmaf(Mi[q], x[q], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) y[i] = s + (add ? add[i] : 0.f);
+    }
+  } else {         // M[q][i] = (the matrix)[i][q]: a thread per output, coalesced along q rows
+    for (int i = threadIdx.x; i < D; i += kDnThreads) {
+      float s = add ? add[i] : 0.f;
+      for (int q = 0; q < D; ++q) s = fmaf(M[(size_t)q * D + i], x[q], s);
+      y[i] = s;
+    }
+  }
+  __syncthreads();
+}
+
+// One CTA per (b, chunk): the chunk's recurrence from a zero delta; its last
+// delta is the chunk's offset d.
+__global__ void __launch_bounds__(kDnThreads) dn_offsets(const Dn2Params p) {
+  __shared__ float xs[2][kDnMaxD];
+  const int D = p.D;
+  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = 0.f;
+  __syncthreads();
+  int cur = 0;
+  for (int pp = 0; pp < kDnChunk; ++pp) {
+    const size_t bt = (size_t)b * p.Tp + (size_t)k * kDnChunk + pp;
+    dn_matvec(p.J + bt * D * D, (pp & 1) != 0, xs[cur], p.rhs + bt * D, xs[cur ^ 1], D);
+    cur ^= 1;
+  }
+  for (int i = threadIdx.x; i < D; i += blockDim.x) p.d[(size_t)blockIdx.x * D + i] = xs[cur][i];
+}
+
+// One CTA per b: the delta entering each chunk, chunk by chunk (x <- P_k x + d_k).
+__global__ void __launch_bounds__(kDnThreads) dn_carry2(const Dn2Params p) {
+  __shared__ float xs[2][kDnMaxD];
+  const int D = p.D, b = blockIdx.x;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = 0.f;
+  __syncthreads();
+  int cur = 0;
+  for (int k = 0; k < p.nC; ++k) {
+    const size_t o = (size_t)b * p.nC + k;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) p.carry[o * D + i] = xs[cur][i];
+    dn_matvec(p.P + o * D * D, true, xs[cur], p.d + o * D, xs[cur ^ 1], D);
+    cur ^= 1;
+  }
+}
+
+// One CTA per (b, chunk): the chunk re-run from its delta; ds added to h.
+__global__ void __launch_bounds__(kDnThreads) dn_apply2(const Dn2Params p) {
+  __shared__ float xs[2][kDnMaxD];
+  const int D = p.D;
+  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = p.carry[(size_t)blockIdx.x * D + i];
+  __syncthreads();
+  int cur = 0;
+  for (int pp = 0; pp < kDnChunk; ++pp) {
+    const int t = k * kDnChunk + pp;
+    if (t >= p.T) break;
+    const size_t bt = (size_t)b * p.Tp + t;
+    dn_matvec(p.J + bt * D * D, (pp & 1) != 0, xs[cur], p.rhs + bt * D, xs[cur ^ 1], D);
+    cur ^= 1;
+    for (int i = threadIdx.x; i < D; i += blockDim.x)
+      p.h[((size_t)b * p.T + t) * D + i] += xs[cur][i];
+  }
+}
+
 struct DnLayout {
   size_t rmax, Q, J, rhs, P, d, carry, total;
 };
+
+// tensor-core path workspace: [0, 256) residual maximum and the GEMMs' error
+// flag, then W^T, Q, W h0, the level-0 blocks, tree levels 1..4, -r, d, carry
+struct Dn2Layout {
+  size_t Wt, Q, Q0, J, lvl[kDnLevels], rhs, d, carry, total;
+};
+
+Dn2Layout dn2_layout(int B, int T, int D) {
+  const size_t nC = (size_t)(T + kDnChunk - 1) / kDnChunk, Tp = nC * kDnChunk;
+  const size_t DD = (size_t)D * D;
+  Dn2Layout L;
+  L.Wt = 256;
+  L.Q = L.Wt + align256(3 * DD * 4);
+  L.Q0 = L.Q + align256((size_t)B * T * 3 * D * 4);
+  L.J = L.Q0 + align256((size_t)B * 3 * D * 4);
+  size_t o = L.J + align256((size_t)B * Tp * DD * 4);
+  for (int l = 0; l < kDnLevels; ++l) {
+    L.lvl[l] = o;
+    o += align256((size_t)B * (Tp >> (l + 1)) * DD * 4);
+  }
+  L.rhs = o;
+  L.d = L.rhs + align256((size_t)B * Tp * D * 4);
+  L.carry = L.d + align256((size_t)B * nC * D * 4);
+  L.total = L.carry + align256((size_t)B * nC * D * 4);
+  return L;
+}
 
 DnLayout dn_layout(int B, int T, int D) {
   const size_t BT = (size_t)B * T, nC = (size_t)(T + kDnChunk - 1) / kDnChunk;
@@ -299,14 +507,138 @@ DnLayout dn_layout(int B, int T, int D) {
 
 }  // namespace
 
-int dense_max_d() { return kDnMaxD; }
-size_t dense_ws_bytes(int B, int T, int D) { return dn_layout(B, T, D).total; }
+int tc_operand_map(CUtensorMap* map, const float* base, int K, int rows, int Z, long long zstride);
+int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, float* C, int M, int N, int K,
+                   int Z, int store_mode, int* err, cudaStream_t stream);
+
+int dense_max_d(bool simt) { return simt ? kDnMaxDSimt : kDnMaxD; }
+size_t dense_ws_bytes(int B, int T, int D) {
+  return std::max(dn_layout(B, T, D).total, dn2_layout(B, T, D).total);
+}
+
+namespace {
+// Tensor-core path; see the file comment.
+int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, const float* h0,
+                   float* h, int B, int T, int D, float tol, int max_iters, pararnn_stats* stats,
+                   void* workspace, cudaStream_t stream) {
+  const Dn2Layout L = dn2_layout(B, T, D);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  Dn2Params p;
+  p.u = u;
+  p.W = W;
+  p.Wt = reinterpret_cast<float*>(ws + L.Wt);
+  p.bias = bias;
+  p.h0 = h0;
+  p.h = h;
+  float* Q = reinterpret_cast<float*>(ws + L.Q);
+  float* Q0 = reinterpret_cast<float*>(ws + L.Q0);
+  p.Q = Q;
+  p.Q0 = Q0;
+  p.J = reinterpret_cast<float*>(ws + L.J);
+  p.P = reinterpret_cast<float*>(ws + L.lvl[kDnLevels - 1]);
+  p.rhs = reinterpret_cast<float*>(ws + L.rhs);
+  p.d = reinterpret_cast<float*>(ws + L.d);
+  p.carry = reinterpret_cast<float*>(ws + L.carry);
+  p.rmax = reinterpret_cast<unsigned*>(ws);
+  int* err = reinterpret_cast<int*>(ws + 4);
+  p.B = B;
+  p.T = T;
+  p.D = D;
+  p.nC = (T + kDnChunk - 1) / kDnChunk;
+  p.Tp = p.nC * kDnChunk;
+  const size_t BT = (size_t)B * T, DD = (size_t)D * D;
+  const int nprod0 = B * p.Tp;  // level-0 blocks
+
+  // operand maps: the states and h0 against the stacked matrices; per tree
+  // level, odd blocks (left factors) against even ones (right factors)
+  CUtensorMap mh, mh0, mw, ml[kDnLevels], mr[kDnLevels];
+  int rc = tc_operand_map(&mh, h, D, (int)BT, 1, (long long)BT * D);
+  rc |= tc_operand_map(&mw, W, D, 3 * D, 1, 3LL * DD);
+  if (h0) rc |= tc_operand_map(&mh0, h0, D, B, 1, (long long)B * D);
+  for (int l = 0; l < kDnLevels; ++l) {
+    const float* in = l == 0 ? p.J : reinterpret_cast<float*>(ws + L.lvl[l - 1]);
+    const int nout = nprod0 >> (l + 1);
+    rc |= tc_operand_map(&ml[l], in + DD, D, D, nout, 2LL * DD);
+    rc |= tc_operand_map(&mr[l], in, D, D, nout, 2LL * DD);
+  }
+  if (rc) return (int)cudaErrorInvalidValue;
+
+  cudaError_t e = cudaMemsetAsync(h, 0, BT * D * 4, stream);  // initial guess: zero
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, 8, stream);  // residual maximum, error flag
+  if (e != cudaSuccess) return (int)e;
+  dn_transpose_w<<<dim3((D + 31) / 32, (D + 31) / 32, 3), dim3(32, 8), 0, stream>>>(
+      W, reinterpret_cast<float*>(ws + L.Wt), D);
+  int ge = 0;
+  if (h0)
+    ge = launch_tc_gemm(mh0, mw, Q0, B, 3 * D, D, 1, 0, err, stream);
+  else
+    e = cudaMemsetAsync(Q0, 0, (size_t)B * 3 * D * 4, stream);
+  if (ge) return ge;
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return (int)e;
+  pararnn_stats st = {0, 0.f, PARARNN_STATUS_CONVERGED, 0};
+  for (int k = 0;; ++k) {
+    e = cudaMemsetAsync(p.rmax, 0, sizeof(unsigned), stream);
+    if (e != cudaSuccess) return (int)e;
+    ge = launch_tc_gemm(mh, mw, Q, (int)BT, 3 * D, D, 1, 0, err, stream);
+    if (ge) return ge;
+    const unsigned nblk = (unsigned)((size_t)B * p.Tp);
+    if (bf16)
+      dn_assemble2<true><<<nblk, kDnThreads, 0, stream>>>(p);
+    else
+      dn_assemble2<false><<<nblk, kDnThreads, 0, stream>>>(p);
+    unsigned hdr[2] = {0u, 0u};
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return (int)e;
+    if (hdr[1] != 0u) {  // a tensor-core GEMM's wait ran out
+      st.status = PARARNN_STATUS_TIMEOUT;
+      break;
+    }
+    float r;
+    std::memcpy(&r, &hdr[0], sizeof r);  // the ordered bits are the float's own
+    st.evals = k + 1;
+    st.max_residual = r;
+    if (!(r == r) || hdr[0] >= 0x7f800000u) {  // NaN or inf
+      st.status = PARARNN_STATUS_NONFINITE;
+      break;
+    }
+    if (k == max_iters) {  // residual-only evaluation at the cap
+      if (!(r < tol)) st.status = PARARNN_STATUS_NOT_CONVERGED;
+      break;
+    }
+    // chunk maps: four levels of pairwise block products
+    for (int l = 0; l < kDnLevels; ++l) {
+      float* out = reinterpret_cast<float*>(ws + L.lvl[l]);
+      ge = launch_tc_gemm(ml[l], mr[l], out, D, D, D, nprod0 >> (l + 1),
+                          l + 1 < kDnLevels ? 2 : 0, err, stream);
+      if (ge) return ge;
+    }
+    const unsigned nmaps = (unsigned)((size_t)B * p.nC);
+    dn_offsets<<<nmaps, kDnThreads, 0, stream>>>(p);
+    dn_carry2<<<(unsigned)B, kDnThreads, 0, stream>>>(p);
+    dn_apply2<<<nmaps, kDnThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+    st.iters = k + 1;
+    if (r < tol) break;  // the update of the first certified iteration is applied
+  }
+  e = cudaMemcpyAsync(stats, &st, sizeof(st), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // st lives on this stack
+  return (int)e;
+}
+}  // namespace
 
 // The host-driven loop; arguments are validated by the caller.  Writes
 // *stats (device) at the end.  Returns 0 or a CUDA error.
-int dense_gru_solve(bool bf16, const void* u, const float* W, const float* bias, const float* h0,
-                    float* h, int B, int T, int D, float tol, int max_iters, pararnn_stats* stats,
-                    void* workspace, cudaStream_t stream) {
+int dense_gru_solve(bool bf16, bool simt, const void* u, const float* W, const float* bias,
+                    const float* h0, float* h, int B, int T, int D, float tol, int max_iters,
+                    pararnn_stats* stats, void* workspace, cudaStream_t stream) {
+  if (!simt)
+    return dense_solve_tc(bf16, u, W, bias, h0, h, B, T, D, tol, max_iters, stats, workspace,
+                          stream);
   const DnLayout L = dn_layout(B, T, D);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   DnParams p;

@@ -120,8 +120,16 @@ def _cases(pr):
     for name, over, code in [
             ("D_above_max", dict(a8=520), -1), ("no_W", dict(a2=None), -1),
             ("dtype", dict(a1=9), -2), ("W_misaligned", dict(a2=0x2002), -5),
+            ("W_not_16_aligned", dict(a2=0x2004), -5), ("h_not_16_aligned", dict(a5=0x3008), -5),
             ("ws_too_small", dict(a12=1024), -3)]:
         C["dense_" + name] = ((lambda o: lambda lib: _dense(lib, pr, **o))(over), code)
+    for name, args, code in [
+            ("K_not_multiple_of_4", (0x1000, 0x2000, 0x3000, 8, 8, 6, 1, 0, 0x4000, None), -1),
+            ("bad_store_mode", (0x1000, 0x2000, 0x3000, 8, 8, 8, 1, 3, 0x4000, None), -1),
+            ("no_err", (0x1000, 0x2000, 0x3000, 8, 8, 8, 1, 0, None, None), -1),
+            ("A_misaligned", (0x1004, 0x2000, 0x3000, 8, 8, 8, 1, 0, 0x4000, None), -5)]:
+        C["dense_matmul_" + name] = ((lambda a_: lambda lib: lib.pararnn_dense_matmul(*a_))(args),
+                                     code)
     # sequence sharding: ParaGRU shard B=1, Ts=8, D=32
     def _seval(lib, **over):
         a = [pr.PARARNN_GRU, 0x1000, pr.PARARNN_BF16, 0x2000, None, None, None, None, 0x3000,
