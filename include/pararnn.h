@@ -86,8 +86,23 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
 #define PARARNN_STATUS_TIMEOUT 3
 
 /* opts.flags */
-#define PARARNN_FLAG_INJECT_WITHHOLD 1u /* testing: chunk `inject_chunk` never
-                                           publishes its look-back record */
+#define PARARNN_FLAG_INJECT_WITHHOLD 1u /* testing: a part of the solve's
+                                           exchange is withheld so that the
+                                           bounded waits for it run out
+                                           (TIMEOUT): in the chunked forward
+                                           solves cluster chunk inject_chunk
+                                           never publishes its look-back
+                                           record; in the row solves the CTA
+                                           of cluster rank inject_chunk
+                                           withholds its exchange at the
+                                           residual-only evaluation of the
+                                           cap (use max_iters to reach it);
+                                           in the segment-queue solve item
+                                           inject_chunk (segment-major:
+                                           segment * tiles + tile) never
+                                           publishes its states to the next
+                                           segment; for the adjoint see
+                                           pararnn_adjoint_ex */
 #define PARARNN_FLAG_FORCE_CHUNKED 2u   /* use the chunked (cluster + decoupled
                                            look-back) solve where the
                                            whole-sequence row kernels would
@@ -205,6 +220,23 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
                     float* du, float* da, float* dbias, float* dc0, float* dh0,
                     int B, int T, int D, int* status, void* workspace,
                     size_t ws_bytes, pararnn_stream_t stream);
+
+/* pararnn_adjoint with options: opts->timeout_us bounds every cross-block
+ * wait (0 or NULL opts: 2 s); with PARARNN_FLAG_INJECT_WITHHOLD in
+ * opts->flags, for testing, a part of the exchange is withheld so that the
+ * waits for it run out and *status becomes PARARNN_STATUS_TIMEOUT: in the
+ * look-back adjoint (fp32 u or T > 4096) the chunk whose ticket is
+ * opts->inject_chunk (the tile's chunks take tickets last first) publishes
+ * no records; in the whole-sequence adjoint (bf16 u, T <= 4096) the CTA of
+ * cluster rank opts->inject_chunk withholds its map in its cluster's last
+ * tile.  Other opts fields are ignored.  NULL opts = pararnn_adjoint. */
+int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a,
+                       const float* bias, const float* c0, const float* h0,
+                       const float* c, const float* h, const float* dLdh,
+                       float* du, float* da, float* dbias, float* dc0,
+                       float* dh0, int B, int T, int D, int* status,
+                       void* workspace, size_t ws_bytes,
+                       const pararnn_opts* opts, pararnn_stream_t stream);
 
 /* Adjoint without a caller-supplied workspace.  (The pages have no
  * counterpart; this is a library convenience.)  For callers that cannot hand

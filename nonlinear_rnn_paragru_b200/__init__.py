@@ -21,7 +21,7 @@ __all__ = [
     "PARARNN_F32", "PARARNN_BF16", "PARARNN_GRU", "PARARNN_LSTM",
     "PararnnOpts", "PararnnError", "library_path", "load_library",
     "pararnn_workspace_size", "pararnn_workspace_init", "pararnn_gru_solve",
-    "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_noalloc",
+    "pararnn_lstm_solve", "pararnn_adjoint", "pararnn_adjoint_ex", "pararnn_adjoint_noalloc",
     "pararnn_seq_baseline", "pararnn_gru_step", "pararnn_lstm_step",
     "pararnn_unfused_workspace_size", "pararnn_solve_unfused", "solve_unfused",
     "pararnn_dense_workspace_size", "pararnn_dense_gru_solve", "dense_gru_solve",
@@ -88,6 +88,8 @@ def load_library():
                                 fp, fp, fp, i, i, i, ip, vp, sz, vp]),
         "pararnn_seq_baseline": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, i, i,
                                      i, vp]),
+        "pararnn_adjoint_ex": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, fp, fp, fp,
+                                   fp, fp, fp, i, i, i, ip, vp, sz, op, vp]),
         "pararnn_adjoint_noalloc": (i, [i, vp, i, fp, fp, fp, fp, fp, fp, fp,
                                         fp, fp, fp, fp, fp, i, i, i, ip, vp]),
         "pararnn_unfused_workspace_size": (sz, [i, i, i, i]),
@@ -208,6 +210,18 @@ def pararnn_adjoint(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, dbias, dc0,
         _iptr(status), _wptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)),
         "pararnn_adjoint")
+
+
+def pararnn_adjoint_ex(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, dbias, dc0,
+                       dh0, status, workspace, opts, stream=None):
+    _check(load_library().pararnn_adjoint_ex(
+        cell, _uptr(u), _dtype_code(u), _ptr(a), _ptr(bias), _ptr(c0),
+        _ptr(h0), _ptr(c), _ptr(h), _ptr(dLdh), _ptr(du), _ptr(da),
+        _ptr(dbias), _ptr(dc0), _ptr(dh0), u.shape[0], u.shape[1], u.shape[3],
+        _iptr(status), _wptr(workspace),
+        workspace.numel() * workspace.element_size(),
+        ctypes.byref(opts) if opts is not None else None, _stream(stream)),
+        "pararnn_adjoint_ex")
 
 
 def pararnn_adjoint_noalloc(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, dbias,
@@ -376,7 +390,7 @@ def lstm_solve(u, a, bias=None, c0=None, h0=None, *, tol=1e-6, max_iters=64,
 
 
 def adjoint(cell, u, a, bias, h0, h, dLdh, c0=None, c=None, *, workspace=None,
-            want_dbias=True, want_dh0=True, stream=None, out=None):
+            want_dbias=True, want_dh0=True, stream=None, out=None, opts=None):
     B, T, G, D = u.shape
     dev = u.device
     o = out or {}
@@ -390,8 +404,12 @@ def adjoint(cell, u, a, bias, h0, h, dLdh, c0=None, c=None, *, workspace=None,
     status = o.get("status") if o.get("status") is not None else torch.zeros(1, dtype=torch.int32, device=dev)
     ws = workspace if workspace is not None else Workspace(dev)
     buf = ws.get(pararnn_workspace_size(cell, B, T, D, 0, 1), stream)
-    pararnn_adjoint(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, db, dc0, dh0,
-                    status, buf, stream)
+    if opts is None:
+        pararnn_adjoint(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, db, dc0, dh0,
+                        status, buf, stream)
+    else:
+        pararnn_adjoint_ex(cell, u, a, bias, c0, h0, c, h, dLdh, du, da, db, dc0, dh0,
+                           status, buf, opts, stream)
     return {"du": du, "da": da, "dbias": db, "dh0": dh0, "dc0": dc0,
             "status": status}
 

@@ -136,6 +136,7 @@ struct AdjParams {
   float *du, *da, *dbias, *dc0, *dh0;
   int B, T, D, nDT, nC;
   uint64_t timeout_ns;
+  int inject_chunk;  // testing: the chunk with this ticket publishes no records (-1: none)
   WsHeader* hdr;
   unsigned* rec_flags;
   float* rec_vals;
@@ -301,9 +302,10 @@ __global__ void __launch_bounds__(kAdjThreads, Cell::kMinBlocks)
     const int stride = 1;
     const size_t rec = (size_t)ticket;
     float* rv = p.rec_vals + rec * (size_t)(kChan * rec_floats<E>());
+    const bool publish = ticket != p.inject_chunk;
     if (v > 0) {
       rec_put_agg(rv, lane, cur);
-      publish_flag(&p.rec_flags[rec], make_flag(epoch, kRecAgg, true));
+      if (publish) publish_flag(&p.rec_flags[rec], make_flag(epoch, kRecAgg, true));
       bool ok;
       if (!lookback<E, V>(p.rec_flags, p.rec_vals, ticket - v, v, 0, stride, epoch, p.timeout_ns,
                           kin, ok)) {
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(kAdjThreads, Cell::kMinBlocks)
       }
     }
     rec_put_incl(rv, lane, cur.apply(kin));
-    publish_flag(&p.rec_flags[rec], make_flag(epoch, kRecIncl, true));
+    if (publish) publish_flag(&p.rec_flags[rec], make_flag(epoch, kRecIncl, true));
     if (status) atomicMax(&ctl[3], status);
     // the incoming carry of every warp, as a constant map
     for (int w = 0; w < kAdjNW; ++w) {
@@ -483,7 +485,7 @@ int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, 
                    const float* bias, const float* c0, const float* h0, const float* c,
                    const float* h, const float* dLdh, float* du, float* da, float* dbias,
                    float* dc0, float* dh0, int B, int T, int D, int* status, void* ws,
-                   cudaStream_t stream) {
+                   uint64_t timeout_ns, int inject_chunk, cudaStream_t stream) {
   const int tc = adjoint_chunk_steps(cell);
   const int G = cell == PARARNN_GRU ? 3 : 4;
   const AdjLayout Lw = adj_layout(cell, B, T, D);
@@ -507,7 +509,8 @@ int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, 
   p.D = D;
   p.nDT = (D + kChan - 1) / kChan;
   p.nC = (T + tc - 1) / tc;
-  p.timeout_ns = 2000000000ull;
+  p.timeout_ns = timeout_ns;
+  p.inject_chunk = inject_chunk;
   p.hdr = reinterpret_cast<WsHeader*>(w);
   p.rec_flags = reinterpret_cast<unsigned*>(w + Lw.flags);
   p.rec_vals = reinterpret_cast<float*>(w + Lw.vals);

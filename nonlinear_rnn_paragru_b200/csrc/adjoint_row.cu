@@ -119,6 +119,8 @@ struct ArParams {
   int B, T, D;
   uint64_t timeout_ns;
   int* status;
+  int withhold_rank;  // testing: this cluster rank withholds its map in its
+                      // cluster's last tile (-1: none)
 };
 
 // affine map x -> P x + d, as float2 (P, d); (f o g)(x) = f(g(x))
@@ -310,7 +312,10 @@ __global__ void __launch_bounds__(kArThreads, 2)
       if (w > warp) cw = ar_after(sh.wagg[par][w][c], cw);
     float cin_cta = 0.f;  // carry entering this CTA from the steps after it
     if (CLS > 1) {
-      if (warp == 0 && kk == 0 && rank > 0) {
+      // testing: a withheld map in the cluster's last tile (no later
+      // exchange reuses a barrier whose phase did not complete)
+      const bool withhold = rank == p.withhold_rank && next >= ntiles;
+      if (warp == 0 && kk == 0 && rank > 0 && !withhold) {
         const float2 m = ar_after(inc, cw);  // the CTA's map of channel c
         for (int r = 0; r < rank; ++r)
           ar_st_async_v2(ar_mapa(smem_u32(&sh.mbox[ms][rank][c]), r), m,
@@ -319,9 +324,9 @@ __global__ void __launch_bounds__(kArThreads, 2)
       // The last rank receives nothing, so it neither waits nor re-arms: a
       // zero-byte re-arm completes the next phase at once, and a warp yet to
       // wait would then wait for the phase after that one.
-      if (rank < CLS - 1 &&
-          !mbar_wait_bounded(&sh.mbar[ms], (n / kArSlots) & 1, p.timeout_ns) && status == 0)
-        status = PARARNN_STATUS_TIMEOUT;
+      const bool got =
+          rank == CLS - 1 || mbar_wait_bounded(&sh.mbar[ms], (n / kArSlots) & 1, p.timeout_ns);
+      if (!got && status == 0) status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
       for (int r = CLS - 1; r > 0; --r) {
         if (r > rank) {
@@ -330,7 +335,9 @@ __global__ void __launch_bounds__(kArThreads, 2)
         }
       }
       __syncwarp();
-      if (tid == 0 && rank < CLS - 1) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
+      // a phase that did not complete is not re-armed: a second arrival on
+      // it would be one more than the barrier counts
+      if (tid == 0 && rank < CLS - 1 && got) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
     }
     const float cwarp = fmaf(cw.x, cin_cta, cw.y);
     const float cchunk = fmaf(xm.x, cwarp, xm.y);
@@ -451,6 +458,7 @@ struct AlParams {
   int B, T, D;
   uint64_t timeout_ns;
   int* status;
+  int withhold_rank;  // as for ArParams
 };
 
 struct AlCell {
@@ -680,7 +688,8 @@ __global__ void __launch_bounds__(kArThreads, 2)
       }
     float2 cin_cta = af2(0.f, 0.f);
     if (CLS > 1) {
-      if (warp == 0 && kk == 0 && rank > 0) {
+      const bool withhold = rank == p.withhold_rank && next >= ntiles;  // testing
+      if (warp == 0 && kk == 0 && rank > 0 && !withhold) {
         const Aff2 m = inc.after(cw);  // the CTA's map of channel c
         const float4 m0 = make_float4(m.m00, m.m01, m.m10, m.m11);
         const float4 m1 = make_float4(m.d0, m.d1, 0.f, 0.f);
@@ -691,9 +700,9 @@ __global__ void __launch_bounds__(kArThreads, 2)
         }
       }
       // the last rank receives nothing: no wait, no re-arm (as for ParaGRU)
-      if (rank < CLS - 1 &&
-          !mbar_wait_bounded(&sh.mbar[ms], (n / kAlSlots) & 1, p.timeout_ns) && status == 0)
-        status = PARARNN_STATUS_TIMEOUT;
+      const bool got =
+          rank == CLS - 1 || mbar_wait_bounded(&sh.mbar[ms], (n / kAlSlots) & 1, p.timeout_ns);
+      if (!got && status == 0) status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
       for (int r = CLS - 1; r > 0; --r) {
         if (r > rank) {
@@ -702,7 +711,7 @@ __global__ void __launch_bounds__(kArThreads, 2)
         }
       }
       __syncwarp();
-      if (tid == 0 && rank < CLS - 1) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
+      if (tid == 0 && rank < CLS - 1 && got) mbar_arrive_expect_tx(&sh.mbar[ms], rx);
     }
     const float2 cchunk = xm.apply(cw.apply(cin_cta));
     const float2 cx = My.apply(cchunk);  // entering step 7 from step 8
@@ -868,7 +877,8 @@ static int launch_ar_t(const CUtensorMap* maps, const ArParams& p, cudaStream_t 
 // maps: u (box 8 x 3 x 19), h (box 8 x 20), dL/dh (box 8 x 19)
 int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bias,
                        const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
-                       int T, int D, int* status, void* ws, cudaStream_t stream) {
+                       int T, int D, int* status, void* ws, uint64_t timeout_ns,
+                       int withhold_rank, cudaStream_t stream) {
   ArParams p;
   p.a = a;
   p.bias = bias;
@@ -879,8 +889,9 @@ int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bia
   p.B = B;
   p.T = T;
   p.D = D;
-  p.timeout_ns = 2000000000ull;
+  p.timeout_ns = timeout_ns;
   p.status = status;
+  p.withhold_rank = withhold_rank;
   const int cls = adjoint_row_cluster(T);
   adjoint_row_init<<<1, 1, 0, stream>>>(status);
   if (cudaGetLastError() != cudaSuccess) return 1;
@@ -933,7 +944,8 @@ static int launch_al_t(const CUtensorMap* maps, const AlParams& p, cudaStream_t 
 int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float* bias,
                             const float* c0, const float* h0, float* du, float* da,
                             float* dbias, float* dc0, float* dh0, int B, int T, int D,
-                            int* status, void* ws, cudaStream_t stream) {
+                            int* status, void* ws, uint64_t timeout_ns, int withhold_rank,
+                            cudaStream_t stream) {
   AlParams p;
   p.a = a;
   p.bias = bias;
@@ -946,8 +958,9 @@ int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float
   p.B = B;
   p.T = T;
   p.D = D;
-  p.timeout_ns = 2000000000ull;
+  p.timeout_ns = timeout_ns;
   p.status = status;
+  p.withhold_rank = withhold_rank;
   const int cls = adjoint_row_cluster(T);
   adjoint_row_init<<<1, 1, 0, stream>>>(status);
   if (cudaGetLastError() != cudaSuccess) return 1;

@@ -37,11 +37,13 @@ int adjoint_row_box_steps(int which);
 size_t adjoint_row_part_bytes(int G, int B, int T, int D);
 int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bias,
                        const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
-                       int T, int D, int* status, void* ws, cudaStream_t stream);
+                       int T, int D, int* status, void* ws, uint64_t timeout_ns,
+                       int withhold_rank, cudaStream_t stream);
 int launch_adjoint_row_lstm(const CUtensorMap* maps, const float* a, const float* bias,
                             const float* c0, const float* h0, float* du, float* da,
                             float* dbias, float* dc0, float* dh0, int B, int T, int D,
-                            int* status, void* ws, cudaStream_t stream);
+                            int* status, void* ws, uint64_t timeout_ns, int withhold_rank,
+                            cudaStream_t stream);
 size_t unfused_ws_bytes(int cell, int B, int T, int D);
 int dense_max_d(bool simt);
 int tc_operand_map(CUtensorMap* map, const float* base, int K, int rows, int Z, long long zstride);
@@ -76,7 +78,7 @@ int launch_adjoint(int cell, bool bf16, const CUtensorMap* maps, const void* u, 
                    const float* bias, const float* c0, const float* h0, const float* c,
                    const float* h, const float* dLdh, float* du, float* da, float* dbias,
                    float* dc0, float* dh0, int B, int T, int D, int* status, void* ws,
-                   cudaStream_t stream);
+                   uint64_t timeout_ns, int inject_chunk, cudaStream_t stream);
 }  // namespace pararnn
 
 using namespace pararnn;
@@ -422,6 +424,19 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
                     const float* dLdh, float* du, float* da, float* dbias, float* dc0, float* dh0,
                     int B, int T, int D, int* status, void* workspace, size_t ws_bytes,
                     pararnn_stream_t stream) {
+  return pararnn_adjoint_ex(cell, u, u_dtype, a, bias, c0, h0, c, h, dLdh, du, da, dbias, dc0,
+                            dh0, B, T, D, status, workspace, ws_bytes, nullptr, stream);
+}
+
+int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, const float* bias,
+                       const float* c0, const float* h0, const float* c, const float* h,
+                       const float* dLdh, float* du, float* da, float* dbias, float* dc0,
+                       float* dh0, int B, int T, int D, int* status, void* workspace,
+                       size_t ws_bytes, const pararnn_opts* opts, pararnn_stream_t stream) {
+  const uint64_t timeout_ns =
+      1000ull * ((opts && opts->timeout_us) ? opts->timeout_us : kDefaultTimeoutUs);
+  const bool inject = opts && (opts->flags & PARARNN_FLAG_INJECT_WITHHOLD);
+  const int inject_chunk = inject ? opts->inject_chunk : -1;
   if (cell != PARARNN_GRU && cell != PARARNN_LSTM) return PARARNN_ERR_INVALID_ARG;
   int rc = check_sizes(B, T, D);
   if (rc) return rc;
@@ -451,7 +466,7 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
       if (!rc) rc = make_s_map(&rmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
       if (rc) return rc;
       e = launch_adjoint_row(rmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status, workspace,
-                             (cudaStream_t)stream);
+                             timeout_ns, inject_chunk, (cudaStream_t)stream);
     } else {  // u, c and h (states before each step), dL/dh
       rc = make_u_map(&rmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
       if (!rc) rc = make_s_map(&rmaps[1], c, B, T, D, adjoint_row_box_steps(1), ch);
@@ -459,7 +474,8 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
       if (!rc) rc = make_s_map(&rmaps[3], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
       if (rc) return rc;
       e = launch_adjoint_row_lstm(rmaps, a, bias, c0, h0, du, da, dbias, dc0, dh0, B, T, D,
-                                  status, workspace, (cudaStream_t)stream);
+                                  status, workspace, timeout_ns, inject_chunk,
+                                  (cudaStream_t)stream);
     }
     return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
   }
@@ -472,7 +488,7 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a, const 
   if (rc) return rc;
   const int e = launch_adjoint(cell, u_dtype == PARARNN_BF16, maps, u, a, bias, c0, h0, c, h, dLdh,
                                du, da, dbias, dc0, dh0, B, T, D, status, workspace,
-                               (cudaStream_t)stream);
+                               timeout_ns, inject_chunk, (cudaStream_t)stream);
   return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
 }
 

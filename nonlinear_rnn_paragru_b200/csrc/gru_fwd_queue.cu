@@ -66,6 +66,7 @@ struct QParams {
   unsigned* seg_done;   // [ntiles] segments of each tile stored (zero at launch)
   int* chan_k;          // [B * D] or null
   pararnn_stats* stats;
+  int withhold_item;    // testing: this item never publishes its segment (-1: none)
 };
 
 template <int NW>
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     __syncthreads();
     // publish the previous item: every thread's state stores precede the
     // barrier above; the fence and release order them before the count
-    if (tid == 0 && prev_item >= 0) {
+    if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
       __threadfence();
       st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
     }
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     item = next;
   }
   __syncthreads();
-  if (tid == 0 && prev_item >= 0) {
+  if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
     __threadfence();
     st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
   }
@@ -459,6 +460,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.seg_done = seg_done;
   p.chan_k = f.chan_k;
   p.stats = f.stats;
+  p.withhold_item = (f.flags & PARARNN_FLAG_INJECT_WITHHOLD) ? f.inject_chunk : -1;
   return launch_queue_t<4>(map, p, stream);
 }
 

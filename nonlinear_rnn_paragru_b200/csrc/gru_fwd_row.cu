@@ -408,7 +408,12 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       float din_cta = 0.f;          // delta entering this CTA
       float prev_cta_last = h0v;    // state before this CTA's first step
       if (CLS > 1) {
-        if (warp == kRowWarps - 1) {
+        // testing: the CTA of rank inject_chunk withholds its last exchange
+        // (the residual-only evaluation at the cap), so its peers' bounded
+        // waits run out
+        const bool withhold =
+            cap && (p.flags & PARARNN_FLAG_INJECT_WITHHOLD) && rank == p.inject_chunk;
+        if (warp == kRowWarps - 1 && !withhold) {
           // the CTA map of channel c: last warp's inclusive map after the
           // warps before it; to every CTA after this one.  Lanes r < CLS
           // send the residual maximum to CTA r.
@@ -423,8 +428,8 @@ __global__ void __launch_bounds__(kRowThreads, 2)
             st_async_b32(mapa_u32(smem_u32(&sh.mbox[par].cmax[rank]), lane),
                          __float_as_uint(cmax), mapa_u32(smem_u32(&sh.mbar[par]), lane));
         }
-        if (!mbar_wait_bounded(&sh.mbar[par], mpar, p.timeout_ns) && status == 0)
-          status = PARARNN_STATUS_TIMEOUT;
+        const bool got = mbar_wait_bounded(&sh.mbar[par], mpar, p.timeout_ns);
+        if (!got && status == 0) status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
         for (int r = 0; r < CLS; ++r) {
           if (r != rank) tmax = fmax_nan(tmax, sh.mbox[par].cmax[r]);
@@ -435,9 +440,12 @@ __global__ void __launch_bounds__(kRowThreads, 2)
           }
         }
         // re-arm this mailbox for its next phase; every thread of the CTA
-        // has passed the wait before any peer can send that phase's bytes
+        // has passed the wait before any peer can send that phase's bytes.
+        // A phase that did not complete is not re-armed (a second arrival on
+        // it would be one more than the barrier counts): later waits on it
+        // run out too and the solve reports TIMEOUT.
         __syncwarp();
-        if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[par], rx);
+        if (tid == 0 && got) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
       final_m = tmax;
       const bool own_ok = tmax < p.tol;

@@ -440,7 +440,11 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       float2 din_cta = lf2(0.f, 0.f);            // delta entering this CTA
       float2 prev_cta_last = lf2(c0v, h0v);      // state before this CTA's first step
       if (CLS > 1) {
-        if (warp == kLrWarps - 1) {
+        // testing: the CTA of rank inject_chunk withholds its last exchange
+        // (the residual-only evaluation at the cap)
+        const bool withhold =
+            cap && (p.flags & PARARNN_FLAG_INJECT_WITHHOLD) && rank == p.inject_chunk;
+        if (warp == kLrWarps - 1 && !withhold) {
           const float cmax = tmax;
           if (kk == kLrK - 1) {
             const Aff2 cm = inc.after(cw);  // the CTA's map of channel c
@@ -456,8 +460,8 @@ __global__ void __launch_bounds__(kLrThreads, 1)
             lr_st_async_b32(lr_mapa(smem_u32(&sh.mbox[par].cmax[rank]), lane),
                             __float_as_uint(cmax), lr_mapa(smem_u32(&sh.mbar[par]), lane));
         }
-        if (!mbar_wait_bounded(&sh.mbar[par], mpar, p.timeout_ns) && status == 0)
-          status = PARARNN_STATUS_TIMEOUT;
+        const bool got = mbar_wait_bounded(&sh.mbar[par], mpar, p.timeout_ns);
+        if (!got && status == 0) status = PARARNN_STATUS_TIMEOUT;
 #pragma unroll
         for (int r = 0; r < CLS; ++r) {
           if (r != rank) tmax = fmax_nan(tmax, sh.mbox[par].cmax[r]);
@@ -468,8 +472,10 @@ __global__ void __launch_bounds__(kLrThreads, 1)
             if (r == rank - 1) prev_cta_last = lf2(m1.z, m1.w);
           }
         }
+        // a phase that did not complete is not re-armed (see the ParaGRU
+        // row kernel)
         __syncwarp();
-        if (tid == 0) mbar_arrive_expect_tx(&sh.mbar[par], rx);
+        if (tid == 0 && got) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
       final_m = tmax;
       const bool own_ok = tmax < p.tol;

@@ -193,3 +193,31 @@ def test_nan_input_reports_nonfinite(cuda_ok, cell, wl):
     x["u"][0, 200, 0, 3] = float("nan")
     g = _gpu_adjoint(cell, x, h, c)
     assert int(g["status"][0]) == 2          # PARARNN_STATUS_NONFINITE
+
+
+@pytest.mark.parametrize("cell,wl,T,inject", [
+    (pr.PARARNN_GRU, 4, 700, 0),     # fp32 u: look-back; ticket 0 (the last chunk) withholds
+    (pr.PARARNN_GRU, 2, 1500, 2),    # bf16 u: whole sequence, cluster rank 2 withholds
+    (pr.PARARNN_LSTM, 5, 1500, 1)])
+def test_withheld_exchange_times_out(cuda_ok, cell, wl, T, inject):
+    x = make_inputs(WORKLOADS[wl].scaled(B=1, T=T, D=8 if wl != 4 else 32), with_grad=True)
+    if cell == pr.PARARNN_GRU:
+        h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+        c = None
+    else:
+        c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    d = "cuda"
+    opts = pr._opts(flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=inject,
+                    timeout_us=20000)
+    out = pr.adjoint(cell, x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d),
+                     torch.as_tensor(h, dtype=torch.float32).to(d).contiguous(), x["dLdh"].to(d),
+                     c0=(x["c0"].to(d) if c is not None else None),
+                     c=(torch.as_tensor(c, dtype=torch.float32).to(d).contiguous()
+                        if c is not None else None), opts=opts)
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 3          # PARARNN_STATUS_TIMEOUT
+    # the next call on the same device is clean
+    if cell == pr.PARARNN_GRU:
+        _check_gru(x, h)
+    else:
+        _check_lstm(x, c, h)

@@ -322,3 +322,32 @@ def test_segment_queue_capped_iterates(cuda_ok):
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=1)
     assert st["status"] == "not_converged" and st["iters"] == 1 and st["evals"] == 2
     assert np.abs(h - r["h"]).max() < TOL_STATE
+
+
+# ---- injected faults (host-set): a part of the exchange is withheld, the
+# bounded waits for it run out, the call reports TIMEOUT, and the next call
+# on the same device converges
+def test_row_kernel_withheld_mailbox_times_out(cuda_ok):
+    # one 8-channel tile of 3000 steps: a cluster of 4 CTAs exchanging maps
+    # through mailboxes; rank 1 withholds its exchange at the cap evaluation
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=3000, D=8))
+    opts = pr._opts(1e-6, 2, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=1,
+                    timeout_us=20000)
+    _, st, _ = _solve(x, opts=opts, max_iters=2)
+    assert st["status"] == "timeout", st
+    h, st2, _ = _solve(x)
+    assert st2["status"] == "converged"
+    assert np.abs(h - _ref(x)).max() < TOL_STATE
+
+
+def test_segment_queue_withheld_segment_times_out(cuda_ok):
+    # item 5 (segment 0 of tile 5) never publishes: segment 1 of tile 5
+    # waits for it until its bounded wait runs out
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=1024, D=4800))
+    opts = pr._opts(1e-6, 64, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=5,
+                    timeout_us=20000)
+    _, st, _ = _solve(x, opts=opts)
+    assert st["status"] == "timeout", st
+    h, st2, _ = _solve(x)
+    assert st2["status"] == "converged"
+    assert np.abs(h - _ref(x)).max() < TOL_STATE

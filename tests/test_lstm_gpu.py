@@ -197,3 +197,14 @@ def test_nan_input_reports_nonfinite(cuda_ok, flags):
     _, _, st, _ = _solve(x, flags=flags, max_iters=8)
     assert st["status"] == "nonfinite", st
     _check(make_inputs(WORKLOADS[3].scaled(B=1, T=900, D=32)), flags=flags)
+
+
+def test_row_kernel_withheld_mailbox_times_out(cuda_ok):
+    # one tile of 1500 steps: a cluster of 4 CTAs of 512 steps; rank 1
+    # withholds its exchange at the cap evaluation
+    x = make_inputs(WORKLOADS[3].scaled(B=1, T=1500, D=8))
+    opts = pr._opts(1e-6, 2, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=1,
+                    timeout_us=20000)
+    _, _, st, _ = _solve(x, opts=opts, max_iters=2)
+    assert st["status"] == "timeout", st
+    _check(x)
