@@ -54,6 +54,9 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal serves the four sigmoids of a step pair, one the pair's two
 #     tanh);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
+#   lstm_newton_queue (ParaLSTM, bf16 u, T <= 4096, at least one 8-channel
+#     tile per SM: every 512-step segment in one launch): the cell pass of
+#     lstm_newton_row;
 #   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096, in segments where
 #     smaller clusters fill the SMs): 5 ex2 + 1.5 rcp (one
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
@@ -78,6 +81,8 @@ def fwd_plan(w, sms=None):
     if w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms:
         return "gru_newton_queue", 4, 512
     if w.cell == "lstm":
+        if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms:
+            return "lstm_newton_queue", 6.5, 512
         if w.u_dtype == "bf16" and w.T <= 4096:
             cls, seg = 1, w.T
             while cls * 512 < w.T:
@@ -117,7 +122,8 @@ def fwd_segments(w, sms=None):
 
 def fwd_launches(w, sms=None):
     """Launches of the forward kernel per solve."""
-    return 1 if fwd_plan(w, sms)[0] == "gru_newton_queue" else len(fwd_segments(w, sms))
+    queue = fwd_plan(w, sms)[0] in ("gru_newton_queue", "lstm_newton_queue")
+    return 1 if queue else len(fwd_segments(w, sms))
 # algorithmic HBM bytes per token-channel: inputs read once, outputs written once
 def fwd_bytes(w):
     ue = 2 if w.u_dtype == "bf16" else 4

@@ -115,11 +115,10 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            products on CUDA cores (exact
                                            Newton steps, D <= 128) instead of
                                            tf32 tensor-core products */
-#define PARARNN_FLAG_FORCE_ROW 4u       /* ParaGRU with bf16 u: launch the
-                                           row kernel segment by segment
-                                           instead of the one-launch
-                                           segment-queue solve (kept for
-                                           comparison) */
+#define PARARNN_FLAG_FORCE_ROW 4u       /* bf16 u: launch the row kernel
+                                           segment by segment instead of the
+                                           one-launch segment-queue solve
+                                           (kept for comparison) */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */

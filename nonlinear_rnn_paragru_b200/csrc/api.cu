@@ -31,6 +31,8 @@ int lstm_row_cta_steps();
 int lstm_row_box_steps();
 int lstm_row_channels();
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
+int launch_lstm_queue(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
+int lstm_queue_steps();
 int adjoint_row_cluster(int T);
 int adjoint_row_channels();
 int adjoint_row_box_steps(int which);
@@ -289,6 +291,9 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.t_len = T;
   p.seg = 0;
   p.ld_h0 = D;
+  p.seg_done = reinterpret_cast<unsigned*>(ws + L.seg);
+  p.nitems = 0;
+  p.withhold_item = (p.flags & PARARNN_FLAG_INJECT_WITHHOLD) ? p.inject_chunk : -1;
 
   // Row kernels: a cluster of CTAs per 8-channel tile holds a whole sequence
   // of up to 4096 steps (ParaGRU: bf16 or fp32 u; ParaLSTM: bf16 u).  Where a
@@ -309,17 +314,22 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const bool row_lstm = cell == PARARNN_LSTM && bf16 && lstm_row_cluster(T) > 0 && !force;
   // ParaGRU with bf16 u and at least one 8-channel tile per resident CTA of
   // the segment-queue solve: all segments of all tiles in one launch
-  const bool queue_gru = row_gru && bf16 && !(opts && (opts->flags & PARARNN_FLAG_FORCE_ROW)) &&
+  const bool force_row = opts && (opts->flags & PARARNN_FLAG_FORCE_ROW);
+  const bool queue_gru = row_gru && bf16 && !force_row &&
                          tiles8 >= (long long)std::max(1, gru_queue_resident());
+  // ParaLSTM (bf16 u, T <= 4096) with at least one 8-channel tile per SM
+  // (one CTA per SM): every 512-step segment in one launch
+  const bool queue_lstm = row_lstm && !force_row && tiles8 >= sm_count();
   const size_t nch = (size_t)B * D;
   const int nhist = max_iters + 2;
-  unsigned* const seg_done = reinterpret_cast<unsigned*>(ws + L.seg);
-  const size_t nflags = queue_gru ? (size_t)tiles8
+  unsigned* const seg_done = p.seg_done;
+  const size_t nflags = (queue_gru || queue_lstm) ? (size_t)tiles8
                                   : ((row_gru || row_lstm) ? 0 : (size_t)ncc * (size_t)(max_iters + 1));
   const size_t ninit = std::max(p.chan_k ? nch : (size_t)1, nflags);
   const unsigned igrid = (unsigned)std::min<size_t>((ninit + 255) / 256, 1024);
   fwd_init_kernel<<<igrid, 256, 0, stream>>>(p.hdr, stats, p.chan_k, nch, iter_hist, nhist,
-                                             queue_gru ? seg_done : p.rec_flags, nflags);
+                                             (queue_gru || queue_lstm) ? seg_done : p.rec_flags,
+                                             nflags);
   if (cudaGetLastError() != cudaSuccess) return PARARNN_ERR_CUDA;
   int e = 0;
   if (queue_gru) {
@@ -327,6 +337,14 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
     rc = make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels());
     if (rc) return rc;
     e = launch_gru_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
+  } else if (queue_lstm) {
+    CUtensorMap rmap;
+    rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(), lstm_row_channels());
+    if (rc) return rc;
+    FwdParams pq = p;
+    pq.nitems = (int)std::min<long long>((long long)tiles8 * cdiv(T, lstm_queue_steps()),
+                                         0x7fffffffLL);
+    e = launch_lstm_queue(rmap, pq, stream);
   } else if (row_gru) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());

@@ -185,6 +185,12 @@ struct FwdParams {
   const void* u;
   int t_base, t_len, seg;
   long long ld_h0;
+  // segment-queue solves: per-tile segment counts (zero at launch), the
+  // number of (tile, segment) items, and the item that withholds its
+  // publication for testing (-1: none); the item counter is hdr->ticket
+  unsigned* seg_done;
+  int nitems;
+  int withhold_item;
 };
 
 }  // namespace pararnn

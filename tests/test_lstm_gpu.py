@@ -208,3 +208,29 @@ def test_row_kernel_withheld_mailbox_times_out(cuda_ok):
     _, _, st, _ = _solve(x, opts=opts, max_iters=2)
     assert st["status"] == "timeout", st
     _check(x)
+
+
+# ---- the segment-queue solve (bf16 u, T <= 4096, at least one 8-channel tile
+# per SM): every 512-step segment of every tile in one launch
+@pytest.mark.parametrize("B,T,D", [(1, 1300, 1200), (2, 700, 640)])
+def test_segment_queue_matches_oracle(cuda_ok, B, T, D):
+    x = make_inputs(WORKLOADS[5].scaled(B=B, T=T, D=D))
+    g = torch.Generator().manual_seed(31)
+    x["c0"] = torch.randn((B, D), generator=g)
+    x["h0"] = torch.randn((B, D), generator=g) * 0.5
+    rc, rh = _ref(x)
+    for flags in (0, pr.PARARNN_FLAG_FORCE_ROW):
+        c, h, st, hist = _solve(x, flags=flags, hist=True)
+        err = max(np.abs(c - rc).max(), np.abs(h - rh).max())
+        assert err < TOL_STATE, (flags, err, st)
+        assert st["status"] == "converged", (flags, st)
+        assert hist.sum() == B * D
+
+
+def test_segment_queue_withheld_segment_times_out(cuda_ok):
+    x = make_inputs(WORKLOADS[3].scaled(B=1, T=1024, D=1200))
+    opts = pr._opts(1e-6, 64, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=3,
+                    timeout_us=20000)
+    _, _, st, _ = _solve(x, opts=opts)
+    assert st["status"] == "timeout", st
+    _check(x)
