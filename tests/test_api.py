@@ -117,7 +117,7 @@ def test_bench_plan_follows_the_library_dispatch_rules():
     assert plan[4] == ("gru_newton_row", 4, 4096)     # T > 4096, 256 tiles >= 148
     assert plan[5] == ("lstm_newton_queue", 6.5, 512)  # 2048 tiles
     assert bench.fwd_launches(WORKLOADS[3], sms=148) == 1
-    assert bench.fwd_plan(WORKLOADS[3].scaled(B=1, D=512), sms=148) == ("lstm_newton_row", 6.5, 4096)
+    assert bench.fwd_plan(WORKLOADS[3].scaled(B=1, D=512), sms=148) == ("lstm_newton_row", 6.5, 2048)
     assert len(bench.fwd_segments(WORKLOADS[4], sms=148)) == 16
     # few tiles keep one launch over the whole sequence
     assert bench.fwd_plan(WORKLOADS[2].scaled(B=1, D=64), sms=148)[2] == 4096
