@@ -414,7 +414,46 @@ def extra_measurements(w, x, pr, fwd_ms):
                          "achieved_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
     except Exception as e:
         res["decode"] = {"error": str(e)[:300]}
+    try:
+        res["dense"] = dense_measurement(pr)
+    except Exception as e:
+        res["dense"] = {"error": str(e)[:300]}
     return res
+
+
+def dense_measurement(pr, B=1, T=1024, D=512):
+    """Dense-Jacobian DEER (the GRU with full recurrent matrices) at one size:
+    time per solve (CUDA events around whole solves, which synchronise on the
+    host every iteration) and the tensor-core contractions' algorithmic
+    FLOPs per Newton iteration: the chunk maps' tree, B*Tp*(1/2+1/4+1/8+1/16)
+    products of 2 D^3, and the pre-activations, 2 B T D 3D.  `frac` divides
+    their rate over the whole solve (a lower bound for the GEMM kernel alone)
+    by a tf32 peak: the measured bf16 GEMM peak times the nominal tf32/bf16
+    ratio (1.1 / 2.25)."""
+    import math
+    w = WORKLOADS[2].scaled(B=B, T=T, D=D)
+    x = make_inputs(w, device="cuda")
+    g = torch.Generator().manual_seed(5)
+    W = ((torch.rand((3, D, D), generator=g) * 2 - 1) * (1.5 / math.sqrt(D))).cuda()
+    ws = pr.Workspace("cuda")
+    h, st = pr.dense_gru_solve(x["u"], W, x["bias"], x["h0"], workspace=ws)
+    s = pr.read_stats(st)
+    ms = time_events(lambda: pr.dense_gru_solve(x["u"], W, x["bias"], x["h0"], workspace=ws), 3)
+    Tp = -(-T // 16) * 16
+    tree = B * Tp * (15 / 16) * 2 * D ** 3
+    pre = 2 * B * T * D * 3 * D
+    # the pre-activations run at every evaluation, the tree at every update
+    flops = s["iters"] * tree + s["evals"] * pre
+    peaks, src = measured_peaks()
+    tf32_peak = peaks["bf16_tflops"] * (1.1 / 2.25)
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"dense GRU B={B} T={T} D={D} fp32 u(bf16 values)", "ms_per_solve": round(ms, 3),
+            "iters": s["iters"], "evals": s["evals"], "status": s["status"],
+            "tensor_tflop_per_solve": round(flops / 1e12, 4),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
+                         "peak": round(tf32_peak, 1), "unit": "TFLOP/s (tf32)",
+                         "frac": round(achieved / tf32_peak, 4),
+                         "peak_source": f"bf16 {peaks['bf16_tflops']} ({src}) x 1.1/2.25"}}
 
 
 def cpu_baseline(w, seconds_hint=10.0):

@@ -242,21 +242,25 @@ __global__ void __launch_bounds__(kDnThreads) dn_chunk_maps(const DnParams p) {
   for (int i = threadIdx.x; i < D; i += blockDim.x) p.d[o + i] = xa[i];
 }
 
-// One CTA per b: the delta entering each chunk, chunk by chunk.
+// One CTA per b: the delta entering each chunk, chunk by chunk; a warp per
+// row of the chunk map, so its loads are coalesced along the row.
 __global__ void __launch_bounds__(kDnThreads) dn_carry(const DnParams p) {
   __shared__ float x[2][kDnMaxD];
   const int D = p.D, b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < D; i += blockDim.x) x[0][i] = 0.f;
   __syncthreads();
   int cur = 0;
   for (int k = 0; k < p.nC; ++k) {
     const size_t o = ((size_t)b * p.nC + k) * D;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) {
-      p.carry[o + i] = x[cur][i];
-      float s = p.d[o + i];
+    for (int i = threadIdx.x; i < D; i += blockDim.x) p.carry[o + i] = x[cur][i];
+    for (int i = warp; i < D; i += kDnThreads / 32) {
       const float* Pi = p.P + (o + i) * D;
-      for (int q = 0; q < D; ++q) s = fmaf(Pi[q], x[cur][q], s);
-      x[cur ^ 1][i] = s;
+      float s = 0.f;
+      for (int q = lane; q < D; q += 32) s = fmaf(Pi[q], x[cur][q], s);
+#pragma unroll
+      for (int sh = 16; sh > 0; sh >>= 1) s += __shfl_xor_sync(0xffffffffu, s, sh);
+      if (lane == 0) x[cur ^ 1][i] = s + p.d[o + i];
     }
     __syncthreads();
     cur ^= 1;
