@@ -141,8 +141,8 @@ __device__ __forceinline__ void ar_cell(const ArCell& k, float2 HP, float2 UZ, f
   const float2 ONE = af2(1.f, 1.f), M1 = af2(-1.f, -1.f), M2 = af2(-2.f, -2.f);
   const float2 F4 = af2(4.f, 4.f), M4 = af2(-4.f, -4.f);
   const float2 TZ = afma(k.AZ2, HP, UZ), TR = afma(k.AR2, HP, UR);
-  const float2 EZ = af2(ex2(fminf(TZ.x, 31.f)), ex2(fminf(TZ.y, 31.f)));
-  const float2 ER = af2(ex2(fminf(TR.x, 31.f)), ex2(fminf(TR.y, 31.f)));
+  const float2 EZ = af2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
+  const float2 ER = af2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
   const float2 PZ = aadd(ONE, EZ), PR = aadd(ONE, ER);
   const float2 PP = amul(PZ, PR);
   const float inv = rcp(PP.x * PP.y);
@@ -150,7 +150,7 @@ __device__ __forceinline__ void ar_cell(const ArCell& k, float2 HP, float2 UZ, f
   const float2 Z = amul(PR, INV), R = amul(PZ, INV);
   RH = amul(R, HP);
   const float2 TC = afma(k.AC2, RH, UC);
-  const float2 EC = af2(ex2(fminf(TC.x, 31.f)), ex2(fminf(TC.y, 31.f)));
+  const float2 EC = af2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));
   const float2 PC = aadd(ONE, EC);
   const float ic = rcp(PC.x * PC.y);
   const float2 TT = af2(PC.y * ic, PC.x * ic);
@@ -477,7 +477,7 @@ __device__ __forceinline__ void al_cell(const AlCell& k, float2 CP, float2 HP, f
   const float2 ONE = af2(1.f, 1.f), M1 = af2(-1.f, -1.f), M2 = af2(-2.f, -2.f);
   const float2 F4 = af2(4.f, 4.f), M4 = af2(-4.f, -4.f);
   const float2 TL = af2(2.f * kLog2e, 2.f * kLog2e);
-  auto cl = [](float2 v) { return af2(fminf(v.x, 21.f), fminf(v.y, 21.f)); };
+  auto cl = [](float2 v) { return af2(fmin_nan(v.x, 21.f), fmin_nan(v.y, 21.f)); };
   auto e2 = [](float2 v) { return af2(ex2(v.x), ex2(v.y)); };
   const float2 EI = e2(cl(afma(k.AI2, HP, UI))), EF = e2(cl(afma(k.AF2, HP, UF)));
   const float2 EO = e2(cl(afma(k.AO2, HP, UO))), EG = e2(cl(afma(k.AG2, HP, UG)));

@@ -36,6 +36,14 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
   return y;
 }
+// min that returns NaN if either operand is NaN: the clamps of exponent
+// arguments, so that a NaN input stays NaN (fminf would return the bound and
+// turn it into a saturated gate) and the solve reports it as non-finite.
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+  float y;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
 
 // ------------------------------------------------------- memory ordering --
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {

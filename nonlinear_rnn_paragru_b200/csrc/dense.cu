@@ -13,9 +13,11 @@
 //            + diag(z (1 - c^2)) [diag(r) W_c + diag((W_c h) r (1 - r)) W_r].
 // Each Newton iteration, with the host checking the residual as in the
 // unfused tier, runs (tensor-core path, the default):
-//   pre-activations  Q = h W^T for every step: a tcgen05 tf32 GEMM of the
-//                    states [B*T, D] by the stacked matrices [3D, D]
-//                    (tc_gemm.cu), W h0 once per solve;
+//   pre-activations  Q = h W^T for every step: tcgen05 GEMMs of the states
+//                    [B*T, D] by the stacked matrices [3D, D] (tc_gemm.cu) in
+//                    split tf32 (three products of hi/lo parts), so they, the
+//                    residual and the fixed point carry fp32 accuracy; W h0
+//                    once per solve;
 //   dn_assemble2     one CTA per (b, step): gates, residual, -r_t and the
 //                    block J_t to HBM, row-major at odd positions of its
 //                    16-step chunk and transposed at even ones;
@@ -29,9 +31,10 @@
 //                    delta), the delta entering each chunk chunk by chunk,
 //                    and every chunk re-run from its delta, ds added to h
 //                    (matrix-vector products, coalesced in either layout).
-// tf32 products make each Newton step inexact (about 1e-3 relative in the
-// chunk maps); the residual is evaluated in fp32, so the fixed point is that
-// of the cell and the iteration still converges, in a step or two more.  The
+// The chunk maps' tf32 products make each Newton step inexact (about 1e-3
+// relative); the residual is evaluated to fp32 accuracy, so the fixed point
+// is that of the cell and the iteration still converges, linearly near the
+// root.  The
 // CUDA-core path (fp32 products, exact steps, D <= 128) is kept for
 // comparison (PARARNN_FLAG_DENSE_SIMT): dn_pre, dn_assemble, dn_chunk_maps
 // (a D x D x D product per step in shared memory), dn_carry, dn_apply.
@@ -311,6 +314,23 @@ struct Dn2Params {
   int B, T, D, nC, Tp;
 };
 
+// x = hi + lo with hi = x with the 13 low mantissa bits cleared (exactly the
+// value a tf32 product reads) and lo = x - hi (exact in fp32).  A product
+// hi_a hi_b + hi_a lo_b + lo_a hi_b then carries the fp32 product to about
+// 2^-21 relative (the dropped lo_a lo_b and the tf32 reading of lo are below
+// it): the split-tf32 technique, used here for the pre-activations, on which
+// the residual and so the fixed point depend.
+__global__ void dn_split(const float* __restrict__ x, float* __restrict__ hi,
+                         float* __restrict__ lo, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    hi[i] = h;
+    lo[i] = v - h;
+  }
+}
+
 // W_g^T for each gate: Wt[g][j][i] = W[g][i][j]
 __global__ void dn_transpose_w(const float* __restrict__ W, float* __restrict__ Wt, int D) {
   __shared__ float tile[32][33];
@@ -338,8 +358,10 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
   const int b = (int)(bt / p.Tp), t = (int)(bt - (size_t)b * p.Tp);
   const size_t DD = (size_t)D * D;
   float* Jt = p.J + bt * DD;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (t >= p.T) {
-    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) Jt[e] = (e / D == e % D) ? 1.f : 0.f;
+    for (int i = warp; i < D; i += kDnThreads / 32)
+      for (int j = lane; j < D; j += 32) Jt[(size_t)i * D + j] = (i == j) ? 1.f : 0.f;
     for (int i = threadIdx.x; i < D; i += blockDim.x) p.rhs[bt * D + i] = 0.f;
     return;
   }
@@ -372,18 +394,25 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
     for (int w = 0; w < kDnThreads / 32; ++w) mm = max(mm, wmax[w]);
     atomicMax(p.rmax, mm);
   }
-  // J[i][j] = [i == j] (1 - z_i) + co1_i Wz[i][j] + co2_i Wc[i][j] + co3_i Wr[i][j]
-  if (t & 1) {  // row-major, element e = i * D + j
-    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) {
-      const int i = (int)(e / D), j = (int)(e - (size_t)i * D);
-      Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.W[e] + co[2][i] * p.W[2 * DD + e] +
-              co[3][i] * p.W[DD + e];
+  // J[i][j] = [i == j] (1 - z_i) + co1_i Wz[i][j] + co2_i Wc[i][j] + co3_i Wr[i][j];
+  // a warp per row of the stored layout, lanes along it (coalesced)
+  if (t & 1) {  // row-major: row i, element (i, j) at i * D + j
+    for (int i = warp; i < D; i += kDnThreads / 32) {
+      const float c0 = co[0][i], c1 = co[1][i], c2 = co[2][i], c3 = co[3][i];
+      const size_t r0 = (size_t)i * D;
+      for (int j = lane; j < D; j += 32) {
+        const size_t e = r0 + j;
+        Jt[e] = (i == j ? c0 : 0.f) + c1 * p.W[e] + c2 * p.W[2 * DD + e] + c3 * p.W[DD + e];
+      }
     }
-  } else {      // transposed, element e = j * D + i (W^T read contiguously)
-    for (size_t e = threadIdx.x; e < DD; e += blockDim.x) {
-      const int j = (int)(e / D), i = (int)(e - (size_t)j * D);
-      Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.Wt[e] + co[2][i] * p.Wt[2 * DD + e] +
-              co[3][i] * p.Wt[DD + e];
+  } else {      // transposed: row j holds column j, element (i, j) at j * D + i
+    for (int j = warp; j < D; j += kDnThreads / 32) {
+      const size_t r0 = (size_t)j * D;
+      for (int i = lane; i < D; i += 32) {
+        const size_t e = r0 + i;
+        Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.Wt[e] + co[2][i] * p.Wt[2 * DD + e] +
+                co[3][i] * p.Wt[DD + e];
+      }
     }
   }
 }
@@ -471,7 +500,7 @@ struct DnLayout {
 // tensor-core path workspace: [0, 256) residual maximum and the GEMMs' error
 // flag, then W^T, Q, W h0, the level-0 blocks, tree levels 1..4, -r, d, carry
 struct Dn2Layout {
-  size_t Wt, Q, Q0, J, lvl[kDnLevels], rhs, d, carry, total;
+  size_t Wt, Wsp, hsp, h0sp, Q, Q0, J, lvl[kDnLevels], rhs, d, carry, total;
 };
 
 Dn2Layout dn2_layout(int B, int T, int D) {
@@ -479,7 +508,10 @@ Dn2Layout dn2_layout(int B, int T, int D) {
   const size_t DD = (size_t)D * D;
   Dn2Layout L;
   L.Wt = 256;
-  L.Q = L.Wt + align256(3 * DD * 4);
+  L.Wsp = L.Wt + align256(3 * DD * 4);                       // W hi, lo
+  L.hsp = L.Wsp + 2 * align256(3 * DD * 4);                  // h hi, lo
+  L.h0sp = L.hsp + 2 * align256((size_t)B * T * D * 4);      // h0 hi, lo
+  L.Q = L.h0sp + 2 * align256((size_t)B * D * 4);
   L.Q0 = L.Q + align256((size_t)B * T * 3 * D * 4);
   L.J = L.Q0 + align256((size_t)B * 3 * D * 4);
   size_t o = L.J + align256((size_t)B * Tp * DD * 4);
@@ -555,10 +587,22 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
 
   // operand maps: the states and h0 against the stacked matrices; per tree
   // level, odd blocks (left factors) against even ones (right factors)
-  CUtensorMap mh, mh0, mw, ml[kDnLevels], mr[kDnLevels];
-  int rc = tc_operand_map(&mh, h, D, (int)BT, 1, (long long)BT * D);
-  rc |= tc_operand_map(&mw, W, D, 3 * D, 1, 3LL * DD);
-  if (h0) rc |= tc_operand_map(&mh0, h0, D, B, 1, (long long)B * D);
+  // split-tf32 operands of the pre-activations: h, W and h0 as hi + lo
+  float* Whi = reinterpret_cast<float*>(ws + L.Wsp);
+  float* Wlo = reinterpret_cast<float*>(ws + L.Wsp + align256(3 * DD * 4));
+  float* hhi = reinterpret_cast<float*>(ws + L.hsp);
+  float* hlo = reinterpret_cast<float*>(ws + L.hsp + align256(BT * D * 4));
+  float* h0hi = reinterpret_cast<float*>(ws + L.h0sp);
+  float* h0lo = reinterpret_cast<float*>(ws + L.h0sp + align256((size_t)B * D * 4));
+  CUtensorMap mhh, mhl, mh0h, mh0l, mwh, mwl, ml[kDnLevels], mr[kDnLevels];
+  int rc = tc_operand_map(&mhh, hhi, D, (int)BT, 1, (long long)BT * D);
+  rc |= tc_operand_map(&mhl, hlo, D, (int)BT, 1, (long long)BT * D);
+  rc |= tc_operand_map(&mwh, Whi, D, 3 * D, 1, 3LL * DD);
+  rc |= tc_operand_map(&mwl, Wlo, D, 3 * D, 1, 3LL * DD);
+  if (h0) {
+    rc |= tc_operand_map(&mh0h, h0hi, D, B, 1, (long long)B * D);
+    rc |= tc_operand_map(&mh0l, h0lo, D, B, 1, (long long)B * D);
+  }
   for (int l = 0; l < kDnLevels; ++l) {
     const float* in = l == 0 ? p.J : reinterpret_cast<float*>(ws + L.lvl[l - 1]);
     const int nout = nprod0 >> (l + 1);
@@ -572,11 +616,22 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
   if (e != cudaSuccess) return (int)e;
   dn_transpose_w<<<dim3((D + 31) / 32, (D + 31) / 32, 3), dim3(32, 8), 0, stream>>>(
       W, reinterpret_cast<float*>(ws + L.Wt), D);
+  const unsigned sgrid = 8 * 148;
+  dn_split<<<sgrid, 256, 0, stream>>>(W, Whi, Wlo, 3 * DD);
+  // C = A B^T to fp32 accuracy from split operands: hi hi, then + hi lo, + lo hi
+  auto split_gemm = [&](const CUtensorMap& ah, const CUtensorMap& al, float* C, int M) {
+    int r = launch_tc_gemm(ah, mwh, C, M, 3 * D, D, 1, 0, err, stream);
+    if (!r) r = launch_tc_gemm(ah, mwl, C, M, 3 * D, D, 1, 3, err, stream);
+    if (!r) r = launch_tc_gemm(al, mwh, C, M, 3 * D, D, 1, 3, err, stream);
+    return r;
+  };
   int ge = 0;
-  if (h0)
-    ge = launch_tc_gemm(mh0, mw, Q0, B, 3 * D, D, 1, 0, err, stream);
-  else
+  if (h0) {
+    dn_split<<<sgrid, 256, 0, stream>>>(h0, h0hi, h0lo, (size_t)B * D);
+    ge = split_gemm(mh0h, mh0l, Q0, B);
+  } else {
     e = cudaMemsetAsync(Q0, 0, (size_t)B * 3 * D * 4, stream);
+  }
   if (ge) return ge;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
@@ -584,7 +639,8 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
   for (int k = 0;; ++k) {
     e = cudaMemsetAsync(p.rmax, 0, sizeof(unsigned), stream);
     if (e != cudaSuccess) return (int)e;
-    ge = launch_tc_gemm(mh, mw, Q, (int)BT, 3 * D, D, 1, 0, err, stream);
+    dn_split<<<sgrid, 256, 0, stream>>>(h, hhi, hlo, BT * D);
+    ge = split_gemm(mhh, mhl, Q, (int)BT);
     if (ge) return ge;
     const unsigned nblk = (unsigned)((size_t)B * p.Tp);
     if (bf16)

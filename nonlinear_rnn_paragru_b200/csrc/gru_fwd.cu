@@ -86,8 +86,8 @@ __device__ __forceinline__ float gru_pass(const unsigned char* __restrict__ rows
     const float ht = h[i];
     // z = 1/(1+ez), r = 1/(1+er) share one reciprocal; arguments are clamped
     // so that (1+ez)(1+er) stays finite (sigmoid below 2^-63 reads as 2^-63).
-    const float ez = ex2(fminf(fmaf(az2, hp, zr.x), 63.f));
-    const float er = ex2(fminf(fmaf(ar2, hp, zr.y), 63.f));
+    const float ez = ex2(fmin_nan(fmaf(az2, hp, zr.x), 63.f));
+    const float er = ex2(fmin_nan(fmaf(ar2, hp, zr.y), 63.f));
     const float pz = 1.f + ez, pr = 1.f + er;
     const float inv = rcp(pz * pr);
     const float z = pr * inv;

@@ -69,17 +69,26 @@ struct QParams {
   int withhold_item;    // testing: this item never publishes its segment (-1: none)
 };
 
-template <int NW>
+// NW warps per CTA, L steps per thread (chunk)
+template <int NW, int L>
 struct QCfg {
   static constexpr int kThreads = NW * 32;
-  static constexpr int kSteps = NW * kRowK * kRowL;        // steps per item
-  static constexpr int kChunks = kSteps / kRowL;
-  static constexpr int kU = kChunks * kRowS;               // fp32 argument bytes
+  static constexpr int kH = L / 2;                          // step pairs per chunk
+  static constexpr int kSteps = NW * kRowK * L;             // steps per item
+  static constexpr int kChunks = kSteps / L;
+  static constexpr int kS = 3 * L * kRowC * 4 + 64;         // chunk slot
+  static constexpr int kU = kChunks * kS;                   // fp32 argument bytes
   static constexpr int kNBox = kSteps / kRowBox;
   static constexpr int kStage = kU - kNBox * kRowBoxBytes;  // bf16 staging at the top
+  static constexpr int kBlocks = kChunks * kH / kThreads;   // expansion blocks
+  static_assert(kNBox >= 1 && kSteps % kRowBox == 0, "whole TMA boxes per item");
   static_assert(kStage % 128 == 0 && kRowBoxBytes % 128 == 0, "TMA destinations");
-  static_assert(kThreads == (kChunks / 2) * kRowH, "the expansion: one (chunk, pair) per thread");
-  static_assert((kChunks / 2) * kRowS <= kStage, "in-place expansion order");
+  static_assert(kBlocks * kThreads == kChunks * kH, "the expansion: one (chunk, pair) per thread");
+  // two blocks: block 0 (the first half of the chunks) writes below every
+  // staged byte; one block reads everything before it writes anything
+  static_assert(kBlocks == 1 || (kBlocks == 2 && (kChunks / 2) * kS <= kStage),
+                "in-place expansion order");
+  static_assert(kS % 128 == 64, "a warp's four chunks in alternate 64-byte bank halves");
   static_assert(NW == 4 || NW == 8, "the CTA's residual maximum is read as float4s");
 };
 
@@ -119,16 +128,17 @@ __device__ __forceinline__ int q_draw(unsigned* counter) {
   return (int)min(atomicAdd(counter, 1u), 0x7fffffffu);
 }
 
-template <int NW>
-__global__ void __launch_bounds__(NW * 32, 16 / NW)
+template <int NW, int L, int MINB>
+__global__ void __launch_bounds__(NW * 32, MINB)
     gru_newton_queue(const __grid_constant__ CUtensorMap map, const QParams p) {
-  using Cfg = QCfg<NW>;
+  using Cfg = QCfg<NW, L>;
+  constexpr int kH = Cfg::kH;
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ QShared<NW> sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = lane % kRowC, kk = lane / kRowC;
   const int q = warp * kRowK + kk;  // chunk index within the item
-  const unsigned char* base = smem + q * kRowS;
+  const unsigned char* base = smem + q * Cfg::kS;
 
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
@@ -168,12 +178,12 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     // two blocks (each block's rows are read before any of its slots is
     // written; block 0 writes below all staging bytes)
     {
-      const int qb = tid / kRowH, i = tid % kRowH;
+      const int qb = tid / kH, i = tid % kH;
       const int sw = row_swizzle(i);
 #pragma unroll 1
-      for (int blk = 0; blk < 2; ++blk) {
-        const int qq = blk * (Cfg::kChunks / 2) + qb;
-        const int ta = qq * kRowL + i, tb = ta + kRowH;
+      for (int blk = 0; blk < Cfg::kBlocks; ++blk) {
+        const int qq = blk * (Cfg::kChunks / Cfg::kBlocks) + qb;
+        const int ta = qq * L + i, tb = ta + kH;
         const bool pa = ta >= t_len, pbd = tb >= t_len;
         float xa[3][kRowC], xb[3][kRowC];
 #pragma unroll
@@ -193,7 +203,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
           }
         }
         __syncthreads();
-        unsigned char* dst = smem + qq * kRowS + i * kRowC * 8;
+        unsigned char* dst = smem + qq * Cfg::kS + i * kRowC * 8;
 #pragma unroll
         for (int g = 0; g < 3; ++g) {
           const float sc = (g == 2) ? 2.f * kLog2e : -kLog2e;
@@ -205,7 +215,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
               if (pa) o.x = 3e30f;
               if (pbd) o.y = 3e30f;
             }
-            *reinterpret_cast<float2*>(dst + g * kRowH * kRowC * 8 + (cc ^ sw) * 8) = o;
+            *reinterpret_cast<float2*>(dst + g * kH * kRowC * 8 + (cc ^ sw) * 8) = o;
           }
         }
         __syncthreads();
@@ -251,9 +261,9 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
       }
     }
 
-    float2 H[kRowH], P[kRowH];
+    float2 H[kH], P[kH];
 #pragma unroll
-    for (int i = 0; i < kRowH; ++i) {
+    for (int i = 0; i < kH; ++i) {
       H[i] = f2(0.f, 0.f);
       P[i] = f2(1.f, 1.f);
     }
@@ -264,13 +274,13 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
       const bool cap = (k >= p.max_iters);
       const int par = phase & 1;
       ++phase;
-      const float last_pre = H[kRowH - 1].y;
+      const float last_pre = H[kH - 1].y;
       float2 DL, PA;
       float m;
       if (cap)
-        m = row_pass<false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+        m = row_pass<kH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else
-        m = row_pass<true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+        m = row_pass<kH, true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       if (!dval) m = 0.f;
       // the chunk's map: second half after the first
       float IP = PA.y * PA.x, Id = fmaf(PA.y, DL.x, DL.y);
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
       hb = first ? h0v : prev_last + din;
       const float2 DIN = f2(din, fmaf(PA.x, din, DL.x));
 #pragma unroll
-      for (int i = 0; i < kRowH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
+      for (int i = 0; i < kH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
       updates = k + 1;
       if (own_ok) break;
     }
@@ -356,16 +366,16 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
     const int it_len = min(Cfg::kSteps, p.T - it_base);
     bool bad = false;
     if (id < p.D) {
-      const int tq = q * kRowL;
+      const int tq = q * L;
       float* out = p.h + ((size_t)ib * p.T + it_base + tq) * p.D + id;
 #pragma unroll
-      for (int i = 0; i < kRowH; ++i) {
+      for (int i = 0; i < kH; ++i) {
         if (tq + i < it_len) {
           out[(size_t)i * p.D] = H[i].x;
           bad |= !isfinite(H[i].x);
         }
-        if (tq + kRowH + i < it_len) {
-          out[(size_t)(kRowH + i) * p.D] = H[i].y;
+        if (tq + kH + i < it_len) {
+          out[(size_t)(kH + i) * p.D] = H[i].y;
           bad |= !isfinite(H[i].y);
         }
       }
@@ -390,32 +400,32 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW)
   if (lane == 0 && st) atomicMax(&p.stats->status, st);
 }
 
-template <int NW>
-int launch_queue_t(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
-  using Cfg = QCfg<NW>;
-  auto kern = gru_newton_queue<NW>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kU);
+// the configuration the library runs: 4 warps per CTA, 16-step chunks
+// (256-step segments), at least 5 CTAs per SM
+constexpr int kQW = 4, kQL = 16, kQMinB = 5;
+using QRun = QCfg<kQW, kQL>;
+
+int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
+  auto kern = gru_newton_queue<kQW, kQL, kQMinB>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QRun::kU);
   if (e != cudaSuccess) return (int)e;
   int dev = 0, sms = 148, per_sm = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Cfg::kThreads, Cfg::kU) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QRun::kThreads, QRun::kU) !=
           cudaSuccess ||
       per_sm < 1)
     per_sm = 1;
   cudaGetLastError();
   // persistent: every CTA resident at once (the queue's progress argument)
   const long long grid = std::min<long long>((long long)sms * per_sm, p.nitems);
-  kern<<<(unsigned)std::max<long long>(grid, 1), Cfg::kThreads, Cfg::kU, stream>>>(map, p);
+  kern<<<(unsigned)std::max<long long>(grid, 1), QRun::kThreads, QRun::kU, stream>>>(map, p);
   return (int)cudaGetLastError();
 }
 
 }  // namespace
 
-// Warps per CTA of the segment-queue solve (segments of 128 * this steps).
-int gru_queue_warps() { return 4; }
-int gru_queue_steps() { return QCfg<4>::kSteps; }
+int gru_queue_steps() { return QRun::kSteps; }
 int gru_queue_channels() { return kRowC; }
 int gru_queue_box_steps() { return kRowBox; }
 
@@ -425,11 +435,11 @@ int gru_queue_resident() {
   int dev = 0, sms = 148, per_sm = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  auto kern = gru_newton_queue<4>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<4>::kU) !=
+  auto kern = gru_newton_queue<kQW, kQL, kQMinB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QRun::kU) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QCfg<4>::kThreads,
-                                                    QCfg<4>::kU) != cudaSuccess)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, QRun::kThreads, QRun::kU) !=
+          cudaSuccess)
     per_sm = 0;
   cudaGetLastError();
   return sms * per_sm;
@@ -450,7 +460,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.D = f.D;
   p.nDTc = (f.D + kRowC - 1) / kRowC;
   p.ntiles = f.B * p.nDTc;
-  p.nseg = (f.T + QCfg<4>::kSteps - 1) / QCfg<4>::kSteps;
+  p.nseg = (f.T + QRun::kSteps - 1) / QRun::kSteps;
   if ((long long)p.ntiles * p.nseg >= (1LL << 31)) return 1;
   p.nitems = p.ntiles * p.nseg;
   p.max_iters = f.max_iters;
@@ -461,7 +471,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.chan_k = f.chan_k;
   p.stats = f.stats;
   p.withhold_item = (f.flags & PARARNN_FLAG_INJECT_WITHHOLD) ? f.inject_chunk : -1;
-  return launch_queue_t<4>(map, p, stream);
+  return launch_queue(map, p, stream);
 }
 
 }  // namespace pararnn

@@ -346,9 +346,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       float2 DL, PA;
       float m;
       if (cap)
-        m = row_pass<false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+        m = row_pass<kRowH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else
-        m = row_pass<true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+        m = row_pass<kRowH, true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       if (!dval) m = 0.f;
       // the chunk's map: second half after the first
       float IP = PA.y * PA.x, Id = fmaf(PA.y, DL.x, DL.y);

@@ -28,15 +28,15 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(
 // channel slot of channel c in pair row i is c ^ row_swizzle(i)
 __host__ __device__ constexpr int row_swizzle(int i) { return (i >> 1) & 7; }
 
-// One pass over a chunk: H[i] = (h_i, h_{i+16}) is the iterate, hb the state
+// One pass over a chunk of 2 kH steps: H[i] = (h_i, h_{i+kH}) is the iterate, hb the state
 // before the chunk.  With kFull the two half-chunks are scanned from a zero
 // incoming delta: H becomes the local solution, P the running products, and
 // DL / PA the halves' (delta out, product).  Returns max |h_t - f_t|.
 // AZ2, AR2, AC2: the h coefficients of the three arguments (-log2e a_z,
 // -log2e a_r, 2 log2e a_c); AZ = a_z.
-template <bool kFull>
+template <int kH, bool kFull>
 __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base, int c8, float hb,
-                                          float2 (&H)[kRowH], float2 (&P)[kRowH], float2 AZ2,
+                                          float2 (&H)[kH], float2 (&P)[kH], float2 AZ2,
                                           float2 AR2, float2 AC2, float2 AZ, float2& DLo,
                                           float2& PAo) {
   const float2 ONE = f2(1.f, 1.f), M1 = f2(-1.f, -1.f), M2 = f2(-2.f, -2.f);
@@ -45,21 +45,21 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
   const float2 TL = f2(2.f * kRowLn2, 2.f * kRowLn2), MTL = f2(-2.f * kRowLn2, -2.f * kRowLn2);
   float m = 0.f;
   float2 DL = f2(0.f, 0.f), PA = ONE;
-  float2 HP = f2(hb, H[kRowH - 1].x);  // states before steps 0 and 16
+  float2 HP = f2(hb, H[kH - 1].x);  // states before steps 0 and 16
 #pragma unroll
-  for (int i = 0; i < kRowH; ++i) {
+  for (int i = 0; i < kH; ++i) {
     const unsigned char* bi = base + ((c8 ^ (row_swizzle(i) * 8)) + i * kRowC * 8);
     const float2 UZ = *reinterpret_cast<const float2*>(bi);
-    const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kRowH * kRowC * 8);
-    const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kRowH * kRowC * 8);
+    const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kH * kRowC * 8);
+    const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kH * kRowC * 8);
     const float2 HT = H[i];
     // z, r = 1/(1+e) with e = 2^(argument).  One reciprocal serves the four
     // sigmoids of the pair and one the two tanh: every argument is clamped
     // at 31, so the product of four (1+e) stays below 2^124 (the clamp moves
     // a sigmoid or tanh by under 1e-9).
     const float2 TZ = ffma2(AZ2, HP, UZ), TR = ffma2(AR2, HP, UR);
-    const float2 EZ = f2(ex2(fminf(TZ.x, 31.f)), ex2(fminf(TZ.y, 31.f)));
-    const float2 ER = f2(ex2(fminf(TR.x, 31.f)), ex2(fminf(TR.y, 31.f)));
+    const float2 EZ = f2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
+    const float2 ER = f2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
     const float2 PZ = fadd2(ONE, EZ), PR = fadd2(ONE, ER);
     const float2 PP = fmul2(PZ, PR);
     const float inv = rcp(PP.x * PP.y);
@@ -67,7 +67,7 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
     const float2 Z = fmul2(PR, INV), R = fmul2(PZ, INV);
     const float2 RH = fmul2(R, HP);
     const float2 TC = ffma2(AC2, RH, UC);
-    const float2 EC = f2(ex2(fminf(TC.x, 31.f)), ex2(fminf(TC.y, 31.f)));  // e^{2y}
+    const float2 EC = f2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));  // e^{2y}
     const float2 PC = fadd2(ONE, EC);
     const float ic = rcp(PC.x * PC.y);
     const float2 TT = f2(PC.y * ic, PC.x * ic);             // t = 1/(1+e^{2y})

@@ -84,9 +84,9 @@ __device__ __forceinline__ float lstm_pass(const unsigned char* __restrict__ row
     const float ct = c[s], ht = h[s];
     // sigmoids of i, f, o share one reciprocal (arguments clamped so the
     // product of the three denominators stays finite)
-    const float ei = ex2(fminf(fmaf(k.ai2, hp, uu.x), 40.f));
-    const float ef = ex2(fminf(fmaf(k.af2, hp, uu.y), 40.f));
-    const float eo = ex2(fminf(fmaf(k.ao2, hp, uu.w), 40.f));
+    const float ei = ex2(fmin_nan(fmaf(k.ai2, hp, uu.x), 40.f));
+    const float ef = ex2(fmin_nan(fmaf(k.af2, hp, uu.y), 40.f));
+    const float eo = ex2(fmin_nan(fmaf(k.ao2, hp, uu.w), 40.f));
     const float eg = ex2(fmaf(k.ag2, hp, uu.z));
     const float pi = 1.f + ei, pf = 1.f + ef, po = 1.f + eo;
     const float pfo = pf * po;

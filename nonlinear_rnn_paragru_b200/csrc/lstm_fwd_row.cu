@@ -105,7 +105,7 @@ __device__ __forceinline__ float2 lfma(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 lmul(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 ladd(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 lclamp(float2 a, float hi) {
-  return lf2(fminf(a.x, hi), fminf(a.y, hi));
+  return lf2(fmin_nan(a.x, hi), fmin_nan(a.y, hi));
 }
 __device__ __forceinline__ float2 lex2(float2 a) { return lf2(ex2(a.x), ex2(a.y)); }
 __device__ __forceinline__ int lr_swizzle(int i) { return i >> 1; }

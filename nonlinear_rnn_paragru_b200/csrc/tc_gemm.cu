@@ -54,7 +54,8 @@ struct TcParams {
   float* C;
   int M, N, K, Z;
   int store_mode;  // 0: C[z] row-major M x N; 1: C[z] transposed (N x M);
-                   // 2: row-major for odd z, transposed for even z
+                   // 2: row-major for odd z, transposed for even z;
+                   // 3: C[z] row-major, the product added to what C holds
   int* err;        // set to 1 by a CTA whose wait ran out
 };
 
@@ -199,6 +200,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const int col = n0 + c0 + j;
             if (col < p.N) Cz[(size_t)col * p.M + row] = __uint_as_float(r[j]);
           }
+        } else if (p.store_mode == 3) {
+          float* dst = Cz + (size_t)row * p.N + n0 + c0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (n0 + c0 + j < p.N) dst[j] += __uint_as_float(r[j]);
         } else {
           float* dst = Cz + (size_t)row * p.N + n0 + c0;
           if (n0 + c0 + 32 <= p.N && (p.N & 3) == 0) {
