@@ -228,7 +228,17 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * opts->inject_chunk (the tile's chunks take tickets last first) publishes
  * no records; in the whole-sequence adjoint (bf16 u, T <= 4096) the CTA of
  * cluster rank opts->inject_chunk withholds its map in its cluster's last
- * tile.  Other opts fields are ignored.  NULL opts = pararnn_adjoint. */
+ * tile; in the ParaGRU queue adjoint item opts->inject_chunk (r * tiles +
+ * tile for the segment r from the end) never publishes its carry.  With
+ * PARARNN_FLAG_FORCE_ROW in opts->flags the whole-sequence kernels run where
+ * the queue adjoint would.  Other opts fields are ignored.  NULL opts =
+ * pararnn_adjoint.
+ * Kernels: ParaGRU with bf16 u and at least one 8-channel tile per resident
+ * CTA of the queue adjoint (4 per SM) takes the queue adjoint (every 256-step
+ * segment of every tile in one launch, last segments first, each segment's
+ * carry from the segment after it); other bf16 problems with T <= 4096 the
+ * whole-sequence kernels (a cluster of CTAs per tile); the rest the chunked
+ * look-back adjoint. */
 int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a,
                        const float* bias, const float* c0, const float* h0,
                        const float* c, const float* h, const float* dLdh,

@@ -37,6 +37,7 @@
 
 #include <algorithm>
 
+#include "adjoint_cell.cuh"
 #include "common.cuh"
 #include "lookback.cuh"
 
@@ -46,28 +47,13 @@ namespace cga = cooperative_groups;
 
 constexpr int kArThreads = 256;
 constexpr int kArWarps = 8;
-constexpr int kArC = 8;                       // channels per tile
-constexpr int kArK = 32 / kArC;               // chunks per warp
-constexpr int kArL = 16;                      // steps per chunk
-constexpr int kArH = kArL / 2;                // step pairs per chunk
 constexpr int kArSteps = kArWarps * kArK * kArL;  // 512 steps per CTA
 constexpr int kArChunks = kArSteps / kArL;        // 32
-constexpr int kArUStep = 3 * kArC * 2;        // 48 bytes per step of u
-constexpr int kArSStep = kArC * 4;            // 32 bytes per step of h or dL/dh
-constexpr int kArUBox = kArL + kArK - 1;      // 19 steps
-constexpr int kArHBox = kArL + kArK;          // 20 steps (one more: h_{t-1})
-constexpr int kArGBox = kArL + kArK - 1;      // 19 steps
-constexpr int kArUOff = 0, kArHOff = 1024, kArGOff = 1664;
-constexpr int kArS = 2304;                    // chunk slot
 constexpr int kArSmem = kArChunks * kArS;     // 73728
 constexpr int kArMaxCluster = 8;
 constexpr int kArTmax = kArSteps * kArMaxCluster;  // 4096
 constexpr unsigned kArTileBytes =
     kArChunks * (kArUBox * kArUStep + kArHBox * kArSStep + kArGBox * kArSStep);
-static_assert(kArUBox * kArUStep <= kArHOff && kArHOff + kArHBox * kArSStep <= kArGOff &&
-                  kArGOff + kArGBox * kArSStep <= kArS && kArS % 128 == 0 &&
-                  kArHOff % 128 == 0 && kArGOff % 128 == 0,
-              "chunk slot layout");
 static_assert(kArWarps == kArC, "one scan row per channel");
 // mailbox ring: slots used round robin by tile, a cluster barrier every
 // kArSyncEvery tiles (see the tile loop)
@@ -83,10 +69,6 @@ struct ArShared {
   uint64_t mbar[kArSlots];               // mailbox barriers, by slot
 };
 
-__device__ __forceinline__ float2 af2(float x, float y) { return make_float2(x, y); }
-__device__ __forceinline__ float2 afma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-__device__ __forceinline__ float2 amul(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 aadd(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 __device__ __forceinline__ uint32_t ar_mapa(uint32_t addr, int rank) {
   uint32_t r;
@@ -123,50 +105,6 @@ struct ArParams {
                       // cluster's last tile (-1: none)
 };
 
-// affine map x -> P x + d, as float2 (P, d); (f o g)(x) = f(g(x))
-__device__ __forceinline__ float2 ar_after(float2 f, float2 g) {
-  return af2(f.x * g.x, fmaf(f.x, g.y, f.y));
-}
-
-struct ArCell {
-  float2 AZ2, AR2, AC2, AZ, AR, AC;  // scaled (argument) and raw weights, both lanes
-};
-
-// The cell at a step pair: from the previous state HP and the pre-scaled
-// arguments UZ, UR, UC, the Jacobian A = df/dh and the pieces
-// GZ = df/du_z, GR = df/du_r, GC = df/du_c, RH = r h.
-__device__ __forceinline__ void ar_cell(const ArCell& k, float2 HP, float2 UZ, float2 UR,
-                                        float2 UC, float2& A, float2& GZ, float2& GR,
-                                        float2& GC, float2& RH) {
-  const float2 ONE = af2(1.f, 1.f), M1 = af2(-1.f, -1.f), M2 = af2(-2.f, -2.f);
-  const float2 F4 = af2(4.f, 4.f), M4 = af2(-4.f, -4.f);
-  const float2 TZ = afma(k.AZ2, HP, UZ), TR = afma(k.AR2, HP, UR);
-  const float2 EZ = af2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
-  const float2 ER = af2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
-  const float2 PZ = aadd(ONE, EZ), PR = aadd(ONE, ER);
-  const float2 PP = amul(PZ, PR);
-  const float inv = rcp(PP.x * PP.y);
-  const float2 INV = af2(PP.y * inv, PP.x * inv);
-  const float2 Z = amul(PR, INV), R = amul(PZ, INV);
-  RH = amul(R, HP);
-  const float2 TC = afma(k.AC2, RH, UC);
-  const float2 EC = af2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));
-  const float2 PC = aadd(ONE, EC);
-  const float ic = rcp(PC.x * PC.y);
-  const float2 TT = af2(PC.y * ic, PC.x * ic);
-  const float2 C = afma(M2, TT, ONE);                 // tanh
-  const float2 CMH = afma(HP, M1, C);
-  const float2 OMZ = afma(Z, M1, ONE);
-  const float2 ZZ = amul(Z, OMZ);                     // z(1-z)
-  const float2 RR = amul(R, afma(R, M1, ONE));        // r(1-r)
-  GZ = amul(CMH, ZZ);                                 // (c-h) z(1-z)
-  GC = amul(Z, amul(TT, afma(TT, M4, F4)));           // z (1-c^2)
-  const float2 GCA = amul(GC, k.AC);
-  GR = amul(GCA, amul(HP, RR));                       // z(1-c^2) a_c h r(1-r)
-  const float2 Q = afma(amul(k.AR, HP), RR, R);       // r + a_r h r(1-r)
-  A = afma(GCA, Q, afma(amul(k.AZ, ZZ), CMH, OMZ));
-}
-
 // Warp 0: the tile's boxes (u, h_{t-1}, dL/dh per chunk; lane q issues
 // chunk q's three) and its a, bias, h0 rows, all on `bar`.
 __device__ __forceinline__ void ar_issue(unsigned char* smem, ArShared& sh,
@@ -191,20 +129,6 @@ __device__ __forceinline__ void ar_issue(unsigned char* smem, ArShared& sh,
   tma_load_4d(slot + kArUOff, mu, &sh.bar, d0, 0, ts, b);
   tma_load_3d(slot + kArHOff, mh, &sh.bar, d0, ts - 1, b);
   tma_load_3d(slot + kArGOff, mg, &sh.bar, d0, ts, b);
-}
-
-// pre-scaled arguments of a step pair: -log2e u_z + b'_z, ... from bf16 rows
-__device__ __forceinline__ void ar_args(const unsigned char* ux, const unsigned char* uy, float2 S,
-                                        float2 BZ, float2 BR, float2 BC, float2& UZ, float2& UR,
-                                        float2& UC) {
-  const unsigned short* rx = reinterpret_cast<const unsigned short*>(ux);
-  const unsigned short* ry = reinterpret_cast<const unsigned short*>(uy);
-  const float2 SC = af2(2.f * kLog2e, 2.f * kLog2e);
-  UZ = afma(S, af2(__uint_as_float((unsigned)rx[0] << 16), __uint_as_float((unsigned)ry[0] << 16)), BZ);
-  UR = afma(S, af2(__uint_as_float((unsigned)rx[kArC] << 16),
-                   __uint_as_float((unsigned)ry[kArC] << 16)), BR);
-  UC = afma(SC, af2(__uint_as_float((unsigned)rx[2 * kArC] << 16),
-                    __uint_as_float((unsigned)ry[2 * kArC] << 16)), BC);
 }
 
 template <int CLS>
@@ -829,6 +753,13 @@ __global__ void adjoint_row_reduce(const float* __restrict__ part, float* da, fl
 }
 
 __global__ void adjoint_row_init(int* status) { *status = 0; }
+
+// da, dbias from per-(tile, part) partial sums (parts: cluster ranks, or the
+// segments of the queue adjoint), in a fixed order
+void adjoint_row_reduce_launch(const float* part, float* da, float* dbias, int B, int D, int cls,
+                               int G, cudaStream_t stream) {
+  adjoint_row_reduce<<<(G * D * 32 + 255) / 256, 256, 0, stream>>>(part, da, dbias, B, D, cls, G);
+}
 
 int adjoint_row_cluster(int T) {
   if (T > kArTmax) return 0;

@@ -37,6 +37,12 @@ int adjoint_row_cluster(int T);
 int adjoint_row_channels();
 int adjoint_row_box_steps(int which);
 size_t adjoint_row_part_bytes(int G, int B, int T, int D);
+size_t adjoint_queue_bytes(int B, int T, int D);
+int adjoint_queue_resident();
+int launch_adjoint_queue(const CUtensorMap* maps, const float* a, const float* bias,
+                         const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
+                         int T, int D, int* status, void* ws, uint64_t timeout_ns,
+                         int withhold_item, cudaStream_t stream);
 int launch_adjoint_row(const CUtensorMap* maps, const float* a, const float* bias,
                        const float* h0, float* du, float* da, float* dbias, float* dh0, int B,
                        int T, int D, int* status, void* ws, uint64_t timeout_ns,
@@ -471,6 +477,23 @@ int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, con
     return PARARNN_ERR_MISALIGNED;
   if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const int G = cell == PARARNN_GRU ? 3 : 4;
+  const bool force_row = opts && (opts->flags & PARARNN_FLAG_FORCE_ROW);
+  // ParaGRU, bf16 projections, at least one 8-channel tile per resident CTA
+  // of the queue adjoint: every 256-step segment in one launch, last first
+  if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && !force_row &&
+      (long long)B * ((D + 7) / 8) >= (long long)std::max(1, adjoint_queue_resident()) &&
+      kWsHeaderBytes + adjoint_queue_bytes(B, T, D) <= ws_bytes) {
+    const int ch = adjoint_row_channels();
+    CUtensorMap qmaps[3];  // u, h (states before each step), dL/dh
+    rc = make_u_map(&qmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
+    if (!rc) rc = make_s_map(&qmaps[1], h, B, T, D, adjoint_row_box_steps(1), ch);
+    if (!rc) rc = make_s_map(&qmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+    if (rc) return rc;
+    const int e = launch_adjoint_queue(qmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status,
+                                       static_cast<unsigned char*>(workspace) + kWsHeaderBytes,
+                                       timeout_ns, inject_chunk, (cudaStream_t)stream);
+    return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
+  }
   // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
   // 8-channel tile holds the whole sequence (no look-back)
   if (u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&

@@ -221,3 +221,48 @@ def test_withheld_exchange_times_out(cuda_ok, cell, wl, T, inject):
         _check_gru(x, h)
     else:
         _check_lstm(x, c, h)
+
+
+# ---- the ParaGRU queue adjoint (bf16 u, at least one 8-channel tile per
+# resident CTA: 4 x 148 = 592 on a B200): every 256-step segment in one
+# launch, last segments first, each segment's carry from the one after it
+@pytest.mark.parametrize("B,T,D", [(1, 700, 4800), (2, 1300, 2400), (1, 256, 4800)])
+def test_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
+    x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
+    x["h0"] = torch.randn((B, D), generator=torch.Generator().manual_seed(37)) * 0.5
+    h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+    _check_gru(x, h)
+    # and the whole-sequence kernel on the same inputs
+    d = "cuda"
+    hh = torch.as_tensor(h, dtype=torch.float32).to(d).contiguous()
+    q = pr.adjoint(pr.PARARNN_GRU, x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d),
+                   hh, x["dLdh"].to(d))
+    r = pr.adjoint(pr.PARARNN_GRU, x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d),
+                   hh, x["dLdh"].to(d), opts=pr._opts(flags=pr.PARARNN_FLAG_FORCE_ROW))
+    torch.cuda.synchronize()
+    for k in ("du", "da", "dbias", "dh0"):
+        assert _rel(q[k].cpu().numpy(), r[k].cpu().numpy()) <= TOL_GRAD, k
+
+
+def test_queue_adjoint_is_bitwise_reproducible(cuda_ok):
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=900, D=4800))
+    h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+    a = _gpu_adjoint(pr.PARARNN_GRU, x, h)
+    b = _gpu_adjoint(pr.PARARNN_GRU, x, h)
+    for k in ("du", "da", "dbias", "dh0"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_queue_adjoint_withheld_carry_times_out(cuda_ok):
+    # item 5 (the last segment of tile 5) never publishes its carry: the
+    # segment before it waits until its bounded wait runs out
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=600, D=4800))
+    h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+    d = "cuda"
+    opts = pr._opts(flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=5, timeout_us=20000)
+    out = pr.adjoint(pr.PARARNN_GRU, x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d),
+                     torch.as_tensor(h, dtype=torch.float32).to(d).contiguous(), x["dLdh"].to(d),
+                     opts=opts)
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 3
+    _check_gru(x, h)
