@@ -47,7 +47,7 @@ NCU_TRAFFIC_BYTES = {
 # The forward kernel a workload runs and its special-function (MUFU)
 # operations per element and cell evaluation, as the kernel issues them:
 #   gru_newton_queue (ParaGRU with bf16 u and at least one 8-channel tile per
-#     resident CTA, five CTAs per SM: every 256-step segment of every tile in
+#     resident CTA, four CTAs per SM: every 512-step segment of every tile in
 #     one launch): the cell pass of gru_newton_row, 3 ex2 + 1 rcp;
 #   gru_newton_row (ParaGRU with T <= 4096, or longer with at least one
 #     8-channel tile per SM, then in 4096-step segments): 3 ex2 + 1 rcp (one
@@ -62,13 +62,13 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
-QUEUE_CTAS_PER_SM = 5   # residency of gru_newton_queue (96 registers, 27 KB smem)
+QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue (128 registers, 53 KB smem)
 
 
 def fwd_plan(w, sms=None):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
     as the library dispatches it: the segment-queue kernels solve every
-    256-step (ParaGRU) or 512-step (ParaLSTM) segment of a problem with bf16 u and at least one
+    512-step segment of a problem with bf16 u and at least one
     8-channel tile per resident CTA in one launch; otherwise the row kernels
     solve a sequence in segments of k x 1024 (ParaGRU, two CTAs per SM) or
     k x 512 steps (ParaLSTM, one CTA per SM), one launch each, k the smallest
@@ -79,7 +79,7 @@ def fwd_plan(w, sms=None):
         sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles8 = w.B * ((w.D + 7) // 8)
     if w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms:
-        return "gru_newton_queue", 4, 256
+        return "gru_newton_queue", 4, 512
     if w.cell == "lstm":
         if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms:
             return "lstm_newton_queue", 6.5, 512

@@ -400,9 +400,12 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   if (lane == 0 && st) atomicMax(&p.stats->status, st);
 }
 
-// the configuration the library runs: 4 warps per CTA, 16-step chunks
-// (256-step segments), at least 5 CTAs per SM
-constexpr int kQW = 4, kQL = 16, kQMinB = 5;
+// the configuration the library runs: 4 warps per CTA, 32-step chunks
+// (512-step segments), 4 CTAs per SM.  Measured on configuration 2 (B200,
+// CUDA events): 345 us, against 354 us for 16-step chunks at 5 CTAs per SM
+// (96 registers) and 366 us at 6 (80 registers, a few spills): more resident
+// warps did not pay for the doubled per-step scan work
+constexpr int kQW = 4, kQL = 32, kQMinB = 4;
 using QRun = QCfg<kQW, kQL>;
 
 int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {

@@ -10,10 +10,6 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
-    config.addinivalue_line(
-        "markers",
-        "gpu_pending: GPU parity tests of code that has not yet run on a B200; not "
-        "selected by -m gpu until they have passed there (run them with -m gpu_pending)")
 
 
 @pytest.fixture(scope="session")

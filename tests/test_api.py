@@ -108,7 +108,7 @@ def test_bench_plan_follows_the_library_dispatch_rules():
     from nonlinear_rnn_paragru_b200.inputs import WORKLOADS
     plan = {k: bench.fwd_plan(w, sms=148) for k, w in WORKLOADS.items()}
     assert plan[1] == ("gru_newton_row", 4, 256)      # 8 tiles: one launch
-    assert plan[2] == ("gru_newton_queue", 4, 256)    # 1024 tiles >= 5 x 148 resident CTAs
+    assert plan[2] == ("gru_newton_queue", 4, 512)    # 1024 tiles >= 4 x 148 resident CTAs
     assert bench.fwd_launches(WORKLOADS[2], sms=148) == 1
     # fewer tiles than resident queue CTAs: the row kernel, launch by segment
     assert bench.fwd_plan(WORKLOADS[2].scaled(B=2), sms=148) == ("gru_newton_row", 4, 2048)

@@ -286,7 +286,7 @@ def test_nan_input_reports_nonfinite(cuda_ok, flags):
 
 
 # ---- the segment-queue solve (bf16 u, at least one 8-channel tile per
-# resident CTA: 5 x 148 = 740 on a B200): every 256-step segment of every tile
+# resident CTA: 4 x 148 = 592 on a B200): every 512-step segment of every tile
 # in one launch, each segment from the state its predecessor converged to
 @pytest.mark.parametrize("B,T,D", [(1, 1300, 6000), (2, 2100, 3000), (3, 257, 2000)])
 def test_segment_queue_matches_oracle(cuda_ok, B, T, D):
@@ -302,7 +302,7 @@ def test_segment_queue_matches_oracle(cuda_ok, B, T, D):
 
 
 def test_segment_queue_channel_index_one_segment(cuda_ok):
-    # T <= 256: one item per tile, so the per-channel index is the oracle's
+    # T <= 512: one item per tile, so the per-channel index is the oracle's
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=250, D=6000))
     ci = torch.full((1, 6000), -5, dtype=torch.int32, device="cuda")
     h, st, hist = _solve(x, hist=True, chan_iters=ci)
@@ -317,7 +317,7 @@ def test_segment_queue_channel_index_one_segment(cuda_ok):
 def test_segment_queue_capped_iterates(cuda_ok):
     # with the cap at one update, every segment returns the first Newton
     # iterate from the state its predecessor ended with
-    # (one segment: T <= 256; across segments the capped iterate of a
+    # (one segment: T <= 512; across segments the capped iterate of a
     # segment starts from its predecessor's, not from the whole-sequence
     # iterate)
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=256, D=6000))
@@ -346,7 +346,7 @@ def test_row_kernel_withheld_mailbox_times_out(cuda_ok):
 def test_segment_queue_withheld_segment_times_out(cuda_ok):
     # item 5 (segment 0 of tile 5) never publishes: segment 1 of tile 5
     # waits for it until its bounded wait runs out
-    x = make_inputs(WORKLOADS[2].scaled(B=1, T=512, D=6000))
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=1024, D=6000))
     opts = pr._opts(1e-6, 64, flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=5,
                     timeout_us=20000)
     _, st, _ = _solve(x, opts=opts)
