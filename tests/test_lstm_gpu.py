@@ -162,11 +162,51 @@ def test_channel_iteration_index_matches_oracle(cuda_ok, B, T, D, flags):
     np.testing.assert_array_equal(hist, np.bincount(k_gpu.ravel(), minlength=66))
 
 
+def _sensitivity(x, c, h):
+    """Per (b, d) channel: max_t of the row-sum norm of sum_{s<=t} prod_{s<k<=t}
+    A_k, from the oracle's fp64 2x2 Jacobians along the trajectory (c, h): a
+    per-step residual of size r moves the state of a near-fixed point by at
+    most r times this (to first order)."""
+    u = x["u"].double().numpy()
+    a, bias = x["a"].double().numpy(), x["bias"].double().numpy()
+    B, T, _, D = u.shape
+    n = B * D
+    ag = np.tile(a.T, (B, 1))
+    bg = np.tile(bias.T, (B, 1))
+    S = np.zeros((n, 2, 2))
+    best = np.zeros(n)
+    cp = np.zeros(n)
+    hp = np.zeros(n)
+    eye = np.eye(2)
+    for t in range(T):
+        ut = u[:, t].transpose(0, 2, 1).reshape(n, 4)
+        _, _, A, _, _ = oracle.lstm_step(cp, hp, ut, ag, bg)
+        S = np.einsum("nij,njk->nik", A, S) + eye
+        best = np.maximum(best, np.abs(S).sum(axis=2).max(axis=1))
+        cp, hp = c[:, t].reshape(n), h[:, t].reshape(n)
+    return best.reshape(B, D)
+
+
 def test_config5_full_size(cuda_ok):
-    # B=4, T=2048, D=4096, u ~ N(0, 4/sqrt(D)): 512-step segments on all SMs
-    st, hist = _check(make_inputs(WORKLOADS[5]), hist=True)
+    # B=4, T=2048, D=4096, u ~ N(0, 4/sqrt(D)): 512-step segments on all SMs.
+    # A few channels of this recurrence amplify a per-step perturbation by up
+    # to about 2e5 (reading 18): no fp32 trajectory matches the fp64 one to
+    # 1e-4 there.  The solve guarantees its residual; the states are held to
+    # 1e-4 where that bound allows and to the bound elsewhere.
+    x = make_inputs(WORKLOADS[5])
+    c, h, st, hist = _solve(x, hist=True)
+    assert st["status"] == "converged" and st["max_residual"] < 1e-6, st
     assert hist.sum() == 4 * 4096 and hist[-1] == 0
-    assert st["max_residual"] < 1e-6
+    resc, resh = oracle.lstm_residual(x["u"], x["a"], x["bias"], x["c0"], x["h0"],
+                                      c.astype(np.float64), h.astype(np.float64))
+    assert max(np.abs(resc).max(), np.abs(resh).max()) < 1e-6
+    rc, rh = _ref(x)
+    err = np.maximum(np.abs(c - rc).max(axis=1), np.abs(h - rh).max(axis=1))   # [B, D]
+    sens = _sensitivity(x, rc, rh)
+    bound = np.maximum(TOL_STATE, 1e-6 * sens)
+    assert (err <= bound).all(), (err.max(), float(np.argmax(err)), sens.max())
+    assert (sens <= 100).mean() > 0.95          # most channels: the plain 1e-4
+    assert (err[sens <= 100] < TOL_STATE).all()
 
 
 def test_config5_fwd_then_adjoint_end_to_end(cuda_ok):
