@@ -40,6 +40,7 @@
 // (a D x D x D product per step in shared memory), dn_carry, dn_apply.
 // Layouts: u [B][T][3][D], W [3][D][D] row-major (row i of W_g feeds unit i),
 // bias [3][D], h0 [B][D], h [B][T][D].  D <= 512.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -417,80 +418,152 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
   }
 }
 
-// y = M x + add over a CTA (M D x D in global memory, row-major or
-// transposed; x, y in shared memory); ends with a CTA barrier.
-__device__ __forceinline__ void dn_matvec(const float* __restrict__ M, bool rowmajor,
-                                          const float* x, const float* __restrict__ add, float* y,
-                                          int D) {
-  if (rowmajor) {  // a warp per row: coalesced along the row
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = warp; i < D; i += kDnThreads / 32) {
+// ---- the sequential passes, a cluster of CL CTAs per chain: CTA rank r owns
+// the rows [r R, r R + R) of every matrix-vector product (R = D / CL), keeps the
+// whole vector x in its shared memory, and sends its rows of the next x to
+// every CTA of the cluster (distributed shared memory) before one cluster
+// barrier per step.  Each chain reads its D x D matrices with CL SMs' worth
+// of loads in flight instead of one.
+namespace cgd = cooperative_groups;
+
+struct DnVec {
+  float x[2][kDnMaxD];       // the vector, double-buffered by step parity
+  float part[2 * kDnMaxD];   // transposed layout: partial sums of the q groups, [qg][row]
+};
+
+// y[i] = sum_q M[i][q] x[q] + add[i] for this CTA's rows i in [r0, r0 + R),
+// M row-major or stored transposed (M[q][i]); the result goes to x_next of
+// every CTA of the cluster.  Ends with the cluster barrier.
+__device__ __forceinline__ void dn_cmatvec(cgd::cluster_group& cl, DnVec& v, int cur,
+                                           const float* __restrict__ M, bool rowmajor,
+                                           const float* __restrict__ add, int D, int r0, int R,
+                                           float* __restrict__ yout) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* x = v.x[cur];
+  float* y_local = v.x[cur ^ 1];
+  const int ncl = (int)cl.num_blocks();
+  if (rowmajor) {  // a warp per row, lanes along it
+    for (int ii = warp; ii < R; ii += kDnThreads / 32) {
+      const int i = r0 + ii;
       const float* Mi = M + (size_t)i * D;
       float s = 0.f;
       for (int q = lane; q < D; q += 32) s = fmaf(Mi[q], x[q], s);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) y[i] = s + (add ? add[i] : 0.f);
+      if (lane == 0) {
+        s += add ? add[i] : 0.f;
+        for (int r = 0; r < ncl; ++r) cl.map_shared_rank(y_local, r)[i] = s;
+        if (yout) yout[i] = s;
+      }
     }
-  } else {         // M[q][i] = (the matrix)[i][q]: a thread per output, coalesced along q rows
-    for (int i = threadIdx.x; i < D; i += kDnThreads) {
+  } else {  // threads over (row offset, quarter of q): rows contiguous in M[q][.]
+    const int nq = kDnThreads / R >= 4 ? 4 : (kDnThreads / R >= 2 ? 2 : 1);
+    const int qlen = (D + nq - 1) / nq;
+    for (int e = threadIdx.x; e < R * nq; e += kDnThreads) {
+      const int ii = e % R, qg = e / R;
+      const int i = r0 + ii;
+      const int q0 = qg * qlen, q1 = min(D, q0 + qlen);
+      float s = 0.f;
+      for (int q = q0; q < q1; ++q) s = fmaf(M[(size_t)q * D + i], x[q], s);
+      v.part[qg * R + ii] = s;
+    }
+    __syncthreads();
+    for (int ii = threadIdx.x; ii < R; ii += kDnThreads) {
+      const int i = r0 + ii;
       float s = add ? add[i] : 0.f;
-      for (int q = 0; q < D; ++q) s = fmaf(M[(size_t)q * D + i], x[q], s);
-      y[i] = s;
+      for (int qg = 0; qg < nq; ++qg) s += v.part[qg * R + ii];
+      for (int r = 0; r < ncl; ++r) cl.map_shared_rank(y_local, r)[i] = s;
+      if (yout) yout[i] = s;
     }
   }
-  __syncthreads();
+  cl.sync();
 }
 
-// One CTA per (b, chunk): the chunk's recurrence from a zero delta; its last
-// delta is the chunk's offset d.
+// One cluster per (b, chunk): the chunk's recurrence from a zero delta; its
+// last delta is the chunk's offset d.
 __global__ void __launch_bounds__(kDnThreads) dn_offsets(const Dn2Params p) {
-  __shared__ float xs[2][kDnMaxD];
-  const int D = p.D;
-  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = 0.f;
-  __syncthreads();
+  __shared__ DnVec v;
+  cgd::cluster_group cl = cgd::this_cluster();
+  const int D = p.D, ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int R = D / ncl, r0 = rank * R;
+  const int chain = blockIdx.x / ncl;
+  const int b = chain / p.nC, k = chain - b * p.nC;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) v.x[0][i] = 0.f;
+  cl.sync();
   int cur = 0;
   for (int pp = 0; pp < kDnChunk; ++pp) {
     const size_t bt = (size_t)b * p.Tp + (size_t)k * kDnChunk + pp;
-    dn_matvec(p.J + bt * D * D, (pp & 1) != 0, xs[cur], p.rhs + bt * D, xs[cur ^ 1], D);
+    const bool last = pp == kDnChunk - 1;
+    dn_cmatvec(cl, v, cur, p.J + bt * D * D, (pp & 1) != 0, p.rhs + bt * D, D, r0, R,
+               last ? p.d + (size_t)chain * D : nullptr);
     cur ^= 1;
   }
-  for (int i = threadIdx.x; i < D; i += blockDim.x) p.d[(size_t)blockIdx.x * D + i] = xs[cur][i];
 }
 
-// One CTA per b: the delta entering each chunk, chunk by chunk (x <- P_k x + d_k).
+// One cluster per b: the delta entering each chunk, chunk by chunk
+// (x <- P_k x + d_k).
 __global__ void __launch_bounds__(kDnThreads) dn_carry2(const Dn2Params p) {
-  __shared__ float xs[2][kDnMaxD];
-  const int D = p.D, b = blockIdx.x;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = 0.f;
-  __syncthreads();
+  __shared__ DnVec v;
+  cgd::cluster_group cl = cgd::this_cluster();
+  const int D = p.D, ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int R = D / ncl, r0 = rank * R;
+  const int b = blockIdx.x / ncl;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) v.x[0][i] = 0.f;
+  cl.sync();
   int cur = 0;
   for (int k = 0; k < p.nC; ++k) {
     const size_t o = (size_t)b * p.nC + k;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) p.carry[o * D + i] = xs[cur][i];
-    dn_matvec(p.P + o * D * D, true, xs[cur], p.d + o * D, xs[cur ^ 1], D);
+    for (int ii = threadIdx.x; ii < R; ii += blockDim.x) p.carry[o * D + r0 + ii] = v.x[cur][r0 + ii];
+    dn_cmatvec(cl, v, cur, p.P + o * D * D, true, p.d + o * D, D, r0, R, nullptr);
     cur ^= 1;
   }
 }
 
-// One CTA per (b, chunk): the chunk re-run from its delta; ds added to h.
+// One cluster per (b, chunk): the chunk re-run from its delta; ds added to h.
 __global__ void __launch_bounds__(kDnThreads) dn_apply2(const Dn2Params p) {
-  __shared__ float xs[2][kDnMaxD];
-  const int D = p.D;
-  const int b = blockIdx.x / p.nC, k = blockIdx.x - b * p.nC;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) xs[0][i] = p.carry[(size_t)blockIdx.x * D + i];
-  __syncthreads();
+  __shared__ DnVec v;
+  cgd::cluster_group cl = cgd::this_cluster();
+  const int D = p.D, ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
+  const int R = D / ncl, r0 = rank * R;
+  const int chain = blockIdx.x / ncl;
+  const int b = chain / p.nC, k = chain - b * p.nC;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) v.x[0][i] = p.carry[(size_t)chain * D + i];
+  cl.sync();
   int cur = 0;
   for (int pp = 0; pp < kDnChunk; ++pp) {
     const int t = k * kDnChunk + pp;
-    if (t >= p.T) break;
+    if (t >= p.T) break;  // the same for every CTA of the cluster
     const size_t bt = (size_t)b * p.Tp + t;
-    dn_matvec(p.J + bt * D * D, (pp & 1) != 0, xs[cur], p.rhs + bt * D, xs[cur ^ 1], D);
+    dn_cmatvec(cl, v, cur, p.J + bt * D * D, (pp & 1) != 0, p.rhs + bt * D, D, r0, R, nullptr);
     cur ^= 1;
-    for (int i = threadIdx.x; i < D; i += blockDim.x)
-      p.h[((size_t)b * p.T + t) * D + i] += xs[cur][i];
+    for (int ii = threadIdx.x; ii < R; ii += blockDim.x)
+      p.h[((size_t)b * p.T + t) * D + r0 + ii] += v.x[cur][r0 + ii];
   }
+}
+
+// CTAs per chain of the sequential passes: D / 64, from 1 to 8, dividing D
+int dn_cluster(int D) {
+  for (int c = 8; c > 1; c /= 2)
+    if (D % (8 * c) == 0 && D / c >= 64) return c;
+  return 1;
+}
+
+template <class K>
+cudaError_t dn_launch_cluster(K kern, unsigned chains, int D, const Dn2Params& p,
+                              cudaStream_t stream) {
+  const int cl = dn_cluster(D);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(chains * (unsigned)cl);
+  cfg.blockDim = dim3(kDnThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 struct DnLayout {
@@ -677,10 +750,10 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
       if (ge) return ge;
     }
     const unsigned nmaps = (unsigned)((size_t)B * p.nC);
-    dn_offsets<<<nmaps, kDnThreads, 0, stream>>>(p);
-    dn_carry2<<<(unsigned)B, kDnThreads, 0, stream>>>(p);
-    dn_apply2<<<nmaps, kDnThreads, 0, stream>>>(p);
-    e = cudaGetLastError();
+    e = dn_launch_cluster(dn_offsets, nmaps, D, p, stream);
+    if (e == cudaSuccess) e = dn_launch_cluster(dn_carry2, (unsigned)B, D, p, stream);
+    if (e == cudaSuccess) e = dn_launch_cluster(dn_apply2, nmaps, D, p, stream);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
     st.iters = k + 1;
     if (r < tol) break;  // the update of the first certified iteration is applied
