@@ -204,7 +204,9 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.001):
+        # a 1 ms period: a timed region of 20 steps of under 1 ms still
+        # carries several samples (one NVML query takes well under 1 ms)
         self.index, self.period = index, period
         self.mhz, self.reasons = [], set()
         self.max_mhz = None
