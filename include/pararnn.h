@@ -234,11 +234,14 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * the queue adjoint would.  Other opts fields are ignored.  NULL opts =
  * pararnn_adjoint.
  * Kernels: ParaGRU with bf16 u and at least one 8-channel tile per resident
- * CTA of the queue adjoint (4 per SM) takes the queue adjoint (every 256-step
+ * CTA of the queue adjoint (5 per SM) takes the queue adjoint (every 256-step
  * segment of every tile in one launch, last segments first, each segment's
  * carry from the segment after it); other bf16 problems with T <= 4096 the
  * whole-sequence kernels (a cluster of CTAs per tile); the rest the chunked
- * look-back adjoint. */
+ * look-back adjoint.  The first two stage the rows of a, bias, h0 and c0 by
+ * 1-D bulk copies and are taken only when those pointers are 16-byte aligned
+ * (4-byte aligned rows take the look-back adjoint: same results within
+ * rounding, slower). */
 int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a,
                        const float* bias, const float* c0, const float* h0,
                        const float* c, const float* h, const float* dLdh,

@@ -12,23 +12,28 @@
 // numbered so that every tile's last segment comes first (item = r * ntiles +
 // tile for the segment r from the end) and drawn from a counter one ahead.
 // A CTA of 4 warps holds a segment (lane = (chunk k = lane / 8, channel c =
-// lane % 8), 16 steps per thread, the cell of adjoint_cell.cuh):
+// lane % 8), 16 steps per thread, the cell of adjoint_cell.cuh); every warp
+// stages its own four chunks and its own copy of the tile's parameters on its
+// own mbarrier, and loads the next item's as soon as its pass 2 is done:
 //   pass 1: each chunk's map carry_in -> carry_out, backwards;
 //   scan: a suffix scan over the warp's four chunks by shuffles, and over the
-//     warps from shared memory after one CTA barrier;
-//   carry: the first chunk's threads wait (bounded acquire poll) for the
-//     segment after this one to publish the carry entering this segment's
-//     last step, then publish the carry this segment passes to the segment
-//     before it (its map applied to that carry) -- before pass 2, so the
+//     warps from shared memory after one CTA barrier (the only one per item);
+//   carry: a segment publishes the carry it passes to the segment before it
+//     as one 64-bit word per channel (the value's bits and the count of
+//     segments published from the end), so that a single relaxed load, issued
+//     when the item starts and checked after pass 1 (a bounded poll if it is
+//     not there yet), brings both; the word is written before pass 2, so the
 //     chain of segments advances one map application per segment;
 //   pass 2: the exact recurrence from the true carry, du written and da /
-//     dbias partials summed per item (reduced afterwards in a fixed order,
-//     bitwise reproducible).
-// The lowest-numbered item that is not done is always being worked on and
-// never waits, so the queue cannot deadlock while all CTAs are resident; a
-// wait that runs out sets TIMEOUT.  Four CTAs share an SM (one tile's boxes in
-// flight each), against two CTAs of 8 warps in clusters exchanging maps every
-// tile for the whole-sequence kernel.
+//     dbias partial sums kept per warp, summed over the warps in a fixed order
+//     after the next item's barrier (reduced over the items afterwards in a
+//     fixed order: bitwise reproducible).
+// The lowest-numbered item that has not published is always being worked on
+// and never waits, so the queue cannot deadlock while all CTAs are resident;
+// a wait that runs out sets TIMEOUT.  Five CTAs share an SM (92 registers a
+// thread, 40 KB of shared memory a CTA; 251 us against 274 us with four for
+// B=8 T=4096 D=1024), against two CTAs of 8 warps in clusters exchanging maps
+// every tile for the whole-sequence kernel.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -46,14 +51,15 @@ constexpr int kAqThreads = kAqWarps * 32;
 constexpr int kAqChunks = kAqWarps * kArK;        // 16
 constexpr int kAqSteps = kAqChunks * kArL;        // 256 steps per item
 constexpr int kAqSmem = kAqChunks * kArS;         // 36864
-constexpr unsigned kAqTileBytes =
-    kAqChunks * (kArUBox * kArUStep + kArHBox * kArSStep + kArGBox * kArSStep);
+constexpr unsigned kAqWarpBytes =
+    kArK * (kArUBox * kArUStep + kArHBox * kArSStep + kArGBox * kArSStep);
 
 struct AqParams {
   const float *a, *bias, *h0;
   float *du, *dh0, *part;
-  float* carry;        // [ntiles][8]: the carry a segment passes to the one before it
-  unsigned* done;      // [ntiles]: segments published from the end (zero at launch)
+  // [ntiles][8]: the carry a segment passes to the one before it, as
+  // (float bits) | (segments published from the end of the tile) << 32
+  unsigned long long* carry;
   unsigned* counter;   // item tickets (zero at launch)
   int B, T, D, nDTc, ntiles, nseg, nitems;
   uint64_t timeout_ns;
@@ -62,12 +68,12 @@ struct AqParams {
 };
 
 struct AqShared {
-  float2 wagg[kAqWarps][kArC];  // per (warp, channel) suffix map of the warp
-  float red[kAqWarps][6][kArC]; // partial sums per warp
-  float par[7][kArC];           // a (3 rows), bias (3 rows), h0 of the item's channels
-  float cin[kArC];              // carry entering the item's last step, per channel
-  uint64_t bar;
-  int nx[2];                    // this and the next item, by parity
+  uint64_t bar[kAqWarps];           // per warp: its chunks' boxes and parameters
+  float par[kAqWarps][7][kArC];     // per warp: a (3 rows), bias (3 rows), h0
+  float2 wagg[2][kAqWarps][kArC];   // by item parity: per (warp, channel) suffix map
+  float red[2][kAqWarps][6][kArC];  // by item parity: partial sums per warp
+  float cin[2][kArC];               // by item parity: carry entering the last step
+  int nx[2];                        // the item after this one, by parity
 };
 
 __device__ __forceinline__ void aq_bulk(void* dst, const void* src, unsigned bytes,
@@ -77,31 +83,42 @@ __device__ __forceinline__ void aq_bulk(void* dst, const void* src, unsigned byt
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ unsigned long long aq_ld_word(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void aq_st_word(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
-// Warp 0: the item's boxes (u, h_{t-1}, dL/dh per chunk; lane q issues chunk
-// q's three) and its a, bias, h0 rows, all on `bar`.
+// Warp `warp`: its four chunks' boxes (u, h_{t-1}, dL/dh; lane k issues chunk
+// k's three) and its copy of the a, bias, h0 rows of the item at (b, d0, t0),
+// all on the warp's mbarrier.  The rows are 16-byte aligned (the caller
+// checks the pointers; d0 is a multiple of 8 and D of 8).
 __device__ __forceinline__ void aq_issue(unsigned char* smem, AqShared& sh,
                                          const CUtensorMap* mu, const CUtensorMap* mh,
-                                         const CUtensorMap* mg, const AqParams& p, int b,
-                                         int d0, int t0, int lane) {
+                                         const CUtensorMap* mg, const AqParams& p, int warp,
+                                         int b, int d0, int t0, int lane) {
   const unsigned pb = kArC * 4;
+  uint64_t* bar = &sh.bar[warp];
   if (lane == 0) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(&sh.bar, kAqTileBytes + 3 * pb + (p.bias ? 3 * pb : 0) +
-                                       (p.h0 ? pb : 0));
-    for (int g = 0; g < 3; ++g) {
-      aq_bulk(&sh.par[g][0], p.a + (size_t)g * p.D + d0, pb, &sh.bar);
-      if (p.bias) aq_bulk(&sh.par[3 + g][0], p.bias + (size_t)g * p.D + d0, pb, &sh.bar);
-    }
-    if (p.h0) aq_bulk(&sh.par[6][0], p.h0 + (size_t)b * p.D + d0, pb, &sh.bar);
+    mbar_arrive_expect_tx(bar, kAqWarpBytes + 3 * pb + (p.bias ? 3 * pb : 0) + (p.h0 ? pb : 0));
   }
   __syncwarp();
-  if (lane < kAqChunks) {
-    const int q = lane, k = q % kArK, ts = t0 + q * kArL - k;
+  if (lane < kArK) {
+    const int q = warp * kArK + lane, ts = t0 + q * kArL - lane;
     unsigned char* slot = smem + q * kArS;
-    tma_load_4d(slot + kArUOff, mu, &sh.bar, d0, 0, ts, b);
-    tma_load_3d(slot + kArHOff, mh, &sh.bar, d0, ts - 1, b);
-    tma_load_3d(slot + kArGOff, mg, &sh.bar, d0, ts, b);
+    tma_load_4d(slot + kArUOff, mu, bar, d0, 0, ts, b);
+    tma_load_3d(slot + kArHOff, mh, bar, d0, ts - 1, b);
+    tma_load_3d(slot + kArGOff, mg, bar, d0, ts, b);
+  } else if (lane < kArK + 3) {
+    const int g = lane - kArK;
+    aq_bulk(&sh.par[warp][g][0], p.a + (size_t)g * p.D + d0, pb, bar);
+    if (p.bias) aq_bulk(&sh.par[warp][3 + g][0], p.bias + (size_t)g * p.D + d0, pb, bar);
+  } else if (lane == kArK + 3 && p.h0) {
+    aq_bulk(&sh.par[warp][6][0], p.h0 + (size_t)b * p.D + d0, pb, bar);
   }
 }
 
@@ -109,7 +126,7 @@ __device__ __forceinline__ int aq_draw(unsigned* counter) {
   return (int)min(atomicAdd(counter, 1u), 0x7fffffffu);
 }
 
-__global__ void __launch_bounds__(kAqThreads, 4)
+__global__ void __launch_bounds__(kAqThreads, 5)
     adjoint_queue(const __grid_constant__ CUtensorMap mu, const __grid_constant__ CUtensorMap mh,
                   const __grid_constant__ CUtensorMap mg, const AqParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -118,37 +135,50 @@ __global__ void __launch_bounds__(kAqThreads, 4)
   const int c = lane % kArC, kk = lane / kArC;
   const int q = warp * kArK + kk;
 
-  if (tid < 7 * kArC) (&sh.par[0][0])[tid] = 0.f;
-  if (tid == 0) {
-    mbar_init(&sh.bar, 1);
-    sh.nx[0] = aq_draw(p.counter);
-  }
+  for (int i = tid; i < kAqWarps * 7 * kArC; i += kAqThreads) (&sh.par[0][0][0])[i] = 0.f;
+  if (tid < kAqWarps) mbar_init(&sh.bar[tid], 1);
+  if (tid == 0) sh.nx[0] = aq_draw(p.counter);
   __syncthreads();
   int item = sh.nx[0];
-  if (warp == 0 && item < p.nitems) {
+  if (item < p.nitems) {
     const int tile = item % p.ntiles, seg = p.nseg - 1 - item / p.ntiles;
-    aq_issue(smem, sh, &mu, &mh, &mg, p, tile / p.nDTc, (tile % p.nDTc) * kArC, seg * kAqSteps,
-             lane);
+    aq_issue(smem, sh, &mu, &mh, &mg, p, warp, tile / p.nDTc, (tile % p.nDTc) * kArC,
+             seg * kAqSteps, lane);
   }
   const unsigned char* slot = smem + q * kArS;
   const unsigned char* ubase = slot + kArUOff + kk * kArUStep + c * 2;
   const float* hbase = reinterpret_cast<const float*>(slot + kArHOff + kk * kArSStep) + c;
   const float* gbase = reinterpret_cast<const float*>(slot + kArGOff + kk * kArSStep) + c;
+  const float* pw = &sh.par[warp][0][0] + c;
   int status = 0;
-  for (int n = 0; item < p.nitems; ++n) {
-    if (tid == 0) sh.nx[(n + 1) & 1] = aq_draw(p.counter);
+  int n = 0, prev_part = -1;  // prev_part: the partial-sum row of the item before
+  bool live = true;           // false once a wait for this warp's boxes ran out
+  int fail_par = 0;
+  for (; item < p.nitems; ++n) {
+    const int par = n & 1;
+    if (tid == 0) sh.nx[par ^ 1] = aq_draw(p.counter);
     const int tile = item % p.ntiles, r = item / p.ntiles, seg = p.nseg - 1 - r;
     const int b = tile / p.nDTc, d0 = (tile % p.nDTc) * kArC;
     const int d = d0 + c;
     const bool dval = d < p.D;
     const int t0 = seg * kAqSteps;
     const bool first = (seg == 0 && q == 0);  // the chunk holding step 0
-    if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
+    // the carry word of the segment after this one, fetched now, read after pass 1
+    unsigned long long cword = 0ull;
+    if (tid < kArC && r > 0) cword = aq_ld_word(&p.carry[(size_t)tile * kArC + c]);
+    if (live) {
+      // a phase that did not complete is never re-armed: the warp stops loading
+      if (!__all_sync(kAqFull, mbar_wait_bounded(&sh.bar[warp], (unsigned)par, p.timeout_ns))) {
+        live = false;
+        fail_par = par;
+        status = PARARNN_STATUS_TIMEOUT;
+      }
+    }
     ArCell k;
     float2 S, BZ, BR, BC;
     float h0v;
     {
-      const float az = sh.par[0][c], ar = sh.par[1][c], ac = sh.par[2][c];
+      const float az = pw[0 * kArC], ar = pw[1 * kArC], ac = pw[2 * kArC];
       k.AZ = af2(az, az);
       k.AR = af2(ar, ar);
       k.AC = af2(ac, ac);
@@ -157,12 +187,12 @@ __global__ void __launch_bounds__(kAqThreads, 4)
       k.AR2 = af2(ar2, ar2);
       k.AC2 = af2(ac2, ac2);
       S = af2(-kLog2e, -kLog2e);
-      const float bz = -kLog2e * sh.par[3][c], br = -kLog2e * sh.par[4][c],
-                  bc = 2.f * kLog2e * sh.par[5][c];
+      const float bz = -kLog2e * pw[3 * kArC], br = -kLog2e * pw[4 * kArC],
+                  bc = 2.f * kLog2e * pw[5 * kArC];
       BZ = af2(bz, bz);
       BR = af2(br, br);
       BC = af2(bc, bc);
-      h0v = sh.par[6][c];
+      h0v = pw[6 * kArC];
     }
 
     // ---- pass 1: the two half-chunk maps, backwards
@@ -189,43 +219,49 @@ __global__ void __launch_bounds__(kAqThreads, 4)
     // the carry entering the warp -> the carry entering this chunk
     float2 xm = af2(__shfl_down_sync(kAqFull, inc.x, kArC), __shfl_down_sync(kAqFull, inc.y, kArC));
     if (kk == kArK - 1) xm = af2(1.f, 0.f);
-    if (kk == 0) sh.wagg[warp][c] = inc;
+    if (kk == 0) sh.wagg[par][warp][c] = inc;
     // the carry entering this segment's last step: zero for the last segment,
-    // else published by the segment after it
+    // else the word the segment after it published (count r)
     if (tid < kArC) {
       float cin = 0.f;
       if (r > 0) {
-        const unsigned* f = &p.done[tile];
-        if (ld_acquire(f) < (unsigned)r) {
+        if ((unsigned)(cword >> 32) < (unsigned)r) {
           const uint64_t w0 = globaltimer_ns();
-          while (ld_acquire(f) < (unsigned)r) {
+          do {
+            cword = aq_ld_word(&p.carry[(size_t)tile * kArC + c]);
+            if ((unsigned)(cword >> 32) >= (unsigned)r) break;
             if (globaltimer_ns() - w0 > p.timeout_ns) {
               status = PARARNN_STATUS_TIMEOUT;
               break;
             }
-          }
+          } while (true);
         }
-        cin = __ldcg(&p.carry[(size_t)tile * kArC + c]);
+        cin = __uint_as_float((unsigned)cword);
       }
-      sh.cin[c] = cin;
+      sh.cin[par][c] = cin;
     }
     __syncthreads();
+    // every warp is done with the item before: its partial sums, in warp order
+    if (prev_part >= 0 && tid < 6 * kArC) {
+      const int j = tid / kArC, cc = tid % kArC;
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kAqWarps; ++w) s += sh.red[par ^ 1][w][j][cc];
+      p.part[(size_t)prev_part * (6 * kArC) + tid] = s;
+    }
     // the warps after this one: the segment's incoming carry -> this warp's
     float2 cw = af2(1.f, 0.f);
 #pragma unroll
     for (int w = kAqWarps - 1; w > 0; --w)
-      if (w > warp) cw = ar_after(sh.wagg[w][c], cw);
-    const float cin_seg = sh.cin[c];
+      if (w > warp) cw = ar_after(sh.wagg[par][w][c], cw);
+    const float cin_seg = sh.cin[par][c];
     // publish the carry this segment passes to the one before it: its map
     // (the warp-0 chunk-0 suffix after the other warps) applied to cin_seg
-    if (warp == 0 && kk == 0) {
+    if (warp == 0 && kk == 0 && item != p.withhold_item) {
       const float2 m = ar_after(inc, cw);
-      if (item != p.withhold_item) {
-        p.carry[(size_t)tile * kArC + c] = fmaf(m.x, cin_seg, m.y);
-        __threadfence();
-      }
-      __syncwarp(0xffu);
-      if (lane == 0 && item != p.withhold_item) st_release(&p.done[tile], (unsigned)r + 1u);
+      aq_st_word(&p.carry[(size_t)tile * kArC + c],
+                 (unsigned long long)__float_as_uint(fmaf(m.x, cin_seg, m.y)) |
+                     ((unsigned long long)(r + 1) << 32));
     }
     const float cwarp = fmaf(cw.x, cin_seg, cw.y);
     const float cchunk = fmaf(xm.x, cwarp, xm.y);
@@ -271,8 +307,15 @@ __global__ void __launch_bounds__(kAqThreads, 4)
       }
     }
     if (first && dval && p.dh0) p.dh0[(size_t)b * p.D + d] = CARRY.x;
-    // partial sums of the item: over the two halves, the warp's chunks, then
-    // the warps in order
+    // this warp's slots and parameters are free: the next item's
+    const int next = sh.nx[par ^ 1];
+    __syncwarp();
+    if (live && next < p.nitems) {
+      const int nt = next % p.ntiles, ns = p.nseg - 1 - next / p.ntiles;
+      aq_issue(smem, sh, &mu, &mh, &mg, p, warp, nt / p.nDTc, (nt % p.nDTc) * kArC,
+               ns * kAqSteps, lane);
+    }
+    // the warp's partial sums: over the two halves, then the warp's chunks
     float v[6] = {SAZ.x + SAZ.y, SAR.x + SAR.y, SAC.x + SAC.y,
                   SBZ.x + SBZ.y, SBR.x + SBR.y, SBC.x + SBC.y};
 #pragma unroll
@@ -283,36 +326,34 @@ __global__ void __launch_bounds__(kAqThreads, 4)
     }
     if (kk == 0)
 #pragma unroll
-      for (int j = 0; j < 6; ++j) sh.red[warp][j][c] = v[j];
+      for (int j = 0; j < 6; ++j) sh.red[par][warp][j][c] = v[j];
     if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
-    __syncthreads();
-    // every pass of this item is done: the slots take the next item
-    const int next = sh.nx[(n + 1) & 1];
-    if (warp == 0 && next < p.nitems) {
-      const int nt = next % p.ntiles, ns = p.nseg - 1 - next / p.ntiles;
-      aq_issue(smem, sh, &mu, &mh, &mg, p, nt / p.nDTc, (nt % p.nDTc) * kArC, ns * kAqSteps,
-               lane);
-    }
-    if (tid < 6 * kArC) {
-      const int j = tid / kArC, cc = tid % kArC;
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kAqWarps; ++w) s += sh.red[w][j][cc];
-      p.part[((size_t)tile * p.nseg + seg) * (6 * kArC) + tid] = s;
-    }
+    prev_part = tile * p.nseg + seg;
     item = next;
   }
+  // the last item's partial sums
+  __syncthreads();
+  if (prev_part >= 0 && tid < 6 * kArC) {
+    const int j = tid / kArC, cc = tid % kArC;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAqWarps; ++w) s += sh.red[(n - 1) & 1][w][j][cc];
+    p.part[(size_t)prev_part * (6 * kArC) + tid] = s;
+  }
+  // copies still in flight into this warp's slots: wait for them (bounded)
+  if (!live) mbar_wait_bounded(&sh.bar[warp], (unsigned)fail_par, p.timeout_ns);
   const int st = __reduce_max_sync(kAqFull, status);
   if (lane == 0 && st) atomicMax(p.status, st);
 }
 
-__global__ void adjoint_queue_init(int* status, unsigned* counter, unsigned* done, int ntiles) {
+__global__ void adjoint_queue_init(int* status, unsigned* counter, unsigned long long* carry,
+                                   int nwords) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i == 0) {
     *status = 0;
     *counter = 0u;
   }
-  for (int j = i; j < ntiles; j += gridDim.x * blockDim.x) done[j] = 0u;
+  for (int j = i; j < nwords; j += gridDim.x * blockDim.x) carry[j] = 0ull;
 }
 
 }  // namespace
@@ -326,8 +367,7 @@ int adjoint_queue_steps() { return kAqSteps; }
 size_t adjoint_queue_bytes(int B, int T, int D) {
   const size_t ntiles = (size_t)B * ((D + kArC - 1) / kArC);
   const size_t nseg = (size_t)(T + kAqSteps - 1) / kAqSteps;
-  return align256(ntiles * nseg * 6 * kArC * 4) + align256(ntiles * kArC * 4) +
-         align256(ntiles * 4) + 256;
+  return align256(ntiles * nseg * 6 * kArC * 4) + align256(ntiles * kArC * 8) + 256;
 }
 
 // Resident CTAs of the queue adjoint on the current device.
@@ -370,13 +410,12 @@ int launch_adjoint_queue(const CUtensorMap* maps, const float* a, const float* b
   unsigned char* w = static_cast<unsigned char*>(ws);
   p.part = reinterpret_cast<float*>(w);
   w += align256((size_t)p.nitems * 6 * kArC * 4);
-  p.carry = reinterpret_cast<float*>(w);
-  w += align256((size_t)p.ntiles * kArC * 4);
-  p.done = reinterpret_cast<unsigned*>(w);
-  w += align256((size_t)p.ntiles * 4);
+  p.carry = reinterpret_cast<unsigned long long*>(w);
+  w += align256((size_t)p.ntiles * kArC * 8);
   p.counter = reinterpret_cast<unsigned*>(w);
-  adjoint_queue_init<<<(unsigned)std::min(1024, (p.ntiles + 255) / 256 + 1), 256, 0, stream>>>(
-      status, p.counter, p.done, p.ntiles);
+  const int nwords = p.ntiles * kArC;
+  adjoint_queue_init<<<(unsigned)std::min(1024, (nwords + 255) / 256 + 1), 256, 0, stream>>>(
+      status, p.counter, p.carry, nwords);
   cudaError_t e = cudaFuncSetAttribute(adjoint_queue, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kAqSmem);
   if (e != cudaSuccess) return (int)e;

@@ -478,9 +478,13 @@ int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, con
   if (ws_bytes < adjoint_ws_bytes(cell, B, T, D)) return PARARNN_ERR_WORKSPACE_TOO_SMALL;
   const int G = cell == PARARNN_GRU ? 3 : 4;
   const bool force_row = opts && (opts->flags & PARARNN_FLAG_FORCE_ROW);
+  // the queue and whole-sequence kernels stage each tile's rows of a, bias,
+  // h0 (c0) with 1-D bulk copies, which take 16-byte aligned addresses only
+  const bool rows16 = aligned(a, 16) && (!bias || aligned(bias, 16)) &&
+                      (!h0 || aligned(h0, 16)) && (!c0 || aligned(c0, 16));
   // ParaGRU, bf16 projections, at least one 8-channel tile per resident CTA
   // of the queue adjoint: every 256-step segment in one launch, last first
-  if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && !force_row &&
+  if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && !force_row && rows16 &&
       (long long)B * ((D + 7) / 8) >= (long long)std::max(1, adjoint_queue_resident()) &&
       kWsHeaderBytes + adjoint_queue_bytes(B, T, D) <= ws_bytes) {
     const int ch = adjoint_row_channels();
@@ -496,7 +500,7 @@ int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, con
   }
   // bf16 projections, sequences of up to 4096 steps: a cluster of CTAs per
   // 8-channel tile holds the whole sequence (no look-back)
-  if (u_dtype == PARARNN_BF16 && adjoint_row_cluster(T) > 0 &&
+  if (u_dtype == PARARNN_BF16 && rows16 && adjoint_row_cluster(T) > 0 &&
       kWsHeaderBytes + adjoint_row_part_bytes(G, B, T, D) <= ws_bytes) {
     const int ch = adjoint_row_channels();
     CUtensorMap rmaps[4];

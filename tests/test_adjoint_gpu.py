@@ -224,9 +224,9 @@ def test_withheld_exchange_times_out(cuda_ok, cell, wl, T, inject):
 
 
 # ---- the ParaGRU queue adjoint (bf16 u, at least one 8-channel tile per
-# resident CTA: 4 x 148 = 592 on a B200): every 256-step segment in one
+# resident CTA: 5 x 148 = 740 on a B200): every 256-step segment in one
 # launch, last segments first, each segment's carry from the one after it
-@pytest.mark.parametrize("B,T,D", [(1, 700, 4800), (2, 1300, 2400), (1, 256, 4800)])
+@pytest.mark.parametrize("B,T,D", [(1, 700, 6000), (2, 1300, 3000), (1, 256, 6000)])
 def test_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
     x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
     x["h0"] = torch.randn((B, D), generator=torch.Generator().manual_seed(37)) * 0.5
@@ -245,7 +245,7 @@ def test_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
 
 
 def test_queue_adjoint_is_bitwise_reproducible(cuda_ok):
-    x = make_inputs(WORKLOADS[2].scaled(B=1, T=900, D=4800))
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=900, D=6000))
     h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
     a = _gpu_adjoint(pr.PARARNN_GRU, x, h)
     b = _gpu_adjoint(pr.PARARNN_GRU, x, h)
@@ -256,7 +256,7 @@ def test_queue_adjoint_is_bitwise_reproducible(cuda_ok):
 def test_queue_adjoint_withheld_carry_times_out(cuda_ok):
     # item 5 (the last segment of tile 5) never publishes its carry: the
     # segment before it waits until its bounded wait runs out
-    x = make_inputs(WORKLOADS[2].scaled(B=1, T=600, D=4800))
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=600, D=6000))
     h = oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
     d = "cuda"
     opts = pr._opts(flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=5, timeout_us=20000)
@@ -266,3 +266,50 @@ def test_queue_adjoint_withheld_carry_times_out(cuda_ok):
     torch.cuda.synchronize()
     assert int(out["status"][0]) == 3
     _check_gru(x, h)
+
+
+def _offset_view(t, d="cuda"):
+    # the same values one float past a 16-byte boundary (4-byte aligned only)
+    buf = torch.empty(t.numel() + 4, dtype=t.dtype, device=d)
+    v = buf[1:1 + t.numel()].view(t.shape)
+    v.copy_(t.to(d))
+    assert v.data_ptr() % 16 == 4
+    return v
+
+
+@pytest.mark.parametrize("cell,B,T,D", [(pr.PARARNN_GRU, 1, 700, 6000),
+                                        (pr.PARARNN_GRU, 2, 1000, 64),
+                                        (pr.PARARNN_LSTM, 1, 700, 48)])
+def test_adjoint_rows_4byte_aligned(cuda_ok, cell, B, T, D):
+    # rows of a, bias, h0 (c0) that are 4-byte but not 16-byte aligned cannot
+    # be staged by bulk copies: the call takes the look-back adjoint, whose
+    # gradients match BPTT and the aligned call's
+    lstm = cell == pr.PARARNN_LSTM
+    x = make_inputs(WORKLOADS[3 if lstm else 2].scaled(B=B, T=T, D=D), with_grad=True)
+    d = "cuda"
+    if lstm:
+        c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+        ref = oracle.lstm_bptt(x["u"], x["a"], x["bias"], x["c0"], x["h0"],
+                               c.astype(np.float32).astype(np.float64),
+                               h.astype(np.float32).astype(np.float64), x["dLdh"])
+        keys = ("du", "da", "dbias", "dh0", "dc0")
+    else:
+        c, h = None, oracle.gru_seq(x["u"], x["a"], x["bias"], x["h0"])
+        ref = oracle.gru_bptt(x["u"], x["a"], x["bias"], x["h0"],
+                              h.astype(np.float32).astype(np.float64), x["dLdh"])
+        keys = ("du", "da", "dbias", "dh0")
+    hh = torch.as_tensor(h, dtype=torch.float32).to(d).contiguous()
+    cc = torch.as_tensor(c, dtype=torch.float32).to(d).contiguous() if lstm else None
+    outs = []
+    for shift in (False, True):
+        prep = _offset_view if shift else (lambda t: t.to(d))
+        outs.append(pr.adjoint(cell, x["u"].to(d), prep(x["a"]), prep(x["bias"]),
+                               prep(x["h0"]), hh, x["dLdh"].to(d),
+                               c0=prep(x["c0"]) if lstm else None, c=cc))
+    torch.cuda.synchronize()
+    for o in outs:
+        assert int(o["status"][0]) == 0
+        for k in keys:
+            assert _rel(o[k].cpu().numpy(), ref[k]) <= TOL_GRAD, k
+    for k in keys:
+        assert _rel(outs[1][k].cpu().numpy(), outs[0][k].cpu().numpy()) <= TOL_GRAD, k
