@@ -36,6 +36,12 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
   return y;
 }
+// the same over three operands, in one instruction
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
 // min that returns NaN if either operand is NaN: the clamps of exponent
 // arguments, so that a NaN input stays NaN (fminf would return the bound and
 // turn it into a saturated gate) and the solve reports it as non-finite.

@@ -46,54 +46,71 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
   float m = 0.f;
   float2 DL = f2(0.f, 0.f), PA = ONE;
   float2 HP = f2(hb, H[kH - 1].x);  // states before steps 0 and 16
+  static_assert(kH % 2 == 0, "the pass takes its step pairs two at a time");
 #pragma unroll
-  for (int i = 0; i < kH; ++i) {
-    const unsigned char* bi = base + ((c8 ^ (row_swizzle(i) * 8)) + i * kRowC * 8);
-    const float2 UZ = *reinterpret_cast<const float2*>(bi);
-    const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kH * kRowC * 8);
-    const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kH * kRowC * 8);
-    const float2 HT = H[i];
-    // z, r = 1/(1+e) with e = 2^(argument).  One reciprocal serves the four
-    // sigmoids of the pair and one the two tanh: every argument is clamped
-    // at 31, so the product of four (1+e) stays below 2^124 (the clamp moves
-    // a sigmoid or tanh by under 1e-9).
-    const float2 TZ = ffma2(AZ2, HP, UZ), TR = ffma2(AR2, HP, UR);
-    const float2 EZ = f2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
-    const float2 ER = f2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
-    const float2 PZ = fadd2(ONE, EZ), PR = fadd2(ONE, ER);
-    const float2 PP = fmul2(PZ, PR);
-    const float inv = rcp(PP.x * PP.y);
-    const float2 INV = f2(PP.y * inv, PP.x * inv);          // 1/(pz pr) per step
-    const float2 Z = fmul2(PR, INV), R = fmul2(PZ, INV);
-    const float2 RH = fmul2(R, HP);
-    const float2 TC = ffma2(AC2, RH, UC);
-    const float2 EC = f2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));  // e^{2y}
-    const float2 PC = fadd2(ONE, EC);
-    const float ic = rcp(PC.x * PC.y);
-    const float2 TT = f2(PC.y * ic, PC.x * ic);             // t = 1/(1+e^{2y})
-    const float2 C = ffma2(M2, TT, ONE);                    // tanh(y) = 1 - 2t
-    const float2 CMH = ffma2(HP, M1, C);
-    const float2 F = ffma2(Z, CMH, HP);
-    const float2 DF = ffma2(F, M1, HT);
-    m = fmax_nan(m, fabsf(DF.x));
-    m = fmax_nan(m, fabsf(DF.y));
-    if (kFull) {
-      // A = (1-z) + a_z z(1-z)(c-h) + (1-c^2) z a_c (r + a_r h r(1-r)),
-      // with 1-c^2 = 4t(1-t)
-      const float2 OMZ = ffma2(Z, M1, ONE);
-      const float2 A1 = ffma2(fmul2(AZ, fmul2(Z, OMZ)), CMH, OMZ);
-      const float2 T1 = fmul2(TT, ffma2(TT, MTL, TL));   // 2 ln2 t(1-t)
-      const float2 S = fmul2(fmul2(Z, T1), AC2);
-      const float2 RR = fmul2(R, ffma2(R, PL, NL));      // -ln2 r(1-r)
-      const float2 Q = ffma2(fmul2(AR2, HP), RR, R);
-      const float2 A = ffma2(S, Q, A1);
-      const float2 HN = ffma2(A, DL, F);
-      DL = ffma2(HT, M1, HN);
-      PA = fmul2(PA, A);
-      H[i] = HN;
-      P[i] = PA;
+  for (int i = 0; i < kH; i += 2) {
+    // two step pairs at a time: the gates of both, then one reciprocal for
+    // the four tanh factors, then their Jacobians and scan steps
+    float2 HPs[2], HTs[2], Z2[2], R2[2], PC2[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int ii = i + j;
+      const unsigned char* bi = base + ((c8 ^ (row_swizzle(ii) * 8)) + ii * kRowC * 8);
+      const float2 UZ = *reinterpret_cast<const float2*>(bi);
+      const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kH * kRowC * 8);
+      const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kH * kRowC * 8);
+      const float2 hp = j == 0 ? HP : HTs[0];
+      HPs[j] = hp;
+      HTs[j] = H[ii];
+      // z, r = 1/(1+e) with e = 2^(argument).  One reciprocal serves the four
+      // sigmoids of a pair and one the four tanh of two pairs: every argument
+      // is clamped at 31, so a product of four (1+e) stays below 2^124 (the
+      // clamp moves a sigmoid or tanh by under 1e-9).
+      const float2 TZ = ffma2(AZ2, hp, UZ), TR = ffma2(AR2, hp, UR);
+      const float2 EZ = f2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
+      const float2 ER = f2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
+      const float2 PZ = fadd2(ONE, EZ), PR = fadd2(ONE, ER);
+      const float2 PP = fmul2(PZ, PR);
+      const float inv = rcp(PP.x * PP.y);
+      const float2 INV = f2(PP.y * inv, PP.x * inv);        // 1/(pz pr) per step
+      Z2[j] = fmul2(PR, INV);
+      R2[j] = fmul2(PZ, INV);
+      const float2 TC = ffma2(AC2, fmul2(R2[j], hp), UC);
+      const float2 EC = f2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));  // e^{2y}
+      PC2[j] = fadd2(ONE, EC);
     }
-    HP = HT;
+    const float w0 = PC2[0].x * PC2[0].y, w1 = PC2[1].x * PC2[1].y;
+    const float ic = rcp(w0 * w1);
+    const float i0 = w1 * ic, i1 = w0 * ic;                  // 1/w0, 1/w1
+    const float2 TTs[2] = {f2(PC2[0].y * i0, PC2[0].x * i0),
+                           f2(PC2[1].y * i1, PC2[1].x * i1)};  // t = 1/(1+e^{2y})
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int ii = i + j;
+      const float2 hp = HPs[j], HT = HTs[j], Z = Z2[j], R = R2[j], TT = TTs[j];
+      const float2 C = ffma2(M2, TT, ONE);                  // tanh(y) = 1 - 2t
+      const float2 CMH = ffma2(hp, M1, C);
+      const float2 F = ffma2(Z, CMH, hp);
+      const float2 DF = ffma2(F, M1, HT);
+      m = fmax3_nan(m, fabsf(DF.x), fabsf(DF.y));
+      if (kFull) {
+        // A = (1-z) + a_z z(1-z)(c-h) + (1-c^2) z a_c (r + a_r h r(1-r)),
+        // with 1-c^2 = 4t(1-t)
+        const float2 OMZ = ffma2(Z, M1, ONE);
+        const float2 A1 = ffma2(fmul2(AZ, fmul2(Z, OMZ)), CMH, OMZ);
+        const float2 T1 = fmul2(TT, ffma2(TT, MTL, TL));   // 2 ln2 t(1-t)
+        const float2 S = fmul2(fmul2(Z, T1), AC2);
+        const float2 RR = fmul2(R, ffma2(R, PL, NL));      // -ln2 r(1-r)
+        const float2 Q = ffma2(fmul2(AR2, hp), RR, R);
+        const float2 A = ffma2(S, Q, A1);
+        const float2 HN = ffma2(A, DL, F);
+        DL = ffma2(HT, M1, HN);
+        PA = fmul2(PA, A);
+        H[ii] = HN;
+        P[ii] = PA;
+      }
+    }
+    HP = HTs[1];
   }
   DLo = DL;
   PAo = PA;
