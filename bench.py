@@ -65,6 +65,11 @@ NCU_TRAFFIC_BYTES = {
 QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue (128 registers, 53 KB smem)
 
 
+# --force-row: the bf16 problems take the whole-sequence (row) kernels where
+# the segment queues would (PARARNN_FLAG_FORCE_ROW on the solve and adjoint)
+FORCE_ROW = False
+
+
 def fwd_plan(w, sms=None):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
     as the library dispatches it: the segment-queue kernels solve every
@@ -78,10 +83,11 @@ def fwd_plan(w, sms=None):
     if sms is None:
         sms = torch.cuda.get_device_properties(0).multi_processor_count
     tiles8 = w.B * ((w.D + 7) // 8)
-    if w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms:
+    if (w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms
+            and not FORCE_ROW):
         return "gru_newton_queue", 4, 512
     if w.cell == "lstm":
-        if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms:
+        if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms and not FORCE_ROW:
             return "lstm_newton_queue", 6.5, 512
         if w.u_dtype == "bf16" and w.T <= 4096:
             cls, seg = 1, w.T
@@ -147,6 +153,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the unfused-tier and decode-step measurements")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--force-row", action="store_true",
+                    help="bf16 problems: the whole-sequence kernels instead of the segment queues")
     return ap.parse_args()
 
 
@@ -275,7 +283,7 @@ class Path:
         self.hist = (torch.empty(66, dtype=torch.int32, device=d) if w.histogram else None)
         self.ws = pr.Workspace(d)
         self.wsa = pr.Workspace(d)
-        self.opts = pr._opts(1e-6, 64)
+        self.opts = pr._opts(1e-6, 64, flags=pr.PARARNN_FLAG_FORCE_ROW if FORCE_ROW else 0)
         cell = pr.PARARNN_LSTM if self.lstm else pr.PARARNN_GRU
         self.fbuf = self.ws.get(pr.pararnn_workspace_size(cell, B, T, D, 64, 0))
         if w.adjoint:
@@ -337,9 +345,14 @@ class Path:
         x = x or self.x
         pr = self.pr
         cell = pr.PARARNN_LSTM if self.lstm else pr.PARARNN_GRU
-        pr.pararnn_adjoint(cell, x["u"], x["a"], x["bias"], x.get("c0"), x["h0"], self.c,
-                           self.h, x["dLdh"], self.du, self.da, self.db, self.dc0, self.dh0,
-                           self.status, self.abuf)
+        if FORCE_ROW:
+            pr.pararnn_adjoint_ex(cell, x["u"], x["a"], x["bias"], x.get("c0"), x["h0"], self.c,
+                                  self.h, x["dLdh"], self.du, self.da, self.db, self.dc0,
+                                  self.dh0, self.status, self.abuf, self.opts)
+        else:
+            pr.pararnn_adjoint(cell, x["u"], x["a"], x["bias"], x.get("c0"), x["h0"], self.c,
+                               self.h, x["dLdh"], self.du, self.da, self.db, self.dc0, self.dh0,
+                               self.status, self.abuf)
 
     def step(self, x=None):
         self.forward(x)
@@ -582,6 +595,7 @@ def run_ours(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name + (" fwd+adjoint" if w.adjoint else " fwd"),
+                   "kernels": "whole-sequence (--force-row)" if FORCE_ROW else "library default",
                    "cell": w.cell, "B": w.B, "T": w.T, "D": w.D, "u_dtype": w.u_dtype,
                    "tol": 1e-6, "l2": "inputs larger than L2 (u alone exceeds 126 MB)",
                    "parallelism": f"{world} independent replica(s)"},
@@ -622,7 +636,9 @@ def run_reference(args, world, rank):
 
 
 def main():
+    global FORCE_ROW
     args = parse()
+    FORCE_ROW = args.force_row
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
