@@ -38,21 +38,20 @@ UNIT = "tokch/s"
 # DRAM bytes (read + write) of one launch of the dominant kernel, taken with
 # ncu on this build for the workload in the key.  None when not captured for
 # the kernel as it stands.
-NCU_TRAFFIC_BYTES = {
-    # one 1024-step segment's launch (the solve is four of them)
-    ("gru_newton_row", "gru_b8_t4096_d1024_bf16"): 50_585_600 + 7_483_392,
-    # one 512-step segment's launch (the solve is eight of them)
-    ("lstm_newton_row", "lstm_b8_t4096_d1024_bf16"): 33_703_168 + 5_925_120,
-}
-# The forward kernel a workload runs and its special-function (MUFU)
-# operations per element and cell evaluation, as the kernel issues them:
+NCU_TRAFFIC_BYTES = {}
+# Special-function (MUFU) work per element and cell evaluation.  The roofline
+# counts the cell in its plain form, the algorithmic figure: ParaGRU 3 exp + 3
+# reciprocals, ParaLSTM 5 exp + 5 reciprocals.  The kernels issue fewer, and
+# the second element of fwd_plan() is that issued count for an exact
+# evaluation:
 #   gru_newton_queue (ParaGRU with bf16 u and at least one 8-channel tile per
 #     resident CTA, four CTAs per SM: every 512-step segment of every tile in
-#     one launch): the cell pass of gru_newton_row, 3 ex2 + 1 rcp;
+#     one launch): the cell pass of gru_newton_row, 3 ex2 + 0.75 rcp for an
+#     exact evaluation; the inexact early evaluations issue 3 tanh;
 #   gru_newton_row (ParaGRU with T <= 4096, or longer with at least one
-#     8-channel tile per SM, then in 4096-step segments): 3 ex2 + 1 rcp (one
-#     reciprocal serves the four sigmoids of a step pair, one the pair's two
-#     tanh);
+#     8-channel tile per SM, then in 4096-step segments): 3 ex2 + 0.75 rcp (one
+#     reciprocal serves the four sigmoids of a step pair, one the four tanh of
+#     two pairs);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
 #   lstm_newton_queue (ParaLSTM, bf16 u, T <= 4096, at least one 8-channel
 #     tile per SM: every 512-step segment in one launch): the cell pass of
@@ -62,6 +61,7 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
+MUFU_ALGORITHMIC = {"gru": 6, "lstm": 10}
 QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue (128 registers, 53 KB smem)
 
 
@@ -85,7 +85,7 @@ def fwd_plan(w, sms=None):
     tiles8 = w.B * ((w.D + 7) // 8)
     if (w.cell == "gru" and w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms
             and not FORCE_ROW):
-        return "gru_newton_queue", 4, 512
+        return "gru_newton_queue", 3.75, 512
     if w.cell == "lstm":
         if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms and not FORCE_ROW:
             return "lstm_newton_queue", 6.5, 512
@@ -111,9 +111,9 @@ def fwd_plan(w, sms=None):
                 seg = k * 1024
                 break
             k *= 2
-        return "gru_newton_row", 4, seg
+        return "gru_newton_row", 3.75, seg
     if tiles8 >= sms:
-        return "gru_newton_row", 4, 4096
+        return "gru_newton_row", 3.75, 4096
     return "gru_newton_fused", 5, w.T
 
 
@@ -312,33 +312,46 @@ class Path:
     def element_evaluations(self, x=None):
         """Cell evaluations performed by one solve, summed over (b, t, d).
 
-        Every tile stops on its own, so this is counted from the per-channel
-        convergence histogram: a channel whose tile first passed the test at
-        iteration k was evaluated k + 1 times.  Exact for the row and queue
-        kernels (a tile is a whole sequence or segment): a sequence the library
-        solves segment by segment is solved here one segment per call, each from
-        the state the one before ended in, which is the arithmetic the segmented
-        solve does.  For the chunked kernels a channel reports its slowest
-        chunk, so this is an upper bound there.  Untimed.
+        Every tile stops on its own, after the first evaluation at which all
+        its channels are below tol, so a tile of channels d0..d0+w-1 was
+        evaluated 1 + max over its channels of the per-channel iteration index
+        (opts.chan_iters) times, and each of its channels that often.  Tiles
+        are 8 channels for the row and segment-queue kernels, whose tiles hold
+        a whole sequence or segment: this is exact there.  A sequence the
+        library solves segment by segment is solved here one segment per call,
+        each from the state the one before ended in, which is the arithmetic
+        the segmented solve does.  For the chunked kernels (32-channel tiles)
+        a channel reports its slowest chunk, so this is an upper bound there.
+        Untimed.
         """
         x = x or self.x
         pr = self.pr
+        kern = fwd_kernel(self.w)[0]
+        width = 32 if kern.endswith("_fused") else 8
+        B, D = self.w.B, self.w.D
         evals = 0
         c_in, h_in = x.get("c0"), x["h0"]
+        ci = torch.zeros((B, D), dtype=torch.int32, device="cuda")
+        opts = self.pr._opts(1e-6, 64, flags=self.opts.flags, chan_iters=ci)
         for s0, n in fwd_segments(self.w):
-            hb = torch.zeros(66, dtype=torch.int32, device="cuda")
             u = x["u"][:, s0:s0 + n].contiguous()
-            h = torch.empty((self.w.B, n, self.w.D), dtype=torch.float32, device="cuda")
+            h = torch.empty((B, n, D), dtype=torch.float32, device="cuda")
             if self.lstm:
                 c = torch.empty_like(h)
-                pr.pararnn_lstm_solve(u, x["a"], x["bias"], c_in, h_in, c, h, self.opts,
-                                      self.stats, hb, self.fbuf)
+                pr.pararnn_lstm_solve(u, x["a"], x["bias"], c_in, h_in, c, h, opts,
+                                      self.stats, None, self.fbuf)
                 c_in = c[:, -1].contiguous()
             else:
-                pr.pararnn_gru_solve(u, x["a"], x["bias"], h_in, h, self.opts, self.stats,
-                                     hb, self.fbuf)
+                pr.pararnn_gru_solve(u, x["a"], x["bias"], h_in, h, opts, self.stats,
+                                     None, self.fbuf)
             h_in = h[:, -1].contiguous()
-            evals += n * sum(m * (k + 1) for k, m in enumerate(hb.cpu().tolist()))
+            k = ci.cpu().long()
+            pad = (-D) % width
+            if pad:
+                k = torch.nn.functional.pad(k, (0, pad))
+            tile_k = k.view(B, -1, width).amax(dim=2)          # [B, tiles]
+            per_ch = tile_k.repeat_interleave(width, dim=1)[:, :D]
+            evals += n * int((per_ch + 1).sum())
         return evals
 
     def backward(self, x=None):
@@ -540,18 +553,21 @@ def run_ours(args, world, rank):
     peaks, src = measured_peaks()
     f_mhz = clk["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
     mufu_peak = 148 * 16 * f_mhz * 1e6 / 1e12          # Tops/s
-    kern, mufu_per_eval = fwd_kernel(w)
+    kern, issued_per_eval = fwd_kernel(w)
+    mufu_per_eval = MUFU_ALGORITHMIC[w.cell]
     elem_evals = path.element_evaluations()
     mufu_done = elem_evals * mufu_per_eval / (fwd_ms * 1e-3) / 1e12
     hbm_ach = w.tokch * fwd_bytes(w) / (fwd_ms * 1e-3) / 1e9
     traffic = NCU_TRAFFIC_BYTES.get((kern, w.name))
     roofline = {"bound": "alu", "kernel": kern, "achieved": round(mufu_done, 3),
-                "peak": round(mufu_peak, 3), "unit": "Tops/s (MUFU ex2+rcp)",
+                "peak": round(mufu_peak, 3),
+                "unit": "Tops/s (MUFU; algorithmic %d ops per element evaluation)" % mufu_per_eval,
                 "frac": round(mufu_done / mufu_peak, 4), "traffic": traffic,
                 "peak_source": f"148 SMs x 16 MUFU/clk x {f_mhz:.0f} MHz sampled",
                 "ops_per_launch": elem_evals * mufu_per_eval / fwd_launches(w),
                 "launches_per_solve": fwd_launches(w),
-                "mean_evals": round(elem_evals / w.tokch, 3)}
+                "mean_evals": round(elem_evals / w.tokch, 3),
+                "issued_per_exact_eval": issued_per_eval}
     hbm = {"fwd_achieved_gbs": round(hbm_ach, 1), "peak_gbs": peaks["hbm_gbs"],
            "frac": round(hbm_ach / peaks["hbm_gbs"], 4), "peak_kind": src,
            "fwd_bytes_per_tokch": fwd_bytes(w)}

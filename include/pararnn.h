@@ -119,6 +119,19 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            segment by segment instead of the
                                            one-launch segment-queue solve
                                            (kept for comparison) */
+#define PARARNN_FLAG_EXACT_STEPS 16u    /* every Newton evaluation exact.
+                                           Without it the ParaGRU
+                                           segment-queue solve evaluates the
+                                           cell with the one-instruction tanh
+                                           (gates within about 2^-11
+                                           relative) while the item's max |r|
+                                           is above 0.1, and decides
+                                           convergence on exact evaluations
+                                           only: the converged states are
+                                           the same, the iterates before that
+                                           are inexact Newton iterates.  With
+                                           it, a solve capped at n updates
+                                           returns the n-th exact iterate. */
 
 typedef struct {
   float tol;          /* stop when max|r| < tol; <= 0 -> 1e-6 */
@@ -135,7 +148,9 @@ typedef struct {
                          before the first evaluation from which the channel's
                          own max_t |r_t| stays below tol (max_iters + 1 if it
                          never got there).  Where the sequence is solved in
-                         segments, the largest index over the segments.
+                         segments, the largest index over the segments.  An
+                         inexact evaluation (see PARARNN_FLAG_EXACT_STEPS)
+                         never counts as below tol.
                          4-byte aligned; the call overwrites every entry. */
 } pararnn_opts;
 

@@ -39,6 +39,7 @@ PARARNN_FLAG_INJECT_WITHHOLD = 1
 PARARNN_FLAG_FORCE_CHUNKED = 2
 PARARNN_FLAG_FORCE_ROW = 4
 PARARNN_FLAG_DENSE_SIMT = 8
+PARARNN_FLAG_EXACT_STEPS = 16
 STATUS_NAMES = {0: "converged", 1: "not_converged", 2: "nonfinite", 3: "timeout"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))

@@ -36,6 +36,14 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
   return y;
 }
+// tanh by the one-instruction hardware approximation (relative error about
+// 2^-11): only for the inexact early Newton evaluations, never for one that
+// decides convergence
+__device__ __forceinline__ float tanh_apx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // the same over three operands, in one instruction
 __device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
   float y;

@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "gru_row_pass.cuh"
@@ -61,6 +62,7 @@ struct QParams {
   int nitems;           // ntiles * nseg (below 2^31: B*T*D <= 2^40)
   int max_iters;
   float tol;
+  float apx_tau;        // inexact evaluations while the item's residual is above this (0: none)
   uint64_t timeout_ns;
   unsigned* counter;    // item tickets (zero at launch)
   unsigned* seg_done;   // [ntiles] segments of each tile stored (zero at launch)
@@ -270,15 +272,22 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     float hb = first ? h0v : 0.f;  // state before this chunk
     int last_bad = -1, updates = 0, k = 0;
     float final_m = 0.f;
-    for (;; ++k) {
-      const bool cap = (k >= p.max_iters);
+    bool apx = p.apx_tau > 0.f;  // CTA-uniform: set from the item's residual maximum
+    // one Newton iteration of the item (kMode 0: exact evaluation and update,
+    // 1: inexact evaluation and update, 2: exact residual only, at the cap);
+    // true when the item is done
+    auto iterate = [&](auto mode) -> bool {
+      constexpr int kMode = decltype(mode)::value;
+      constexpr bool cap = kMode == 2, apx_eval = kMode == 1;
       const int par = phase & 1;
       ++phase;
       const float last_pre = H[kH - 1].y;
       float2 DL, PA;
       float m;
-      if (cap)
+      if constexpr (cap)
         m = row_pass<kH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+      else if constexpr (apx_eval)
+        m = row_pass_apx<kH>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else
         m = row_pass<kH, true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       if (!dval) m = 0.f;
@@ -315,7 +324,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (!(chm < p.tol)) last_bad = k;
+        if (apx_eval || !(chm < p.tol)) last_bad = k;
       }
       // the delta entering this warp: the maps of the warps before it applied
       // to the zero delta entering the item; and the item's residual maximum
@@ -334,11 +343,14 @@ __global__ void __launch_bounds__(NW * 32, MINB)
         tmax = fmax_nan(tmax, fmax_nan(fmax_nan(v.x, v.y), fmax_nan(v.z, v.w)));
       }
       final_m = tmax;
-      const bool own_ok = tmax < p.tol;
-      if (cap) {
+      // an inexact evaluation never decides convergence; the first one whose
+      // residual is at most apx_tau hands over to exact evaluations
+      const bool own_ok = !apx_eval && tmax < p.tol;
+      if (apx_eval && tmax <= p.apx_tau) apx = false;
+      if constexpr (cap) {
         updates = k;
         if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        break;
+        return true;
       }
       const float din = first ? 0.f : fmaf(xP, cd, xd);  // delta entering this chunk
       float prev_last = __shfl_up_sync(kFull, last_pre, kRowC);
@@ -348,7 +360,17 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 #pragma unroll
       for (int i = 0; i < kH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
       updates = k + 1;
-      if (own_ok) break;
+      return own_ok;
+    };
+    // inexact iterations while the residual is large, then exact ones to
+    // convergence or the cap (k: the evaluation's index)
+    for (; apx && k < p.max_iters; ++k) iterate(std::integral_constant<int, 1>{});
+    for (;; ++k) {
+      if (k >= p.max_iters) {
+        iterate(std::integral_constant<int, 2>{});
+        break;
+      }
+      if (iterate(std::integral_constant<int, 0>{})) break;
     }
     // every thread is past its last pass of this item (the barrier of the last
     // exchange): the staging area takes the next item
@@ -406,6 +428,11 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 // (96 registers) and 366 us at 6 (80 registers, a few spills): more resident
 // warps did not pay for the doubled per-step scan work
 constexpr int kQW = 4, kQL = 32, kQMinB = 4;
+// inexact (one-instruction tanh) evaluations while the item's max |r| is above
+// 0.1: on configuration-2 inputs the first three evaluations of a segment,
+// after which the exact ones converge in as many evaluations as from exact
+// steps throughout (fp64 model of the iteration with 2^-11 gate errors)
+constexpr float kQApxTau = 0.1f;
 using QRun = QCfg<kQW, kQL>;
 
 int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
@@ -468,6 +495,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.nitems = p.ntiles * p.nseg;
   p.max_iters = f.max_iters;
   p.tol = f.tol;
+  p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kQApxTau;
   p.timeout_ns = f.timeout_ns;
   p.counter = counter;
   p.seg_done = seg_done;

@@ -117,4 +117,61 @@ __device__ __forceinline__ float row_pass(const unsigned char* __restrict__ base
   return m;
 }
 
+// The pass of row_pass<kH, true> with every gate from the one-instruction
+// tanh: sigma(x) = 1/2 + 1/2 tanh(x/2), c = tanh(y).  The stored arguments
+// are -log2e x (z, r) and 2 log2e y (c), so x/2 and y are those times -ln2/2
+// and ln2/2.  An inexact evaluation (gates within about 2^-11 relative) for
+// the Newton iterations far from the root: the fixed point is fixed by the
+// residual alone ("Параллельность RNN?", §1.2), so the solve takes these
+// while the residual is large and decides convergence on exact evaluations
+// only.  Same arguments and results as row_pass<kH, true>.
+template <int kH>
+__device__ __forceinline__ float row_pass_apx(const unsigned char* __restrict__ base, int c8,
+                                              float hb, float2 (&H)[kH], float2 (&P)[kH],
+                                              float2 AZ2, float2 AR2, float2 AC2, float2 AZ,
+                                              float2& DLo, float2& PAo) {
+  const float2 ONE = f2(1.f, 1.f), M1 = f2(-1.f, -1.f), HALF = f2(0.5f, 0.5f);
+  const float2 KG = f2(-0.5f * kRowLn2, -0.5f * kRowLn2), KC = f2(0.5f * kRowLn2, 0.5f * kRowLn2);
+  const float2 MKC = f2(-0.5f * kRowLn2, -0.5f * kRowLn2);
+  // a_r = -ln2 AR2 and a_c = ln2/2 AC2: the constants ride on r(1-r), 1-c^2
+  const float2 NL = f2(-kRowLn2, -kRowLn2), PL = f2(kRowLn2, kRowLn2);
+  float m = 0.f;
+  float2 DL = f2(0.f, 0.f), PA = ONE;
+  float2 HP = f2(hb, H[kH - 1].x);  // states before steps 0 and 16
+#pragma unroll
+  for (int i = 0; i < kH; ++i) {
+    const unsigned char* bi = base + ((c8 ^ (row_swizzle(i) * 8)) + i * kRowC * 8);
+    const float2 UZ = *reinterpret_cast<const float2*>(bi);
+    const float2 UR = *reinterpret_cast<const float2*>(bi + 1 * kH * kRowC * 8);
+    const float2 UC = *reinterpret_cast<const float2*>(bi + 2 * kH * kRowC * 8);
+    const float2 HT = H[i];
+    const float2 XZ = fmul2(ffma2(AZ2, HP, UZ), KG), XR = fmul2(ffma2(AR2, HP, UR), KG);  // x/2
+    const float2 Z = ffma2(HALF, f2(tanh_apx(XZ.x), tanh_apx(XZ.y)), HALF);
+    const float2 R = ffma2(HALF, f2(tanh_apx(XR.x), tanh_apx(XR.y)), HALF);
+    const float2 Y = fmul2(ffma2(AC2, fmul2(R, HP), UC), KC);                         // y
+    const float2 C = f2(tanh_apx(Y.x), tanh_apx(Y.y));
+    const float2 CMH = ffma2(HP, M1, C);
+    const float2 F = ffma2(Z, CMH, HP);
+    const float2 DF = ffma2(F, M1, HT);
+    m = fmax3_nan(m, fabsf(DF.x), fabsf(DF.y));
+    // A = (1-z) + a_z z(1-z)(c-h) + (1-c^2) z a_c (r + a_r h r(1-r))
+    const float2 OMZ = ffma2(Z, M1, ONE);
+    const float2 A1 = ffma2(fmul2(AZ, fmul2(Z, OMZ)), CMH, OMZ);
+    const float2 OMC = ffma2(fmul2(C, MKC), C, KC);      // ln2/2 (1 - c^2)
+    const float2 S = fmul2(fmul2(Z, OMC), AC2);
+    const float2 RR = fmul2(R, ffma2(R, PL, NL));        // -ln2 r(1-r)
+    const float2 Q = ffma2(fmul2(AR2, HP), RR, R);
+    const float2 A = ffma2(S, Q, A1);
+    const float2 HN = ffma2(A, DL, F);
+    DL = ffma2(HT, M1, HN);
+    PA = fmul2(PA, A);
+    H[i] = HN;
+    P[i] = PA;
+    HP = HT;
+  }
+  DLo = DL;
+  PAo = PA;
+  return m;
+}
+
 }  // namespace pararnn

@@ -107,14 +107,14 @@ def test_bench_plan_follows_the_library_dispatch_rules():
     import bench
     from nonlinear_rnn_paragru_b200.inputs import WORKLOADS
     plan = {k: bench.fwd_plan(w, sms=148) for k, w in WORKLOADS.items()}
-    assert plan[1] == ("gru_newton_row", 4, 256)      # 8 tiles: one launch
-    assert plan[2] == ("gru_newton_queue", 4, 512)    # 1024 tiles >= 4 x 148 resident CTAs
+    assert plan[1] == ("gru_newton_row", 3.75, 256)      # 8 tiles: one launch
+    assert plan[2] == ("gru_newton_queue", 3.75, 512)    # 1024 tiles >= 4 x 148 resident CTAs
     assert bench.fwd_launches(WORKLOADS[2], sms=148) == 1
     # fewer tiles than resident queue CTAs: the row kernel, launch by segment
-    assert bench.fwd_plan(WORKLOADS[2].scaled(B=2), sms=148) == ("gru_newton_row", 4, 2048)
+    assert bench.fwd_plan(WORKLOADS[2].scaled(B=2), sms=148) == ("gru_newton_row", 3.75, 2048)
     assert bench.fwd_launches(WORKLOADS[2].scaled(B=2), sms=148) == 2
     assert plan[3] == ("lstm_newton_queue", 6.5, 512)  # 1024 tiles >= 148 SMs
-    assert plan[4] == ("gru_newton_row", 4, 4096)     # T > 4096, 256 tiles >= 148
+    assert plan[4] == ("gru_newton_row", 3.75, 4096)     # T > 4096, 256 tiles >= 148
     assert plan[5] == ("lstm_newton_queue", 6.5, 512)  # 2048 tiles
     assert bench.fwd_launches(WORKLOADS[3], sms=148) == 1
     assert bench.fwd_plan(WORKLOADS[3].scaled(B=1, D=512), sms=148) == ("lstm_newton_row", 6.5, 2048)
@@ -133,3 +133,11 @@ def test_dense_workspace_sizes():
     assert pr.pararnn_dense_workspace_size(2, 300, 64) >= 2 * 300 * 64 * 64 * 4
     assert pr.pararnn_dense_workspace_size(2, 300, 520) == 0     # D above the maximum
     assert pr.pararnn_dense_workspace_size(2, 300, 60) == 0      # D % 8
+
+
+def test_flag_constants_match_header():
+    src = open(os.path.join(ROOT, "include", "pararnn.h")).read()
+    flags = dict(re.findall(r"#define (PARARNN_FLAG_\w+) (\d+)u", src))
+    assert len(flags) >= 5
+    for name, val in flags.items():
+        assert getattr(pr, name) == int(val), name

@@ -303,9 +303,10 @@ def test_segment_queue_matches_oracle(cuda_ok, B, T, D):
 
 def test_segment_queue_channel_index_one_segment(cuda_ok):
     # T <= 512: one item per tile, so the per-channel index is the oracle's
+    # (exact steps throughout: the oracle's index is that of exact Newton)
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=250, D=6000))
     ci = torch.full((1, 6000), -5, dtype=torch.int32, device="cuda")
-    h, st, hist = _solve(x, hist=True, chan_iters=ci)
+    h, st, hist = _solve(x, hist=True, chan_iters=ci, flags=pr.PARARNN_FLAG_EXACT_STEPS)
     k_gpu = ci.cpu().numpy()
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=64)
     diff = np.abs(k_gpu - r["chan_k"])
@@ -321,10 +322,60 @@ def test_segment_queue_capped_iterates(cuda_ok):
     # segment starts from its predecessor's, not from the whole-sequence
     # iterate)
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=256, D=6000))
-    h, st, _ = _solve(x, max_iters=1)
+    h, st, _ = _solve(x, max_iters=1, flags=pr.PARARNN_FLAG_EXACT_STEPS)
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=1)
     assert st["status"] == "not_converged" and st["iters"] == 1 and st["evals"] == 2
     assert np.abs(h - r["h"]).max() < TOL_STATE
+
+
+def _scan_sensitivity(x, hprev):
+    """Per channel: max_t sum_{s<=t} prod_{s<k<=t} |A_k|, with A_t the fp64
+    Jacobian of the cell at (hprev_{t-1}, u_t): an error e_s added at each
+    step of the linear scan h_t = f_t + A_t h_{t-1} moves h_t by at most
+    this times max |e_s|."""
+    u = x["u"].double().numpy()[0]            # [T, 3, D]
+    a = x["a"].double().numpy().T             # [D, 3]
+    bias = x["bias"].double().numpy().T
+    T, _, D = u.shape
+    s = np.zeros(D)
+    best = np.zeros(D)
+    hp = x["h0"].double().numpy()[0]
+    for t in range(T):
+        _, A, _, _ = oracle.gru_step(hp, u[t].T, a, bias)
+        s = np.abs(A) * s + 1.0
+        best = np.maximum(best, s)
+        hp = hprev[t]
+    return best
+
+
+def test_segment_queue_inexact_first_iterate(cuda_ok):
+    # Without PARARNN_FLAG_EXACT_STEPS the first evaluations of a segment use
+    # the one-instruction tanh (gates within 2^-10 relative, with margin).
+    # The first iterate is then h~_t = f~_t + A~_t h~_{t-1} instead of
+    # h_t = f_t + A_t h_{t-1}, both evaluated at the initial guess.  With
+    # |h| <= 1 the gate errors give |f~ - f| <= 1.5 d and |A~ - A| <= 8 d
+    # (d = 2^-10, from the derivatives of f and A in the gates), so per channel
+    # |h~ - h| <= S (1.5 d + 8 d max|h~|), S the scan's sensitivity.  A sign or
+    # scaling slip in the inexact cell moves the iterate by O(S).
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=256, D=6000))
+    h, st, _ = _solve(x, max_iters=1)
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=1)
+    assert st["status"] == "not_converged" and st["iters"] == 1
+    err = np.abs(h[0] - r["h"][0]).max(axis=0)                  # per channel
+    S = _scan_sensitivity(x, np.zeros((256, 6000)))
+    d = 2.0 ** -10
+    bound = S * (1.5 * d + 8 * d * np.abs(h[0]).max(axis=0))
+    assert (err <= bound).all(), (float((err / bound).max()), float(S.max()))
+    assert err.max() > 1e-6            # the inexact evaluation was taken
+    # and the solve converges to the same states in at most one more
+    # evaluation than with exact steps throughout
+    he, ste, _ = _solve(x, flags=pr.PARARNN_FLAG_EXACT_STEPS)
+    hi, sti, _ = _solve(x)
+    ref = _ref(x)
+    for hh, ss in ((he, ste), (hi, sti)):
+        assert ss["status"] == "converged" and ss["max_residual"] < 1e-6, ss
+        assert np.abs(hh - ref).max() < TOL_STATE
+    assert sti["evals"] <= ste["evals"] + 1, (sti, ste)
 
 
 # ---- injected faults (host-set): a part of the exchange is withheld, the
