@@ -38,7 +38,10 @@ UNIT = "tokch/s"
 # DRAM bytes (read + write) of one launch of the dominant kernel, taken with
 # ncu on this build for the workload in the key.  None when not captured for
 # the kernel as it stands.
-NCU_TRAFFIC_BYTES = {}
+NCU_TRAFFIC_BYTES = {
+    # one launch (the whole solve), profiles/gru_newton_queue_b8_t4096_d1024.md
+    ("gru_newton_queue", "gru_b8_t4096_d1024_bf16"): 201_561_344 + 102_954_496,
+}
 # Special-function (MUFU) work per element and cell evaluation.  The roofline
 # counts the cell in its plain form, the algorithmic figure: ParaGRU 3 exp + 3
 # reciprocals, ParaLSTM 5 exp + 5 reciprocals.  The kernels issue fewer, and
