@@ -56,16 +56,17 @@ NCU_TRAFFIC_BYTES = {
 #     reciprocal serves the four sigmoids of a step pair, one the four tanh of
 #     two pairs);
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
-#   lstm_newton_queue (ParaLSTM, bf16 u, T <= 4096, at least one 8-channel
-#     tile per SM: every 512-step segment in one launch): the cell pass of
-#     lstm_newton_row;
+#   lstm_newton_queue (ParaLSTM, bf16 u, at least one 8-channel tile per
+#     resident CTA, four CTAs per SM: every 128-step segment in one launch):
+#     5 ex2 + 1.5 rcp for an exact evaluation; the inexact early evaluations
+#     issue 5 tanh;
 #   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096, in segments where
 #     smaller clusters fill the SMs): 5 ex2 + 1.5 rcp (one
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
 #     one for the two tanh(c'));
 #   lstm_newton_fused (ParaLSTM otherwise): 5 ex2 + 3 rcp.
 MUFU_ALGORITHMIC = {"gru": 6, "lstm": 10}
-QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue (128 registers, 53 KB smem)
+QUEUE_CTAS_PER_SM = 4   # residency of gru_newton_queue and lstm_newton_queue (128 registers)
 
 
 # --force-row: the bf16 problems take the whole-sequence (row) kernels where
@@ -76,8 +77,8 @@ FORCE_ROW = False
 def fwd_plan(w, sms=None):
     """(kernel, MUFU ops per evaluation, segment length) of the forward solve
     as the library dispatches it: the segment-queue kernels solve every
-    512-step segment of a problem with bf16 u and at least one
-    8-channel tile per resident CTA in one launch; otherwise the row kernels
+    512-step (ParaGRU) or 128-step (ParaLSTM) segment of a problem with bf16 u
+    and at least one 8-channel tile per resident CTA in one launch; otherwise the row kernels
     solve a sequence in segments of k x 1024 (ParaGRU, two CTAs per SM) or
     k x 512 steps (ParaLSTM, one CTA per SM), one launch each, k the smallest
     cluster size below the one the whole sequence needs at which its
@@ -90,8 +91,8 @@ def fwd_plan(w, sms=None):
             and not FORCE_ROW):
         return "gru_newton_queue", 3.75, 512
     if w.cell == "lstm":
-        if w.u_dtype == "bf16" and w.T <= 4096 and tiles8 >= sms and not FORCE_ROW:
-            return "lstm_newton_queue", 6.5, 512
+        if w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms and not FORCE_ROW:
+            return "lstm_newton_queue", 6.5, 128
         if w.u_dtype == "bf16" and w.T <= 4096:
             cls, seg = 1, w.T
             while cls * 512 < w.T:

@@ -115,17 +115,19 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            products on CUDA cores (exact
                                            Newton steps, D <= 128) instead of
                                            tf32 tensor-core products */
-#define PARARNN_FLAG_FORCE_ROW 4u       /* bf16 u: launch the row kernel
-                                           segment by segment instead of the
-                                           one-launch segment-queue solve
-                                           (kept for comparison) */
+#define PARARNN_FLAG_FORCE_ROW 4u       /* bf16 u: the whole-sequence (row)
+                                           kernels, launched segment by
+                                           segment, where the one-launch
+                                           segment-queue solves (forward of
+                                           both cells, ParaGRU adjoint) would
+                                           run (kept for comparison) */
 #define PARARNN_FLAG_EXACT_STEPS 16u    /* every Newton evaluation exact.
-                                           Without it the ParaGRU
-                                           segment-queue solve evaluates the
+                                           Without it the segment-queue
+                                           solves (both cells) evaluate the
                                            cell with the one-instruction tanh
                                            (gates within about 2^-11
                                            relative) while the item's max |r|
-                                           is above 0.1, and decides
+                                           is above 0.1, and decide
                                            convergence on exact evaluations
                                            only: the converged states are
                                            the same, the iterates before that
@@ -185,8 +187,12 @@ int pararnn_workspace_init(void* workspace, size_t ws_bytes,
  * Newton starts from h = 0 at every t, applies the page's update until the
  * residual of an iterate is below tol everywhere upstream (and then applies
  * that last update), or until max_iters updates have been applied.  Channels
- * are independent; each 8-channel tile stops on its own.  A sequence of up
- * to 4096 steps is held by a cluster of k CTAs of 1024 steps per tile; when a
+ * are independent; each 8-channel tile stops on its own.  With bf16 u and at
+ * least one 8-channel tile per resident CTA of the segment-queue solve
+ * (B * D / 8 >= 4 * SMs), one launch solves every 512-step segment of every
+ * tile, each segment from the state the one before it converged to (stats
+ * and iter_hist take the maximum over the segments).  Otherwise a sequence of
+ * up to 4096 steps is held by a cluster of k CTAs of 1024 steps per tile; when a
  * smaller cluster of k' CTAs already gives two CTAs per SM
  * (k' * B * D / 8 >= 2 * SMs), it is solved in segments of k' * 1024 steps.
  * A longer sequence with at least one 8-channel tile (B * D / 8) per SM is
@@ -203,7 +209,11 @@ int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
 /* ParaLSTM forward solve.  As pararnn_gru_solve with u [B][T][4][D]
  * (i, f, g, o), a/bias [4][D], initial cell state c0 (NULL = zeros) and both
  * state trajectories out: c [B][T][D], h [B][T][D].  The residual norm is the
- * max over both components.  With bf16 u and T <= 4096 a tile's sequence is
+ * max over both components.  With bf16 u and at least one 8-channel tile per
+ * resident CTA of the segment-queue solve (B * D / 8 >= 4 * SMs), one launch
+ * solves every 128-step segment of every tile (any T), each segment from the
+ * (c, h) the one before it converged to.  Otherwise, with bf16 u and
+ * T <= 4096, a tile's sequence is
  * held by a cluster of k CTAs of 512 steps each; when a smaller cluster of
  * k' CTAs already puts one CTA on every SM (k' * B * D / 8 >= SMs), the
  * sequence is solved in segments of k' * 512 steps instead, each starting

@@ -31,8 +31,10 @@ int lstm_row_cta_steps();
 int lstm_row_box_steps();
 int lstm_row_channels();
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
-int launch_lstm_queue(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
-int lstm_queue_steps();
+int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+                      unsigned* seg_done, cudaStream_t stream);
+int lstm_queue_resident();
+int lstm_queue_box_steps();
 int adjoint_row_cluster(int T);
 int adjoint_row_channels();
 int adjoint_row_box_steps(int which);
@@ -323,9 +325,11 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   const bool force_row = opts && (opts->flags & PARARNN_FLAG_FORCE_ROW);
   const bool queue_gru = row_gru && bf16 && !force_row &&
                          tiles8 >= (long long)std::max(1, gru_queue_resident());
-  // ParaLSTM (bf16 u, T <= 4096) with at least one 8-channel tile per SM
-  // (one CTA per SM): every 512-step segment in one launch
-  const bool queue_lstm = row_lstm && !force_row && tiles8 >= sm_count();
+  // ParaLSTM (bf16 u, any T) with at least one 8-channel tile per resident CTA
+  // of the segment-queue solve (four per SM): every 128-step segment in one
+  // launch
+  const bool queue_lstm = cell == PARARNN_LSTM && bf16 && !force && !force_row &&
+                          tiles8 >= (long long)std::max(1, lstm_queue_resident());
   const size_t nch = (size_t)B * D;
   const int nhist = max_iters + 2;
   unsigned* const seg_done = p.seg_done;
@@ -345,12 +349,9 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
     e = launch_gru_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
   } else if (queue_lstm) {
     CUtensorMap rmap;
-    rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_row_box_steps(), lstm_row_channels());
+    rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_queue_box_steps(), lstm_row_channels());
     if (rc) return rc;
-    FwdParams pq = p;
-    pq.nitems = (int)std::min<long long>((long long)tiles8 * cdiv(T, lstm_queue_steps()),
-                                         0x7fffffffLL);
-    e = launch_lstm_queue(rmap, pq, stream);
+    e = launch_lstm_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
   } else if (row_gru) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());

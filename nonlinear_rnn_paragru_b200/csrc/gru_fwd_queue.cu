@@ -159,6 +159,9 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   int status = 0;
   unsigned phase = 0;  // exchange phases so far, over all items
   int prev_item = -1;
+  // CTA-uniform: 0 while the staged boxes arrive, else 1 + the phase parity of
+  // the wait that ran out (no box is issued after that)
+  int dead = 0;
   for (int n = 0; item < p.nitems; ++n) {
     __syncthreads();
     // publish the previous item: every thread's state stores precede the
@@ -175,7 +178,13 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     const bool dval = d < p.D;
     const int t_base = seg * Cfg::kSteps;
     const int t_len = min(Cfg::kSteps, p.T - t_base);
-    if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
+    bool got = true;
+    if (!dead) {
+      got = mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns);
+      if (!got) status = PARARNN_STATUS_TIMEOUT;
+    }
+    // a phase that did not complete is never re-armed: no more boxes then
+    if (!dead && !__syncthreads_and(got)) dead = 1 + (n & 1);
     // ---- expand the staged bf16 rows [t][gate][8 ch] into fp32 arguments in
     // two blocks (each block's rows are read before any of its slots is
     // written; block 0 writes below all staging bytes)
@@ -375,7 +384,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     // every thread is past its last pass of this item (the barrier of the last
     // exchange): the staging area takes the next item
     const int next = sh.nx[(n + 1) & 1];
-    if (tid == 0 && next < p.nitems) {
+    if (tid == 0 && !dead && next < p.nitems) {
       const int ntile = next % p.ntiles;
       q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, ntile / p.nDTc,
               (ntile % p.nDTc) * kRowC, (next / p.ntiles) * Cfg::kSteps);
@@ -418,6 +427,8 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     __threadfence();
     st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
   }
+  // boxes still in flight into the staging area: wait for them (bounded)
+  if (dead && tid == 0) mbar_wait_bounded(&sh.bar, (unsigned)(dead - 1), p.timeout_ns);
   const int st = __reduce_max_sync(kFull, status);
   if (lane == 0 && st) atomicMax(&p.stats->status, st);
 }

@@ -97,7 +97,6 @@ struct LrShared {
   __align__(16) float par[2][10][kLrC];
   uint64_t bar;                       // the staging area's mbarrier
   uint64_t mbar[2];                   // mailbox mbarriers, by parity
-  int nx[2];                          // queue mode: this and the next item, by parity
 };
 
 __device__ __forceinline__ float2 lf2(float x, float y) { return make_float2(x, y); }
@@ -261,17 +260,9 @@ __host__ __device__ constexpr unsigned lr_rx_bytes(int rank, int cls) {
   return (unsigned)(rank * kLrC * 32 + (cls - 1) * 4);
 }
 
-// kQ (with CLS = 1): the segment-queue mode.  Items (tile, 512-step segment)
-// are numbered segment-major and drawn from a counter one ahead, so every
-// segment of every tile is solved by one launch with the tiles balanced
-// dynamically; a segment's CTA waits (bounded acquire poll) until the tile's
-// previous segment has published its states, reads its initial (c, h) from
-// them, and publishes its own with a release store after storing them (see
-// gru_fwd_queue.cu for why the queue cannot deadlock).
-template <int CLS, bool kQ>
+template <int CLS>
 __global__ void __launch_bounds__(kLrThreads, 1)
     lstm_newton_row(const __grid_constant__ CUtensorMap map, const FwdParams p) {
-  static_assert(!kQ || CLS == 1, "the queue mode runs without clusters");
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ LrShared sh;
   cgl::cluster_group cluster = cgl::this_cluster();
@@ -285,19 +276,11 @@ __global__ void __launch_bounds__(kLrThreads, 1)
   const int t0 = rank * kLrSteps;            // first step of this CTA
   const unsigned rx = lr_rx_bytes(rank, CLS);
 
-  // the current unit of work: a tile (row mode) or an item (queue mode)
-  int cur = clus, limit = ntiles;
-  if constexpr (kQ) {
-    if (tid == 0) sh.nx[0] = (int)min(atomicAdd(&p.hdr->ticket, 1u), 0x7fffffffu);
-    __syncthreads();
-    cur = sh.nx[0];
-    limit = p.nitems;
-  }
+  int cur = clus;  // the current tile
   // the first tile's parameters; later tiles' are loaded a tile ahead
-  if (tid < 10 * kLrC && cur < limit) {
-    const int tl = kQ ? cur % ntiles : cur;
-    const int b = tl / nDTc;
-    (&sh.par[0][0][0])[tid] = lr_param(p, tid, b, (tl - b * nDTc) * kLrC);
+  if (tid < 10 * kLrC && cur < ntiles) {
+    const int b = cur / nDTc;
+    (&sh.par[0][0][0])[tid] = lr_param(p, tid, b, (cur - b * nDTc) * kLrC);
   }
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
@@ -310,32 +293,26 @@ __global__ void __launch_bounds__(kLrThreads, 1)
   }
   __syncthreads();
   if (CLS > 1) cluster.sync();  // the peers' mailbox barriers are armed before anyone sends
-  if (tid == 0 && cur < limit) {
-    const int tl = kQ ? cur % ntiles : cur;
-    const int b = tl / nDTc;
-    lr_issue(smem, sh, &map, b, (tl - b * nDTc) * kLrC,
-             kQ ? (cur / ntiles) * kLrSteps : p.t_base + t0);
+  if (tid == 0 && cur < ntiles) {
+    const int b = cur / nDTc;
+    lr_issue(smem, sh, &map, b, (cur - b * nDTc) * kLrC, p.t_base + t0);
   }
-  int prev_item = -1;  // queue mode: the item whose states are yet to be published
   const unsigned char* base = smem + q * kLrS;
   int status = 0;
   int n = 0;
   unsigned phase = 0;  // exchange phases so far, over all tiles
-  for (; cur < limit; ++n) {
-    const int tile = kQ ? cur % ntiles : cur;
-    const int seg = kQ ? cur / ntiles : 0;
-    const int t_base = kQ ? seg * kLrSteps : p.t_base;   // the launch's (item's) first step
-    const int t_len = kQ ? min(kLrSteps, p.T - t_base) : p.t_len;
-    if (kQ && tid == 0) sh.nx[(n + 1) & 1] = (int)min(atomicAdd(&p.hdr->ticket, 1u), 0x7fffffffu);
+  for (; cur < ntiles; ++n) {
+    const int tile = cur;
+    const int t_base = p.t_base;   // the launch's first step
+    const int t_len = p.t_len;
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kLrC;
     const int d = d0 + c;
     const bool dval = d < p.D;
-    int next = kQ ? -1 : tile + nclus;  // queue mode: read after the barrier below
-    // the next tile's parameters: loaded now (queue mode: after the
-    // barrier below), stored at the end of this tile
+    const int next = tile + nclus;
+    // the next tile's parameters: loaded now, stored at the end of this tile
     const int pj = tid - 32;
     float pnext = 0.f;
-    if (!kQ && pj >= 0 && pj < 10 * kLrC && next < ntiles) {
+    if (pj >= 0 && pj < 10 * kLrC && next < ntiles) {
       const int b2 = next / nDTc;
       pnext = lr_param(p, pj, b2, (next - b2 * nDTc) * kLrC);
     }
@@ -391,44 +368,10 @@ __global__ void __launch_bounds__(kLrThreads, 1)
     }
     float c0v = sh.par[pb][8][c], h0v = sh.par[pb][9][c];
     __syncthreads();
-    int next_t = p.t_base + t0;  // first step of the next unit's boxes
-    if constexpr (kQ) {
-      // publish the previous item: every thread's state stores precede the
-      // barrier above
-      if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
-        __threadfence();
-        st_release(&p.seg_done[prev_item % ntiles], (unsigned)(prev_item / ntiles) + 1u);
-      }
-      next = sh.nx[(n + 1) & 1];
-      const int ntile = next % ntiles;
-      next_t = (next / ntiles) * kLrSteps;
-      if (pj >= 0 && pj < 10 * kLrC && next < limit) {
-        const int b2 = ntile / nDTc;
-        pnext = lr_param(p, pj, b2, (ntile - b2 * nDTc) * kLrC);
-      }
-      // the item's initial state: (c0, h0), or the last states of the tile's
-      // previous segment once its CTA has published them
-      if (q == 0 && seg > 0) {
-        const unsigned* f = &p.seg_done[tile];
-        if (ld_acquire(f) < (unsigned)seg) {
-          const uint64_t w0 = globaltimer_ns();
-          while (ld_acquire(f) < (unsigned)seg) {
-            if (globaltimer_ns() - w0 > p.timeout_ns) {
-              status = PARARNN_STATUS_TIMEOUT;
-              break;
-            }
-          }
-        }
-        const size_t ip = ((size_t)b * p.T + t_base - 1) * p.D + d;
-        c0v = dval ? __ldcg(p.c + ip) : 0.f;
-        h0v = dval ? __ldcg(p.h + ip) : 0.f;
-      }
-    }
     // the staging area and the parameter rows are free: the next tile's
-    if (tid == 0 && next < limit) {
-      const int nt = kQ ? next % ntiles : next;
-      const int b2 = nt / nDTc;
-      lr_issue(smem, sh, &map, b2, (nt - b2 * nDTc) * kLrC, next_t);
+    if (tid == 0 && next < ntiles) {
+      const int b2 = next / nDTc;
+      lr_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kLrC, p.t_base + t0);
     }
     const bool first = (rank == 0 && q == 0);  // chunk holding step 0
 
@@ -600,15 +543,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       atomicMax(&p.stats->evals, kit + 1);
       atomicMax(reinterpret_cast<int*>(&p.stats->max_residual), __float_as_int(final_m));
     }
-    prev_item = cur;
     cur = next;
-  }
-  if constexpr (kQ) {
-    __syncthreads();
-    if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
-      __threadfence();
-      st_release(&p.seg_done[prev_item % ntiles], (unsigned)(prev_item / ntiles) + 1u);
-    }
   }
   const int st = __reduce_max_sync(kFull, status);
   if (lane == 0 && st) atomicMax(&p.stats->status, st);
@@ -628,13 +563,13 @@ int lstm_row_box_steps() { return kLrBox; }
 int lstm_row_cta_steps() { return kLrSteps; }
 int lstm_row_channels() { return kLrC; }
 
-template <int CLS, bool kQ = false>
+template <int CLS>
 static int launch_lr_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
   const long long ntiles = (long long)p.B * ((p.D + kLrC - 1) / kLrC);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  auto kern = lstm_newton_row<CLS, kQ>;
+  auto kern = lstm_newton_row<CLS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLrSmem);
   if (e != cudaSuccess) return (int)e;
   cudaLaunchConfig_t cfg = {};
@@ -654,20 +589,11 @@ static int launch_lr_t(const CUtensorMap& map, const FwdParams& p, cudaStream_t 
   if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) == cudaSuccess && active > 0)
     nclus = std::min(nclus, active);
   cudaGetLastError();
-  // queue mode: persistent, every CTA resident at once (the queue's progress
-  // argument), at most one per item
-  nclus = (int)std::min<long long>(nclus, kQ ? (long long)p.nitems : ntiles);
+  nclus = (int)std::min<long long>(nclus, ntiles);
   if (nclus < 1) nclus = 1;
   cfg.gridDim = dim3(nclus * CLS);
   return (int)cudaLaunchKernelEx(&cfg, kern, map, p);
 }
-
-// Every 512-step segment of every tile (bf16 u) in one launch; p.seg_done
-// (ntiles entries) and hdr->ticket must be zero at launch.
-int launch_lstm_queue(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
-  return launch_lr_t<1, true>(map, p, stream);
-}
-int lstm_queue_steps() { return kLrSteps; }
 
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream) {
   switch (lstm_row_cluster(p.t_len)) {
