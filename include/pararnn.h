@@ -253,15 +253,16 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * opts->inject_chunk (the tile's chunks take tickets last first) publishes
  * no records; in the whole-sequence adjoint (bf16 u, T <= 4096) the CTA of
  * cluster rank opts->inject_chunk withholds its map in its cluster's last
- * tile; in the ParaGRU queue adjoint item opts->inject_chunk (r * tiles +
- * tile for the segment r from the end) never publishes its carry.  With
+ * tile; in the queue adjoints item opts->inject_chunk (r * tiles + tile for
+ * the segment r from the end) never publishes its carry.  With
  * PARARNN_FLAG_FORCE_ROW in opts->flags the whole-sequence kernels run where
  * the queue adjoint would.  Other opts fields are ignored.  NULL opts =
  * pararnn_adjoint.
- * Kernels: ParaGRU with bf16 u and at least one 8-channel tile per resident
- * CTA of the queue adjoint (5 per SM) takes the queue adjoint (every 256-step
- * segment of every tile in one launch, last segments first, each segment's
- * carry from the segment after it); other bf16 problems with T <= 4096 the
+ * Kernels: bf16 u with at least one 8-channel tile per resident CTA of the
+ * queue adjoint (5 per SM for ParaGRU, 4 for ParaLSTM) takes the queue
+ * adjoint (every 256-step segment of every tile in one launch, last segments
+ * first, each segment's carry from the segment after it); other bf16
+ * problems with T <= 4096 the
  * whole-sequence kernels (a cluster of CTAs per tile); the rest the chunked
  * look-back adjoint.  The first two stage the rows of a, bias, h0 and c0 by
  * 1-D bulk copies and are taken only when those pointers are 16-byte aligned

@@ -92,4 +92,82 @@ __device__ __forceinline__ void ar_args(const unsigned char* ux, const unsigned 
                     __uint_as_float((unsigned)ry[2 * kArC] << 16)), BC);
 }
 
+// ---------------------------------------------------------------- ParaLSTM --
+// A chunk's staged inputs for the ParaLSTM adjoints: u (bf16 [t][i f g o]
+// [8 ch], 19 steps), c_{t-1} and h_{t-1} (fp32, 20 steps) and dL/dh (fp32,
+// 19 steps) in a 3200-byte slot.  The u rows are 64 bytes, so chunks k and
+// k + 2 of a warp share bank windows there (two-way); the 32-byte state rows
+// are conflict-free as for ParaGRU.
+constexpr int kAlUStep = 4 * kArC * 2;        // 64 bytes per step of u
+constexpr int kAlUOff = 0, kAlCOff = 1280, kAlHOff = 1920, kAlGOff = 2560;
+constexpr int kAlS = 3200;                    // chunk slot
+
+struct AlCell {
+  float2 AI2, AF2, AG2, AO2;  // h coefficients of the arguments (-log2e a; 2 log2e a for g)
+  float2 AI, AF, AG, AO;      // raw weights
+};
+
+// The cell at a step pair from (CP, HP) = (c_{t-1}, h_{t-1}) and the
+// pre-scaled arguments: the Jacobian entries A00 = f, A01 = X = dc'/dh,
+// A10 = dh'/dc, A11 = dh'/dh, and the pieces of du: du_{i,f,g} = (gci, gcf,
+// gcg) (lambda_c + kk lambda_h), du_o = dot lambda_h.
+__device__ __forceinline__ void al_cell(const AlCell& k, float2 CP, float2 HP, float2 UI,
+                                        float2 UF, float2 UG, float2 UO, float2& F, float2& X,
+                                        float2& KK, float2& A11, float2& GCI, float2& GCF,
+                                        float2& GCG, float2& DOT) {
+  const float2 ONE = af2(1.f, 1.f), M1 = af2(-1.f, -1.f), M2 = af2(-2.f, -2.f);
+  const float2 F4 = af2(4.f, 4.f), M4 = af2(-4.f, -4.f);
+  const float2 TL = af2(2.f * kLog2e, 2.f * kLog2e);
+  auto cl = [](float2 v) { return af2(fmin_nan(v.x, 21.f), fmin_nan(v.y, 21.f)); };
+  auto e2 = [](float2 v) { return af2(ex2(v.x), ex2(v.y)); };
+  const float2 EI = e2(cl(afma(k.AI2, HP, UI))), EF = e2(cl(afma(k.AF2, HP, UF)));
+  const float2 EO = e2(cl(afma(k.AO2, HP, UO))), EG = e2(cl(afma(k.AG2, HP, UG)));
+  const float2 PI = aadd(ONE, EI), PF = aadd(ONE, EF), PO = aadd(ONE, EO);
+  const float2 PFO = amul(PF, PO), PIO = amul(PI, PO), PIF = amul(PI, PF);
+  const float2 Q = amul(PI, PFO);
+  const float iq = rcp(Q.x * Q.y);
+  const float2 IQ = af2(Q.y * iq, Q.x * iq);
+  const float2 I = amul(PFO, IQ), O = amul(PIF, IQ);
+  F = amul(PIO, IQ);
+  const float2 PG = aadd(ONE, EG);
+  const float ig = rcp(PG.x * PG.y);
+  const float2 TG = af2(PG.y * ig, PG.x * ig);
+  const float2 G = afma(M2, TG, ONE);
+  const float2 CN = afma(F, CP, amul(I, G));
+  const float2 EC = e2(cl(amul(TL, CN)));
+  const float2 PC = aadd(ONE, EC);
+  const float icn = rcp(PC.x * PC.y);
+  const float2 TC1 = af2(PC.y * icn, PC.x * icn);
+  const float2 TC = afma(M2, TC1, ONE);
+  const float2 DI = amul(I, afma(I, M1, ONE));
+  const float2 DF = amul(F, afma(F, M1, ONE));
+  const float2 DO = amul(O, afma(O, M1, ONE));
+  const float2 DG = amul(TG, afma(TG, M4, F4));       // 1 - g^2
+  const float2 DT = amul(TC1, afma(TC1, M4, F4));     // 1 - tanh^2(c')
+  GCI = amul(G, DI);
+  GCF = amul(CP, DF);
+  GCG = amul(I, DG);
+  KK = amul(O, DT);
+  DOT = amul(DO, TC);
+  X = afma(GCF, k.AF, afma(GCI, k.AI, amul(GCG, k.AG)));
+  A11 = afma(DOT, k.AO, amul(KK, X));
+}
+
+// pre-scaled arguments of a step pair from bf16 rows [i f g o][8 ch]
+__device__ __forceinline__ void al_args(const unsigned char* ux, const unsigned char* uy,
+                                        const float2 (&BS)[4], float2& UI, float2& UF,
+                                        float2& UG, float2& UO) {
+  const unsigned short* rx = reinterpret_cast<const unsigned short*>(ux);
+  const unsigned short* ry = reinterpret_cast<const unsigned short*>(uy);
+  const float2 S = af2(-kLog2e, -kLog2e), SG = af2(2.f * kLog2e, 2.f * kLog2e);
+  auto ld = [&](int g) {
+    return af2(__uint_as_float((unsigned)rx[g * kArC] << 16),
+               __uint_as_float((unsigned)ry[g * kArC] << 16));
+  };
+  UI = afma(S, ld(0), BS[0]);
+  UF = afma(S, ld(1), BS[1]);
+  UG = afma(SG, ld(2), BS[2]);
+  UO = afma(S, ld(3), BS[3]);
+}
+
 }  // namespace pararnn

@@ -279,7 +279,7 @@ def _offset_view(t, d="cuda"):
 
 @pytest.mark.parametrize("cell,B,T,D", [(pr.PARARNN_GRU, 1, 700, 6000),
                                         (pr.PARARNN_GRU, 2, 1000, 64),
-                                        (pr.PARARNN_LSTM, 1, 700, 48)])
+                                        (pr.PARARNN_LSTM, 1, 700, 4800)])
 def test_adjoint_rows_4byte_aligned(cuda_ok, cell, B, T, D):
     # rows of a, bias, h0 (c0) that are 4-byte but not 16-byte aligned cannot
     # be staged by bulk copies: the call takes the look-back adjoint, whose
@@ -313,3 +313,53 @@ def test_adjoint_rows_4byte_aligned(cuda_ok, cell, B, T, D):
             assert _rel(o[k].cpu().numpy(), ref[k]) <= TOL_GRAD, k
     for k in keys:
         assert _rel(outs[1][k].cpu().numpy(), outs[0][k].cpu().numpy()) <= TOL_GRAD, k
+
+
+# ---- the ParaLSTM queue adjoint (bf16 u, at least one 8-channel tile per
+# resident CTA: 4 x 148 = 592 on a B200)
+def _lstm_queue_inputs(B, T, D):
+    x = make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D), with_grad=True)
+    g = torch.Generator().manual_seed(41)
+    x["c0"] = torch.randn((B, D), generator=g) * 0.5
+    x["h0"] = torch.randn((B, D), generator=g) * 0.5
+    c, h = oracle.lstm_seq(x["u"], x["a"], x["bias"], x["c0"], x["h0"])
+    return x, c, h
+
+
+@pytest.mark.parametrize("B,T,D", [(1, 700, 4800), (2, 1300, 2400), (1, 256, 4800)])
+def test_lstm_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
+    x, c, h = _lstm_queue_inputs(B, T, D)
+    _check_lstm(x, c, h)
+    # and the whole-sequence kernel on the same inputs
+    d = "cuda"
+    hh = torch.as_tensor(h, dtype=torch.float32).to(d).contiguous()
+    cc = torch.as_tensor(c, dtype=torch.float32).to(d).contiguous()
+    args = (pr.PARARNN_LSTM, x["u"].to(d), x["a"].to(d), x["bias"].to(d), x["h0"].to(d), hh,
+            x["dLdh"].to(d))
+    q = pr.adjoint(*args, c0=x["c0"].to(d), c=cc)
+    r = pr.adjoint(*args, c0=x["c0"].to(d), c=cc, opts=pr._opts(flags=pr.PARARNN_FLAG_FORCE_ROW))
+    torch.cuda.synchronize()
+    for k in ("du", "da", "dbias", "dh0", "dc0"):
+        assert _rel(q[k].cpu().numpy(), r[k].cpu().numpy()) <= TOL_GRAD, k
+
+
+def test_lstm_queue_adjoint_is_bitwise_reproducible(cuda_ok):
+    x, c, h = _lstm_queue_inputs(1, 900, 4800)
+    a = _gpu_adjoint(pr.PARARNN_LSTM, x, h, c)
+    b = _gpu_adjoint(pr.PARARNN_LSTM, x, h, c)
+    for k in ("du", "da", "dbias", "dh0", "dc0"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_lstm_queue_adjoint_withheld_carry_times_out(cuda_ok):
+    # item 5 (the last segment of tile 5) never publishes its carry
+    x, c, h = _lstm_queue_inputs(1, 600, 4800)
+    d = "cuda"
+    opts = pr._opts(flags=pr.PARARNN_FLAG_INJECT_WITHHOLD, inject_chunk=5, timeout_us=20000)
+    out = pr.adjoint(pr.PARARNN_LSTM, x["u"].to(d), x["a"].to(d), x["bias"].to(d),
+                     x["h0"].to(d), torch.as_tensor(h, dtype=torch.float32).to(d).contiguous(),
+                     x["dLdh"].to(d), c0=x["c0"].to(d),
+                     c=torch.as_tensor(c, dtype=torch.float32).to(d).contiguous(), opts=opts)
+    torch.cuda.synchronize()
+    assert int(out["status"][0]) == 3
+    _check_lstm(x, c, h)
