@@ -123,7 +123,8 @@ enum { PARARNN_GRU = 0, PARARNN_LSTM = 1 };
                                            run (kept for comparison) */
 #define PARARNN_FLAG_EXACT_STEPS 16u    /* every Newton evaluation exact.
                                            Without it the segment-queue
-                                           solves (both cells) evaluate the
+                                           solves (both cells) and the
+                                           ParaGRU row kernels evaluate the
                                            cell with the one-instruction tanh
                                            (gates within about 2^-11
                                            relative) while the item's max |r|

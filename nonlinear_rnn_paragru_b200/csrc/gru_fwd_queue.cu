@@ -439,11 +439,6 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 // (96 registers) and 366 us at 6 (80 registers, a few spills): more resident
 // warps did not pay for the doubled per-step scan work
 constexpr int kQW = 4, kQL = 32, kQMinB = 4;
-// inexact (one-instruction tanh) evaluations while the item's max |r| is above
-// 0.1: on configuration-2 inputs the first three evaluations of a segment,
-// after which the exact ones converge in as many evaluations as from exact
-// steps throughout (fp64 model of the iteration with 2^-11 gate errors)
-constexpr float kQApxTau = 0.1f;
 using QRun = QCfg<kQW, kQL>;
 
 int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
@@ -506,7 +501,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.nitems = p.ntiles * p.nseg;
   p.max_iters = f.max_iters;
   p.tol = f.tol;
-  p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kQApxTau;
+  p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kApxTau;
   p.timeout_ns = f.timeout_ns;
   p.counter = counter;
   p.seg_done = seg_done;

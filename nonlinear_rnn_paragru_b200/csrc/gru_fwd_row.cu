@@ -53,6 +53,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "gru_row_pass.cuh"
@@ -337,16 +338,23 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     float hb = first ? h0v : 0.f;  // state before this chunk
     int last_bad = -1, updates = 0, k = 0;
     float final_m = 0.f;
-    for (;; ++k) {
-      const bool cap = (k >= p.max_iters);
+    bool apx = p.apx_tau > 0.f;  // cluster-uniform: set from the tile's residual maximum
+    // one Newton iteration of the tile (kMode 0: exact evaluation and update,
+    // 1: inexact evaluation and update, 2: exact residual only, at the cap);
+    // true when the tile is done
+    auto iterate = [&](auto mode) -> bool {
+      constexpr int kMode = decltype(mode)::value;
+      constexpr bool cap = kMode == 2, apx_eval = kMode == 1;
       const int par = phase & 1;
       const unsigned mpar = (phase >> 1) & 1;  // phase parity of mbar[par]
       ++phase;
       const float last_pre = H[kRowH - 1].y;
       float2 DL, PA;
       float m;
-      if (cap)
+      if constexpr (cap)
         m = row_pass<kRowH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
+      else if constexpr (apx_eval)
+        m = row_pass_apx<kRowH>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else
         m = row_pass<kRowH, true>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       if (!dval) m = 0.f;
@@ -388,7 +396,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < kRowWarps; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (!(chm < p.tol)) last_bad = k;
+        if (apx_eval || !(chm < p.tol)) last_bad = k;
       }
       // maps of the warps before this one: CTA incoming delta -> delta
       // entering this warp; and the CTA's residual maximum
@@ -448,11 +456,14 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         if (tid == 0 && got) mbar_arrive_expect_tx(&sh.mbar[par], rx);
       }
       final_m = tmax;
-      const bool own_ok = tmax < p.tol;
-      if (cap) {
+      // an inexact evaluation never decides convergence; the first one whose
+      // residual is at most apx_tau hands over to exact evaluations
+      const bool own_ok = !apx_eval && tmax < p.tol;
+      if (apx_eval && tmax <= p.apx_tau) apx = false;
+      if constexpr (cap) {
         updates = k;
         if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        break;
+        return true;
       }
       const float cin = fmaf(cP, din_cta, cd);  // delta entering this warp
       const float din = first ? 0.f : fmaf(xP, cin, xd);
@@ -464,7 +475,17 @@ __global__ void __launch_bounds__(kRowThreads, 2)
 #pragma unroll
       for (int i = 0; i < kRowH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
       updates = k + 1;
-      if (own_ok) break;
+      return own_ok;
+    };
+    // inexact iterations while the residual is large, then exact ones to
+    // convergence or the cap (k: the evaluation's index)
+    for (; apx && k < p.max_iters; ++k) iterate(std::integral_constant<int, 1>{});
+    for (;; ++k) {
+      if (k >= p.max_iters) {
+        iterate(std::integral_constant<int, 2>{});
+        break;
+      }
+      if (iterate(std::integral_constant<int, 0>{})) break;
     }
     // every thread of the CTA is past its last pass of this tile (the
     // barrier of the last exchange): the staging area takes the next tile

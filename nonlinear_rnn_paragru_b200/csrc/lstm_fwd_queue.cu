@@ -75,7 +75,6 @@ constexpr int kLqBoxBytes = kLqSteps * kLqG * kLqC * 2;  // 8192: one box of 128
 constexpr int kLqStage = kLqU;                      // bf16 staging after the arguments
 constexpr int kLqSmem = kLqStage + kLqBoxBytes;
 constexpr int kLqMinB = 4;                          // CTAs per SM
-constexpr float kLqApxTau = 0.1f;
 static_assert(kLqS % 128 == 64, "a warp's four chunks in alternate 64-byte bank halves");
 static_assert(kLqStage % 128 == 0, "TMA destination");
 static_assert(2 * kLqThreads == kLqChunks * kLqH * kLqG, "the expansion: two gates per thread");
@@ -589,7 +588,7 @@ int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* coun
   p.nitems = (int)nitems;
   p.max_iters = f.max_iters;
   p.tol = f.tol;
-  p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kLqApxTau;
+  p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kApxTau;
   p.timeout_ns = f.timeout_ns;
   p.counter = counter;
   p.seg_done = seg_done;

@@ -89,7 +89,7 @@ def test_residual_of_result_is_small(cuda_ok):
 
 def test_iteration_histogram_matches_oracle_counts(cuda_ok):
     x = make_inputs(WORKLOADS[4].scaled(B=1, T=2048, D=64))
-    _, st, hist = _solve(x, hist=True, max_iters=32)
+    _, st, hist = _solve(x, hist=True, max_iters=32, flags=pr.PARARNN_FLAG_EXACT_STEPS)
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=32)
     # counts are reported, not asserted equal: fp32 vs fp64 may differ by one
     ks = np.nonzero(hist)[0]
@@ -100,9 +100,10 @@ def test_iteration_histogram_matches_oracle_counts(cuda_ok):
 @pytest.mark.parametrize("n", [1, 2, 3])
 def test_capped_iterates_match_oracle_newton(cuda_ok, n):
     # with the cap at n updates the solver returns the n-th Newton iterate
-    # (states after n updates of the page's scheme) and NOT_CONVERGED
+    # (states after n updates of the page's scheme) and NOT_CONVERGED; exact
+    # steps throughout
     x = make_inputs(WORKLOADS[2].scaled(B=1, T=1300, D=64))
-    h, st, _ = _solve(x, max_iters=n)
+    h, st, _ = _solve(x, max_iters=n, flags=pr.PARARNN_FLAG_EXACT_STEPS)
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=0.0, max_iters=n)
     assert st["status"] == "not_converged"
     assert st["iters"] == n and st["evals"] == n + 1
@@ -247,7 +248,7 @@ def test_channel_iteration_index_matches_oracle(cuda_ok, B, T, D, wl, flags):
     # sequences here are solved in one launch (no segments).
     x = make_inputs(WORKLOADS[wl].scaled(B=B, T=T, D=D))
     ci = torch.full((B, D), -5, dtype=torch.int32, device="cuda")
-    h, st, hist = _solve(x, hist=True, chan_iters=ci, flags=flags)
+    h, st, hist = _solve(x, hist=True, chan_iters=ci, flags=flags | pr.PARARNN_FLAG_EXACT_STEPS)
     k_gpu = ci.cpu().numpy()
     r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=1e-6, max_iters=64)
     diff = np.abs(k_gpu - r["chan_k"])
