@@ -76,6 +76,7 @@ constexpr int kLqStage = kLqU;                      // bf16 staging after the ar
 constexpr int kLqSmem = kLqStage + kLqBoxBytes;
 constexpr int kLqMinB = 4;                          // CTAs per SM
 static_assert(kLqS % 128 == 64, "a warp's four chunks in alternate 64-byte bank halves");
+static_assert(kLqW % 4 == 0, "the item's residual maximum is read as float4s");
 static_assert(kLqStage % 128 == 0, "TMA destination");
 static_assert(2 * kLqThreads == kLqChunks * kLqH * kLqG, "the expansion: two gates per thread");
 
@@ -452,8 +453,12 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
                     fmaf(m0.z, cin.x, fmaf(m0.w, cin.y, m1.y)));
         }
       }
-      const float4 wm4 = *reinterpret_cast<const float4*>(&sh.wmax[par][0]);
-      const float tmax = fmax_nan(fmax_nan(wm4.x, wm4.y), fmax_nan(wm4.z, wm4.w));
+      float tmax = 0.f;
+#pragma unroll
+      for (int w4 = 0; w4 < kLqW; w4 += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(&sh.wmax[par][w4]);
+        tmax = fmax_nan(tmax, fmax_nan(fmax_nan(v.x, v.y), fmax_nan(v.z, v.w)));
+      }
       final_m = tmax;
       // an inexact evaluation never decides convergence; the first one whose
       // residual is at most apx_tau hands over to exact evaluations
