@@ -348,47 +348,53 @@ __global__ void dn_transpose_w(const float* __restrict__ W, float* __restrict__ 
   }
 }
 
-// One CTA per (b, padded step t): gates from the pre-activations of h_{t-1},
-// residual, -r_t and J_t; padded steps (t >= T) get J = I and -r = 0.
+// One CTA per (b, four consecutive padded steps t0..t0+3): gates from the
+// pre-activations of h_{t-1}, residual, -r_t and J_t for each; padded steps
+// (t >= T) get J = I and -r = 0.  The two odd steps are stored row-major and
+// the two even ones transposed, so every float4 of a W (Wt) row is loaded
+// once for two steps.
+constexpr int kDnAsm = 4;  // steps per assembly CTA (Tp is a multiple of 16)
 template <bool kBF16>
 __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
-  __shared__ float co[4][kDnMaxD];
+  __shared__ __align__(16) float co[kDnAsm][4][kDnMaxD];
   __shared__ unsigned wmax[kDnThreads / 32];
   const int D = p.D;
-  const size_t bt = blockIdx.x;  // b * Tp + t
-  const int b = (int)(bt / p.Tp), t = (int)(bt - (size_t)b * p.Tp);
+  const int groups = p.Tp / kDnAsm;
+  const int b = (int)(blockIdx.x / groups), t0 = (int)(blockIdx.x % groups) * kDnAsm;
   const size_t DD = (size_t)D * D;
-  float* Jt = p.J + bt * DD;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (t >= p.T) {
-    for (int i = warp; i < D; i += kDnThreads / 32)
-      for (int j = lane; j < D; j += 32) Jt[(size_t)i * D + j] = (i == j) ? 1.f : 0.f;
-    for (int i = threadIdx.x; i < D; i += blockDim.x) p.rhs[bt * D + i] = 0.f;
-    return;
-  }
-  const size_t bs = (size_t)b * p.T + t;  // (b, t) in the unpadded arrays
-  const float* q3 = t > 0 ? p.Q + (bs - 1) * 3 * D : p.Q0 + (size_t)b * 3 * D;
   unsigned m = 0;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) {
-    const float hp = t > 0 ? p.h[(bs - 1) * D + i] : (p.h0 ? p.h0[(size_t)b * D + i] : 0.f);
-    const size_t iu = bs * 3 * D + i;
-    const float z = dn_sig(q3[i] + dn_u<kBF16>(p.u, iu) + (p.bias ? p.bias[i] : 0.f));
-    const float r = dn_sig(q3[D + i] + dn_u<kBF16>(p.u, iu + D) + (p.bias ? p.bias[D + i] : 0.f));
-    const float q = q3[2 * D + i];
-    const float c =
-        tanhf(dn_u<kBF16>(p.u, iu + 2 * (size_t)D) + (p.bias ? p.bias[2 * D + i] : 0.f) + r * q);
-    const float f = fmaf(z, c - hp, hp);
-    const float res = p.h[bs * D + i] - f;
-    p.rhs[bt * D + i] = -res;
-    m = max(m, dn_abs_bits(res));
-    const float gc = z * (1.f - c * c);
-    co[0][i] = 1.f - z;
-    co[1][i] = (c - hp) * z * (1.f - z);
-    co[2][i] = gc * r;
-    co[3][i] = gc * q * r * (1.f - r);
+#pragma unroll 1
+  for (int st = 0; st < kDnAsm; ++st) {
+    const int t = t0 + st;
+    const size_t bt = (size_t)b * p.Tp + t;
+    if (t >= p.T) {
+      for (int i = threadIdx.x; i < D; i += blockDim.x) p.rhs[bt * D + i] = 0.f;
+      continue;
+    }
+    const size_t bs = (size_t)b * p.T + t;  // (b, t) in the unpadded arrays
+    const float* q3 = t > 0 ? p.Q + (bs - 1) * 3 * D : p.Q0 + (size_t)b * 3 * D;
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+      const float hp = t > 0 ? p.h[(bs - 1) * D + i] : (p.h0 ? p.h0[(size_t)b * D + i] : 0.f);
+      const size_t iu = bs * 3 * D + i;
+      const float z = dn_sig(q3[i] + dn_u<kBF16>(p.u, iu) + (p.bias ? p.bias[i] : 0.f));
+      const float r = dn_sig(q3[D + i] + dn_u<kBF16>(p.u, iu + D) + (p.bias ? p.bias[D + i] : 0.f));
+      const float q = q3[2 * D + i];
+      const float c =
+          tanhf(dn_u<kBF16>(p.u, iu + 2 * (size_t)D) + (p.bias ? p.bias[2 * D + i] : 0.f) + r * q);
+      const float f = fmaf(z, c - hp, hp);
+      const float res = p.h[bs * D + i] - f;
+      p.rhs[bt * D + i] = -res;
+      m = max(m, dn_abs_bits(res));
+      const float gc = z * (1.f - c * c);
+      co[st][0][i] = 1.f - z;
+      co[st][1][i] = (c - hp) * z * (1.f - z);
+      co[st][2][i] = gc * r;
+      co[st][3][i] = gc * q * r * (1.f - r);
+    }
   }
   m = __reduce_max_sync(0xffffffffu, m);
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  if (lane == 0) wmax[warp] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
     unsigned mm = 0;
@@ -396,23 +402,63 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
     atomicMax(p.rmax, mm);
   }
   // J[i][j] = [i == j] (1 - z_i) + co1_i Wz[i][j] + co2_i Wc[i][j] + co3_i Wr[i][j];
-  // a warp per row of the stored layout, lanes along it (coalesced)
-  if (t & 1) {  // row-major: row i, element (i, j) at i * D + j
-    for (int i = warp; i < D; i += kDnThreads / 32) {
-      const float c0 = co[0][i], c1 = co[1][i], c2 = co[2][i], c3 = co[3][i];
-      const size_t r0 = (size_t)i * D;
-      for (int j = lane; j < D; j += 32) {
-        const size_t e = r0 + j;
-        Jt[e] = (i == j ? c0 : 0.f) + c1 * p.W[e] + c2 * p.W[2 * DD + e] + c3 * p.W[DD + e];
+  // a warp per stored row, lanes along it in float4s (coalesced, every load
+  // of the row in flight before the stores)
+  constexpr int kQ4 = kDnMaxD / 128;
+  const int D4 = D >> 2;
+#pragma unroll 1
+  for (int parity = 1; parity >= 0; --parity) {  // odd steps row-major, even transposed
+    const float* Wsrc = parity ? p.W : p.Wt;
+    const int sa = parity, sb = parity + 2;       // the group's two steps of this parity
+    const bool va = t0 + sa < p.T, vb = t0 + sb < p.T;
+    float* Ja = p.J + ((size_t)b * p.Tp + t0 + sa) * DD;
+    float* Jb = p.J + ((size_t)b * p.Tp + t0 + sb) * DD;
+    for (int row = warp; row < D; row += kDnThreads / 32) {
+      float4 wz[kQ4], wr[kQ4], wc[kQ4];
+#pragma unroll
+      for (int k = 0; k < kQ4; ++k) {
+        const int q4 = lane + 32 * k;
+        if (q4 < D4) {
+          const float4* base = reinterpret_cast<const float4*>(Wsrc + (size_t)row * D) + q4;
+          wz[k] = __ldg(base);
+          wr[k] = __ldg(base + DD / 4);
+          wc[k] = __ldg(base + 2 * DD / 4);
+        }
       }
-    }
-  } else {      // transposed: row j holds column j, element (i, j) at j * D + i
-    for (int j = warp; j < D; j += kDnThreads / 32) {
-      const size_t r0 = (size_t)j * D;
-      for (int i = lane; i < D; i += 32) {
-        const size_t e = r0 + i;
-        Jt[e] = (i == j ? co[0][i] : 0.f) + co[1][i] * p.Wt[e] + co[2][i] * p.Wt[2 * DD + e] +
-                co[3][i] * p.Wt[DD + e];
+#pragma unroll
+      for (int k = 0; k < kQ4; ++k) {
+        const int q4 = lane + 32 * k;
+        if (q4 >= D4) continue;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const int s = which ? sb : sa;
+          const bool valid = which ? vb : va;
+          float* Jt = which ? Jb : Ja;
+          float4 o;
+          if (!valid) {  // padded step: the identity
+            o = make_float4(row == 4 * q4 ? 1.f : 0.f, row == 4 * q4 + 1 ? 1.f : 0.f,
+                            row == 4 * q4 + 2 ? 1.f : 0.f, row == 4 * q4 + 3 ? 1.f : 0.f);
+          } else if (parity) {  // row-major: element (row, j), row coefficients
+            const float c1 = co[s][1][row], c2 = co[s][2][row], c3 = co[s][3][row];
+            o.x = fmaf(c1, wz[k].x, fmaf(c2, wc[k].x, c3 * wr[k].x));
+            o.y = fmaf(c1, wz[k].y, fmaf(c2, wc[k].y, c3 * wr[k].y));
+            o.z = fmaf(c1, wz[k].z, fmaf(c2, wc[k].z, c3 * wr[k].z));
+            o.w = fmaf(c1, wz[k].w, fmaf(c2, wc[k].w, c3 * wr[k].w));
+            const int dj = row - 4 * q4;  // the diagonal element, if in this float4
+            if (dj >= 0 && dj < 4) (&o.x)[dj] += co[s][0][row];
+          } else {  // transposed: stored row j = row holds column j, element (i, j)
+            const float4 c1 = reinterpret_cast<const float4*>(co[s][1])[q4];
+            const float4 c2 = reinterpret_cast<const float4*>(co[s][2])[q4];
+            const float4 c3 = reinterpret_cast<const float4*>(co[s][3])[q4];
+            o.x = fmaf(c1.x, wz[k].x, fmaf(c2.x, wc[k].x, c3.x * wr[k].x));
+            o.y = fmaf(c1.y, wz[k].y, fmaf(c2.y, wc[k].y, c3.y * wr[k].y));
+            o.z = fmaf(c1.z, wz[k].z, fmaf(c2.z, wc[k].z, c3.z * wr[k].z));
+            o.w = fmaf(c1.w, wz[k].w, fmaf(c2.w, wc[k].w, c3.w * wr[k].w));
+            const int di = row - 4 * q4;
+            if (di >= 0 && di < 4) (&o.x)[di] += co[s][0][row];
+          }
+          reinterpret_cast<float4*>(Jt + (size_t)row * D)[q4] = o;
+        }
       }
     }
   }
@@ -427,7 +473,7 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
 namespace cgd = cooperative_groups;
 
 struct DnVec {
-  float x[2][kDnMaxD];       // the vector, double-buffered by step parity
+  __align__(16) float x[2][kDnMaxD];  // the vector, double-buffered by step parity
   float part[2 * kDnMaxD];   // transposed layout: partial sums of the q groups, [qg][row]
 };
 
@@ -442,18 +488,52 @@ __device__ __forceinline__ void dn_cmatvec(cgd::cluster_group& cl, DnVec& v, int
   const float* x = v.x[cur];
   float* y_local = v.x[cur ^ 1];
   const int ncl = (int)cl.num_blocks();
-  if (rowmajor) {  // a warp per row, lanes along it
-    for (int ii = warp; ii < R; ii += kDnThreads / 32) {
-      const int i = r0 + ii;
-      const float* Mi = M + (size_t)i * D;
-      float s = 0.f;
-      for (int q = lane; q < D; q += 32) s = fmaf(Mi[q], x[q], s);
+  if (rowmajor) {
+    // a warp per row, lanes along it in float4s, four rows at a time: every
+    // lane has its 4 x (D / 128) loads in flight before the first fma (the
+    // chain reads a fresh D x D matrix each step, so the pass is bound by
+    // how many loads are in flight)
+    constexpr int kRows = 4, kQ4 = kDnMaxD / 128;
+    const int D4 = D >> 2;
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    for (int i0 = warp * kRows; i0 < R; i0 += (kDnThreads / 32) * kRows) {
+      float4 mv[kRows][kQ4];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) {
-        s += add ? add[i] : 0.f;
-        for (int r = 0; r < ncl; ++r) cl.map_shared_rank(y_local, r)[i] = s;
-        if (yout) yout[i] = s;
+      for (int rr = 0; rr < kRows; ++rr)
+#pragma unroll
+        for (int k = 0; k < kQ4; ++k) {
+          const int q4 = lane + 32 * k;
+          mv[rr][k] = (i0 + rr < R && q4 < D4)
+                          ? __ldg(reinterpret_cast<const float4*>(M + (size_t)(r0 + i0 + rr) * D) + q4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      float s[kRows];
+#pragma unroll
+      for (int rr = 0; rr < kRows; ++rr) {
+        s[rr] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kQ4; ++k) {
+          const int q4 = lane + 32 * k;
+          if (q4 < D4) {
+            const float4 xv = x4[q4];
+            s[rr] = fmaf(mv[rr][k].x, xv.x, s[rr]);
+            s[rr] = fmaf(mv[rr][k].y, xv.y, s[rr]);
+            s[rr] = fmaf(mv[rr][k].z, xv.z, s[rr]);
+            s[rr] = fmaf(mv[rr][k].w, xv.w, s[rr]);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s[rr] += __shfl_xor_sync(0xffffffffu, s[rr], o);
+      }
+      if (lane < kRows && i0 + lane < R) {
+        float sv = s[0];
+#pragma unroll
+        for (int rr = 1; rr < kRows; ++rr)
+          if (lane == rr) sv = s[rr];
+        const int i = r0 + i0 + lane;
+        sv += add ? add[i] : 0.f;
+        for (int r = 0; r < ncl; ++r) cl.map_shared_rank(y_local, r)[i] = sv;
+        if (yout) yout[i] = sv;
       }
     }
   } else {  // threads over (row offset, quarter of q): rows contiguous in M[q][.]
@@ -463,9 +543,15 @@ __device__ __forceinline__ void dn_cmatvec(cgd::cluster_group& cl, DnVec& v, int
       const int ii = e % R, qg = e / R;
       const int i = r0 + ii;
       const int q0 = qg * qlen, q1 = min(D, q0 + qlen);
-      float s = 0.f;
-      for (int q = q0; q < q1; ++q) s = fmaf(M[(size_t)q * D + i], x[q], s);
-      v.part[qg * R + ii] = s;
+      // eight independent sums, so that eight loads are in flight
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int q = q0;
+      for (; q + 8 <= q1; q += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s8[u] = fmaf(__ldg(M + (size_t)(q + u) * D + i), x[q + u], s8[u]);
+      }
+      for (; q < q1; ++q) s8[0] = fmaf(__ldg(M + (size_t)q * D + i), x[q], s8[0]);
+      v.part[qg * R + ii] = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
     }
     __syncthreads();
     for (int ii = threadIdx.x; ii < R; ii += kDnThreads) {
@@ -715,7 +801,7 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
     dn_split<<<sgrid, 256, 0, stream>>>(h, hhi, hlo, BT * D);
     ge = split_gemm(mhh, mhl, Q, (int)BT);
     if (ge) return ge;
-    const unsigned nblk = (unsigned)((size_t)B * p.Tp);
+    const unsigned nblk = (unsigned)((size_t)B * (p.Tp / kDnAsm));
     if (bf16)
       dn_assemble2<true><<<nblk, kDnThreads, 0, stream>>>(p);
     else
