@@ -41,8 +41,11 @@
 //
 // Data.  u arrives by one TMA box of 128 steps into a staging area, is
 // expanded into fp32 arguments (-log2e u + b' for i, f, o; 2 log2e u + b' for
-// g) laid out per chunk as [gate][pair i][channel] {step i, step i + 4},
-// channel c at slot c ^ (i >> 1), and the next item's box is issued as soon
+// g) laid out per chunk q as [gate][pair i][channel] {step i, step i + 4},
+// channel c at slot c ^ ((q + 2 (i >> 1)) & 7): the expansion's lanes, which
+// cover 8 chunks x 4 pairs of one channel, then write each 256-byte row
+// with every bank pair twice, and a warp's reads in the pass stay one
+// 64-byte window per chunk.  The next item's box is issued as soon
 // as the expansion is done.  a, bias (and c0, h0 for a first segment) of the
 // next item's channels are loaded during the current item.  Steps past T get
 // i and o shut and f open.
@@ -135,7 +138,8 @@ struct LqPar {
 // delta: C, H become the local solution, P the running products, Mx / My
 // the halves' maps.  Returns max over steps of max(|c_t - c'_t|, |h_t - h'_t|).
 template <int kMode>
-__device__ __forceinline__ float lq_pass(const unsigned char* __restrict__ base, int c8, float cb,
+__device__ __forceinline__ float lq_pass(const unsigned char* __restrict__ base, int so0, int so1,
+                                         float cb,
                                          float hb, float2 (&C)[kLqH], float2 (&H)[kLqH],
                                          float2 (&P00)[kLqH], float2 (&P01)[kLqH],
                                          float2 (&P10)[kLqH], float2 (&P11)[kLqH],
@@ -150,7 +154,7 @@ __device__ __forceinline__ float lq_pass(const unsigned char* __restrict__ base,
   float2 CP = qf2(cb, C[kLqH - 1].x), HP = qf2(hb, H[kLqH - 1].x);  // before steps 0 and 4
 #pragma unroll
   for (int i = 0; i < kLqH; ++i) {
-    const unsigned char* bi = base + ((c8 ^ ((i >> 1) * 8)) + i * kLqC * 8);
+    const unsigned char* bi = base + ((i >> 1) ? so1 : so0) + i * kLqC * 8;
     const float2 UI = *reinterpret_cast<const float2*>(bi);
     const float2 UF = *reinterpret_cast<const float2*>(bi + 1 * kLqRowB);
     const float2 UG = *reinterpret_cast<const float2*>(bi + 2 * kLqRowB);
@@ -267,6 +271,8 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
   const int c = lane % kLqC, kk = lane / kLqC;
   const int q = warp * kLqK + kk;  // chunk index within the item
   const unsigned char* base = smem + q * kLqS;
+  // this thread's channel slot in its chunk for pairs 0, 1 and for pairs 2, 3
+  const int so0 = (c ^ (q & 7)) * 8, so1 = (c ^ ((q + 2) & 7)) * 8;
 
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
@@ -312,7 +318,7 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     {
       const int unit = tid % (kLqChunks * kLqH), half = tid / (kLqChunks * kLqH);
       const int qq = unit / kLqH, i = unit % kLqH;
-      const int sw = i >> 1;
+      const int sw = (qq + 2 * (i >> 1)) & 7;
       const int ta = qq * kLqL + i, tb = ta + kLqH;  // steps within the item
       const bool pa = ta >= t_len, pbd = tb >= t_len;
       unsigned char* dst = smem + qq * kLqS + i * kLqC * 8;
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       ++phase;
       const float lastc = C[kLqH - 1].y, lasth = H[kLqH - 1].y;
       Aff2 Mx, My;
-      float m = lq_pass<kMode>(base, c * 8, cb, hb, C, H, P00, P01, P10, P11, k, Mx, My);
+      float m = lq_pass<kMode>(base, so0, so1, cb, hb, C, H, P00, P01, P10, P11, k, Mx, My);
       if (!dval) m = 0.f;
       // the chunk's map: second half after the first
       Aff2 inc = My.after(Mx);
