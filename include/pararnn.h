@@ -369,8 +369,12 @@ size_t pararnn_dense_workspace_size(int B, int T, int D);
  * can be checked on its own: C[z] = A[z] B[z]^T for z < Z, with A[z] M x K
  * and B[z] N x K row-major fp32 (A[z] at A + z M K, B[z] at Bm + z N K),
  * tf32 products (tcgen05.mma kind::tf32) accumulated in fp32.  C[z] at
- * C + z M N: row-major M x N (store_mode 0), transposed N x M (1), or
- * row-major for odd z and transposed for even z (2).  K a multiple of 4; A,
+ * C + z M N: row-major M x N (store_mode 0), transposed N x M (1),
+ * row-major for odd z and transposed for even z (2), or row-major with the
+ * product added to what C holds (3).  Launches with at least one 128 x 256
+ * output tile per SM run a persistent kernel (one CTA per SM, 128 x 256
+ * tiles, two accumulators in tensor memory), smaller ones one CTA per
+ * 128 x 128 tile.  K a multiple of 4; A,
  * Bm, C 16-byte aligned.  *err (device int) is set to 1 if a bounded wait ran
  * out (the affected tiles are not written); it is not cleared. */
 int pararnn_dense_matmul(const float* A, const float* Bm, float* C, int M,

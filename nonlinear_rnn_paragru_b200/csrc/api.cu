@@ -664,7 +664,7 @@ int pararnn_solve_unfused(int cell, const void* u, int u_dtype, const float* a, 
 int pararnn_dense_matmul(const float* A, const float* Bm, float* C, int M, int N, int K, int Z,
                          int store_mode, int* err, pararnn_stream_t stream) {
   if (!A || !Bm || !C || !err || M < 1 || N < 1 || K < 1 || Z < 1 || (K % 4) != 0 ||
-      store_mode < 0 || store_mode > 2)
+      store_mode < 0 || store_mode > 3)
     return PARARNN_ERR_INVALID_ARG;
   if ((long long)M * N * Z >= (1LL << 40) || M >= (1 << 30) || N >= (1 << 30))
     return PARARNN_ERR_TOO_LARGE;

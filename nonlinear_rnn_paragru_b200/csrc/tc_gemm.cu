@@ -23,6 +23,15 @@
 // Every wait is bounded: a wait that runs out sets *err, the CTA skips its
 // stores, and it frees its tensor memory before returning.  Loads past the
 // matrices' edges read zeros (TMA out-of-bounds fill); stores are masked.
+//
+// Large launches (at least one 128 x 256 output tile per SM) take the
+// persistent form instead, one CTA per SM working off tiles in a fixed
+// order: 128 x 256 tiles (a third less operand traffic per product than
+// 128 x 128), a 4-stage ring of 48 KB stages, and two 128 x 256 accumulators
+// in tensor memory (all 512 columns), so the epilogue of one tile overlaps
+// the products of the next.  Warp 0 loads, warp 1 issues the products,
+// warps 2-5 (tensor-memory lane quarters 2, 3, 0, 1) read the accumulators
+// and store.
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
@@ -229,6 +238,211 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                  : "memory");
 }
 
+// ------------------------------------------------------ persistent form --
+constexpr int kPgBM = 128, kPgBN = 256;
+constexpr int kPgStages = 4;
+constexpr int kPgABytes = kPgBM * kTcBK * 4;                  // 16384
+constexpr int kPgBBytes = kPgBN * kTcBK * 4;                  // 32768: two 128-row boxes
+constexpr int kPgStageBytes = kPgABytes + kPgBBytes;
+constexpr int kPgSmem = kPgStages * kPgStageBytes + 1024;     // + alignment slack
+constexpr int kPgThreads = 192;
+constexpr uint32_t kPgCols = 512;                              // two fp32 accumulators, N = 256
+constexpr uint32_t kPgIdesc = (1u << 4) | (2u << 7) | (2u << 10) |
+                              ((uint32_t)(kPgBN >> 3) << 17) | ((uint32_t)(kPgBM >> 4) << 24);
+static_assert(kPgBN % kTcBM == 0, "the B tile is whole boxes of the operand map");
+
+struct PgShared {
+  uint64_t full[kPgStages], empty[kPgStages];
+  uint64_t acc_full[2], acc_empty[2], done;
+  uint32_t tmem;
+  int fail;
+};
+
+__device__ __forceinline__ void pg_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool pg_failed(const PgShared& sh) {
+  return *reinterpret_cast<const volatile int*>(&sh.fail) != 0;
+}
+__device__ __forceinline__ void pg_fail(PgShared& sh) {
+  *reinterpret_cast<volatile int*>(&sh.fail) = 1;
+}
+__device__ __forceinline__ void pg_mma(uint32_t tmem, uint64_t da, uint64_t db, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+      "l"(da), "l"(db), "r"(kPgIdesc), "r"(acc)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kPgThreads, 1)
+    tc_gemm_tf32_persistent(const __grid_constant__ CUtensorMap ma,
+                            const __grid_constant__ CUtensorMap mb, const TcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ PgShared sh;
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tm = (p.M + kPgBM - 1) / kPgBM, tn = (p.N + kPgBN - 1) / kPgBN;
+  const int ntiles = tm * tn * p.Z;
+  const int nk = (p.K + kTcBK - 1) / kTcBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPgStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.acc_full[a], 1);
+      mbar_init(&sh.acc_empty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&sh.done, 1);
+    sh.fail = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sh.tmem)),
+                 "r"(kPgCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // producer: every tile's K slices into the ring
+      int it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !pg_failed(sh); tile += gridDim.x) {
+        const int z = tile / (tm * tn), rem = tile - z * (tm * tn);
+        const int m0 = (rem % tm) * kPgBM, n0 = (rem / tm) * kPgBN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kPgStages;
+          if (it >= kPgStages &&
+              !mbar_wait_bounded(&sh.empty[s], ((it / kPgStages) - 1) & 1, kTcTimeoutNs)) {
+            pg_fail(sh);
+            break;
+          }
+          unsigned char* st = smem + s * kPgStageBytes;
+          mbar_arrive_expect_tx(&sh.full[s], (unsigned)kPgStageBytes);
+          tma_load_3d(st, &ma, &sh.full[s], kb * kTcBK, m0, z);
+#pragma unroll
+          for (int h = 0; h < kPgBN / kTcBM; ++h)
+            tma_load_3d(st + kPgABytes + h * kTcBM * kTcBK * 4, &mb, &sh.full[s], kb * kTcBK,
+                        n0 + h * kTcBM, z);
+        }
+      }
+      // loads still in flight (a failed run): wait for them, bounded
+      if (pg_failed(sh))
+        for (int back = 1; back <= kPgStages && it - back >= 0; ++back) {
+          const int j = it - back;
+          mbar_wait_bounded(&sh.full[j % kPgStages], (j / kPgStages) & 1, kTcTimeoutNs);
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // products: a tile into accumulator j & 1, once the epilogue has read
+      // what that accumulator held two tiles before
+      int it = 0, j = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !pg_failed(sh); tile += gridDim.x, ++j) {
+        const int ab = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(&sh.acc_empty[ab], ((j >> 1) - 1) & 1, kTcTimeoutNs)) {
+          pg_fail(sh);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(ab * kPgBN);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kPgStages;
+          if (!mbar_wait_bounded(&sh.full[s], (it / kPgStages) & 1, kTcTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + s * kPgStageBytes), b0 = a0 + kPgABytes;
+#pragma unroll
+          for (int k = 0; k < kTcBK / 8; ++k)  // K = 8 tf32 (32 bytes) per instruction
+            pg_mma(d, tc_sdesc(a0 + k * 32), tc_sdesc(b0 + k * 32), (kb | k) != 0);
+          tc_commit(&sh.empty[s]);  // the stage is free once these products are done
+        }
+        if (!ok) {
+          pg_fail(sh);
+          break;
+        }
+        tc_commit(&sh.acc_full[ab]);
+      }
+      tc_commit(&sh.done);  // every product issued is done
+    }
+  } else {
+    // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (rows)
+    const int eq = warp & 3;
+    const bool trans_all = p.store_mode == 1;
+    int j = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !pg_failed(sh); tile += gridDim.x, ++j) {
+      const int ab = j & 1;
+      if (!mbar_wait_bounded(&sh.acc_full[ab], (j >> 1) & 1, kTcTimeoutNs)) {
+        pg_fail(sh);
+        break;
+      }
+      tc_fence_after();
+      const int z = tile / (tm * tn), rem = tile - z * (tm * tn);
+      const int m0 = (rem % tm) * kPgBM, n0 = (rem / tm) * kPgBN;
+      const int row = m0 + eq * 32 + lane;
+      const bool trans = trans_all || (p.store_mode == 2 && (z & 1) == 0);
+      float* Cz = p.C + (size_t)z * p.M * p.N;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kPgBN; c0 += 32) {
+        if (n0 + c0 >= p.N) break;
+        uint32_t r[32];
+        tc_ld32(tmem + ((uint32_t)(eq * 32) << 16) + (uint32_t)(ab * kPgBN + c0), r);
+        if (row < p.M) {
+          if (trans) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+              const int col = n0 + c0 + jj;
+              if (col < p.N) Cz[(size_t)col * p.M + row] = __uint_as_float(r[jj]);
+            }
+          } else if (p.store_mode == 3) {
+            float* dst = Cz + (size_t)row * p.N + n0 + c0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (n0 + c0 + jj < p.N) dst[jj] += __uint_as_float(r[jj]);
+          } else {
+            float* dst = Cz + (size_t)row * p.N + n0 + c0;
+            if (n0 + c0 + 32 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+              for (int jj = 0; jj < 32; jj += 4)
+                *reinterpret_cast<float4*>(dst + jj) =
+                    make_float4(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]),
+                                __uint_as_float(r[jj + 2]), __uint_as_float(r[jj + 3]));
+            } else {
+#pragma unroll
+              for (int jj = 0; jj < 32; ++jj)
+                if (n0 + c0 + jj < p.N) dst[jj] = __uint_as_float(r[jj]);
+            }
+          }
+        }
+      }
+      // this warp has read its quarter of the accumulator: the products may
+      // reuse it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) pg_arrive(&sh.acc_empty[ab]);
+    }
+  }
+  // every product done before the tensor memory goes back (bounded)
+  if (tid == 0 && !mbar_wait_bounded(&sh.done, 0, kTcTimeoutNs)) pg_fail(sh);
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && sh.fail) atomicExch(p.err, 1);
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPgCols)
+                 : "memory");
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tc_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -278,6 +492,17 @@ int launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, float* C, int M
   p.err = err;
   const long long tiles = (long long)((M + kTcBM - 1) / kTcBM) * ((N + kTcBN - 1) / kTcBN) * Z;
   if (tiles >= (1LL << 31)) return (int)cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long ptiles = (long long)((M + kPgBM - 1) / kPgBM) * ((N + kPgBN - 1) / kPgBN) * Z;
+  if (ptiles >= sms) {  // the persistent form: one CTA per SM
+    e = cudaFuncSetAttribute(tc_gemm_tf32_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kPgSmem);
+    if (e != cudaSuccess) return (int)e;
+    tc_gemm_tf32_persistent<<<(unsigned)sms, kPgThreads, kPgSmem, stream>>>(ma, mb, p);
+    return (int)cudaGetLastError();
+  }
   tc_gemm_tf32<<<(unsigned)tiles, kTcThreads, kTcSmem, stream>>>(ma, mb, p);
   return (int)cudaGetLastError();
 }

@@ -125,7 +125,7 @@ def _cases(pr):
         C["dense_" + name] = ((lambda o: lambda lib: _dense(lib, pr, **o))(over), code)
     for name, args, code in [
             ("K_not_multiple_of_4", (0x1000, 0x2000, 0x3000, 8, 8, 6, 1, 0, 0x4000, None), -1),
-            ("bad_store_mode", (0x1000, 0x2000, 0x3000, 8, 8, 8, 1, 3, 0x4000, None), -1),
+            ("bad_store_mode", (0x1000, 0x2000, 0x3000, 8, 8, 8, 1, 4, 0x4000, None), -1),
             ("no_err", (0x1000, 0x2000, 0x3000, 8, 8, 8, 1, 0, None, None), -1),
             ("A_misaligned", (0x1004, 0x2000, 0x3000, 8, 8, 8, 1, 0, 0x4000, None), -5)]:
         C["dense_matmul_" + name] = ((lambda a_: lambda lib: lib.pararnn_dense_matmul(*a_))(args),

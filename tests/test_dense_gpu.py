@@ -70,6 +70,32 @@ def test_tensor_core_matmul_matches_fp64(cuda_ok, M, N, K, Z, mode):
         assert rel < 1e-3, (z, rel)
 
 
+# launches with at least one 128 x 256 tile per SM take the persistent form
+# (one CTA per SM, double-buffered accumulators): all four store modes, ragged
+# edges in M, N and K
+@pytest.mark.parametrize("M,N,K,Z,mode", [(512, 512, 256, 40, 0), (300, 520, 96, 60, 2),
+                                          (512, 512, 512, 20, 1), (256, 384, 64, 110, 3)])
+def test_tensor_core_matmul_persistent_matches_fp64(cuda_ok, M, N, K, Z, mode):
+    g = torch.Generator().manual_seed(M + N + K + Z + 1)
+    A = torch.randn((Z, M, K), generator=g)
+    Bm = torch.randn((Z, N, K), generator=g)
+    C0 = torch.randn((Z, M, N), generator=g) if mode == 3 else torch.full((Z, M, N), float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Cd = C0.cuda()
+    pr.pararnn_dense_matmul(A.cuda(), Bm.cuda(), Cd, mode, err)
+    torch.cuda.synchronize()
+    assert int(err[0]) == 0
+    ref = torch.einsum("zmk,znk->zmn", A.double(), Bm.double())
+    if mode == 3:
+        ref = ref + C0.double()
+    got = Cd.cpu().double()
+    for z in range(Z):
+        trans = mode == 1 or (mode == 2 and z % 2 == 0)
+        gz = got[z].reshape(N, M).t() if trans else got[z]
+        bound = 2 * TF32_REL * K * A[z].abs().max() * Bm[z].abs().max()
+        assert (gz - ref[z]).abs().max() <= bound, (z, float((gz - ref[z]).abs().max()))
+
+
 @pytest.mark.parametrize("n", [1, 2])
 def test_simt_capped_iterates_match_oracle_dense_newton(cuda_ok, n):
     x = _inputs(2, 45, 40)   # three 16-step chunks, the last ragged; GEMM tiles ragged
@@ -94,7 +120,7 @@ def test_tensor_core_capped_iterates_within_the_tf32_bound(cuda_ok, n):
 
 @pytest.mark.parametrize("B,T,D,f32,flags", [
     (2, 300, 64, False, 0), (1, 200, 64, True, 0), (1, 70, 128, False, 0), (3, 17, 8, False, 0),
-    (1, 100, 256, False, 0), (1, 64, 512, True, 0),
+    (1, 100, 256, False, 0), (1, 64, 512, True, 0), (1, 300, 512, False, 0),
     (2, 300, 64, False, 8), (1, 70, 128, False, 8)])   # 8 = PARARNN_FLAG_DENSE_SIMT
 def test_converges_to_the_sequential_recurrence(cuda_ok, B, T, D, f32, flags):
     x = _inputs(B, T, D, f32=f32)
