@@ -634,21 +634,34 @@ int dn_cluster(int D) {
   return 1;
 }
 
+// `wide`: a pass with few chains (the carry chain, one per b) takes clusters
+// of 16 CTAs (a non-portable size) where the device can hold one per chain,
+// so that twice as many SMs read each step's matrix
 template <class K>
 cudaError_t dn_launch_cluster(K kern, unsigned chains, int D, const Dn2Params& p,
-                              cudaStream_t stream) {
-  const int cl = dn_cluster(D);
+                              cudaStream_t stream, bool wide = false) {
+  int cl = dn_cluster(D);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(chains * (unsigned)cl);
   cfg.blockDim = dim3(kDnThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cl;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (wide && D % (8 * 16) == 0 && D / 16 >= 32 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+          cudaSuccess) {
+    attr[0].val.clusterDim.x = 16;
+    cfg.gridDim = dim3(chains * 16u);
+    int fit = 0;
+    if (cudaOccupancyMaxActiveClusters(&fit, kern, &cfg) == cudaSuccess && fit >= (int)chains)
+      cl = 16;
+  }
+  cudaGetLastError();
+  attr[0].val.clusterDim.x = cl;
+  cfg.gridDim = dim3(chains * (unsigned)cl);
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -837,7 +850,7 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
     }
     const unsigned nmaps = (unsigned)((size_t)B * p.nC);
     e = dn_launch_cluster(dn_offsets, nmaps, D, p, stream);
-    if (e == cudaSuccess) e = dn_launch_cluster(dn_carry2, (unsigned)B, D, p, stream);
+    if (e == cudaSuccess) e = dn_launch_cluster(dn_carry2, (unsigned)B, D, p, stream, true);
     if (e == cudaSuccess) e = dn_launch_cluster(dn_apply2, nmaps, D, p, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
