@@ -40,6 +40,8 @@ int adjoint_row_channels();
 int adjoint_row_box_steps(int which);
 size_t adjoint_row_part_bytes(int G, int B, int T, int D);
 size_t adjoint_queue_bytes(int B, int T, int D);
+int adjoint_queue_box_steps(int which);
+int adjoint_queue_channels();
 int adjoint_queue_resident();
 size_t adjoint_queue_lstm_bytes(int B, int T, int D);
 int adjoint_queue_lstm_resident();
@@ -491,16 +493,16 @@ int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, con
   // h0 (c0) with 1-D bulk copies, which take 16-byte aligned addresses only
   const bool rows16 = aligned(a, 16) && (!bias || aligned(bias, 16)) &&
                       (!h0 || aligned(h0, 16)) && (!c0 || aligned(c0, 16));
-  // ParaGRU, bf16 projections, at least one 8-channel tile per resident CTA
-  // of the queue adjoint: every 256-step segment in one launch, last first
+  // ParaGRU, bf16 projections, at least one 32-channel tile per resident CTA
+  // of the queue adjoint: every 128-step segment in one launch, last first
   if (cell == PARARNN_GRU && u_dtype == PARARNN_BF16 && !force_row && rows16 &&
-      (long long)B * ((D + 7) / 8) >= (long long)std::max(1, adjoint_queue_resident()) &&
+      (long long)B * ((D + 31) / 32) >= (long long)std::max(1, adjoint_queue_resident()) &&
       kWsHeaderBytes + adjoint_queue_bytes(B, T, D) <= ws_bytes) {
-    const int ch = adjoint_row_channels();
+    const int ch = adjoint_queue_channels();
     CUtensorMap qmaps[3];  // u, h (states before each step), dL/dh
-    rc = make_u_map(&qmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
-    if (!rc) rc = make_s_map(&qmaps[1], h, B, T, D, adjoint_row_box_steps(1), ch);
-    if (!rc) rc = make_s_map(&qmaps[2], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+    rc = make_u_map(&qmaps[0], u, true, B, T, G, D, adjoint_queue_box_steps(0), ch);
+    if (!rc) rc = make_s_map(&qmaps[1], h, B, T, D, adjoint_queue_box_steps(1), ch);
+    if (!rc) rc = make_s_map(&qmaps[2], dLdh, B, T, D, adjoint_queue_box_steps(2), ch);
     if (rc) return rc;
     const int e = launch_adjoint_queue(qmaps, a, bias, h0, du, da, dbias, dh0, B, T, D, status,
                                        static_cast<unsigned char*>(workspace) + kWsHeaderBytes,

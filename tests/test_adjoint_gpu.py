@@ -224,9 +224,10 @@ def test_withheld_exchange_times_out(cuda_ok, cell, wl, T, inject):
 
 
 # ---- the ParaGRU queue adjoint (bf16 u, at least one 8-channel tile per
-# resident CTA: 5 x 148 = 740 on a B200): every 256-step segment in one
+# resident CTA: 4 x 148 = 592 on a B200): every 128-step segment in one
 # launch, last segments first, each segment's carry from the one after it
-@pytest.mark.parametrize("B,T,D", [(1, 700, 6000), (2, 1300, 3000), (1, 256, 6000)])
+@pytest.mark.parametrize("B,T,D", [(1, 700, 6000), (2, 1300, 3000), (1, 256, 6000),
+                                   (1, 130, 4736), (1, 1, 6000), (1, 128, 4800)])
 def test_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
     x = make_inputs(WORKLOADS[2].scaled(B=B, T=T, D=D))
     x["h0"] = torch.randn((B, D), generator=torch.Generator().manual_seed(37)) * 0.5
