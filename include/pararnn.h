@@ -262,8 +262,8 @@ int pararnn_adjoint(int cell, const void* u, int u_dtype, const float* a,
  * Kernels: bf16 u with at least one tile per resident CTA of the queue
  * adjoint takes the queue adjoint (every segment of every tile in one launch,
  * last segments first, each segment's carry from the segment after it):
- * ParaGRU 32-channel tiles in 128-step segments, one 16-warp CTA per SM;
- * ParaLSTM 8-channel tiles in 256-step segments, four CTAs per SM.  Other bf16
+ * 32-channel tiles in 128-step segments, one 16-warp CTA per SM (so at
+ * least 148 tiles of 32 channels on a B200).  Other bf16
  * problems with T <= 4096 the
  * whole-sequence kernels (a cluster of CTAs per tile); the rest the chunked
  * look-back adjoint.  The first two stage the rows of a, bias, h0 and c0 by

@@ -19,8 +19,9 @@
 // boxes are in flight while the warp works on this one.
 //   pass 1: each chunk's map carry_in -> carry_out, backwards, keeping the
 //     cell's results (A, the three df/du, r h) of every step in registers;
-//   scan: the chunk maps of the warps after this one, composed from shared
-//     memory after one CTA barrier (the only one per item);
+//   scan: the carry entering a chunk is the segment's incoming carry taken
+//     through the chunk maps of the warps after it, read from shared memory
+//     after one CTA barrier (the only one per item);
 //   carry: a segment publishes the carry it passes to the segment before it
 //     as one 64-bit word per channel (the value's bits and the count of
 //     segments published from the end), so that a single relaxed load, issued
@@ -67,23 +68,6 @@ static_assert(kAqHOff % 128 == 0 && kAqGOff % 128 == 0 && kAqPOff % 128 == 0 &&
 constexpr int kAqSmem = 2 * kAqW * kAqS;           // 143360
 constexpr unsigned kAqBoxBytes = kAqL * (kAqUStep + 2 * kAqSStep);  // 3584
 
-// n / d for 0 <= n < 2^31 by one multiply-high, the method of Granlund and
-// Montgomery ("Division by invariant integers using multiplication", 1994,
-// Fig. 4.1) with the (N+1)-bit sum kept in 32 bits because n < 2^31.
-struct AqDiv {
-  unsigned m;
-  int l;
-};
-AqDiv aq_div(unsigned d) {
-  int l = 0;
-  while ((1ull << l) < d) ++l;
-  const unsigned long long m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
-  return AqDiv{(unsigned)m, l};
-}
-__device__ __forceinline__ int aq_quot(int n, AqDiv v) {
-  return (int)((__umulhi(v.m, (unsigned)n) + (unsigned)n) >> v.l);
-}
-
 struct AqParams {
   const float *a, *bias, *h0;
   float *du, *dh0, *part;
@@ -92,7 +76,7 @@ struct AqParams {
   unsigned long long* carry;
   unsigned* counter;   // item tickets (zero at launch)
   int B, T, D, nDT, ntiles, nseg, nitems;
-  AqDiv div_tiles, div_nDT;
+  FastDiv div_tiles, div_nDT;
   uint64_t timeout_ns;
   int* status;
   int withhold_item;   // testing: this item never publishes its carry (-1: none)
@@ -112,9 +96,9 @@ struct AqItem {
 };
 __device__ __forceinline__ AqItem aq_decode(const AqParams& p, int item) {
   AqItem it;
-  it.r = aq_quot(item, p.div_tiles);
+  it.r = fast_quot(item, p.div_tiles);
   it.tile = item - it.r * p.ntiles;
-  it.b = aq_quot(it.tile, p.div_nDT);
+  it.b = fast_quot(it.tile, p.div_nDT);
   it.d0 = (it.tile - it.b * p.nDT) * kAqC;
   it.t0 = (p.nseg - 1 - it.r) * kAqSteps;
   return it;
@@ -326,21 +310,20 @@ __global__ void __launch_bounds__(kAqThreads, 1)
       for (int w = 0; w < kAqW; ++w) sum += sh.red[s ^ 1][w][j][cc];
       p.part[(size_t)prev_part * (6 * kAqC) + tid] = sum;
     }
-    // the chunks after this one: the segment's incoming carry -> this chunk's
-    float2 cw = af2(1.f, 0.f);
-#pragma unroll
-    for (int w = kAqW - 1; w > 0; --w)
-      if (w > warp) cw = ar_after(sh.wagg[s][w][lane], cw);
-    const float cin_seg = sh.cin[s][lane];
-    // publish the carry this segment passes to the one before it: its map
-    // (chunk 0's after the others) applied to cin_seg
-    if (warp == 0 && item != p.withhold_item) {
-      const float2 m = ar_after(inc, cw);
-      aq_st_word(&p.carry[(size_t)cur.tile * kAqC + lane],
-                 (unsigned long long)__float_as_uint(fmaf(m.x, cin_seg, m.y)) |
-                     ((unsigned long long)(cur.r + 1) << 32));
+    // the carry entering this chunk: the segment's incoming carry through the
+    // maps of the chunks after this one, last first
+    float cchunk = sh.cin[s][lane];
+#pragma unroll 3
+    for (int w = kAqW - 1; w > warp; --w) {
+      const float2 m = sh.wagg[s][w][lane];
+      cchunk = fmaf(m.x, cchunk, m.y);
     }
-    const float cchunk = fmaf(cw.x, cin_seg, cw.y);
+    // publish the carry this segment passes to the one before it: chunk 0's
+    // map applied to the carry entering chunk 0
+    if (warp == 0 && item != p.withhold_item)
+      aq_st_word(&p.carry[(size_t)cur.tile * kAqC + lane],
+                 (unsigned long long)__float_as_uint(fmaf(inc.x, cchunk, inc.y)) |
+                     ((unsigned long long)(cur.r + 1) << 32));
 
     // ---- pass 2: the exact recurrence from the true carry, du and the sums
     float2 CARRY = af2(fmaf(PM.y, cchunk, DM.y), cchunk);  // entering steps 3 and 7
@@ -494,8 +477,8 @@ int launch_adjoint_queue(const CUtensorMap* maps, const float* a, const float* b
   p.nseg = (T + kAqSteps - 1) / kAqSteps;
   if ((long long)p.ntiles * p.nseg >= (1LL << 31) - 4) return 1;
   p.nitems = p.ntiles * p.nseg;
-  p.div_tiles = aq_div((unsigned)p.ntiles);
-  p.div_nDT = aq_div((unsigned)p.nDT);
+  p.div_tiles = fast_div((unsigned)p.ntiles);
+  p.div_nDT = fast_div((unsigned)p.nDT);
   p.timeout_ns = timeout_ns;
   p.status = status;
   p.withhold_item = withhold_item;

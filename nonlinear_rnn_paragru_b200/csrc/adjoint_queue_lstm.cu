@@ -1,7 +1,6 @@
 // adjoint_queue_lstm.cu -- reverse (adjoint) scan of a solved ParaLSTM
-// trajectory with bf16 input projections for many 8-channel tiles: every
-// 256-step segment of every tile in one persistent launch, last segments
-// first.
+// trajectory with bf16 input projections: every 128-step segment of every
+// 32-channel tile in one persistent launch, last segments first.
 //
 // The ParaGRU queue adjoint (adjoint_queue.cu) with the 2x2 Jacobian
 // ("Параллельность RNN?", §1.3, transposed): lambda = (lambda_c, lambda_h),
@@ -10,17 +9,19 @@
 // (the cell of adjoint_cell.cuh), da = sum_t du_t h_{t-1}, dbias = sum_t du_t,
 // and dL/dc0, dL/dh0 the carry out of the first step.
 //
-// Items (8 channels of one batch row over one segment) are numbered so that
+// Items (32 channels of one batch row over one segment) are numbered so that
 // every tile's last segment comes first (item = r * ntiles + tile for the
-// segment r from the end) and drawn from a counter one ahead.  A CTA of 4
-// warps holds a segment (lane = (chunk k = lane / 8, channel c = lane % 8),
-// 16 steps per thread as 8 packed step pairs); every warp stages its own four
-// chunks and its own copy of the tile's parameter rows on its own mbarrier
-// and loads the next item's as soon as its pass 2 is done:
+// segment r from the end) and drawn from a counter two ahead.  A CTA of 16
+// warps holds a segment: warp w the 8-step chunk w, lane c channel c, the 8
+// steps as 4 packed step pairs (i, i + 4).  Every warp stages its own chunk
+// (u as 64-byte rows, c_{t-1}, h_{t-1} and dL/dh as 128-byte rows) on its own
+// mbarriers, and warp 0 the tile's parameter rows for the whole CTA, in two
+// stages: the next item's boxes are in flight while the CTA works on this one.
 //   pass 1: each chunk's map carry_in -> carry_out (2x2 matrix, 2-vector),
 //     backwards;
-//   scan: a suffix scan over the warp's four chunks by shuffles, and over the
-//     warps from shared memory after one CTA barrier (the only one per item);
+//   scan: the carry entering a chunk is the segment's incoming carry taken
+//     through the maps of the chunks after it, read from shared memory after
+//     one CTA barrier (the only one per item);
 //   carry: a segment publishes the carry it passes to the segment before it
 //     as two 64-bit words per channel, (lambda_c bits, count) and (lambda_h
 //     bits, count), the count being the segments published from the tile's
@@ -29,14 +30,15 @@
 //     bound if not there yet) need no fence; the words are written before
 //     pass 2, so the chain of segments advances one map application per
 //     segment;
-//   pass 2: the exact recurrence from the true carry, du written and the
-//     da / dbias partial sums kept per warp, summed over the warps in a fixed
-//     order after the next item's barrier (reduced over the items afterwards
-//     in a fixed order: bitwise reproducible).
-// The lowest-numbered item that has not published is always being worked on
-// and never waits, so the queue cannot deadlock while all CTAs are resident;
-// a wait that runs out sets TIMEOUT.  Four CTAs share an SM (51.2 KB of
-// staged chunks each).
+//   pass 2: the exact recurrence from the true carry (the cell evaluated
+//     again), du written (a warp stores whole 128-byte lines) and the da /
+//     dbias partial sums kept per warp, summed over the warps in a fixed order
+//     after the next item's barrier and over the items afterwards in a fixed
+//     order: bitwise reproducible.
+// The lowest-numbered item that has not published is always some CTA's
+// current item and never waits (the items a CTA holds but has not started
+// are numbered above its current one), so the queue cannot deadlock while all
+// CTAs are resident; a wait that runs out sets TIMEOUT.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -50,35 +52,63 @@ namespace pararnn {
 namespace {
 
 constexpr unsigned kAlqFull = 0xffffffffu;
-constexpr int kAlqWarps = 4;
-constexpr int kAlqThreads = kAlqWarps * 32;
-constexpr int kAlqChunks = kAlqWarps * kArK;       // 16
-constexpr int kAlqSteps = kAlqChunks * kArL;       // 256 steps per item
-constexpr int kAlqSmem = kAlqChunks * kAlS;        // 51200
-constexpr unsigned kAlqWarpBytes =
-    kArK * (kArUBox * kAlUStep + 2 * kArHBox * kArSStep + kArGBox * kArSStep);
+constexpr int kAlqC = 32;                          // channels per tile (lanes)
+constexpr int kAlqW = 16;                          // warps per CTA = chunks per item
+constexpr int kAlqThreads = kAlqW * 32;
+constexpr int kAlqL = 8;                           // steps per chunk (per thread)
+constexpr int kAlqH = kAlqL / 2;                   // step pairs per chunk
+constexpr int kAlqSteps = kAlqW * kAlqL;           // 128 steps per item
+// a warp's stage: u [8 steps][i f g o][32 ch] bf16, then c_{t-1}, h_{t-1} and
+// dL/dh [8][32] fp32
+constexpr int kAlqUStep = 4 * kAlqC * 2;           // 256 bytes per step of u
+constexpr int kAlqSStep = kAlqC * 4;               // 128 bytes per step of a state
+constexpr int kAlqUOff = 0, kAlqCOff = kAlqL * kAlqUStep;
+constexpr int kAlqHOff = kAlqCOff + kAlqL * kAlqSStep, kAlqGOff = kAlqHOff + kAlqL * kAlqSStep;
+constexpr int kAlqS = kAlqGOff + kAlqL * kAlqSStep;  // 5120 bytes per warp and stage
+constexpr unsigned kAlqBoxBytes = kAlqS;
+// the CTA's parameter rows per stage: a (4 rows), bias (4), c0, h0
+constexpr int kAlqPar = 10 * kAlqC * 4;            // 1280 bytes
+// dynamic shared memory: the warps' stages, the parameter stages, then the
+// scan maps, partial sums, carries, mbarriers and tickets
+constexpr int kAlqParOff = 2 * kAlqW * kAlqS;                       // 163840
+constexpr int kAlqMapOff = kAlqParOff + 2 * kAlqPar;                // [2][16][3][32] float2
+constexpr int kAlqRedOff = kAlqMapOff + 2 * kAlqW * 3 * kAlqC * 8;  // [2][16][8][32] float
+constexpr int kAlqCinOff = kAlqRedOff + 2 * kAlqW * 8 * kAlqC * 4;  // [2][32] float2
+constexpr int kAlqBarOff = kAlqCinOff + 2 * kAlqC * 8;              // [2][16 + 1] u64
+constexpr int kAlqNxOff = kAlqBarOff + 2 * (kAlqW + 1) * 8;         // [2] int
+constexpr int kAlqSmem = kAlqNxOff + 16;
+static_assert(kAlqCOff % 128 == 0 && kAlqHOff % 128 == 0 && kAlqGOff % 128 == 0 &&
+                  kAlqS % 128 == 0 && kAlqParOff % 128 == 0 && kAlqPar % 128 == 0 &&
+                  kAlqBarOff % 8 == 0,
+              "stage layout");
+static_assert(kAlqSmem <= 227 * 1024, "one CTA per SM");
 
 struct AlqParams {
   const float *a, *bias, *c0, *h0;
   float *du, *dc0, *dh0, *part;
-  // [ntiles][8][2]: the carry (lambda_c, lambda_h) a segment passes to the
+  // [ntiles][32][2]: the carry (lambda_c, lambda_h) a segment passes to the
   // one before it, each as (float bits) | (segments published from the end) << 32
   unsigned long long* carry;
   unsigned* counter;   // item tickets (zero at launch)
-  int B, T, D, nDTc, ntiles, nseg, nitems;
+  int B, T, D, nDT, ntiles, nseg, nitems;
+  FastDiv div_tiles, div_nDT;
   uint64_t timeout_ns;
   int* status;
   int withhold_item;   // testing: this item never publishes its carry (-1: none)
 };
 
-struct AlqShared {
-  uint64_t bar[kAlqWarps];            // per warp: its chunks' boxes and parameters
-  float par[kAlqWarps][10][kArC];     // per warp: a (4 rows), bias (4 rows), c0, h0
-  float4 wagg[2][kAlqWarps][kArC][2]; // by item parity: per (warp, channel) suffix map
-  float red[2][kAlqWarps][8][kArC];   // by item parity: partial sums per warp
-  float2 cin[2][kArC];                // by item parity: carry entering the last step
-  int nx[2];                          // the item after this one, by parity
+struct AlqItem {
+  int tile, r, b, d0, t0;
 };
+__device__ __forceinline__ AlqItem alq_decode(const AlqParams& p, int item) {
+  AlqItem it;
+  it.r = fast_quot(item, p.div_tiles);
+  it.tile = item - it.r * p.ntiles;
+  it.b = fast_quot(it.tile, p.div_nDT);
+  it.d0 = (it.tile - it.b * p.nDT) * kAlqC;
+  it.t0 = (p.nseg - 1 - it.r) * kAlqSteps;
+  return it;
+}
 
 __device__ __forceinline__ void alq_bulk(void* dst, const void* src, unsigned bytes,
                                          uint64_t* bar) {
@@ -98,47 +128,51 @@ __device__ __forceinline__ void alq_st_word(unsigned long long* p, unsigned long
 __device__ __forceinline__ unsigned long long alq_word(float v, int count) {
   return (unsigned long long)__float_as_uint(v) | ((unsigned long long)count << 32);
 }
-__device__ __forceinline__ Aff2 alq_shfl_down(const Aff2& a, int o) {
-  return Aff2{__shfl_down_sync(kAlqFull, a.m00, o), __shfl_down_sync(kAlqFull, a.m01, o),
-              __shfl_down_sync(kAlqFull, a.m10, o), __shfl_down_sync(kAlqFull, a.m11, o),
-              __shfl_down_sync(kAlqFull, a.d0, o),  __shfl_down_sync(kAlqFull, a.d1, o)};
-}
 
-// Warp `warp`: its four chunks' boxes (u, c_{t-1}, h_{t-1}, dL/dh; lane k
-// issues chunk k's four), its copy of the a and bias rows and, for a first
-// segment, the c0 and h0 rows of the item at (b, d0, t0), all on the warp's
-// mbarrier.  The rows are 16-byte aligned (the caller checks the pointers;
-// d0 is a multiple of 8 and D of 8).
-__device__ __forceinline__ void alq_issue(unsigned char* smem, AlqShared& sh,
-                                          const CUtensorMap* mu, const CUtensorMap* mc,
-                                          const CUtensorMap* mh, const CUtensorMap* mg,
-                                          const AlqParams& p, int warp, int b, int d0, int t0,
-                                          int lane) {
-  const unsigned pb = kArC * 4;
-  const bool first_seg = t0 == 0;
-  uint64_t* bar = &sh.bar[warp];
+// Warp `warp`: its chunk's four boxes of item `it` (u, c_{t-1}, h_{t-1},
+// dL/dh; lanes 0-3) into stage buffer `st` on mbarrier `bar`; warp 0 also
+// the tile's parameter rows (lanes 4-13: the channels below D, a and bias
+// rows, and c0, h0 for a first segment) into `par` on mbarrier `pbar`.  The
+// rows are 16-byte aligned (the caller checks the pointers; d0 and D are
+// multiples of 8).
+__device__ __forceinline__ void alq_issue(unsigned char* st, uint64_t* bar, float* par,
+                                          uint64_t* pbar, const CUtensorMap* mu,
+                                          const CUtensorMap* mc, const CUtensorMap* mh,
+                                          const CUtensorMap* mg, const AlqParams& p,
+                                          const AlqItem& it, int warp, int lane) {
+  const unsigned pb = (unsigned)min(kAlqC, p.D - it.d0) * 4;
+  const bool first_seg = it.t0 == 0;
   if (lane == 0) {
+    // this warp's reads of the stage (generic proxy) before the copies into it
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(bar, kAlqWarpBytes + 4 * pb + (p.bias ? 4 * pb : 0) +
-                                   ((first_seg && p.c0) ? pb : 0) +
-                                   ((first_seg && p.h0) ? pb : 0));
+    mbar_arrive_expect_tx(bar, kAlqBoxBytes);
+    if (warp == 0)
+      mbar_arrive_expect_tx(pbar, 4 * pb + (p.bias ? 4 * pb : 0) +
+                                      ((first_seg && p.c0) ? pb : 0) +
+                                      ((first_seg && p.h0) ? pb : 0));
   }
   __syncwarp();
-  if (lane < kArK) {
-    const int q = warp * kArK + lane, ts = t0 + q * kArL - lane;
-    unsigned char* slot = smem + q * kAlS;
-    tma_load_4d(slot + kAlUOff, mu, bar, d0, 0, ts, b);
-    tma_load_3d(slot + kAlCOff, mc, bar, d0, ts - 1, b);
-    tma_load_3d(slot + kAlHOff, mh, bar, d0, ts - 1, b);
-    tma_load_3d(slot + kAlGOff, mg, bar, d0, ts, b);
-  } else if (lane < kArK + 4) {
-    const int g = lane - kArK;
-    alq_bulk(&sh.par[warp][g][0], p.a + (size_t)g * p.D + d0, pb, bar);
-    if (p.bias) alq_bulk(&sh.par[warp][4 + g][0], p.bias + (size_t)g * p.D + d0, pb, bar);
-  } else if (lane == kArK + 4 && first_seg && p.c0) {
-    alq_bulk(&sh.par[warp][8][0], p.c0 + (size_t)b * p.D + d0, pb, bar);
-  } else if (lane == kArK + 5 && first_seg && p.h0) {
-    alq_bulk(&sh.par[warp][9][0], p.h0 + (size_t)b * p.D + d0, pb, bar);
+  const int ts = it.t0 + warp * kAlqL;
+  if (lane == 0) {
+    tma_load_4d(st + kAlqUOff, mu, bar, it.d0, 0, ts, it.b);
+  } else if (lane == 1) {
+    tma_load_3d(st + kAlqCOff, mc, bar, it.d0, ts - 1, it.b);
+  } else if (lane == 2) {
+    tma_load_3d(st + kAlqHOff, mh, bar, it.d0, ts - 1, it.b);
+  } else if (lane == 3) {
+    tma_load_3d(st + kAlqGOff, mg, bar, it.d0, ts, it.b);
+  } else if (warp == 0) {
+    if (lane < 8) {
+      const int g = lane - 4;
+      alq_bulk(par + g * kAlqC, p.a + (size_t)g * p.D + it.d0, pb, pbar);
+    } else if (lane < 12) {
+      const int g = lane - 8;
+      if (p.bias) alq_bulk(par + (4 + g) * kAlqC, p.bias + (size_t)g * p.D + it.d0, pb, pbar);
+    } else if (lane == 12) {
+      if (first_seg && p.c0) alq_bulk(par + 8 * kAlqC, p.c0 + (size_t)it.b * p.D + it.d0, pb, pbar);
+    } else if (lane == 13) {
+      if (first_seg && p.h0) alq_bulk(par + 9 * kAlqC, p.h0 + (size_t)it.b * p.D + it.d0, pb, pbar);
+    }
   }
 }
 
@@ -146,66 +180,111 @@ __device__ __forceinline__ int alq_draw(unsigned* counter) {
   return (int)min(atomicAdd(counter, 1u), 0x7fffffffu);
 }
 
-__global__ void __launch_bounds__(kAlqThreads, 4)
+// pre-scaled arguments of a step pair from bf16 rows [i f g o][32 channels]
+__device__ __forceinline__ void alq_args(const unsigned short* rx, const unsigned short* ry,
+                                         const float2 (&BS)[4], float2& UI, float2& UF,
+                                         float2& UG, float2& UO) {
+  const float2 S = af2(-kLog2e, -kLog2e), SG = af2(2.f * kLog2e, 2.f * kLog2e);
+  auto ld = [&](int g) {
+    return af2(__uint_as_float((unsigned)rx[g * kAlqC] << 16),
+               __uint_as_float((unsigned)ry[g * kAlqC] << 16));
+  };
+  UI = afma(S, ld(0), BS[0]);
+  UF = afma(S, ld(1), BS[1]);
+  UG = afma(SG, ld(2), BS[2]);
+  UO = afma(S, ld(3), BS[3]);
+}
+
+__global__ void __launch_bounds__(kAlqThreads, 1)
     adjoint_queue_lstm(const __grid_constant__ CUtensorMap mu,
                        const __grid_constant__ CUtensorMap mc,
                        const __grid_constant__ CUtensorMap mh,
                        const __grid_constant__ CUtensorMap mg, const AlqParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ AlqShared sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = lane % kArC, kk = lane / kArC;
-  const int q = warp * kArK + kk;
+  unsigned char* st0 = smem + warp * kAlqS;             // this warp's stage 0
+  unsigned char* st1 = smem + (kAlqW + warp) * kAlqS;   // and stage 1
+  float* par0 = reinterpret_cast<float*>(smem + kAlqParOff);
+  float* par1 = reinterpret_cast<float*>(smem + kAlqParOff + kAlqPar);
+  float2* wmap = reinterpret_cast<float2*>(smem + kAlqMapOff);   // [2][16][3][32]
+  float* red = reinterpret_cast<float*>(smem + kAlqRedOff);      // [2][16][8][32]
+  float2* cinb = reinterpret_cast<float2*>(smem + kAlqCinOff);   // [2][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAlqBarOff);  // [2][17]: warps, params
+  int* nx = reinterpret_cast<int*>(smem + kAlqNxOff);
 
-  for (int i = tid; i < kAlqWarps * 10 * kArC; i += kAlqThreads) (&sh.par[0][0][0])[i] = 0.f;
-  if (tid < kAlqWarps) mbar_init(&sh.bar[tid], 1);
-  if (tid == 0) sh.nx[0] = alq_draw(p.counter);
-  __syncthreads();
-  int item = sh.nx[0];
-  if (item < p.nitems) {
-    const int tile = item % p.ntiles, seg = p.nseg - 1 - item / p.ntiles;
-    alq_issue(smem, sh, &mu, &mc, &mh, &mg, p, warp, tile / p.nDTc, (tile % p.nDTc) * kArC,
-              seg * kAlqSteps, lane);
+  // parameter rows start at zero (bias, c0 and h0 stay so when absent, c0
+  // and h0 outside first segments); rows of channels at or above D are never
+  // copied: their lanes compute on whatever the stage holds and store nothing
+  for (int i = tid; i < 2 * 10 * kAlqC; i += kAlqThreads) par0[i] = 0.f;
+  if (tid < 2 * (kAlqW + 1)) mbar_init(&bars[tid], 1);
+  if (tid == 0) {
+    nx[0] = alq_draw(p.counter);
+    nx[1] = alq_draw(p.counter);
   }
-  const unsigned char* slot = smem + q * kAlS;
-  const unsigned char* ubase = slot + kAlUOff + kk * kAlUStep + c * 2;
-  const float* cbase = reinterpret_cast<const float*>(slot + kAlCOff + kk * kArSStep) + c;
-  const float* hbase = reinterpret_cast<const float*>(slot + kAlHOff + kk * kArSStep) + c;
-  const float* gbase = reinterpret_cast<const float*>(slot + kAlGOff + kk * kArSStep) + c;
-  const float* pw = &sh.par[warp][0][0] + c;
+  __syncthreads();
+  int item = nx[0], nxt = nx[1];
+  __syncthreads();
+  // pend: per stage, 1 + the parity of a phase armed and not yet waited for
+  // (this warp's boxes; warp 0 also the parameters)
+  int pend0 = 0, pend1 = 0;
+  AlqItem cur = alq_decode(p, item < p.nitems ? item : 0);
+  if (item < p.nitems) {
+    alq_issue(st0, &bars[warp], par0, &bars[kAlqW], &mu, &mc, &mh, &mg, p, cur, warp, lane);
+    pend0 = 1;
+  }
   int status = 0;
-  int n = 0, prev_part = -1;  // prev_part: the partial-sum row of the item before
-  // 0 while this warp's boxes arrive, else 1 + the phase parity of the wait
-  // that ran out (the warp issues no more loads)
-  int dead = 0;
+  bool live = true;    // false once a wait for this warp's boxes ran out
+  int prev_part = -1;  // the partial-sum row of the item before
+  int n = 0;
   for (; item < p.nitems; ++n) {
-    const int par = n & 1;
-    if (tid == 0) sh.nx[par ^ 1] = alq_draw(p.counter);
-    const int tile = item % p.ntiles, r = item / p.ntiles, seg = p.nseg - 1 - r;
-    const int b = tile / p.nDTc, d0 = (tile % p.nDTc) * kArC;
-    const int d = d0 + c;
+    const int s = n & 1;
+    uint64_t* sbar = bars + s * (kAlqW + 1);
+    // the ticket of the item after the next one: stored just before the barrier
+    int ticket = 0;
+    if (tid == 0) ticket = alq_draw(p.counter);
+    // the next item's boxes into the other stage (the CTA is done with it:
+    // every parameter read of the item before precedes its barrier)
+    AlqItem nit = alq_decode(p, nxt < p.nitems ? nxt : 0);
+    if (live && nxt < p.nitems) {
+      alq_issue(s ? st0 : st1, bars + (s ^ 1) * (kAlqW + 1) + warp, s ? par0 : par1,
+                bars + (s ^ 1) * (kAlqW + 1) + kAlqW, &mu, &mc, &mh, &mg, p, nit, warp, lane);
+      if (s) pend0 = 1 + (((n + 1) >> 1) & 1);
+      else pend1 = 1 + (((n + 1) >> 1) & 1);
+    }
+    const int d = cur.d0 + lane;
     const bool dval = d < p.D;
-    const int t0 = seg * kAlqSteps;
-    const bool first = (seg == 0 && q == 0);  // the chunk holding step 0
+    const bool first = (cur.t0 == 0 && warp == 0);  // the chunk holding step 0
     // the carry words of the segment after this one, fetched now, read after pass 1
+    unsigned long long* cwp = &p.carry[((size_t)cur.tile * kAlqC + lane) * 2];
     unsigned long long wc = 0ull, wh = 0ull;
-    unsigned long long* cwp = &p.carry[((size_t)tile * kArC + c) * 2];
-    if (tid < kArC && r > 0) {
+    if (warp == 0 && cur.r > 0) {
       wc = alq_ld_word(cwp);
       wh = alq_ld_word(cwp + 1);
     }
-    if (!dead) {
+    if (live) {
       // a phase that did not complete is never re-armed: the warp stops loading
-      if (!__all_sync(kAlqFull, mbar_wait_bounded(&sh.bar[warp], (unsigned)par, p.timeout_ns))) {
-        dead = 1 + par;
+      const unsigned ph = (unsigned)((n >> 1) & 1);
+      bool ok = mbar_wait_bounded(&sbar[warp], ph, p.timeout_ns);
+      if (ok) ok = mbar_wait_bounded(&sbar[kAlqW], ph, p.timeout_ns);
+      if (__all_sync(kAlqFull, ok)) {
+        if (s) pend1 = 0;
+        else pend0 = 0;
+      } else {
+        live = false;
         status = PARARNN_STATUS_TIMEOUT;
       }
     }
+    const unsigned char* stg = s ? st1 : st0;
+    const unsigned short* ubase = reinterpret_cast<const unsigned short*>(stg + kAlqUOff) + lane;
+    const float* cbase = reinterpret_cast<const float*>(stg + kAlqCOff) + lane;
+    const float* hbase = reinterpret_cast<const float*>(stg + kAlqHOff) + lane;
+    const float* gbase = reinterpret_cast<const float*>(stg + kAlqGOff) + lane;
+    const float* pw = (s ? par1 : par0) + lane;
     AlCell k;
     float2 BS[4];
     float c0v, h0v;
     {
-      const float ai = pw[0 * kArC], af = pw[1 * kArC], ag = pw[2 * kArC], ao = pw[3 * kArC];
+      const float ai = pw[0 * kAlqC], af = pw[1 * kAlqC], ag = pw[2 * kAlqC], ao = pw[3 * kAlqC];
       k.AI = af2(ai, ai);
       k.AF = af2(af, af);
       k.AG = af2(ag, ag);
@@ -216,28 +295,29 @@ __global__ void __launch_bounds__(kAlqThreads, 4)
       k.AO2 = af2(-kLog2e * ao, -kLog2e * ao);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const float bs = (g == 2 ? 2.f * kLog2e : -kLog2e) * pw[(4 + g) * kArC];
+        const float bs = (g == 2 ? 2.f * kLog2e : -kLog2e) * pw[(4 + g) * kAlqC];
         BS[g] = af2(bs, bs);
       }
-      c0v = (seg == 0) ? pw[8 * kArC] : 0.f;
-      h0v = (seg == 0) ? pw[9 * kArC] : 0.f;
+      c0v = first ? pw[8 * kAlqC] : 0.f;
+      h0v = first ? pw[9 * kAlqC] : 0.f;
     }
     auto state = [&](int i, float2& CP, float2& HP, float2& G) {
-      CP = af2(cbase[i * kArC], cbase[(i + kArH) * kArC]);  // (c, h)_{t-1}
-      HP = af2(hbase[i * kArC], hbase[(i + kArH) * kArC]);
+      CP = af2(cbase[i * kAlqC], cbase[(i + kAlqH) * kAlqC]);  // (c, h)_{t-1}
+      HP = af2(hbase[i * kAlqC], hbase[(i + kAlqH) * kAlqC]);
       if (i == 0 && first) {
         CP.x = c0v;
         HP.x = h0v;
       }
-      G = af2(gbase[i * kArC], gbase[(i + kArH) * kArC]);
+      G = af2(gbase[i * kAlqC], gbase[(i + kAlqH) * kAlqC]);
     };
 
     // ---- pass 1: the two half-chunk maps (carry_in -> carry_out), backwards
     float2 M00 = af2(1.f, 1.f), M01 = af2(0.f, 0.f), M10 = M01, M11 = M00, D0 = M01, D1 = M01;
 #pragma unroll
-    for (int i = kArH - 1; i >= 0; --i) {
+    for (int i = kAlqH - 1; i >= 0; --i) {
       float2 UI, UF, UG, UO, CP, HP, G, F, X, KK, A11, GCI, GCF, GCG, DOT;
-      al_args(ubase + i * kAlUStep, ubase + (i + kArH) * kAlUStep, BS, UI, UF, UG, UO);
+      alq_args(ubase + i * (kAlqUStep / 2), ubase + (i + kAlqH) * (kAlqUStep / 2), BS, UI, UF,
+               UG, UO);
       state(i, CP, HP, G);
       al_cell(k, CP, HP, UI, UF, UG, UO, F, X, KK, A11, GCI, GCF, GCG, DOT);
       const float2 A10 = amul(KK, F);
@@ -256,24 +336,18 @@ __global__ void __launch_bounds__(kAlqThreads, 4)
     const Aff2 Mx{M00.x, M01.x, M10.x, M11.x, D0.x, D1.x};
     const Aff2 My{M00.y, M01.y, M10.y, M11.y, D0.y, D1.y};
     // the chunk's map: the first half after the second
-    Aff2 inc = Mx.after(My);
-    // suffix scan over the warp's four chunks of channel c (lanes c + 8k)
-#pragma unroll
-    for (int o = kArC; o < 32; o <<= 1) {
-      const Aff2 nx = alq_shfl_down(inc, o);
-      if (lane + o < 32) inc = inc.after(nx);
-    }
-    // the carry entering the warp -> the carry entering this chunk
-    Aff2 xm = alq_shfl_down(inc, kArC);
-    if (kk == kArK - 1) xm = Aff2::id();
-    if (kk == 0) {
-      sh.wagg[par][warp][c][0] = make_float4(inc.m00, inc.m01, inc.m10, inc.m11);
-      sh.wagg[par][warp][c][1] = make_float4(inc.d0, inc.d1, 0.f, 0.f);
+    const Aff2 inc = Mx.after(My);
+    {
+      float2* mw = wmap + ((s * kAlqW + warp) * 3) * kAlqC + lane;
+      mw[0] = af2(inc.m00, inc.m01);
+      mw[kAlqC] = af2(inc.m10, inc.m11);
+      mw[2 * kAlqC] = af2(inc.d0, inc.d1);
     }
     // the carry entering this segment's last step: zero for the last segment,
     // else the words the segment after it published (count r)
-    if (tid < kArC) {
+    if (warp == 0) {
       float2 cin = af2(0.f, 0.f);
+      const int r = cur.r;
       if (r > 0) {
         if ((unsigned)(wc >> 32) < (unsigned)r || (unsigned)(wh >> 32) < (unsigned)r) {
           const uint64_t w0 = globaltimer_ns();
@@ -289,48 +363,49 @@ __global__ void __launch_bounds__(kAlqThreads, 4)
         }
         cin = af2(__uint_as_float((unsigned)wc), __uint_as_float((unsigned)wh));
       }
-      sh.cin[par][c] = cin;
+      cinb[s * kAlqC + lane] = cin;
     }
+    if (tid == 0) nx[s] = ticket;
     __syncthreads();
+    const int nn = nx[s];  // the item after the next one
     // every warp is done with the item before: its partial sums, in warp order
-    if (prev_part >= 0 && tid < 8 * kArC) {
-      const int j = tid / kArC, cc = tid % kArC;
-      float s = 0.f;
+    if (prev_part >= 0 && tid < 8 * kAlqC) {
+      const float* rp = red + (s ^ 1) * kAlqW * 8 * kAlqC + tid;
+      float sum = 0.f;
 #pragma unroll
-      for (int w = 0; w < kAlqWarps; ++w) s += sh.red[par ^ 1][w][j][cc];
-      p.part[(size_t)prev_part * (8 * kArC) + tid] = s;
+      for (int w = 0; w < kAlqW; ++w) sum += rp[w * 8 * kAlqC];
+      p.part[(size_t)prev_part * (8 * kAlqC) + tid] = sum;
     }
-    // the warps after this one: the segment's incoming carry -> this warp's
-    Aff2 cw = Aff2::id();
-#pragma unroll
-    for (int w = kAlqWarps - 1; w > 0; --w)
-      if (w > warp) {
-        const float4 m4 = sh.wagg[par][w][c][0], v4 = sh.wagg[par][w][c][1];
-        cw = Aff2{m4.x, m4.y, m4.z, m4.w, v4.x, v4.y}.after(cw);
-      }
-    const float2 cin_seg = sh.cin[par][c];
-    // publish the carry this segment passes to the one before it: its map
-    // (the warp-0 chunk-0 suffix after the other warps) applied to cin_seg
-    if (warp == 0 && kk == 0 && item != p.withhold_item) {
-      const float2 out = inc.after(cw).apply(cin_seg);
-      alq_st_word(cwp, alq_word(out.x, r + 1));
-      alq_st_word(cwp + 1, alq_word(out.y, r + 1));
+    // the carry entering this chunk: the segment's incoming carry through the
+    // maps of the chunks after this one, last first
+    float2 cchunk = cinb[s * kAlqC + lane];
+#pragma unroll 2
+    for (int w = kAlqW - 1; w > warp; --w) {
+      const float2* mw = wmap + ((s * kAlqW + w) * 3) * kAlqC + lane;
+      const float2 m0 = mw[0], m1 = mw[kAlqC], dv = mw[2 * kAlqC];
+      cchunk = Aff2{m0.x, m0.y, m1.x, m1.y, dv.x, dv.y}.apply(cchunk);
     }
-    const float2 cchunk = xm.apply(cw.apply(cin_seg));
-    const float2 cx = My.apply(cchunk);  // entering step 7 from step 8
+    // publish the carry this segment passes to the one before it: chunk 0's
+    // map applied to the carry entering chunk 0
+    if (warp == 0 && item != p.withhold_item) {
+      const float2 out = inc.apply(cchunk);
+      alq_st_word(cwp, alq_word(out.x, cur.r + 1));
+      alq_st_word(cwp + 1, alq_word(out.y, cur.r + 1));
+    }
+    const float2 cx = My.apply(cchunk);  // entering step 3 from step 4
 
     // ---- pass 2: the exact recurrence, du and the partial sums
     float2 LC = af2(cx.x, cchunk.x), LH = af2(cx.y, cchunk.y);
     float2 SA[4], SB[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) SA[g] = SB[g] = af2(0.f, 0.f);
-    const int tq = t0 + q * kArL;
-    float* dub = p.du + (((size_t)b * p.T + tq) * 4) * p.D + d;
-    bool bad = false;
+    const int tq = cur.t0 + warp * kAlqL;
+    float* dub = p.du + (((size_t)cur.b * p.T + tq) * 4) * p.D + d;
 #pragma unroll
-    for (int i = kArH - 1; i >= 0; --i) {
+    for (int i = kAlqH - 1; i >= 0; --i) {
       float2 UI, UF, UG, UO, CP, HP, G, F, X, KK, A11, GCI, GCF, GCG, DOT;
-      al_args(ubase + i * kAlUStep, ubase + (i + kArH) * kAlUStep, BS, UI, UF, UG, UO);
+      alq_args(ubase + i * (kAlqUStep / 2), ubase + (i + kAlqH) * (kAlqUStep / 2), BS, UI, UF,
+               UG, UO);
       state(i, CP, HP, G);
       al_cell(k, CP, HP, UI, UF, UG, UO, F, X, KK, A11, GCI, GCF, GCG, DOT);
       const float2 LHE = aadd(LH, G);                      // lambda_h
@@ -348,66 +423,62 @@ __global__ void __launch_bounds__(kAlqThreads, 4)
         if (tq + i < p.T) {
           float* o = dub + (size_t)i * 4 * p.D;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            o[(size_t)g * p.D] = DU[g].x;
-            bad |= !isfinite(DU[g].x);
-          }
+          for (int g = 0; g < 4; ++g) o[(size_t)g * p.D] = DU[g].x;
         }
-        if (tq + kArH + i < p.T) {
-          float* o = dub + (size_t)(kArH + i) * 4 * p.D;
+        if (tq + kAlqH + i < p.T) {
+          float* o = dub + (size_t)(kAlqH + i) * 4 * p.D;
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            o[(size_t)g * p.D] = DU[g].y;
-            bad |= !isfinite(DU[g].y);
-          }
+          for (int g = 0; g < 4; ++g) o[(size_t)g * p.D] = DU[g].y;
         }
       }
     }
     if (first && dval) {
-      if (p.dc0) p.dc0[(size_t)b * p.D + d] = LC.x;
-      if (p.dh0) p.dh0[(size_t)b * p.D + d] = LH.x;
+      if (p.dc0) p.dc0[(size_t)cur.b * p.D + d] = LC.x;
+      if (p.dh0) p.dh0[(size_t)cur.b * p.D + d] = LH.x;
     }
-    // this warp's slots and parameters are free: the next item's
-    const int next = sh.nx[par ^ 1];
-    __syncwarp();
-    if (!dead && next < p.nitems) {
-      const int nt = next % p.ntiles, ns = p.nseg - 1 - next / p.ntiles;
-      alq_issue(smem, sh, &mu, &mc, &mh, &mg, p, warp, nt / p.nDTc, (nt % p.nDTc) * kArC,
-                ns * kAlqSteps, lane);
-    }
-    // the warp's partial sums: over the two halves, then the warp's chunks
+    // the warp's partial sums per channel.  Every du of the chunk enters one
+    // of the dbias sums, so a non-finite du (or an overflowing sum) leaves one
+    // of them non-finite.
     float v[8];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
       v[g] = SA[g].x + SA[g].y;
       v[4 + g] = SB[g].x + SB[g].y;
     }
+    bool bad = false;
+    float* rw = red + (s * kAlqW + warp) * 8 * kAlqC + lane;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      v[j] = dval ? v[j] : 0.f;
-      v[j] += __shfl_xor_sync(kAlqFull, v[j], 8);
-      v[j] += __shfl_xor_sync(kAlqFull, v[j], 16);
+      rw[j * kAlqC] = v[j];
+      bad |= !isfinite(v[j]);
     }
-    if (kk == 0)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) sh.red[par][warp][j][c] = v[j];
-    if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
-    prev_part = tile * p.nseg + seg;
-    item = next;
+    if (dval && bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
+    prev_part = cur.tile * p.nseg + (p.nseg - 1 - cur.r);
+    item = nxt;
+    nxt = nn;
+    cur = nit;
   }
   // the last item's partial sums
   __syncthreads();
-  if (prev_part >= 0 && tid < 8 * kArC) {
-    const int j = tid / kArC, cc = tid % kArC;
-    float s = 0.f;
+  if (prev_part >= 0 && tid < 8 * kAlqC) {
+    const float* rp = red + ((n - 1) & 1) * kAlqW * 8 * kAlqC + tid;
+    float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kAlqWarps; ++w) s += sh.red[(n - 1) & 1][w][j][cc];
-    p.part[(size_t)prev_part * (8 * kArC) + tid] = s;
+    for (int w = 0; w < kAlqW; ++w) sum += rp[w * 8 * kAlqC];
+    p.part[(size_t)prev_part * (8 * kAlqC) + tid] = sum;
   }
-  // copies still in flight into this warp's slots: wait for them (bounded)
-  if (dead) mbar_wait_bounded(&sh.bar[warp], (unsigned)(dead - 1), p.timeout_ns);
-  const int st = __reduce_max_sync(kAlqFull, status);
-  if (lane == 0 && st) atomicMax(p.status, st);
+  // copies still in flight into this warp's stages (warp 0: and the
+  // parameter stages): wait for them (bounded)
+  if (pend0) {
+    mbar_wait_bounded(&bars[warp], (unsigned)(pend0 - 1), p.timeout_ns);
+    if (warp == 0) mbar_wait_bounded(&bars[kAlqW], (unsigned)(pend0 - 1), p.timeout_ns);
+  }
+  if (pend1) {
+    mbar_wait_bounded(&bars[kAlqW + 1 + warp], (unsigned)(pend1 - 1), p.timeout_ns);
+    if (warp == 0) mbar_wait_bounded(&bars[2 * kAlqW + 1], (unsigned)(pend1 - 1), p.timeout_ns);
+  }
+  const int sts = __reduce_max_sync(kAlqFull, status);
+  if (lane == 0 && sts) atomicMax(p.status, sts);
 }
 
 __global__ void adjoint_queue_lstm_init(int* status, unsigned* counter,
@@ -418,6 +489,34 @@ __global__ void adjoint_queue_lstm_init(int* status, unsigned* counter,
     *counter = 0u;
   }
   for (int j = i; j < nwords; j += gridDim.x * blockDim.x) carry[j] = 0ull;
+}
+
+// da[g][d], dbias[g][d] = the items' partial sums of channel d, over the
+// batch rows and segments in a fixed order (a warp per output pair)
+__global__ void adjoint_queue_lstm_reduce(const float* __restrict__ part, float* da,
+                                          float* dbias, int B, int D, int nDT, int nseg) {
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // over 4 * D
+  const int lane = threadIdx.x & 31;
+  if (i >= 4 * D) return;
+  const int g = i / D, d = i - g * D;
+  const int dt = d / kAlqC, cc = d % kAlqC;
+  const int nterm = B * nseg;
+  float sa = 0.f, sb = 0.f;
+  for (int j = lane; j < nterm; j += 32) {
+    const int b = j / nseg, r = j - b * nseg;
+    const float* pp = part + ((size_t)(b * nDT + dt) * nseg + r) * (8 * kAlqC);
+    sa += pp[g * kAlqC + cc];
+    sb += pp[(4 + g) * kAlqC + cc];
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    sa += __shfl_xor_sync(kAlqFull, sa, o);
+    sb += __shfl_xor_sync(kAlqFull, sb, o);
+  }
+  if (lane == 0) {
+    da[i] = sa;
+    if (dbias) dbias[i] = sb;
+  }
 }
 
 int alq_per_sm() {
@@ -433,14 +532,13 @@ int alq_per_sm() {
 
 }  // namespace
 
-void adjoint_row_reduce_launch(const float* part, float* da, float* dbias, int B, int D, int cls,
-                               int G, cudaStream_t stream);
+int adjoint_queue_lstm_channels() { return kAlqC; }
 
 // Workspace bytes past the 256-byte header: partial sums, carry words, count.
 size_t adjoint_queue_lstm_bytes(int B, int T, int D) {
-  const size_t ntiles = (size_t)B * ((D + kArC - 1) / kArC);
+  const size_t ntiles = (size_t)B * ((D + kAlqC - 1) / kAlqC);
   const size_t nseg = (size_t)(T + kAlqSteps - 1) / kAlqSteps;
-  return align256(ntiles * nseg * 8 * kArC * 4) + align256(ntiles * kArC * 2 * 8) + 256;
+  return align256(ntiles * nseg * 8 * kAlqC * 4) + align256(ntiles * kAlqC * 2 * 8) + 256;
 }
 
 // Resident CTAs of the ParaLSTM queue adjoint on the current device.
@@ -451,8 +549,8 @@ int adjoint_queue_lstm_resident() {
   return sms * alq_per_sm();
 }
 
-// maps: u (box 8 x 4 x 19), c and h (box 8 x 20), dL/dh (box 8 x 19); ws: the
-// workspace past its header, adjoint_queue_lstm_bytes(B, T, D) bytes
+// maps: u (box 32 x 4 x 8), c, h and dL/dh (box 32 x 8); ws: the workspace
+// past its header, adjoint_queue_lstm_bytes(B, T, D) bytes
 int launch_adjoint_queue_lstm(const CUtensorMap* maps, const float* a, const float* bias,
                               const float* c0, const float* h0, float* du, float* da,
                               float* dbias, float* dc0, float* dh0, int B, int T, int D,
@@ -469,21 +567,23 @@ int launch_adjoint_queue_lstm(const CUtensorMap* maps, const float* a, const flo
   p.B = B;
   p.T = T;
   p.D = D;
-  p.nDTc = (D + kArC - 1) / kArC;
-  p.ntiles = B * p.nDTc;
+  p.nDT = (D + kAlqC - 1) / kAlqC;
+  p.ntiles = B * p.nDT;
   p.nseg = (T + kAlqSteps - 1) / kAlqSteps;
-  if ((long long)p.ntiles * p.nseg >= (1LL << 31)) return 1;
+  if ((long long)p.ntiles * p.nseg >= (1LL << 31) - 4) return 1;
   p.nitems = p.ntiles * p.nseg;
+  p.div_tiles = fast_div((unsigned)p.ntiles);
+  p.div_nDT = fast_div((unsigned)p.nDT);
   p.timeout_ns = timeout_ns;
   p.status = status;
   p.withhold_item = withhold_item;
   unsigned char* w = static_cast<unsigned char*>(ws);
   p.part = reinterpret_cast<float*>(w);
-  w += align256((size_t)p.nitems * 8 * kArC * 4);
+  w += align256((size_t)p.nitems * 8 * kAlqC * 4);
   p.carry = reinterpret_cast<unsigned long long*>(w);
-  w += align256((size_t)p.ntiles * kArC * 2 * 8);
+  w += align256((size_t)p.ntiles * kAlqC * 2 * 8);
   p.counter = reinterpret_cast<unsigned*>(w);
-  const int nwords = p.ntiles * kArC * 2;
+  const int nwords = p.ntiles * kAlqC * 2;
   adjoint_queue_lstm_init<<<(unsigned)std::min(1024, (nwords + 255) / 256 + 1), 256, 0,
                             stream>>>(status, p.counter, p.carry, nwords);
   const int per_sm = std::max(1, alq_per_sm());
@@ -495,7 +595,8 @@ int launch_adjoint_queue_lstm(const CUtensorMap* maps, const float* a, const flo
       maps[0], maps[1], maps[2], maps[3], p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  adjoint_row_reduce_launch(p.part, da, dbias, B, D, p.nseg, 4, stream);
+  adjoint_queue_lstm_reduce<<<(4 * D * 32 + 255) / 256, 256, 0, stream>>>(p.part, da, dbias, B, D,
+                                                                          p.nDT, p.nseg);
   return (int)cudaGetLastError();
 }
 

@@ -45,6 +45,7 @@ int adjoint_queue_channels();
 int adjoint_queue_resident();
 size_t adjoint_queue_lstm_bytes(int B, int T, int D);
 int adjoint_queue_lstm_resident();
+int adjoint_queue_lstm_channels();
 int launch_adjoint_queue_lstm(const CUtensorMap* maps, const float* a, const float* bias,
                               const float* c0, const float* h0, float* du, float* da,
                               float* dbias, float* dc0, float* dh0, int B, int T, int D,
@@ -509,16 +510,17 @@ int pararnn_adjoint_ex(int cell, const void* u, int u_dtype, const float* a, con
                                        timeout_ns, inject_chunk, (cudaStream_t)stream);
     return e == 0 ? PARARNN_OK : PARARNN_ERR_CUDA;
   }
-  // ParaLSTM likewise (four CTAs per SM)
+  // ParaLSTM likewise (32-channel tiles, one 16-warp CTA per SM)
   if (cell == PARARNN_LSTM && u_dtype == PARARNN_BF16 && !force_row && rows16 &&
-      (long long)B * ((D + 7) / 8) >= (long long)std::max(1, adjoint_queue_lstm_resident()) &&
+      (long long)B * ((D + 31) / 32) >= (long long)std::max(1, adjoint_queue_lstm_resident()) &&
       kWsHeaderBytes + adjoint_queue_lstm_bytes(B, T, D) <= ws_bytes) {
-    const int ch = adjoint_row_channels();
+    const int ch = adjoint_queue_lstm_channels();
+    const int tc = adjoint_queue_box_steps(0);
     CUtensorMap qmaps[4];  // u, c and h (states before each step), dL/dh
-    rc = make_u_map(&qmaps[0], u, true, B, T, G, D, adjoint_row_box_steps(0), ch);
-    if (!rc) rc = make_s_map(&qmaps[1], c, B, T, D, adjoint_row_box_steps(1), ch);
-    if (!rc) rc = make_s_map(&qmaps[2], h, B, T, D, adjoint_row_box_steps(1), ch);
-    if (!rc) rc = make_s_map(&qmaps[3], dLdh, B, T, D, adjoint_row_box_steps(2), ch);
+    rc = make_u_map(&qmaps[0], u, true, B, T, G, D, tc, ch);
+    if (!rc) rc = make_s_map(&qmaps[1], c, B, T, D, tc, ch);
+    if (!rc) rc = make_s_map(&qmaps[2], h, B, T, D, tc, ch);
+    if (!rc) rc = make_s_map(&qmaps[3], dLdh, B, T, D, tc, ch);
     if (rc) return rc;
     const int e = launch_adjoint_queue_lstm(
         qmaps, a, bias, c0, h0, du, da, dbias, dc0, dh0, B, T, D, status,

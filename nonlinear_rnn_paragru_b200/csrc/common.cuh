@@ -140,6 +140,24 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// ------------------------------------------------- division by invariants --
+// n / d for 0 <= n < 2^31 by one multiply-high, the method of Granlund and
+// Montgomery ("Division by invariant integers using multiplication", 1994,
+// Fig. 4.1), with the (N+1)-bit sum kept in 32 bits because n < 2^31.
+struct FastDiv {
+  unsigned m;
+  int l;
+};
+inline FastDiv fast_div(unsigned d) {
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  const unsigned long long m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
+  return FastDiv{(unsigned)m, l};
+}
+__device__ __forceinline__ int fast_quot(int n, FastDiv v) {
+  return (int)((__umulhi(v.m, (unsigned)n) + (unsigned)n) >> v.l);
+}
+
 // ------------------------------------------------------------ workspace --
 // Forward-solve workspace:
 //   [0, 256)           header: epoch, ticket counter

@@ -223,8 +223,8 @@ def test_withheld_exchange_times_out(cuda_ok, cell, wl, T, inject):
         _check_lstm(x, c, h)
 
 
-# ---- the ParaGRU queue adjoint (bf16 u, at least one 8-channel tile per
-# resident CTA: 4 x 148 = 592 on a B200): every 128-step segment in one
+# ---- the ParaGRU queue adjoint (bf16 u, at least one 32-channel tile per
+# resident CTA: 148 on a B200): every 128-step segment in one
 # launch, last segments first, each segment's carry from the one after it
 @pytest.mark.parametrize("B,T,D", [(1, 700, 6000), (2, 1300, 3000), (1, 256, 6000),
                                    (1, 130, 4736), (1, 1, 6000), (1, 128, 4800)])
@@ -316,8 +316,8 @@ def test_adjoint_rows_4byte_aligned(cuda_ok, cell, B, T, D):
         assert _rel(outs[1][k].cpu().numpy(), outs[0][k].cpu().numpy()) <= TOL_GRAD, k
 
 
-# ---- the ParaLSTM queue adjoint (bf16 u, at least one 8-channel tile per
-# resident CTA: 4 x 148 = 592 on a B200)
+# ---- the ParaLSTM queue adjoint (bf16 u, at least one 32-channel tile per
+# resident CTA: 148 on a B200)
 def _lstm_queue_inputs(B, T, D):
     x = make_inputs(WORKLOADS[3].scaled(B=B, T=T, D=D), with_grad=True)
     g = torch.Generator().manual_seed(41)
@@ -327,7 +327,8 @@ def _lstm_queue_inputs(B, T, D):
     return x, c, h
 
 
-@pytest.mark.parametrize("B,T,D", [(1, 700, 4800), (2, 1300, 2400), (1, 256, 4800)])
+@pytest.mark.parametrize("B,T,D", [(1, 700, 4800), (2, 1300, 2400), (1, 256, 4800),
+                                   (1, 1, 4736), (1, 130, 4808)])
 def test_lstm_queue_adjoint_matches_bptt(cuda_ok, B, T, D):
     x, c, h = _lstm_queue_inputs(B, T, D)
     _check_lstm(x, c, h)
