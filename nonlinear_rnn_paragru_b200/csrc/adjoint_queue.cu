@@ -412,6 +412,7 @@ __global__ void adjoint_queue_reduce(const float* __restrict__ part, float* da, 
   const int dt = d / kAqC, cc = d % kAqC;
   const int nterm = B * nseg;
   float sa = 0.f, sb = 0.f;
+#pragma unroll 8
   for (int j = lane; j < nterm; j += 32) {
     const int b = j / nseg, r = j - b * nseg;
     const float* pp = part + ((size_t)(b * nDT + dt) * nseg + r) * (6 * kAqC);

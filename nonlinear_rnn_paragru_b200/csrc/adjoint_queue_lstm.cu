@@ -502,6 +502,7 @@ __global__ void adjoint_queue_lstm_reduce(const float* __restrict__ part, float*
   const int dt = d / kAlqC, cc = d % kAlqC;
   const int nterm = B * nseg;
   float sa = 0.f, sb = 0.f;
+#pragma unroll 8
   for (int j = lane; j < nterm; j += 32) {
     const int b = j / nseg, r = j - b * nseg;
     const float* pp = part + ((size_t)(b * nDT + dt) * nseg + r) * (8 * kAlqC);
