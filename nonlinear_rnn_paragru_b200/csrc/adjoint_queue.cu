@@ -70,12 +70,14 @@ constexpr unsigned kAqBoxBytes = kAqL * (kAqUStep + 2 * kAqSStep);  // 3584
 
 struct AqParams {
   const float *a, *bias, *h0;
+  // part: [6][nDT * 32][B * nseg] per-item partial sums of da (rows 0-2) and
+  // dbias (rows 3-5), the item's term (b * nseg + segment) innermost
   float *du, *dh0, *part;
   // [ntiles][32]: the carry a segment passes to the one before it, as
   // (float bits) | (segments published from the end of the tile) << 32
   unsigned long long* carry;
   unsigned* counter;   // item tickets (zero at launch)
-  int B, T, D, nDT, ntiles, nseg, nitems;
+  int B, T, D, nDT, ntiles, nseg, nitems, nterm;
   FastDiv div_tiles, div_nDT;
   uint64_t timeout_ns;
   int* status;
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kAqThreads, 1)
   }
   int status = 0;
   bool live = true;    // false once a wait for this warp's boxes ran out
-  int prev_part = -1;  // the partial-sum row of the item before
+  long long prev_part = -1;  // the partial-sum offset of the item before
   int n = 0;
   for (; item < p.nitems; ++n) {
     const int s = n & 1;
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kAqThreads, 1)
       float sum = 0.f;
 #pragma unroll
       for (int w = 0; w < kAqW; ++w) sum += sh.red[s ^ 1][w][j][cc];
-      p.part[(size_t)prev_part * (6 * kAqC) + tid] = sum;
+      p.part[prev_part + ((size_t)j * p.nDT * kAqC + cc) * p.nterm] = sum;
     }
     // the carry entering this chunk: the segment's incoming carry through the
     // maps of the chunks after this one, last first
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(kAqThreads, 1)
     const bool bad = !isfinite(v[0]) || !isfinite(v[1]) || !isfinite(v[2]) ||
                      !isfinite(v[3]) || !isfinite(v[4]) || !isfinite(v[5]);
     if (dval && bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
-    prev_part = cur.tile * p.nseg + (p.nseg - 1 - cur.r);
+    prev_part = (long long)cur.d0 * p.nterm + (long long)cur.b * p.nseg + (p.nseg - 1 - cur.r);
     item = nxt;
     nxt = nn;
     cur = nit;
@@ -382,7 +384,7 @@ __global__ void __launch_bounds__(kAqThreads, 1)
     float sum = 0.f;
 #pragma unroll
     for (int w = 0; w < kAqW; ++w) sum += sh.red[(n - 1) & 1][w][j][cc];
-    p.part[(size_t)prev_part * (6 * kAqC) + tid] = sum;
+    p.part[prev_part + ((size_t)j * p.nDT * kAqC + cc) * p.nterm] = sum;
   }
   // copies still in flight into this warp's stages: wait for them (bounded)
   if (pend0) mbar_wait_bounded(&sh.bar[0][warp], (unsigned)(pend0 - 1), p.timeout_ns);
@@ -402,31 +404,23 @@ __global__ void adjoint_queue_init(int* status, unsigned* counter, unsigned long
 }
 
 // da[g][d], dbias[g][d] = the items' partial sums of channel d, over the
-// batch rows and segments in a fixed order (a warp per output pair)
+// batch rows and segments in a fixed order: a warp per output, its lanes
+// reading the output's terms as whole lines
 __global__ void adjoint_queue_reduce(const float* __restrict__ part, float* da, float* dbias,
-                                     int B, int D, int nDT, int nseg) {
-  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // over 3 * D
+                                     int D, int Dp, int nterm) {
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // over 6 * D
   const int lane = threadIdx.x & 31;
-  if (i >= 3 * D) return;
-  const int g = i / D, d = i - g * D;
-  const int dt = d / kAqC, cc = d % kAqC;
-  const int nterm = B * nseg;
-  float sa = 0.f, sb = 0.f;
+  if (i >= 6 * D) return;
+  const int j = i / D, d = i - j * D;
+  const float* pp = part + ((size_t)j * Dp + d) * nterm;
+  float s = 0.f;
 #pragma unroll 8
-  for (int j = lane; j < nterm; j += 32) {
-    const int b = j / nseg, r = j - b * nseg;
-    const float* pp = part + ((size_t)(b * nDT + dt) * nseg + r) * (6 * kAqC);
-    sa += pp[g * kAqC + cc];
-    sb += pp[(3 + g) * kAqC + cc];
-  }
+  for (int t = lane; t < nterm; t += 32) s += pp[t];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    sa += __shfl_xor_sync(kAqFull, sa, o);
-    sb += __shfl_xor_sync(kAqFull, sb, o);
-  }
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(kAqFull, s, o);
   if (lane == 0) {
-    da[i] = sa;
-    if (dbias) dbias[i] = sb;
+    if (j < 3) da[i] = s;
+    else if (dbias) dbias[i - 3 * D] = s;
   }
 }
 
@@ -478,6 +472,7 @@ int launch_adjoint_queue(const CUtensorMap* maps, const float* a, const float* b
   p.nseg = (T + kAqSteps - 1) / kAqSteps;
   if ((long long)p.ntiles * p.nseg >= (1LL << 31) - 4) return 1;
   p.nitems = p.ntiles * p.nseg;
+  p.nterm = B * p.nseg;
   p.div_tiles = fast_div((unsigned)p.ntiles);
   p.div_nDT = fast_div((unsigned)p.nDT);
   p.timeout_ns = timeout_ns;
@@ -508,8 +503,8 @@ int launch_adjoint_queue(const CUtensorMap* maps, const float* a, const float* b
       maps[0], maps[1], maps[2], p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
-  adjoint_queue_reduce<<<(3 * D * 32 + 255) / 256, 256, 0, stream>>>(p.part, da, dbias, B, D,
-                                                                      p.nDT, p.nseg);
+  adjoint_queue_reduce<<<(6 * D * 32 + 255) / 256, 256, 0, stream>>>(p.part, da, dbias, D,
+                                                                      p.nDT * kAqC, p.nterm);
   return (int)cudaGetLastError();
 }
 
