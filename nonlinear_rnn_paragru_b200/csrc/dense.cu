@@ -18,19 +18,22 @@
 //                    split tf32 (three products of hi/lo parts), so they, the
 //                    residual and the fixed point carry fp32 accuracy; W h0
 //                    once per solve;
-//   dn_assemble2     one CTA per (b, step): gates, residual, -r_t and the
-//                    block J_t to HBM, row-major at odd positions of its
+//   dn_assemble2     one CTA per (b, 8 steps, half of the rows): gates,
+//                    residual, -r_t, the four coefficient vectors of J_t and
+//                    the block J_t to HBM, row-major at odd positions of its
 //                    16-step chunk and transposed at even ones;
 //   chunk maps       each chunk's product J_15 ... J_0 as a tree of pairwise
 //                    products, four levels of batched D x D tcgen05 GEMMs (left
 //                    factor row-major, right factor transposed: both operands
 //                    K-major; each level stores its products in the layout the
 //                    next level reads them in);
-//   dn_offsets, dn_carry2, dn_apply2
-//                    the chunk offsets (the chunk's recurrence from a zero
-//                    delta), the delta entering each chunk chunk by chunk,
-//                    and every chunk re-run from its delta, ds added to h
-//                    (matrix-vector products, coalesced in either layout).
+//   dn_spass, dn_carry2, dn_spass
+//                    the chunk offsets (every chunk's recurrence from a zero
+//                    delta), the delta entering each chunk chunk by chunk
+//                    (matrix-vector products with the chunk maps), and every
+//                    chunk re-run from its delta, ds added to h; the two
+//                    chunk passes take J_t through its structure, diag(co0)
+//                    plus row-scaled W_z, W_c, W_r, all chains at once.
 // The chunk maps' tf32 products make each Newton step inexact (about 1e-3
 // relative); the residual is evaluated to fp32 accuracy, so the fixed point
 // is that of the cell and the iteration still converges, linearly near the
@@ -309,6 +312,9 @@ struct Dn2Params {
   float* J;        // [B][Tp][D][D]: odd positions of a chunk row-major, even transposed
   const float* P;  // chunk maps [B][nC][D][D] row-major (the last tree level)
   float* rhs;      // -r [B][Tp][D], zero on padded steps
+  // [B][Tp][4][D]: J_t = diag(co0) + diag(co1) W_z + diag(co2) W_c + diag(co3) W_r
+  // (co0 = 1, the others 0 on padded steps)
+  float* co;
   float* d;        // chunk offsets [B][nC][D]
   float* carry;    // delta entering each chunk [B][nC][D]
   unsigned* rmax;
@@ -348,19 +354,27 @@ __global__ void dn_transpose_w(const float* __restrict__ W, float* __restrict__ 
   }
 }
 
-// One CTA per (b, four consecutive padded steps t0..t0+3): gates from the
-// pre-activations of h_{t-1}, residual, -r_t and J_t for each; padded steps
-// (t >= T) get J = I and -r = 0.  The two odd steps are stored row-major and
-// the two even ones transposed, so every float4 of a W (Wt) row is loaded
-// once for two steps.
-constexpr int kDnAsm = 4;  // steps per assembly CTA (Tp is a multiple of 16)
+// One CTA per (b, eight consecutive padded steps t0..t0+7, half of the rows):
+// gates from the pre-activations of h_{t-1}, residual, -r_t, the coefficients
+// of J_t and, for its rows, J_t for each step; padded steps (t >= T) get J = I,
+// -r = 0 and the identity's coefficients.  The four odd steps are stored
+// row-major and the four even ones transposed, so every float4 of a W (Wt) row
+// is loaded once for four steps.  The two CTAs of a step group compute the
+// same gates; the one holding the first half of the rows stores the vectors.
+constexpr int kDnAsm = 8;     // steps per assembly CTA (Tp is a multiple of 16)
+constexpr int kDnAsmSplit = 2;  // CTAs per step group (row halves)
+constexpr size_t kDnAsmSmem = (size_t)kDnAsm * 4 * kDnMaxD * 4;
 template <bool kBF16>
 __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
-  __shared__ __align__(16) float co[kDnAsm][4][kDnMaxD];
+  extern __shared__ __align__(16) float asm_sm[];
+  float (*co)[4][kDnMaxD] = reinterpret_cast<float (*)[4][kDnMaxD]>(asm_sm);
   __shared__ unsigned wmax[kDnThreads / 32];
   const int D = p.D;
   const int groups = p.Tp / kDnAsm;
-  const int b = (int)(blockIdx.x / groups), t0 = (int)(blockIdx.x % groups) * kDnAsm;
+  const int half = (int)(blockIdx.x % kDnAsmSplit);
+  const int gidx = (int)(blockIdx.x / kDnAsmSplit);
+  const int b = gidx / groups, t0 = (gidx % groups) * kDnAsm;
+  const bool vec_owner = half == 0;
   const size_t DD = (size_t)D * D;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned m = 0;
@@ -369,7 +383,14 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
     const int t = t0 + st;
     const size_t bt = (size_t)b * p.Tp + t;
     if (t >= p.T) {
-      for (int i = threadIdx.x; i < D; i += blockDim.x) p.rhs[bt * D + i] = 0.f;
+      if (vec_owner)
+        for (int i = threadIdx.x; i < D; i += blockDim.x) {
+          p.rhs[bt * D + i] = 0.f;
+          p.co[(bt * 4 + 0) * D + i] = 1.f;
+          p.co[(bt * 4 + 1) * D + i] = 0.f;
+          p.co[(bt * 4 + 2) * D + i] = 0.f;
+          p.co[(bt * 4 + 3) * D + i] = 0.f;
+        }
       continue;
     }
     const size_t bs = (size_t)b * p.T + t;  // (b, t) in the unpadded arrays
@@ -384,36 +405,42 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
           tanhf(dn_u<kBF16>(p.u, iu + 2 * (size_t)D) + (p.bias ? p.bias[2 * D + i] : 0.f) + r * q);
       const float f = fmaf(z, c - hp, hp);
       const float res = p.h[bs * D + i] - f;
-      p.rhs[bt * D + i] = -res;
       m = max(m, dn_abs_bits(res));
       const float gc = z * (1.f - c * c);
-      co[st][0][i] = 1.f - z;
-      co[st][1][i] = (c - hp) * z * (1.f - z);
-      co[st][2][i] = gc * r;
-      co[st][3][i] = gc * q * r * (1.f - r);
+      const float c0 = 1.f - z, c1 = (c - hp) * z * (1.f - z), c2 = gc * r,
+                  c3 = gc * q * r * (1.f - r);
+      co[st][0][i] = c0;
+      co[st][1][i] = c1;
+      co[st][2][i] = c2;
+      co[st][3][i] = c3;
+      if (vec_owner) {
+        p.rhs[bt * D + i] = -res;
+        p.co[(bt * 4 + 0) * D + i] = c0;
+        p.co[(bt * 4 + 1) * D + i] = c1;
+        p.co[(bt * 4 + 2) * D + i] = c2;
+        p.co[(bt * 4 + 3) * D + i] = c3;
+      }
     }
   }
   m = __reduce_max_sync(0xffffffffu, m);
   if (lane == 0) wmax[warp] = m;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && vec_owner) {
     unsigned mm = 0;
     for (int w = 0; w < kDnThreads / 32; ++w) mm = max(mm, wmax[w]);
     atomicMax(p.rmax, mm);
   }
   // J[i][j] = [i == j] (1 - z_i) + co1_i Wz[i][j] + co2_i Wc[i][j] + co3_i Wr[i][j];
-  // a warp per stored row, lanes along it in float4s (coalesced, every load
-  // of the row in flight before the stores)
+  // a warp per stored row of this CTA's half, lanes along it in float4s
+  // (coalesced, every load of the row in flight before the stores)
   constexpr int kQ4 = kDnMaxD / 128;
+  constexpr int kPar = kDnAsm / 2;  // steps of one parity
   const int D4 = D >> 2;
+  const int Dh = D / kDnAsmSplit, rlo = half * Dh, rhi = rlo + Dh;
 #pragma unroll 1
   for (int parity = 1; parity >= 0; --parity) {  // odd steps row-major, even transposed
     const float* Wsrc = parity ? p.W : p.Wt;
-    const int sa = parity, sb = parity + 2;       // the group's two steps of this parity
-    const bool va = t0 + sa < p.T, vb = t0 + sb < p.T;
-    float* Ja = p.J + ((size_t)b * p.Tp + t0 + sa) * DD;
-    float* Jb = p.J + ((size_t)b * p.Tp + t0 + sb) * DD;
-    for (int row = warp; row < D; row += kDnThreads / 32) {
+    for (int row = rlo + warp; row < rhi; row += kDnThreads / 32) {
       float4 wz[kQ4], wr[kQ4], wc[kQ4];
 #pragma unroll
       for (int k = 0; k < kQ4; ++k) {
@@ -430,10 +457,10 @@ __global__ void __launch_bounds__(kDnThreads) dn_assemble2(const Dn2Params p) {
         const int q4 = lane + 32 * k;
         if (q4 >= D4) continue;
 #pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const int s = which ? sb : sa;
-          const bool valid = which ? vb : va;
-          float* Jt = which ? Jb : Ja;
+        for (int which = 0; which < kPar; ++which) {
+          const int s = parity + 2 * which;
+          const bool valid = t0 + s < p.T;
+          float* Jt = p.J + ((size_t)b * p.Tp + t0 + s) * DD;
           float4 o;
           if (!valid) {  // padded step: the identity
             o = make_float4(row == 4 * q4 ? 1.f : 0.f, row == 4 * q4 + 1 ? 1.f : 0.f,
@@ -565,27 +592,6 @@ __device__ __forceinline__ void dn_cmatvec(cgd::cluster_group& cl, DnVec& v, int
   cl.sync();
 }
 
-// One cluster per (b, chunk): the chunk's recurrence from a zero delta; its
-// last delta is the chunk's offset d.
-__global__ void __launch_bounds__(kDnThreads) dn_offsets(const Dn2Params p) {
-  __shared__ DnVec v;
-  cgd::cluster_group cl = cgd::this_cluster();
-  const int D = p.D, ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
-  const int R = D / ncl, r0 = rank * R;
-  const int chain = blockIdx.x / ncl;
-  const int b = chain / p.nC, k = chain - b * p.nC;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) v.x[0][i] = 0.f;
-  cl.sync();
-  int cur = 0;
-  for (int pp = 0; pp < kDnChunk; ++pp) {
-    const size_t bt = (size_t)b * p.Tp + (size_t)k * kDnChunk + pp;
-    const bool last = pp == kDnChunk - 1;
-    dn_cmatvec(cl, v, cur, p.J + bt * D * D, (pp & 1) != 0, p.rhs + bt * D, D, r0, R,
-               last ? p.d + (size_t)chain * D : nullptr);
-    cur ^= 1;
-  }
-}
-
 // One cluster per b: the delta entering each chunk, chunk by chunk
 // (x <- P_k x + d_k).
 __global__ void __launch_bounds__(kDnThreads) dn_carry2(const Dn2Params p) {
@@ -605,25 +611,181 @@ __global__ void __launch_bounds__(kDnThreads) dn_carry2(const Dn2Params p) {
   }
 }
 
-// One cluster per (b, chunk): the chunk re-run from its delta; ds added to h.
-__global__ void __launch_bounds__(kDnThreads) dn_apply2(const Dn2Params p) {
-  __shared__ DnVec v;
-  cgd::cluster_group cl = cgd::this_cluster();
-  const int D = p.D, ncl = (int)cl.num_blocks(), rank = (int)cl.block_rank();
-  const int R = D / ncl, r0 = rank * R;
-  const int chain = blockIdx.x / ncl;
-  const int b = chain / p.nC, k = chain - b * p.nC;
-  for (int i = threadIdx.x; i < D; i += blockDim.x) v.x[0][i] = p.carry[(size_t)chain * D + i];
-  cl.sync();
-  int cur = 0;
+// ---- the chunks' recurrences through the structure of J_t, for all chains
+// at once.  J_t x = co0 x + co1 (W_z x) + co2 (W_c x) + co3 (W_r x): the
+// three products with x take the stacked recurrent matrices, the same for
+// every step, so a step of every chain is one product of W by the matrix of
+// the chains' deltas, and a step reads 4 D coefficients instead of the D x D
+// block.  One persistent CTA per SM owns up to 4 channels i (rows i of W_z,
+// W_r, W_c, held in shared memory k-major); per step it stages the chains'
+// deltas (X[j][chain], chains innermost) in blocks of 64 chains, its warps
+// take eighths of k and their partial sums are added in warp order, and each
+// thread finishes one (channel, chain) of the block.  A grid barrier (bounded
+// wait) separates the steps.  Offsets: from a zero delta, the last step's
+// delta is the chunk offset; apply: from the delta entering the chunk, every
+// step's delta added to h.
+constexpr int kSpCpc = 4;                    // channels per CTA, at most
+constexpr int kSpCb = 64;                    // chains per staged block
+constexpr int kSpKg = kDnThreads / 32;       // k groups (warps)
+struct SpParams {
+  Dn2Params p;
+  float* X;             // [2][D][nchp] chain deltas, chains innermost
+  unsigned* bar;        // grid barrier arrivals (zero at launch)
+  int* err;             // set when a barrier wait runs out
+  int cpc, nch, nchp;   // channels per CTA, chains (B * nC), padded to 4
+  uint64_t timeout_ns;
+};
+constexpr size_t kSpSmem =
+    (size_t)(kDnMaxD * 3 * kSpCpc + kDnMaxD * kSpCb + kSpKg * 6 * kSpCpc * 32) * 4;
+
+// every CTA's stores before this point are visible to every CTA after it;
+// false when the wait ran out
+__device__ __forceinline__ bool sp_grid_sync(unsigned* bar, unsigned target, uint64_t timeout_ns) {
+  __shared__ int ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+    int good = 1;
+    if (ld_acquire(bar) < target) {
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire(bar) < target) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
+          good = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    ok = good;
+  }
+  __syncthreads();
+  return ok != 0;
+}
+
+template <bool kApply>
+__global__ void __launch_bounds__(kDnThreads, 1) dn_spass(const SpParams s) {
+  extern __shared__ __align__(16) float sp_sm[];
+  const Dn2Params& p = s.p;
+  const int D = p.D, nch = s.nch, nchp = s.nchp, cpc = s.cpc;
+  float* Ws = sp_sm;                            // [D][3][kSpCpc]
+  float* Xs = Ws + kDnMaxD * 3 * kSpCpc;        // [D][kSpCb]
+  float* part = Xs + kDnMaxD * kSpCb;           // [kSpKg][2][3][kSpCpc][32]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = blockIdx.x * cpc;
+  const unsigned G = gridDim.x;
+  // this CTA's rows of W_z, W_r, W_c, k-major (rows past D or cpc: zero)
+  for (int e = tid; e < D * 3 * kSpCpc; e += kDnThreads) {
+    const int k = e / (3 * kSpCpc), rem = e % (3 * kSpCpc), m = rem / kSpCpc, il = rem % kSpCpc;
+    const int i = i0 + il;
+    Ws[e] = (il < cpc && i < D) ? p.W[((size_t)m * D + i) * D + k] : 0.f;
+  }
+  // the deltas entering the chunks: zero (offsets) or the carries (apply)
+  float* X0 = s.X;
+  for (int e = tid; e < cpc * nch; e += kDnThreads) {
+    const int il = e / nch, cg = e % nch, i = i0 + il;
+    if (i < D) X0[(size_t)i * nchp + cg] = kApply ? p.carry[(size_t)cg * D + i] : 0.f;
+  }
+  unsigned round = 1;
+  if (!sp_grid_sync(s.bar, round * G, s.timeout_ns)) {
+    if (tid == 0) atomicExch(s.err, 1);
+    return;
+  }
+  const int kq = (D + kSpKg - 1) / kSpKg, k0 = warp * kq, k1 = min(D, k0 + kq);
   for (int pp = 0; pp < kDnChunk; ++pp) {
-    const int t = k * kDnChunk + pp;
-    if (t >= p.T) break;  // the same for every CTA of the cluster
-    const size_t bt = (size_t)b * p.Tp + t;
-    dn_cmatvec(cl, v, cur, p.J + bt * D * D, (pp & 1) != 0, p.rhs + bt * D, D, r0, R, nullptr);
-    cur ^= 1;
-    for (int ii = threadIdx.x; ii < R; ii += blockDim.x)
-      p.h[((size_t)b * p.T + t) * D + r0 + ii] += v.x[cur][r0 + ii];
+    const float* Xc = s.X + (size_t)(pp & 1) * D * nchp;
+    float* Xn = s.X + (size_t)((pp & 1) ^ 1) * D * nchp;
+    for (int cb0 = 0; cb0 < nch; cb0 += kSpCb) {
+      const int ncb = min(kSpCb, nchp - cb0);    // a multiple of 4
+      // this thread's output (channel il, chain c of the block): its
+      // coefficients and -r loaded now, used after the products
+      const int oil = tid / kSpCb, oc = tid % kSpCb;
+      const int oi = i0 + oil, ocg = cb0 + oc;
+      const bool own = oil < cpc && oi < D && ocg < nch;
+      const int ob = own ? ocg / p.nC : 0, okc = own ? ocg - ob * p.nC : 0;
+      const int ot = okc * kDnChunk + pp;
+      const size_t obt = (size_t)ob * p.Tp + ot;
+      float cf0 = 0.f, cf1 = 0.f, cf2 = 0.f, cf3 = 0.f, orhs = 0.f;
+      if (own) {
+        const float* cof = p.co + obt * 4 * D + oi;
+        cf0 = cof[0];
+        cf1 = cof[D];
+        cf2 = cof[2 * D];
+        cf3 = cof[3 * D];
+        orhs = p.rhs[obt * D + oi];
+      }
+      // stage X[.][cb0, cb0 + ncb) (float4s, L2: other CTAs wrote it)
+      const int n4 = ncb >> 2;
+      for (int e = tid; e < D * n4; e += kDnThreads) {
+        const int j = e / n4, c4 = e % n4;
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(Xc + (size_t)j * nchp + cb0) + c4);
+        reinterpret_cast<float4*>(Xs + j * kSpCb)[c4] = v;
+      }
+      __syncthreads();
+      // y[m][il][c] over this warp's k range, chains lane and lane + 32
+      float acc[2][3][kSpCpc];
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+#pragma unroll
+          for (int il = 0; il < kSpCpc; ++il) acc[h2][m][il] = 0.f;
+#pragma unroll 4
+      for (int k = k0; k < k1; ++k) {
+        const float xa = Xs[k * kSpCb + lane], xb = Xs[k * kSpCb + 32 + lane];
+        const float4* w4 = reinterpret_cast<const float4*>(Ws + k * 3 * kSpCpc);
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          const float4 w = w4[m];
+          acc[0][m][0] = fmaf(w.x, xa, acc[0][m][0]);
+          acc[0][m][1] = fmaf(w.y, xa, acc[0][m][1]);
+          acc[0][m][2] = fmaf(w.z, xa, acc[0][m][2]);
+          acc[0][m][3] = fmaf(w.w, xa, acc[0][m][3]);
+          acc[1][m][0] = fmaf(w.x, xb, acc[1][m][0]);
+          acc[1][m][1] = fmaf(w.y, xb, acc[1][m][1]);
+          acc[1][m][2] = fmaf(w.z, xb, acc[1][m][2]);
+          acc[1][m][3] = fmaf(w.w, xb, acc[1][m][3]);
+        }
+      }
+      float* pw = part + (size_t)warp * 2 * 3 * kSpCpc * 32;
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+#pragma unroll
+          for (int il = 0; il < kSpCpc; ++il)
+            pw[((h2 * 3 + m) * kSpCpc + il) * 32 + lane] = acc[h2][m][il];
+      __syncthreads();
+      // the thread's output: the warps' sums in order, then J_t x - r_t
+      if (own) {
+        const int h2 = oc >> 5, ln = oc & 31;
+        float y3[3];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          float sum = 0.f;
+          for (int w = 0; w < kSpKg; ++w)
+            sum += part[(size_t)w * 2 * 3 * kSpCpc * 32 + ((h2 * 3 + m) * kSpCpc + oil) * 32 + ln];
+          y3[m] = sum;
+        }
+        const float x = Xs[oi * kSpCb + oc];
+        // W rows: 0 = W_z, 1 = W_r, 2 = W_c
+        const float y = fmaf(cf0, x, fmaf(cf1, y3[0], fmaf(cf2, y3[2], fmaf(cf3, y3[1], orhs))));
+        Xn[(size_t)oi * nchp + ocg] = y;
+        if (kApply) {
+          if (ot < p.T) p.h[((size_t)ob * p.T + ot) * D + oi] += y;
+        } else if (pp == kDnChunk - 1) {
+          p.d[(size_t)ocg * D + oi] = y;
+        }
+      }
+      __syncthreads();
+    }
+    if (pp + 1 < kDnChunk) {
+      ++round;
+      if (!sp_grid_sync(s.bar, round * G, s.timeout_ns)) {
+        if (tid == 0) atomicExch(s.err, 1);
+        return;
+      }
+    }
   }
 }
 
@@ -665,6 +827,17 @@ cudaError_t dn_launch_cluster(K kern, unsigned chains, int D, const Dn2Params& p
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+// A structured pass, launched cooperatively (all its CTAs resident: its
+// steps are separated by grid barriers), its barrier count zeroed first.
+cudaError_t sp_launch(bool apply, const SpParams& sp, unsigned grid, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(sp.bar, 0, sizeof(unsigned), stream);
+  if (e != cudaSuccess) return e;
+  SpParams a = sp;
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel(apply ? (const void*)dn_spass<true> : (const void*)dn_spass<false>,
+                                     dim3(grid), dim3(kDnThreads), args, kSpSmem, stream);
+}
+
 struct DnLayout {
   size_t rmax, Q, J, rhs, P, d, carry, total;
 };
@@ -672,7 +845,7 @@ struct DnLayout {
 // tensor-core path workspace: [0, 256) residual maximum and the GEMMs' error
 // flag, then W^T, Q, W h0, the level-0 blocks, tree levels 1..4, -r, d, carry
 struct Dn2Layout {
-  size_t Wt, Wsp, hsp, h0sp, Q, Q0, J, lvl[kDnLevels], rhs, d, carry, total;
+  size_t Wt, Wsp, hsp, h0sp, Q, Q0, J, lvl[kDnLevels], rhs, d, carry, co, X, total;
 };
 
 Dn2Layout dn2_layout(int B, int T, int D) {
@@ -694,7 +867,10 @@ Dn2Layout dn2_layout(int B, int T, int D) {
   L.rhs = o;
   L.d = L.rhs + align256((size_t)B * Tp * D * 4);
   L.carry = L.d + align256((size_t)B * nC * D * 4);
-  L.total = L.carry + align256((size_t)B * nC * D * 4);
+  L.co = L.carry + align256((size_t)B * nC * D * 4);
+  L.X = L.co + align256((size_t)B * Tp * 4 * D * 4);
+  const size_t nchp = ((size_t)B * nC + 3) & ~size_t(3);
+  L.total = L.X + align256(2 * (size_t)D * nchp * 4);
   return L;
 }
 
@@ -745,6 +921,7 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
   p.J = reinterpret_cast<float*>(ws + L.J);
   p.P = reinterpret_cast<float*>(ws + L.lvl[kDnLevels - 1]);
   p.rhs = reinterpret_cast<float*>(ws + L.rhs);
+  p.co = reinterpret_cast<float*>(ws + L.co);
   p.d = reinterpret_cast<float*>(ws + L.d);
   p.carry = reinterpret_cast<float*>(ws + L.carry);
   p.rmax = reinterpret_cast<unsigned*>(ws);
@@ -807,6 +984,35 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
   if (ge) return ge;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return (int)e;
+  // the structured passes: one CTA per SM, up to 4 channels each
+  SpParams sp;
+  sp.p = p;
+  sp.X = reinterpret_cast<float*>(ws + L.X);
+  sp.bar = reinterpret_cast<unsigned*>(ws + 8);
+  sp.err = err;
+  sp.nch = B * p.nC;
+  sp.nchp = (sp.nch + 3) & ~3;
+  sp.timeout_ns = 1000000000ull;
+  unsigned sgrid_sp = 0;
+  {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    sp.cpc = std::min(kSpCpc, (D + sms - 1) / sms);
+    sgrid_sp = (unsigned)((D + sp.cpc - 1) / sp.cpc);
+    e = cudaFuncSetAttribute(dn_assemble2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kDnAsmSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dn_assemble2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kDnAsmSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dn_spass<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSpSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dn_spass<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSpSmem);
+    if (e != cudaSuccess) return (int)e;
+  }
   pararnn_stats st = {0, 0.f, PARARNN_STATUS_CONVERGED, 0};
   for (int k = 0;; ++k) {
     e = cudaMemsetAsync(p.rmax, 0, sizeof(unsigned), stream);
@@ -814,11 +1020,11 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
     dn_split<<<sgrid, 256, 0, stream>>>(h, hhi, hlo, BT * D);
     ge = split_gemm(mhh, mhl, Q, (int)BT);
     if (ge) return ge;
-    const unsigned nblk = (unsigned)((size_t)B * (p.Tp / kDnAsm));
+    const unsigned nblk = (unsigned)((size_t)B * (p.Tp / kDnAsm) * kDnAsmSplit);
     if (bf16)
-      dn_assemble2<true><<<nblk, kDnThreads, 0, stream>>>(p);
+      dn_assemble2<true><<<nblk, kDnThreads, kDnAsmSmem, stream>>>(p);
     else
-      dn_assemble2<false><<<nblk, kDnThreads, 0, stream>>>(p);
+      dn_assemble2<false><<<nblk, kDnThreads, kDnAsmSmem, stream>>>(p);
     unsigned hdr[2] = {0u, 0u};
     e = cudaGetLastError();
     if (e == cudaSuccess)
@@ -848,10 +1054,9 @@ int dense_solve_tc(bool bf16, const void* u, const float* W, const float* bias, 
                           l + 1 < kDnLevels ? 2 : 0, err, stream);
       if (ge) return ge;
     }
-    const unsigned nmaps = (unsigned)((size_t)B * p.nC);
-    e = dn_launch_cluster(dn_offsets, nmaps, D, p, stream);
+    e = sp_launch(false, sp, sgrid_sp, stream);
     if (e == cudaSuccess) e = dn_launch_cluster(dn_carry2, (unsigned)B, D, p, stream, true);
-    if (e == cudaSuccess) e = dn_launch_cluster(dn_apply2, nmaps, D, p, stream);
+    if (e == cudaSuccess) e = sp_launch(true, sp, sgrid_sp, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
     st.iters = k + 1;
