@@ -626,7 +626,8 @@ __global__ void __launch_bounds__(kDnThreads) dn_carry2(const Dn2Params p) {
 // step's delta added to h.
 constexpr int kSpCpc = 4;                    // channels per CTA, at most
 constexpr int kSpCb = 64;                    // chains per staged block
-constexpr int kSpKg = kDnThreads / 32;       // k groups (warps)
+constexpr int kSpThreads = 512;
+constexpr int kSpKg = kSpThreads / 32;       // k groups (warps)
 struct SpParams {
   Dn2Params p;
   float* X;             // [2][D][nchp] chain deltas, chains innermost
@@ -664,7 +665,7 @@ __device__ __forceinline__ bool sp_grid_sync(unsigned* bar, unsigned target, uin
 }
 
 template <bool kApply>
-__global__ void __launch_bounds__(kDnThreads, 1) dn_spass(const SpParams s) {
+__global__ void __launch_bounds__(kSpThreads, 1) dn_spass(const SpParams s) {
   extern __shared__ __align__(16) float sp_sm[];
   const Dn2Params& p = s.p;
   const int D = p.D, nch = s.nch, nchp = s.nchp, cpc = s.cpc;
@@ -675,14 +676,14 @@ __global__ void __launch_bounds__(kDnThreads, 1) dn_spass(const SpParams s) {
   const int i0 = blockIdx.x * cpc;
   const unsigned G = gridDim.x;
   // this CTA's rows of W_z, W_r, W_c, k-major (rows past D or cpc: zero)
-  for (int e = tid; e < D * 3 * kSpCpc; e += kDnThreads) {
+  for (int e = tid; e < D * 3 * kSpCpc; e += kSpThreads) {
     const int k = e / (3 * kSpCpc), rem = e % (3 * kSpCpc), m = rem / kSpCpc, il = rem % kSpCpc;
     const int i = i0 + il;
     Ws[e] = (il < cpc && i < D) ? p.W[((size_t)m * D + i) * D + k] : 0.f;
   }
   // the deltas entering the chunks: zero (offsets) or the carries (apply)
   float* X0 = s.X;
-  for (int e = tid; e < cpc * nch; e += kDnThreads) {
+  for (int e = tid; e < cpc * nch; e += kSpThreads) {
     const int il = e / nch, cg = e % nch, i = i0 + il;
     if (i < D) X0[(size_t)i * nchp + cg] = kApply ? p.carry[(size_t)cg * D + i] : 0.f;
   }
@@ -699,7 +700,7 @@ __global__ void __launch_bounds__(kDnThreads, 1) dn_spass(const SpParams s) {
       const int ncb = min(kSpCb, nchp - cb0);    // a multiple of 4
       // this thread's output (channel il, chain c of the block): its
       // coefficients and -r loaded now, used after the products
-      const int oil = tid / kSpCb, oc = tid % kSpCb;
+      const int oil = tid / kSpCb, oc = tid % kSpCb;  // threads past 4 x 64: none
       const int oi = i0 + oil, ocg = cb0 + oc;
       const bool own = oil < cpc && oi < D && ocg < nch;
       const int ob = own ? ocg / p.nC : 0, okc = own ? ocg - ob * p.nC : 0;
@@ -716,7 +717,8 @@ __global__ void __launch_bounds__(kDnThreads, 1) dn_spass(const SpParams s) {
       }
       // stage X[.][cb0, cb0 + ncb) (float4s, L2: other CTAs wrote it)
       const int n4 = ncb >> 2;
-      for (int e = tid; e < D * n4; e += kDnThreads) {
+#pragma unroll 16
+      for (int e = tid; e < D * n4; e += kSpThreads) {
         const int j = e / n4, c4 = e % n4;
         const float4 v = __ldcg(reinterpret_cast<const float4*>(Xc + (size_t)j * nchp + cb0) + c4);
         reinterpret_cast<float4*>(Xs + j * kSpCb)[c4] = v;
@@ -835,7 +837,7 @@ cudaError_t sp_launch(bool apply, const SpParams& sp, unsigned grid, cudaStream_
   SpParams a = sp;
   void* args[] = {&a};
   return cudaLaunchCooperativeKernel(apply ? (const void*)dn_spass<true> : (const void*)dn_spass<false>,
-                                     dim3(grid), dim3(kDnThreads), args, kSpSmem, stream);
+                                     dim3(grid), dim3(kSpThreads), args, kSpSmem, stream);
 }
 
 struct DnLayout {
