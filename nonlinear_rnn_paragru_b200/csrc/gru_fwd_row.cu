@@ -35,8 +35,9 @@
 // predecessor's pre-update last state plus the incoming delta.
 //
 // Data: bf16 u arrives by four TMA boxes of 256 steps into the top of the
-// CTA's 98 KB buffer (fp32 u is read straight from global memory by the
-// expansion, the next tile's rows prefetched into L2 meanwhile); a, bias and
+// CTA's 98 KB buffer, fp32 u by four boxes that fill it from its start (the
+// expansion then takes its second block first, so that it stays in place);
+// the next tile's boxes are prefetched into L2 meanwhile; a, bias and
 // h0 of the next tile's channels are read with plain loads a tile ahead into
 // a double-buffered block.  Once per tile u is expanded in place into the
 // fp32 arguments -log2e u_z + b'_z, -log2e u_r + b'_r, 2 log2e u_c + b'_c
@@ -77,6 +78,13 @@ static_assert(kRowStage % 128 == 0 && kRowBoxBytes % 128 == 0, "TMA destinations
 static_assert(kRowThreads == (kRowChunks / 2) * kRowH, "the expansion: one (chunk, pair) per thread");
 // expansion block 0 (chunks below kRowChunks / 2) writes below every staged byte
 static_assert((kRowChunks / 2) * kRowS <= kRowStage, "in-place expansion order");
+// fp32 u: the four 256-step boxes fill the buffer from its start (96 bytes a
+// step); the expansion takes block 1 first, whose slots lie above every row
+// of block 0, then block 0, whose slots reach into block 1's rows only
+constexpr int kRowBoxBytesF32 = kRowBox * 3 * kRowC * 4;    // 24576
+static_assert(kRowNBox * kRowBoxBytesF32 <= kRowU &&
+                  (kRowChunks / 2) * kRowS >= (kRowChunks / 2) * kRowL * 3 * kRowC * 4,
+              "in-place fp32 expansion order");
 
 struct RowMailbox {  // written by the cluster peers with remote async stores
   float4 map[kRowMaxCluster][kRowC];   // (P, ds, last state before the update, -) by rank
@@ -126,12 +134,17 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned b
 
 // Thread 0: load the tile's four 256-step boxes for CTA `rank` into the
 // staging area, on `bar`.
+// The tile's boxes that hold steps of this CTA's range (nbox of them, 0 to
+// 4; the expansion takes steps past the range as zeros).
+template <bool kF32>
 __device__ __forceinline__ void row_issue(unsigned char* smem, RowShared& sh,
-                                          const CUtensorMap* map, int b, int d0, int t0) {
+                                          const CUtensorMap* map, int b, int d0, int t0,
+                                          int nbox) {
+  constexpr int kStage = kF32 ? 0 : kRowStage, kBox = kF32 ? kRowBoxBytesF32 : kRowBoxBytes;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  mbar_arrive_expect_tx(&sh.bar, (unsigned)(kRowNBox * kRowBoxBytes));
-  for (int j = 0; j < kRowNBox; ++j)
-    tma_load_4d(smem + kRowStage + j * kRowBoxBytes, map, &sh.bar, d0, 0, t0 + j * kRowBox, b);
+  mbar_arrive_expect_tx(&sh.bar, (unsigned)(nbox * kBox));
+  for (int j = 0; j < nbox; ++j)
+    tma_load_4d(smem + kStage + j * kBox, map, &sh.bar, d0, 0, t0 + j * kRowBox, b);
 }
 // Parameter j (0..55) of the tile at (b, d0): a[g][c] (j < 24), bias[g][c]
 // (j < 48, 0 when absent), h0[c] (0 when absent).
@@ -142,8 +155,9 @@ __device__ __forceinline__ float row_param(const FwdParams& p, int j, int b, int
   return p.h0 ? p.h0[(size_t)b * p.ld_h0 + d0 + c] : 0.f;
 }
 // L2 prefetch of a tile's boxes (no shared memory touched).
-__device__ __forceinline__ void row_prefetch(const CUtensorMap* map, int b, int d0, int t0) {
-  for (int j = 0; j < kRowNBox; ++j)
+__device__ __forceinline__ void row_prefetch(const CUtensorMap* map, int b, int d0, int t0,
+                                             int nbox) {
+  for (int j = 0; j < nbox; ++j)
     asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
                  "r"(d0), "r"(0), "r"(t0 + j * kRowBox), "r"(b)
@@ -170,6 +184,8 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   const int nclus = gridDim.x / CLS, clus = blockIdx.x / CLS;
   const int t0 = rank * kRowSteps;           // first step of this CTA in the segment
   const int tg0 = p.t_base + t0;             // ... in the sequence
+  // boxes of this CTA's range that hold steps of the segment
+  const int nbox = min(kRowNBox, max(0, (p.t_len - t0 + kRowBox - 1) / kRowBox));
   const unsigned rx = row_rx_bytes(rank, CLS);
 
   // the first tile's parameters; later tiles' are loaded a tile ahead
@@ -189,9 +205,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   __syncthreads();
   // the peers' mailbox barriers are armed before anyone sends
   if (CLS > 1) cluster.sync();
-  if (!kF32 && tid == 0 && clus < ntiles) {
+  if (tid == 0 && clus < ntiles) {
     const int b = clus / nDTc;
-    row_issue(smem, sh, &map, b, (clus - b * nDTc) * kRowC, tg0);
+    row_issue<kF32>(smem, sh, &map, b, (clus - b * nDTc) * kRowC, tg0, nbox);
   }
   const unsigned char* base = smem + q * kRowS;
   int status = 0;
@@ -228,24 +244,11 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     const int b = tile / nDTc, d0 = (tile - b * nDTc) * kRowC;
     const int d = d0 + c;
     const bool dval = d < p.D;
-    if (!kF32 && tid == 0 && next < ntiles) {
+    if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, tg0);
+      row_prefetch(&map, b2, (next - b2 * nDTc) * kRowC, tg0, nbox);
     }
-    if (kF32 && next < ntiles) {
-      // the next tile's fp32 rows into L2, 12 (step, gate) rows per thread
-      const int b2 = next / nDTc, d2 = (next - b2 * nDTc) * kRowC;
-      const float* ug = static_cast<const float*>(p.u);
-#pragma unroll 4
-      for (int r = tid; r < kRowSteps * 3; r += kRowThreads) {
-        const int t = r / 3, g = r - t * 3;
-        if (t0 + t < p.t_len)
-          asm volatile("prefetch.global.L2 [%0];" ::"l"(
-              ug + (((size_t)b2 * p.T + tg0 + t) * 3 + g) * p.D + d2));
-      }
-    }
-    if (!kF32 && !mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns))
-      status = PARARNN_STATUS_TIMEOUT;
+    if (!mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns)) status = PARARNN_STATUS_TIMEOUT;
     // ---- expand the staged bf16 rows [t][gate][8 ch] into the fp32 arguments
     // in two blocks of 512 steps (each block's rows are read before any of
     // its slots is written; block 0 writes below all staging bytes).  Thread
@@ -254,30 +257,22 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       const int qb = tid / kRowH, i = tid % kRowH;
       const int sw = row_swizzle(i);
 #pragma unroll 1
-      for (int blk = 0; blk < 2; ++blk) {
+      for (int bi = 0; bi < 2; ++bi) {
+        const int blk = kF32 ? 1 - bi : bi;  // fp32: block 1 first (in place)
         const int qq = blk * (kRowChunks / 2) + qb;
         const int ta = qq * kRowL + i, tb = ta + kRowH;  // steps within the CTA
         const bool pa = t0 + ta >= p.t_len, pbd = t0 + tb >= p.t_len;
-        // the 8 channels of gate g at steps ta (xa) and tb (xb): bf16 from
-        // the staging area, fp32 straight from global memory
+        // the 8 channels of gate g at steps ta (xa) and tb (xb) from the
+        // staged rows (bf16 at the top of the buffer, fp32 from its start)
         float xa[3][kRowC], xb[3][kRowC];
         if (kF32) {
-          const float* ug = static_cast<const float*>(p.u);
 #pragma unroll
           for (int g = 0; g < 3; ++g) {
-            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
-            if (!pa) {
-              const float4* ra = reinterpret_cast<const float4*>(
-                  ug + (((size_t)b * p.T + tg0 + ta) * 3 + g) * p.D + d0);
-              a0 = __ldg(ra);
-              a1 = __ldg(ra + 1);
-            }
-            if (!pbd) {
-              const float4* rb = reinterpret_cast<const float4*>(
-                  ug + (((size_t)b * p.T + tg0 + tb) * 3 + g) * p.D + d0);
-              b0 = __ldg(rb);
-              b1 = __ldg(rb + 1);
-            }
+            const float4* ra = reinterpret_cast<const float4*>(smem + (ta * 3 + g) * kRowC * 4);
+            const float4* rb = reinterpret_cast<const float4*>(smem + (tb * 3 + g) * kRowC * 4);
+            const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 a0 = pa ? z4 : ra[0], a1 = pa ? z4 : ra[1];
+            const float4 b0 = pbd ? z4 : rb[0], b1 = pbd ? z4 : rb[1];
             const float fa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float fb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -289,9 +284,10 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         } else {
 #pragma unroll
           for (int g = 0; g < 3; ++g) {
-            const uint4 va = *reinterpret_cast<const uint4*>(
+            const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            const uint4 va = pa ? z4 : *reinterpret_cast<const uint4*>(
                 smem + kRowStage + (ta / kRowBox) * kRowBoxBytes + ((ta % kRowBox) * 3 + g) * 16);
-            const uint4 vb = *reinterpret_cast<const uint4*>(
+            const uint4 vb = pbd ? z4 : *reinterpret_cast<const uint4*>(
                 smem + kRowStage + (tb / kRowBox) * kRowBoxBytes + ((tb % kRowBox) * 3 + g) * 16);
             const unsigned wa[4] = {va.x, va.y, va.z, va.w};
             const unsigned wb[4] = {vb.x, vb.y, vb.z, vb.w};
@@ -489,9 +485,9 @@ __global__ void __launch_bounds__(kRowThreads, 2)
     }
     // every thread of the CTA is past its last pass of this tile (the
     // barrier of the last exchange): the staging area takes the next tile
-    if (!kF32 && tid == 0 && next < ntiles) {
+    if (tid == 0 && next < ntiles) {
       const int b2 = next / nDTc;
-      row_issue(smem, sh, &map, b2, (next - b2 * nDTc) * kRowC, tg0);
+      row_issue<kF32>(smem, sh, &map, b2, (next - b2 * nDTc) * kRowC, tg0, nbox);
     }
     if (pj >= 0 && pj < 7 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
 
