@@ -60,6 +60,7 @@ struct QParams {
   int ntiles;           // B * nDTc
   int nseg;             // segments per sequence
   int nitems;           // ntiles * nseg (below 2^31: B*T*D <= 2^40)
+  FastDiv dv_tiles, dv_ndtc;  // division by ntiles and by nDTc
   int max_iters;
   float tol;
   float apx_tau;        // inexact evaluations while the item's residual is above this (0: none)
@@ -105,6 +106,20 @@ struct QShared {
   int nx[2];                   // this and the next item, by item parity
 };
 
+// An item's segment, tile, batch row and first channel (item = segment *
+// ntiles + tile, tile = row * nDTc + channel block), by multiply-high division
+__device__ __forceinline__ int q_seg(const QParams& p, int item) {
+  return fast_quot(item, p.dv_tiles);
+}
+__device__ __forceinline__ int q_tile(const QParams& p, int item) {
+  return item - q_seg(p, item) * p.ntiles;
+}
+__device__ __forceinline__ int q_row(const QParams& p, int tile) {
+  return fast_quot(tile, p.dv_ndtc);
+}
+__device__ __forceinline__ int q_d0(const QParams& p, int tile) {
+  return (tile - q_row(p, tile) * p.nDTc) * kRowC;
+}
 __device__ __forceinline__ void q_issue(unsigned char* smem, int stage, int nbox, uint64_t* bar,
                                         const CUtensorMap* map, int b, int d0, int t0) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -149,12 +164,12 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   __syncthreads();
   int item = sh.nx[0];
   if (item < p.nitems) {
-    const int tile = item % p.ntiles;
-    const int d0 = (tile % p.nDTc) * kRowC;
+    const int tile = q_tile(p, item);
+    const int d0 = q_d0(p, tile);
     if (tid < 6 * kRowC) (&sh.par[0][0][0])[tid] = q_param(p, tid, d0);
     if (tid == 0)
-      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, tile / p.nDTc, d0,
-              (item / p.ntiles) * Cfg::kSteps);
+      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, q_row(p, tile), d0,
+              q_seg(p, item) * Cfg::kSteps);
   }
   int status = 0;
   unsigned phase = 0;  // exchange phases so far, over all items
@@ -168,12 +183,12 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     // barrier above; the fence and release order them before the count
     if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
       __threadfence();
-      st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+      st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
     }
     if (tid == 0) sh.nx[(n + 1) & 1] = q_draw(p.counter);
     const int pb = n & 1;
-    const int tile = item % p.ntiles, seg = item / p.ntiles;
-    const int b = tile / p.nDTc, d0 = (tile % p.nDTc) * kRowC;
+    const int tile = q_tile(p, item), seg = q_seg(p, item);
+    const int b = q_row(p, tile), d0 = q_d0(p, tile);
     const int d = d0 + c;
     const bool dval = d < p.D;
     const int t_base = seg * Cfg::kSteps;
@@ -239,10 +254,10 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     {
       const int next = sh.nx[(n + 1) & 1];
       if (next < p.nitems) {
-        const int ntile = next % p.ntiles;
-        const int nd0 = (ntile % p.nDTc) * kRowC;
+        const int ntile = q_tile(p, next);
+        const int nd0 = q_d0(p, ntile);
         if (tid == 0)
-          q_prefetch(&map, Cfg::kNBox, ntile / p.nDTc, nd0, (next / p.ntiles) * Cfg::kSteps);
+          q_prefetch(&map, Cfg::kNBox, q_row(p, ntile), nd0, q_seg(p, next) * Cfg::kSteps);
         if (pj >= 0 && pj < 6 * kRowC) pnext = q_param(p, pj, nd0);
       }
     }
@@ -385,15 +400,15 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     // exchange): the staging area takes the next item
     const int next = sh.nx[(n + 1) & 1];
     if (tid == 0 && !dead && next < p.nitems) {
-      const int ntile = next % p.ntiles;
-      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, ntile / p.nDTc,
-              (ntile % p.nDTc) * kRowC, (next / p.ntiles) * Cfg::kSteps);
+      const int ntile = q_tile(p, next);
+      q_issue(smem, Cfg::kStage, Cfg::kNBox, &sh.bar, &map, q_row(p, ntile),
+              q_d0(p, ntile), q_seg(p, next) * Cfg::kSteps);
     }
     if (pj >= 0 && pj < 6 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
     // ---- states straight from registers (indices re-derived from the item)
     item = sh.nx[n & 1];
-    const int itile = item % p.ntiles, it_base = (item / p.ntiles) * Cfg::kSteps;
-    const int ib = itile / p.nDTc, id = (itile % p.nDTc) * kRowC + c;
+    const int itile = q_tile(p, item), it_base = q_seg(p, item) * Cfg::kSteps;
+    const int ib = q_row(p, itile), id = q_d0(p, itile) + c;
     const int it_len = min(Cfg::kSteps, p.T - it_base);
     bool bad = false;
     if (id < p.D) {
@@ -425,7 +440,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   __syncthreads();
   if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
     __threadfence();
-    st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+    st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
   }
   // boxes still in flight into the staging area: wait for them (bounded)
   if (dead && tid == 0) mbar_wait_bounded(&sh.bar, (unsigned)(dead - 1), p.timeout_ns);
@@ -496,6 +511,8 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.D = f.D;
   p.nDTc = (f.D + kRowC - 1) / kRowC;
   p.ntiles = f.B * p.nDTc;
+  p.dv_tiles = fast_div((unsigned)p.ntiles);
+  p.dv_ndtc = fast_div((unsigned)p.nDTc);
   p.nseg = (f.T + QRun::kSteps - 1) / QRun::kSteps;
   if ((long long)p.ntiles * p.nseg >= (1LL << 31)) return 1;
   p.nitems = p.ntiles * p.nseg;

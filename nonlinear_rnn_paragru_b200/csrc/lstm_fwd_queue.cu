@@ -94,6 +94,7 @@ struct LqParams {
   int nDTc;             // 8-channel tiles per batch row
   int ntiles;           // B * nDTc
   int nitems;           // ntiles * segments (below 2^31)
+  FastDiv dv_tiles, dv_ndtc;  // division by ntiles and by nDTc
   int max_iters;
   float tol;
   float apx_tau;        // inexact evaluations while the item's residual is above this (0: none)
@@ -253,6 +254,20 @@ __device__ __forceinline__ float lq_param(const LqParams& p, int j, int b, int d
   if (row == 8) return p.c0 ? p.c0[(size_t)b * p.D + d0 + c] : 0.f;
   return p.h0 ? p.h0[(size_t)b * p.D + d0 + c] : 0.f;
 }
+// An item's segment, tile, batch row and first channel (item = segment *
+// ntiles + tile, tile = row * nDTc + channel block), by multiply-high division
+__device__ __forceinline__ int lq_seg(const LqParams& p, int item) {
+  return fast_quot(item, p.dv_tiles);
+}
+__device__ __forceinline__ int lq_tile(const LqParams& p, int item) {
+  return item - lq_seg(p, item) * p.ntiles;
+}
+__device__ __forceinline__ int lq_row(const LqParams& p, int tile) {
+  return fast_quot(tile, p.dv_ndtc);
+}
+__device__ __forceinline__ int lq_d0(const LqParams& p, int tile) {
+  return (tile - lq_row(p, tile) * p.nDTc) * kLqC;
+}
 __device__ __forceinline__ void lq_issue(unsigned char* smem, uint64_t* bar, const CUtensorMap* map,
                                          int b, int d0, int t0) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -281,9 +296,9 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
   __syncthreads();
   int item = sh.nx[0];
   if (item < p.nitems) {
-    const int tile = item % p.ntiles, b = tile / p.nDTc, d0 = (tile % p.nDTc) * kLqC;
+    const int tile = lq_tile(p, item), b = lq_row(p, tile), d0 = lq_d0(p, tile);
     if (tid < 10 * kLqC) (&sh.par[0][0][0])[tid] = lq_param(p, tid, b, d0);
-    if (tid == 0) lq_issue(smem, &sh.bar, &map, b, d0, (item / p.ntiles) * kLqSteps);
+    if (tid == 0) lq_issue(smem, &sh.bar, &map, b, d0, lq_seg(p, item) * kLqSteps);
   }
   int status = 0;
   unsigned phase = 0;  // exchange phases so far, over all items
@@ -297,12 +312,12 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     // barrier above; the fence and release order them before the count
     if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
       __threadfence();
-      st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+      st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
     }
     if (tid == 0) sh.nx[(n + 1) & 1] = lq_draw(p.counter);
     const int pb = n & 1;
-    const int tile = item % p.ntiles, seg = item / p.ntiles;
-    const int b = tile / p.nDTc, d0 = (tile % p.nDTc) * kLqC;
+    const int tile = lq_tile(p, item), seg = lq_seg(p, item);
+    const int b = lq_row(p, tile), d0 = lq_d0(p, tile);
     const int d = d0 + c;
     const bool dval = d < p.D;
     const int t_base = seg * kLqSteps;
@@ -375,8 +390,8 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     const int pj = tid - 32;
     float pnext = 0.f;
     if (next < p.nitems) {
-      const int ntile = next % p.ntiles, nb = ntile / p.nDTc, nd0 = (ntile % p.nDTc) * kLqC;
-      if (tid == 0 && !dead) lq_issue(smem, &sh.bar, &map, nb, nd0, (next / p.ntiles) * kLqSteps);
+      const int ntile = lq_tile(p, next), nb = lq_row(p, ntile), nd0 = lq_d0(p, ntile);
+      if (tid == 0 && !dead) lq_issue(smem, &sh.bar, &map, nb, nd0, lq_seg(p, next) * kLqSteps);
       if (pj >= 0 && pj < 10 * kLqC) pnext = lq_param(p, pj, nb, nd0);
     }
     const bool first = (q == 0);  // the chunk holding the segment's first step
@@ -544,7 +559,7 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
   __syncthreads();
   if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
     __threadfence();
-    st_release(&p.seg_done[prev_item % p.ntiles], (unsigned)(prev_item / p.ntiles) + 1u);
+    st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
   }
   // a box still in flight into the staging area: wait for it (bounded)
   if (dead && tid == 0) mbar_wait_bounded(&sh.bar, (unsigned)(dead - 1), p.timeout_ns);
@@ -594,6 +609,8 @@ int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* coun
   p.D = f.D;
   p.nDTc = (f.D + kLqC - 1) / kLqC;
   p.ntiles = f.B * p.nDTc;
+  p.dv_tiles = fast_div((unsigned)p.ntiles);
+  p.dv_ndtc = fast_div((unsigned)p.nDTc);
   const long long nitems = (long long)p.ntiles * ((f.T + kLqSteps - 1) / kLqSteps);
   if (nitems >= (1LL << 31)) return 1;
   p.nitems = (int)nitems;
