@@ -180,8 +180,9 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   for (int n = 0; item < p.nitems; ++n) {
     __syncthreads();
     // publish the previous item: every thread's state stores precede the
-    // barrier above; the fence and release order them before the count
-    if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
+    // barrier above; the fence and release order them before the count (warp
+    // 1, while warp 0 draws the next ticket: both wait on memory)
+    if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
       __threadfence();
       st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
     }
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     item = next;
   }
   __syncthreads();
-  if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
+  if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
     __threadfence();
     st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
   }

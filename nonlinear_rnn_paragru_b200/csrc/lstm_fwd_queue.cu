@@ -309,12 +309,16 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
   for (int n = 0; item < p.nitems; ++n) {
     __syncthreads();
     // publish the previous item: every thread's state stores precede the
-    // barrier above; the fence and release order them before the count
-    if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
+    // barrier above; the fence and release order them before the count (warp
+    // 1, while warp 0 draws the next ticket: both wait on memory)
+    if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
       __threadfence();
       st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
     }
-    if (tid == 0) sh.nx[(n + 1) & 1] = lq_draw(p.counter);
+    // the item after this one: drawn now, stored before the item's first
+    // barrier (the atomic's latency overlaps the wait for the boxes)
+    int ticket = 0;
+    if (tid == 0) ticket = lq_draw(p.counter);
     const int pb = n & 1;
     const int tile = lq_tile(p, item), seg = lq_seg(p, item);
     const int b = lq_row(p, tile), d0 = lq_d0(p, tile);
@@ -379,6 +383,7 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       k.ao2 = qf2(ao2, ao2);
     }
     float c0v = sh.par[pb][8][c], h0v = sh.par[pb][9][c];
+    if (tid == 0) sh.nx[(n + 1) & 1] = ticket;  // read after the barrier below
     // a phase that did not complete is never re-armed: no more boxes then
     if (dead) {
       __syncthreads();
@@ -557,7 +562,7 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     item = next;
   }
   __syncthreads();
-  if (tid == 0 && prev_item >= 0 && prev_item != p.withhold_item) {
+  if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
     __threadfence();
     st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
   }
