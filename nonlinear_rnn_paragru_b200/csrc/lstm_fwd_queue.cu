@@ -326,6 +326,26 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     const bool dval = d < p.D;
     const int t_base = seg * kLqSteps;
     const int t_len = min(kLqSteps, p.T - t_base);
+    const bool first = (q == 0);  // the chunk holding the segment's first step
+    // the segment's initial state: (c0, h0), or the last states of the
+    // previous segment once that segment's CTA has published them (waited
+    // for and loaded here, so that the loads overlap the wait for the box)
+    float pc0 = 0.f, ph0 = 0.f;
+    if (first && seg > 0) {
+      const unsigned* f = &p.seg_done[tile];
+      if (ld_acquire(f) < (unsigned)seg) {
+        const uint64_t w0 = globaltimer_ns();
+        while (ld_acquire(f) < (unsigned)seg) {
+          if (globaltimer_ns() - w0 > p.timeout_ns) {
+            status = PARARNN_STATUS_TIMEOUT;
+            break;
+          }
+        }
+      }
+      const size_t ip = ((size_t)b * p.T + t_base - 1) * p.D + d;
+      pc0 = dval ? __ldcg(p.c + ip) : 0.f;
+      ph0 = dval ? __ldcg(p.h + ip) : 0.f;
+    }
     bool got = true;
     if (!dead) {
       got = mbar_wait_bounded(&sh.bar, n & 1, p.timeout_ns);
@@ -399,23 +419,9 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       if (tid == 0 && !dead) lq_issue(smem, &sh.bar, &map, nb, nd0, lq_seg(p, next) * kLqSteps);
       if (pj >= 0 && pj < 10 * kLqC) pnext = lq_param(p, pj, nb, nd0);
     }
-    const bool first = (q == 0);  // the chunk holding the segment's first step
-    // the segment's initial state: (c0, h0), or the last states of the
-    // previous segment once that segment's CTA has published them
     if (first && seg > 0) {
-      const unsigned* f = &p.seg_done[tile];
-      if (ld_acquire(f) < (unsigned)seg) {
-        const uint64_t w0 = globaltimer_ns();
-        while (ld_acquire(f) < (unsigned)seg) {
-          if (globaltimer_ns() - w0 > p.timeout_ns) {
-            status = PARARNN_STATUS_TIMEOUT;
-            break;
-          }
-        }
-      }
-      const size_t ip = ((size_t)b * p.T + t_base - 1) * p.D + d;
-      c0v = dval ? __ldcg(p.c + ip) : 0.f;
-      h0v = dval ? __ldcg(p.h + ip) : 0.f;
+      c0v = pc0;
+      h0v = ph0;
     }
 
     float2 C[kLqH], H[kLqH], P00[kLqH], P01[kLqH], P10[kLqH], P11[kLqH];
