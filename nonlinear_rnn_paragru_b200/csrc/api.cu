@@ -20,7 +20,8 @@ int launch_gru_row(const CUtensorMap& map, const FwdParams& p, bool f32, cudaStr
 int gru_row_max_steps();
 int gru_row_cta_steps();
 int gru_queue_resident();
-int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+int launch_gru_queue(const CUtensorMap& map, const CUtensorMap& hmap, const FwdParams& f,
+                     unsigned* counter,
                      unsigned* seg_done, cudaStream_t stream);
 int launch_lstm_fwd(const CUtensorMap& tmap, bool bf16, const FwdParams& p, int nctas,
                     cudaStream_t stream);
@@ -356,8 +357,10 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   if (queue_gru) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, true, B, T, G, D, gru_row_box_steps(), gru_row_channels());
+    CUtensorMap hmap;  // the states, stored by the same 256-step boxes
+    if (!rc) rc = make_s_map(&hmap, h, B, T, D, gru_row_box_steps(), gru_row_channels());
     if (rc) return rc;
-    e = launch_gru_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
+    e = launch_gru_queue(rmap, hmap, p, &p.hdr->ticket, seg_done, stream);
   } else if (queue_lstm) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_queue_box_steps(), lstm_row_channels());

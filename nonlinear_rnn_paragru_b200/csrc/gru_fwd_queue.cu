@@ -92,6 +92,7 @@ struct QCfg {
   static_assert(kBlocks == 1 || (kBlocks == 2 && (kChunks / 2) * kS <= kStage),
                 "in-place expansion order");
   static_assert(kS % 128 == 64, "a warp's four chunks in alternate 64-byte bank halves");
+  static_assert(kSteps * kRowC * 4 <= kStage, "the states' store buffer below the staging area");
   static_assert(NW == 4 || NW == 8, "the CTA's residual maximum is read as float4s");
 };
 
@@ -147,7 +148,8 @@ __device__ __forceinline__ int q_draw(unsigned* counter) {
 
 template <int NW, int L, int MINB>
 __global__ void __launch_bounds__(NW * 32, MINB)
-    gru_newton_queue(const __grid_constant__ CUtensorMap map, const QParams p) {
+    gru_newton_queue(const __grid_constant__ CUtensorMap map,
+                     const __grid_constant__ CUtensorMap hmap, const QParams p) {
   using Cfg = QCfg<NW, L>;
   constexpr int kH = Cfg::kH;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -179,14 +181,20 @@ __global__ void __launch_bounds__(NW * 32, MINB)
   int dead = 0;
   for (int n = 0; item < p.nitems; ++n) {
     __syncthreads();
-    // publish the previous item: every thread's state stores precede the
-    // barrier above; the fence and release order them before the count (warp
-    // 1, while warp 0 draws the next ticket: both wait on memory)
-    if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
-      __threadfence();
-      st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
+    // publish the previous item: its states' bulk stores (issued by thread 0)
+    // complete, then the proxy fence, the fence and the release order them
+    // before the count.  The wait also frees the stores' shared memory before
+    // this item's expansion writes there.  Warp 1 draws the next ticket
+    // meanwhile: both wait on memory.
+    if (tid == 0 && prev_item >= 0) {
+      bulk_wait_all();
+      if (prev_item != p.withhold_item) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
+      }
     }
-    if (tid == 0) sh.nx[(n + 1) & 1] = q_draw(p.counter);
+    if (tid == 32) sh.nx[(n + 1) & 1] = q_draw(p.counter);
     const int pb = n & 1;
     const int tile = q_tile(p, item), seg = q_seg(p, item);
     const int b = q_row(p, tile), d0 = q_d0(p, tile);
@@ -406,25 +414,35 @@ __global__ void __launch_bounds__(NW * 32, MINB)
               q_d0(p, ntile), q_seg(p, next) * Cfg::kSteps);
     }
     if (pj >= 0 && pj < 6 * kRowC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
-    // ---- states straight from registers (indices re-derived from the item)
+    // ---- states: from registers into the buffer below the staging area
+    // ([step][8 ch], 16 KB; every pass is done and the next item's boxes
+    // land above it), then two 256-step bulk-tensor stores (steps past T are
+    // not written).  Indices re-derived from the item.
     item = sh.nx[n & 1];
     const int itile = q_tile(p, item), it_base = q_seg(p, item) * Cfg::kSteps;
     const int ib = q_row(p, itile), id = q_d0(p, itile) + c;
     const int it_len = min(Cfg::kSteps, p.T - it_base);
     bool bad = false;
-    if (id < p.D) {
+    {
+      float* sts = reinterpret_cast<float*>(smem);
       const int tq = q * L;
-      float* out = p.h + ((size_t)ib * p.T + it_base + tq) * p.D + id;
 #pragma unroll
       for (int i = 0; i < kH; ++i) {
-        if (tq + i < it_len) {
-          out[(size_t)i * p.D] = H[i].x;
-          bad |= !isfinite(H[i].x);
+        sts[(tq + i) * kRowC + c] = H[i].x;
+        sts[(tq + kH + i) * kRowC + c] = H[i].y;
+        if (id < p.D) {
+          bad |= tq + i < it_len && !isfinite(H[i].x);
+          bad |= tq + kH + i < it_len && !isfinite(H[i].y);
         }
-        if (tq + kH + i < it_len) {
-          out[(size_t)(kH + i) * p.D] = H[i].y;
-          bad |= !isfinite(H[i].y);
-        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      if (tid == 0) {
+        const int d0i = q_d0(p, itile);
+#pragma unroll
+        for (int j = 0; j < Cfg::kNBox; ++j)
+          tma_store_3d(&hmap, smem + j * kRowBox * kRowC * 4, d0i, it_base + j * kRowBox, ib);
+        bulk_commit();
       }
     }
     if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
@@ -439,9 +457,13 @@ __global__ void __launch_bounds__(NW * 32, MINB)
     item = next;
   }
   __syncthreads();
-  if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
-    __threadfence();
-    st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
+  if (tid == 0 && prev_item >= 0) {
+    bulk_wait_all();
+    if (prev_item != p.withhold_item) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __threadfence();
+      st_release(&p.seg_done[q_tile(p, prev_item)], (unsigned)q_seg(p, prev_item) + 1u);
+    }
   }
   // boxes still in flight into the staging area: wait for them (bounded)
   if (dead && tid == 0) mbar_wait_bounded(&sh.bar, (unsigned)(dead - 1), p.timeout_ns);
@@ -457,7 +479,8 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 constexpr int kQW = 4, kQL = 32, kQMinB = 4;
 using QRun = QCfg<kQW, kQL>;
 
-int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) {
+int launch_queue(const CUtensorMap& map, const CUtensorMap& hmap, const QParams& p,
+                 cudaStream_t stream) {
   auto kern = gru_newton_queue<kQW, kQL, kQMinB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, QRun::kU);
   if (e != cudaSuccess) return (int)e;
@@ -471,7 +494,7 @@ int launch_queue(const CUtensorMap& map, const QParams& p, cudaStream_t stream) 
   cudaGetLastError();
   // persistent: every CTA resident at once (the queue's progress argument)
   const long long grid = std::min<long long>((long long)sms * per_sm, p.nitems);
-  kern<<<(unsigned)std::max<long long>(grid, 1), QRun::kThreads, QRun::kU, stream>>>(map, p);
+  kern<<<(unsigned)std::max<long long>(grid, 1), QRun::kThreads, QRun::kU, stream>>>(map, hmap, p);
   return (int)cudaGetLastError();
 }
 
@@ -500,8 +523,9 @@ int gru_queue_resident() {
 // One launch solves every segment of every tile; u is bf16 through `map`
 // (boxes of 8 channels x 3 gates x 256 steps).  counter and seg_done must be
 // zero at launch (ntiles entries of seg_done).
-int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
-                     unsigned* seg_done, cudaStream_t stream) {
+// hmap: the states h [B][T][D], box 8 channels x 256 steps
+int launch_gru_queue(const CUtensorMap& map, const CUtensorMap& hmap, const FwdParams& f,
+                     unsigned* counter, unsigned* seg_done, cudaStream_t stream) {
   QParams p;
   p.a = f.a;
   p.bias = f.bias;
@@ -526,7 +550,7 @@ int launch_gru_queue(const CUtensorMap& map, const FwdParams& f, unsigned* count
   p.chan_k = f.chan_k;
   p.stats = f.stats;
   p.withhold_item = (f.flags & PARARNN_FLAG_INJECT_WITHHOLD) ? f.inject_chunk : -1;
-  return launch_queue(map, p, stream);
+  return launch_queue(map, hmap, p, stream);
 }
 
 }  // namespace pararnn
