@@ -32,7 +32,8 @@ int lstm_row_cta_steps();
 int lstm_row_box_steps();
 int lstm_row_channels();
 int launch_lstm_row(const CUtensorMap& map, const FwdParams& p, cudaStream_t stream);
-int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+int launch_lstm_queue(const CUtensorMap& map, const CUtensorMap& cmap, const CUtensorMap& hmap,
+                      const FwdParams& f, unsigned* counter,
                       unsigned* seg_done, cudaStream_t stream);
 int lstm_queue_resident();
 int lstm_queue_box_steps();
@@ -364,8 +365,11 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   } else if (queue_lstm) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, true, B, T, G, D, lstm_queue_box_steps(), lstm_row_channels());
+    CUtensorMap cmap, hmap;  // the states, stored by the same 128-step boxes
+    if (!rc) rc = make_s_map(&cmap, c, B, T, D, lstm_queue_box_steps(), lstm_row_channels());
+    if (!rc) rc = make_s_map(&hmap, h, B, T, D, lstm_queue_box_steps(), lstm_row_channels());
     if (rc) return rc;
-    e = launch_lstm_queue(rmap, p, &p.hdr->ticket, seg_done, stream);
+    e = launch_lstm_queue(rmap, cmap, hmap, p, &p.hdr->ticket, seg_done, stream);
   } else if (row_gru) {
     CUtensorMap rmap;
     rc = make_u_map(&rmap, u, bf16, B, T, G, D, gru_row_box_steps(), gru_row_channels());

@@ -76,7 +76,9 @@ constexpr int kLqS = kLqG * kLqRowB + 64;           // chunk slot: 1088 bytes
 constexpr int kLqU = kLqChunks * kLqS;              // 17408: the item's fp32 arguments
 constexpr int kLqBoxBytes = kLqSteps * kLqG * kLqC * 2;  // 8192: one box of 128 steps
 constexpr int kLqStage = kLqU;                      // bf16 staging after the arguments
-constexpr int kLqSmem = kLqStage + kLqBoxBytes;
+// the item's final (c, h), [128 steps][8 ch] each, for the bulk-tensor stores
+constexpr int kLqStates = kLqStage + kLqBoxBytes;
+constexpr int kLqSmem = kLqStates + 2 * kLqSteps * kLqC * 4;
 constexpr int kLqMinB = 4;                          // CTAs per SM
 static_assert(kLqS % 128 == 64, "a warp's four chunks in alternate 64-byte bank halves");
 static_assert(kLqW % 4 == 0, "the item's residual maximum is read as float4s");
@@ -279,7 +281,9 @@ __device__ __forceinline__ int lq_draw(unsigned* counter) {
 }
 
 __global__ void __launch_bounds__(kLqThreads, kLqMinB)
-    lstm_newton_queue(const __grid_constant__ CUtensorMap map, const LqParams p) {
+    lstm_newton_queue(const __grid_constant__ CUtensorMap map,
+                      const __grid_constant__ CUtensorMap cmap,
+                      const __grid_constant__ CUtensorMap hmap, const LqParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ LqShared sh;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -308,12 +312,18 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
   int dead = 0;
   for (int n = 0; item < p.nitems; ++n) {
     __syncthreads();
-    // publish the previous item: every thread's state stores precede the
-    // barrier above; the fence and release order them before the count (warp
-    // 1, while warp 0 draws the next ticket: both wait on memory)
-    if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
-      __threadfence();
-      st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
+    // publish the previous item: its states' bulk stores (issued by thread
+    // 32) complete, then the proxy fence, the fence and the release order
+    // them before the count.  Warp 0 draws the next ticket meanwhile: both
+    // wait on memory.  The completed stores have also read the states buffer,
+    // which this item fills again at its end.
+    if (tid == 32 && prev_item >= 0) {
+      bulk_wait_all();
+      if (prev_item != p.withhold_item) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
+      }
     }
     // the item after this one: drawn now, stored before the item's first
     // barrier (the atomic's latency overlaps the wait for the boxes)
@@ -537,23 +547,31 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     }
     if (pj >= 0 && pj < 10 * kLqC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
 
-    // ---- states straight from registers
+    // ---- states: from registers into the states buffer ([step][8 ch] for c
+    // and for h), then one bulk-tensor store each (steps past T are not
+    // written)
     bool bad = false;
-    if (dval) {
+    {
+      float* cs = reinterpret_cast<float*>(smem + kLqStates);
+      float* hs = cs + kLqSteps * kLqC;
       const int tq = q * kLqL;
-      const size_t o0 = ((size_t)b * p.T + t_base + tq) * p.D + d;
 #pragma unroll
       for (int i = 0; i < kLqH; ++i) {
-        if (tq + i < t_len) {
-          p.c[o0 + (size_t)i * p.D] = C[i].x;
-          p.h[o0 + (size_t)i * p.D] = H[i].x;
-          bad |= !isfinite(C[i].x) || !isfinite(H[i].x);
+        cs[(tq + i) * kLqC + c] = C[i].x;
+        hs[(tq + i) * kLqC + c] = H[i].x;
+        cs[(tq + kLqH + i) * kLqC + c] = C[i].y;
+        hs[(tq + kLqH + i) * kLqC + c] = H[i].y;
+        if (dval) {
+          bad |= tq + i < t_len && (!isfinite(C[i].x) || !isfinite(H[i].x));
+          bad |= tq + kLqH + i < t_len && (!isfinite(C[i].y) || !isfinite(H[i].y));
         }
-        if (tq + kLqH + i < t_len) {
-          p.c[o0 + (size_t)(kLqH + i) * p.D] = C[i].y;
-          p.h[o0 + (size_t)(kLqH + i) * p.D] = H[i].y;
-          bad |= !isfinite(C[i].y) || !isfinite(H[i].y);
-        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      if (tid == 32) {
+        tma_store_3d(&cmap, cs, d0, t_base, b);
+        tma_store_3d(&hmap, hs, d0, t_base, b);
+        bulk_commit();
       }
     }
     if (bad && status < PARARNN_STATUS_NONFINITE) status = PARARNN_STATUS_NONFINITE;
@@ -568,9 +586,13 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
     item = next;
   }
   __syncthreads();
-  if (tid == 32 && prev_item >= 0 && prev_item != p.withhold_item) {
-    __threadfence();
-    st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
+  if (tid == 32 && prev_item >= 0) {
+    bulk_wait_all();
+    if (prev_item != p.withhold_item) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __threadfence();
+      st_release(&p.seg_done[lq_tile(p, prev_item)], (unsigned)lq_seg(p, prev_item) + 1u);
+    }
   }
   // a box still in flight into the staging area: wait for it (bounded)
   if (dead && tid == 0) mbar_wait_bounded(&sh.bar, (unsigned)(dead - 1), p.timeout_ns);
@@ -606,7 +628,9 @@ int lstm_queue_resident() {
 // One launch solves every 128-step segment of every tile; u is bf16 through
 // `map` (boxes of 8 channels x 4 gates x 128 steps).  counter and seg_done
 // (ntiles entries) must be zero at launch.
-int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* counter,
+// cmap, hmap: the states c, h [B][T][D], box 8 channels x 128 steps
+int launch_lstm_queue(const CUtensorMap& map, const CUtensorMap& cmap, const CUtensorMap& hmap,
+                      const FwdParams& f, unsigned* counter,
                       unsigned* seg_done, cudaStream_t stream) {
   LqParams p;
   p.a = f.a;
@@ -640,8 +664,8 @@ int launch_lstm_queue(const CUtensorMap& map, const FwdParams& f, unsigned* coun
   const int per_sm = std::max(1, lq_per_sm());
   // persistent: every CTA resident at once (the queue's progress argument)
   const long long grid = std::min<long long>((long long)sms * per_sm, p.nitems);
-  lstm_newton_queue<<<(unsigned)std::max<long long>(grid, 1), kLqThreads, kLqSmem, stream>>>(map,
-                                                                                           p);
+  lstm_newton_queue<<<(unsigned)std::max<long long>(grid, 1), kLqThreads, kLqSmem, stream>>>(
+      map, cmap, hmap, p);
   return (int)cudaGetLastError();
 }
 
