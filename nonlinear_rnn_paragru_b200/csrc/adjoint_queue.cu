@@ -40,6 +40,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "adjoint_cell.cuh"
 #include "common.cuh"
@@ -327,40 +328,47 @@ __global__ void __launch_bounds__(kAqThreads, 1)
                  (unsigned long long)__float_as_uint(fmaf(inc.x, cchunk, inc.y)) |
                      ((unsigned long long)(cur.r + 1) << 32));
 
-    // ---- pass 2: the exact recurrence from the true carry, du and the sums
+    // ---- pass 2: the exact recurrence from the true carry, du and the sums;
+    // a chunk inside T with its channel below D (warp-uniform but for a
+    // partial last tile) takes the copy of the loop without per-step tests
     float2 CARRY = af2(fmaf(PM.y, cchunk, DM.y), cchunk);  // entering steps 3 and 7
     float2 SAZ = af2(0.f, 0.f), SAR = SAZ, SAC = SAZ, SBZ = SAZ, SBR = SAZ, SBC = SAZ;
     const int tq = cur.t0 + warp * kAqL;
     float* dub = p.du + (((size_t)cur.b * p.T + tq) * 3) * p.D + d;
+    auto pass2 = [&](auto full) {
+      constexpr bool kFull = decltype(full)::value;
 #pragma unroll
-    for (int i = kAqH - 1; i >= 0; --i) {
-      float2 HP = af2(hbase[i * kAqC], hbase[(i + kAqH) * kAqC]);
-      if (i == 0 && first) HP.x = h0v;
-      const float2 G = af2(gbase[i * kAqC], gbase[(i + kAqH) * kAqC]);
-      const float2 LAM = aadd(G, CARRY);
-      const float2 DZ = amul(KZ[i], LAM), DR = amul(KR[i], LAM), DC = amul(KC[i], LAM);
-      SAZ = afma(DZ, HP, SAZ);
-      SAR = afma(DR, HP, SAR);
-      SAC = afma(DC, KH[i], SAC);
-      SBZ = aadd(SBZ, DZ);
-      SBR = aadd(SBR, DR);
-      SBC = aadd(SBC, DC);
-      CARRY = amul(KA[i], LAM);
-      if (dval) {
-        if (tq + i < p.T) {
-          float* o = dub + (size_t)i * 3 * p.D;
-          o[0] = DZ.x;
-          o[p.D] = DR.x;
-          o[2 * (size_t)p.D] = DC.x;
+      for (int i = kAqH - 1; i >= 0; --i) {
+        float2 HP = af2(hbase[i * kAqC], hbase[(i + kAqH) * kAqC]);
+        if (i == 0 && first) HP.x = h0v;
+        const float2 G = af2(gbase[i * kAqC], gbase[(i + kAqH) * kAqC]);
+        const float2 LAM = aadd(G, CARRY);
+        const float2 DZ = amul(KZ[i], LAM), DR = amul(KR[i], LAM), DC = amul(KC[i], LAM);
+        SAZ = afma(DZ, HP, SAZ);
+        SAR = afma(DR, HP, SAR);
+        SAC = afma(DC, KH[i], SAC);
+        SBZ = aadd(SBZ, DZ);
+        SBR = aadd(SBR, DR);
+        SBC = aadd(SBC, DC);
+        CARRY = amul(KA[i], LAM);
+        float* ox = dub + (size_t)i * 3 * p.D;
+        float* oy = dub + (size_t)(kAqH + i) * 3 * p.D;
+        if (kFull || (dval && tq + i < p.T)) {
+          ox[0] = DZ.x;
+          ox[p.D] = DR.x;
+          ox[2 * (size_t)p.D] = DC.x;
         }
-        if (tq + kAqH + i < p.T) {
-          float* o = dub + (size_t)(kAqH + i) * 3 * p.D;
-          o[0] = DZ.y;
-          o[p.D] = DR.y;
-          o[2 * (size_t)p.D] = DC.y;
+        if (kFull || (dval && tq + kAqH + i < p.T)) {
+          oy[0] = DZ.y;
+          oy[p.D] = DR.y;
+          oy[2 * (size_t)p.D] = DC.y;
         }
       }
-    }
+    };
+    if (dval && tq + kAqL <= p.T)
+      pass2(std::true_type{});
+    else
+      pass2(std::false_type{});
     if (first && dval && p.dh0) p.dh0[(size_t)cur.b * p.D + d] = CARRY.x;
     // the warp's partial sums per channel.  Every du of the chunk enters one
     // of the dbias sums, so a non-finite du (or an overflowing sum) leaves one
