@@ -42,6 +42,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "adjoint_cell.cuh"
 #include "common.cuh"
@@ -394,44 +395,51 @@ __global__ void __launch_bounds__(kAlqThreads, 1)
     }
     const float2 cx = My.apply(cchunk);  // entering step 3 from step 4
 
-    // ---- pass 2: the exact recurrence, du and the partial sums
+    // ---- pass 2: the exact recurrence, du and the partial sums; a chunk
+    // inside T with its channel below D (warp-uniform but for a partial last
+    // tile) takes the copy of the loop without per-step tests
     float2 LC = af2(cx.x, cchunk.x), LH = af2(cx.y, cchunk.y);
     float2 SA[4], SB[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) SA[g] = SB[g] = af2(0.f, 0.f);
     const int tq = cur.t0 + warp * kAlqL;
     float* dub = p.du + (((size_t)cur.b * p.T + tq) * 4) * p.D + d;
+    auto pass2 = [&](auto full) {
+      constexpr bool kFull = decltype(full)::value;
 #pragma unroll
-    for (int i = kAlqH - 1; i >= 0; --i) {
-      float2 UI, UF, UG, UO, CP, HP, G, F, X, KK, A11, GCI, GCF, GCG, DOT;
-      alq_args(ubase + i * (kAlqUStep / 2), ubase + (i + kAlqH) * (kAlqUStep / 2), BS, UI, UF,
-               UG, UO);
-      state(i, CP, HP, G);
-      al_cell(k, CP, HP, UI, UF, UG, UO, F, X, KK, A11, GCI, GCF, GCG, DOT);
-      const float2 LHE = aadd(LH, G);                      // lambda_h
-      const float2 LCH = afma(KK, LHE, LC);                // lambda_c + kk lambda_h
-      const float2 DU[4] = {amul(GCI, LCH), amul(GCF, LCH), amul(GCG, LCH), amul(DOT, LHE)};
+      for (int i = kAlqH - 1; i >= 0; --i) {
+        float2 UI, UF, UG, UO, CP, HP, G, F, X, KK, A11, GCI, GCF, GCG, DOT;
+        alq_args(ubase + i * (kAlqUStep / 2), ubase + (i + kAlqH) * (kAlqUStep / 2), BS, UI, UF,
+                 UG, UO);
+        state(i, CP, HP, G);
+        al_cell(k, CP, HP, UI, UF, UG, UO, F, X, KK, A11, GCI, GCF, GCG, DOT);
+        const float2 LHE = aadd(LH, G);                      // lambda_h
+        const float2 LCH = afma(KK, LHE, LC);                // lambda_c + kk lambda_h
+        const float2 DU[4] = {amul(GCI, LCH), amul(GCF, LCH), amul(GCG, LCH), amul(DOT, LHE)};
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        SA[g] = afma(DU[g], HP, SA[g]);
-        SB[g] = aadd(SB[g], DU[g]);
-      }
-      // carry = A^T lambda = (f (lambda_c + kk lambda_h), X (...) + a_o du_o)
-      LC = amul(F, LCH);
-      LH = afma(X, LCH, amul(k.AO, DU[3]));
-      if (dval) {
-        if (tq + i < p.T) {
-          float* o = dub + (size_t)i * 4 * p.D;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) o[(size_t)g * p.D] = DU[g].x;
+        for (int g = 0; g < 4; ++g) {
+          SA[g] = afma(DU[g], HP, SA[g]);
+          SB[g] = aadd(SB[g], DU[g]);
         }
-        if (tq + kAlqH + i < p.T) {
-          float* o = dub + (size_t)(kAlqH + i) * 4 * p.D;
+        // carry = A^T lambda = (f (lambda_c + kk lambda_h), X (...) + a_o du_o)
+        LC = amul(F, LCH);
+        LH = afma(X, LCH, amul(k.AO, DU[3]));
+        float* ox = dub + (size_t)i * 4 * p.D;
+        float* oy = dub + (size_t)(kAlqH + i) * 4 * p.D;
+        if (kFull || (dval && tq + i < p.T)) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) o[(size_t)g * p.D] = DU[g].y;
+          for (int g = 0; g < 4; ++g) ox[(size_t)g * p.D] = DU[g].x;
+        }
+        if (kFull || (dval && tq + kAlqH + i < p.T)) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) oy[(size_t)g * p.D] = DU[g].y;
         }
       }
-    }
+    };
+    if (dval && tq + kAlqL <= p.T)
+      pass2(std::true_type{});
+    else
+      pass2(std::false_type{});
     if (first && dval) {
       if (p.dc0) p.dc0[(size_t)cur.b * p.D + d] = LC.x;
       if (p.dh0) p.dh0[(size_t)cur.b * p.D + d] = LH.x;
