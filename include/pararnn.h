@@ -187,8 +187,12 @@ int pararnn_workspace_init(void* workspace, size_t ws_bytes,
  *      never got there within the cap.
  * Newton starts from h = 0 at every t, applies the page's update until the
  * residual of an iterate is below tol everywhere upstream (and then applies
- * that last update), or until max_iters updates have been applied.  Channels
- * are independent; each 8-channel tile stops on its own.  With bf16 u and at
+ * that last update), or until max_iters updates have been applied.  The
+ * segment-queue solves check an iterate reached by an exact step from a
+ * residual at most sqrt(tol) with a residual-only evaluation, and return that
+ * iterate itself when it is below tol (ParaLSTM: sqrt(tol / 2) and tol / 2, a
+ * margin for the fp32 rounding of a cell state that is not bounded).  Channels are independent; each
+ * 8-channel tile stops on its own.  With bf16 u and at
  * least one 8-channel tile per resident CTA of the segment-queue solve
  * (B * D / 8 >= 4 * SMs), one launch solves every 512-step segment of every
  * tile, each segment from the state the one before it converged to (stats

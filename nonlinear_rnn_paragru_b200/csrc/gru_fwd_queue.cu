@@ -12,9 +12,12 @@
 // a thread keeps its 32-step chunk's iterate and running Jacobian product in
 // registers, and each iteration runs the cell pass of gru_row_pass.cuh, a
 // shuffle scan over the warp's four chunks, one CTA barrier and a scan over
-// the warps from shared memory, and the fix-up.  The item stops after the
-// update of the first iteration whose residual over the item is below tol
-// (or after a residual-only evaluation at the cap).
+// the warps from shared memory, and the fix-up.  The item stops at the first
+// exact evaluation whose residual over the item is below tol: after its
+// update when the evaluation formed the step, or on the iterate itself when
+// it was a residual-only check (the evaluation after an exact step from a
+// residual at most sqrt(tol)).  At the cap it ends with a residual-only
+// evaluation.
 //
 // Queue.  Items are numbered segment-major (item = s * ntiles + tile) and
 // CTAs draw them from a counter one item ahead, so a CTA's items increase.
@@ -39,6 +42,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <type_traits>
 
 #include "common.cuh"
@@ -63,7 +67,8 @@ struct QParams {
   FastDiv dv_tiles, dv_ndtc;  // division by ntiles and by nDTc
   int max_iters;
   float tol;
-  float apx_tau;        // inexact evaluations while the item's residual is above this (0: none)
+  float apx_tau;
+  float spec_tau;       // a residual-only check follows an exact step from at most this        // inexact evaluations while the item's residual is above this (0: none)
   uint64_t timeout_ns;
   unsigned* counter;    // item tickets (zero at launch)
   unsigned* seg_done;   // [ntiles] segments of each tile stored (zero at launch)
@@ -303,21 +308,23 @@ __global__ void __launch_bounds__(NW * 32, MINB)
       P[i] = f2(1.f, 1.f);
     }
     float hb = first ? h0v : 0.f;  // state before this chunk
-    int last_bad = -1, updates = 0, k = 0;
+    // last_bad: updates applied before the last evaluation that left the
+    // channel at or above tol (histogram); nupd: updates applied so far
+    int last_bad = -1, updates = 0, k = 0, nupd = 0;
     float final_m = 0.f;
     bool apx = p.apx_tau > 0.f;  // CTA-uniform: set from the item's residual maximum
     // one Newton iteration of the item (kMode 0: exact evaluation and update,
-    // 1: inexact evaluation and update, 2: exact residual only, at the cap);
-    // true when the item is done
+    // 1: inexact evaluation and update, 2: exact residual only, at the cap or
+    // as a check that certifies the iterate); true when the item is done
     auto iterate = [&](auto mode) -> bool {
       constexpr int kMode = decltype(mode)::value;
-      constexpr bool cap = kMode == 2, apx_eval = kMode == 1;
+      constexpr bool resid_only = kMode == 2, apx_eval = kMode == 1;
       const int par = phase & 1;
       ++phase;
       const float last_pre = H[kH - 1].y;
       float2 DL, PA;
       float m;
-      if constexpr (cap)
+      if constexpr (resid_only)
         m = row_pass<kH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else if constexpr (apx_eval)
         m = row_pass_apx<kH>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
       unsigned cmu = __float_as_uint(m);
       cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 8));
       cmu = max(cmu, __shfl_xor_sync(kFull, cmu, 16));
-      if (kk == kRowK - 1) {
+      if (!resid_only && kk == kRowK - 1) {
         sh.wagg[par][warp][c] = make_float2(IP, Id);
         sh.wlast[par][warp][c] = last_pre;
       }
@@ -357,7 +364,7 @@ __global__ void __launch_bounds__(NW * 32, MINB)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (apx_eval || !(chm < p.tol)) last_bad = k;
+        if (apx_eval || !(chm < p.tol)) last_bad = nupd;
       }
       // the delta entering this warp: the maps of the warps before it applied
       // to the zero delta entering the item; and the item's residual maximum
@@ -380,10 +387,14 @@ __global__ void __launch_bounds__(NW * 32, MINB)
       // residual is at most apx_tau hands over to exact evaluations
       const bool own_ok = !apx_eval && tmax < p.tol;
       if (apx_eval && tmax <= p.apx_tau) apx = false;
-      if constexpr (cap) {
-        updates = k;
-        if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        return true;
+      if constexpr (resid_only) {
+        updates = nupd;
+        const bool cap = k >= p.max_iters;
+        if (cap && !own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
+        // a check certifies below tol, as an exact evaluation that forms the
+        // step does: a ParaGRU state stays inside (-1, 1), where the fp32
+        // rounding of the states and of this evaluation is about 1e-7
+        return cap || own_ok;
       }
       const float din = first ? 0.f : fmaf(xP, cd, xd);  // delta entering this chunk
       float prev_last = __shfl_up_sync(kFull, last_pre, kRowC);
@@ -392,18 +403,30 @@ __global__ void __launch_bounds__(NW * 32, MINB)
       const float2 DIN = f2(din, fmaf(PA.x, din, DL.x));
 #pragma unroll
       for (int i = 0; i < kH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
-      updates = k + 1;
+      updates = ++nupd;
       return own_ok;
     };
     // inexact iterations while the residual is large, then exact ones to
-    // convergence or the cap (k: the evaluation's index)
+    // convergence or the cap (k: the evaluation's index).  An exact step
+    // from a residual at most spec_tau (sqrt(tol)) lands below tol with
+    // quadratic convergence, so the evaluation after it is a residual-only
+    // check: if it certifies, the item ends on that iterate without forming
+    // the step; if not, the next evaluation forms the step at the same
+    // iterate.
     for (; apx && k < p.max_iters; ++k) iterate(std::integral_constant<int, 1>{});
+    bool spec = false;
     for (;; ++k) {
       if (k >= p.max_iters) {
         iterate(std::integral_constant<int, 2>{});
         break;
       }
+      if (spec) {
+        spec = false;
+        if (iterate(std::integral_constant<int, 2>{})) break;
+        continue;
+      }
       if (iterate(std::integral_constant<int, 0>{})) break;
+      spec = final_m <= p.spec_tau;
     }
     // every thread is past its last pass of this item (the barrier of the last
     // exchange): the staging area takes the next item
@@ -544,6 +567,7 @@ int launch_gru_queue(const CUtensorMap& map, const CUtensorMap& hmap, const FwdP
   p.max_iters = f.max_iters;
   p.tol = f.tol;
   p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kApxTau;
+  p.spec_tau = f.tol > 0.f ? std::sqrt(f.tol) : -1.f;
   p.timeout_ns = f.timeout_ns;
   p.counter = counter;
   p.seg_done = seg_done;

@@ -13,9 +13,11 @@
 // as its scalar form).  Each iteration: the cell pass, a shuffle scan of the
 // chunk maps (2x2 matrix, 2-vector) over the warp's four chunks, one CTA
 // barrier and a composition over the warps from shared memory, and the
-// fix-up.  The item stops after the update of the first exact iteration
-// whose residual over the item is below tol (or after a residual-only
-// evaluation at the cap).
+// fix-up.  The item stops at the first exact evaluation whose residual over
+// the item is below tol: after its update when the evaluation formed the
+// step, or on the iterate itself when it was a residual-only check below
+// tol / 2 (the evaluation after an exact step from a residual at most
+// sqrt(tol / 2)).  At the cap it ends with a residual-only evaluation.
 //
 // Inexact early evaluations.  While the item's max |r| is above 0.1 the cell
 // is evaluated with the one-instruction tanh (sigma(x) = 1/2 + 1/2 tanh(x/2);
@@ -52,6 +54,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <type_traits>
 
 #include "common.cuh"
@@ -100,6 +103,8 @@ struct LqParams {
   int max_iters;
   float tol;
   float apx_tau;        // inexact evaluations while the item's residual is above this (0: none)
+  float spec_tau;       // a residual-only check follows an exact step from at most this
+  float chk_tol;        // and certifies the iterate below this (tol / 2)
   uint64_t timeout_ns;
   unsigned* counter;    // item tickets (zero at launch)
   unsigned* seg_done;   // [ntiles] segments of each tile stored (zero at launch)
@@ -206,7 +211,7 @@ __device__ __forceinline__ float lq_pass(const unsigned char* __restrict__ base,
     }
     const float2 HN = qmul(O, TC);                          // h' = o tanh(c')
     const float2 RC = qfma(CN, M1, CT), RH = qfma(HN, M1, HT);
-    m = fmax3_nan(m, fmax_nan(fabsf(RC.x), fabsf(RC.y)), fmax_nan(fabsf(RH.x), fabsf(RH.y)));
+    m = fmax3_nan(fmax3_nan(m, fabsf(RC.x), fabsf(RC.y)), fabsf(RH.x), fabsf(RH.y));
     if constexpr (kMode != 2) {
       DI = qmul(I, qfma(I, M1, ONE));
       DF = qmul(F, qfma(F, M1, ONE));
@@ -442,14 +447,16 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       P00[i] = P01[i] = P10[i] = P11[i] = qf2(0.f, 0.f);
     }
     float cb = first ? c0v : 0.f, hb = first ? h0v : 0.f;  // state before this chunk
-    int last_bad = -1, updates = 0, kit = 0;
+    // last_bad: updates applied before the last evaluation that left the
+    // channel at or above tol (histogram); nupd: updates applied so far
+    int last_bad = -1, updates = 0, kit = 0, nupd = 0;
     float final_m = 0.f;
     bool apx = p.apx_tau > 0.f;  // CTA-uniform: set from the item's residual maximum
-    // one Newton iteration of the item (kMode as in lq_pass); true when the
-    // item is done
+    // one Newton iteration of the item (kMode as in lq_pass; 2 at the cap or
+    // as a check that certifies the iterate); true when the item is done
     auto iterate = [&](auto mode) -> bool {
       constexpr int kMode = decltype(mode)::value;
-      constexpr bool cap = kMode == 2, apx_eval = kMode == 1;
+      constexpr bool resid_only = kMode == 2, apx_eval = kMode == 1;
       const int par = phase & 1;
       ++phase;
       const float lastc = C[kLqH - 1].y, lasth = H[kLqH - 1].y;
@@ -457,21 +464,23 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       float m = lq_pass<kMode>(base, so0, so1, cb, hb, C, H, P00, P01, P10, P11, k, Mx, My);
       if (!dval) m = 0.f;
       // the chunk's map: second half after the first
-      Aff2 inc = My.after(Mx);
-      // inclusive scan over the warp's four chunks of channel c (lanes c + 8k)
+      Aff2 inc = My.after(Mx), xm = Aff2::id();
+      if constexpr (!resid_only) {
+        // inclusive scan over the warp's four chunks of channel c (lanes c + 8k)
 #pragma unroll
-      for (int o = kLqC; o < 32; o <<= 1) {
-        const Aff2 prev = lq_shfl_up(inc, o);
-        if (lane >= o) inc = inc.after(prev);
+        for (int o = kLqC; o < 32; o <<= 1) {
+          const Aff2 prev = lq_shfl_up(inc, o);
+          if (lane >= o) inc = inc.after(prev);
+        }
+        // exclusive: the delta entering the warp -> the delta entering this chunk
+        xm = lq_shfl_up(inc, kLqC);
+        if (kk == 0) xm = Aff2::id();
       }
-      // exclusive: the delta entering the warp -> the delta entering this chunk
-      Aff2 xm = lq_shfl_up(inc, kLqC);
-      if (kk == 0) xm = Aff2::id();
       const unsigned wm = __reduce_max_sync(kLqFull, __float_as_uint(m));
       unsigned cmu = __float_as_uint(m);
       cmu = max(cmu, __shfl_xor_sync(kLqFull, cmu, 8));
       cmu = max(cmu, __shfl_xor_sync(kLqFull, cmu, 16));
-      if (kk == kLqK - 1) {
+      if (!resid_only && kk == kLqK - 1) {
         sh.wagg[par][warp][c][0] = make_float4(inc.m00, inc.m01, inc.m10, inc.m11);
         sh.wagg[par][warp][c][1] = make_float4(inc.d0, inc.d1, lastc, lasth);
       }
@@ -482,14 +491,14 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < kLqW; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (apx_eval || !(chm < p.tol)) last_bad = kit;
+        if (apx_eval || !(chm < p.tol)) last_bad = nupd;
       }
       // the delta entering this warp: the maps of the warps before it applied
       // to the zero delta entering the item; and the item's residual maximum
       float2 cin = qf2(0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < kLqW - 1; ++w) {
-        if (w < warp) {
+        if (!resid_only && w < warp) {
           const float4 m0 = sh.wagg[par][w][c][0], m1 = sh.wagg[par][w][c][1];
           cin = qf2(fmaf(m0.x, cin.x, fmaf(m0.y, cin.y, m1.x)),
                     fmaf(m0.z, cin.x, fmaf(m0.w, cin.y, m1.y)));
@@ -506,10 +515,14 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
       // residual is at most apx_tau hands over to exact evaluations
       const bool own_ok = !apx_eval && tmax < p.tol;
       if (apx_eval && tmax <= p.apx_tau) apx = false;
-      if constexpr (cap) {
-        updates = kit;
-        if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        return true;
+      if constexpr (resid_only) {
+        updates = nupd;
+        const bool cap = kit >= p.max_iters;
+        if (cap && !own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
+        // a check certifies below tol / 2: the margin covers the fp32
+        // rounding of the states and of this evaluation, so that the exact
+        // residual of the returned states stays below tol
+        return cap || tmax < p.chk_tol;
       }
       const float2 din = first ? qf2(0.f, 0.f) : xm.apply(cin);  // delta entering this chunk
       float2 prev_last = qf2(__shfl_up_sync(kLqFull, lastc, kLqC),
@@ -532,18 +545,30 @@ __global__ void __launch_bounds__(kLqThreads, kLqMinB)
         C[i] = qfma(P00[i], DINC, qfma(P01[i], DINH, C[i]));
         H[i] = qfma(P10[i], DINC, qfma(P11[i], DINH, H[i]));
       }
-      updates = kit + 1;
+      updates = ++nupd;
       return own_ok;
     };
     // inexact iterations while the residual is large, then exact ones to
-    // convergence or the cap (kit: the evaluation's index)
+    // convergence or the cap (kit: the evaluation's index).  An exact step
+    // from a residual at most spec_tau (sqrt(tol / 2)) lands below tol / 2
+    // with quadratic convergence, so the evaluation after it is a
+    // residual-only check: if it certifies, the item ends on that iterate
+    // without forming the step; if not, the next evaluation forms the step at
+    // the same iterate.
     for (; apx && kit < p.max_iters; ++kit) iterate(std::integral_constant<int, 1>{});
+    bool spec = false;
     for (;; ++kit) {
       if (kit >= p.max_iters) {
         iterate(std::integral_constant<int, 2>{});
         break;
       }
+      if (spec) {
+        spec = false;
+        if (iterate(std::integral_constant<int, 2>{})) break;
+        continue;
+      }
       if (iterate(std::integral_constant<int, 0>{})) break;
+      spec = final_m <= p.spec_tau;
     }
     if (pj >= 0 && pj < 10 * kLqC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;
 
@@ -652,6 +677,8 @@ int launch_lstm_queue(const CUtensorMap& map, const CUtensorMap& cmap, const CUt
   p.max_iters = f.max_iters;
   p.tol = f.tol;
   p.apx_tau = (f.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kApxTau;
+  p.chk_tol = 0.5f * f.tol;
+  p.spec_tau = f.tol > 0.f ? std::sqrt(p.chk_tol) : -1.f;
   p.timeout_ns = f.timeout_ns;
   p.counter = counter;
   p.seg_done = seg_done;

@@ -198,7 +198,7 @@ __device__ __forceinline__ float lr_pass(const unsigned char* __restrict__ base,
     const float2 TC = lfma(M2, TC1, ONE);                 // tanh(c')
     const float2 HN = lmul(O, TC);                        // h' = o tanh(c')
     const float2 RC = lfma(CN, M1, CT), RH = lfma(HN, M1, HT);
-    m = fmax_nan(m, fmax_nan(fmax_nan(fabsf(RC.x), fabsf(RC.y)), fmax_nan(fabsf(RH.x), fabsf(RH.y))));
+    m = fmax3_nan(fmax3_nan(m, fabsf(RC.x), fabsf(RC.y)), fabsf(RH.x), fabsf(RH.y));
     if (kFull) {
       const float2 DI = lmul(I, lfma(I, M1, ONE));        // i(1-i)
       const float2 DF = lmul(F, lfma(F, M1, ONE));
