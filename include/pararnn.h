@@ -188,11 +188,10 @@ int pararnn_workspace_init(void* workspace, size_t ws_bytes,
  * Newton starts from h = 0 at every t, applies the page's update until the
  * residual of an iterate is below tol everywhere upstream (and then applies
  * that last update), or until max_iters updates have been applied.  The
- * segment-queue solves check an iterate reached by an exact step from a
- * residual at most sqrt(tol) with a residual-only evaluation, and return that
- * iterate itself when it is below tol (ParaLSTM: sqrt(tol / 2) and tol / 2, a
- * margin for the fp32 rounding of a cell state that is not bounded).  Channels are independent; each
- * 8-channel tile stops on its own.  With bf16 u and at
+ * segment-queue and whole-sequence solves evaluate only the residual of an
+ * iterate reached by an exact step from a residual at most sqrt(tol), and
+ * return that iterate itself when it is below tol.  Channels are
+ * independent; each 8-channel tile stops on its own.  With bf16 u and at
  * least one 8-channel tile per resident CTA of the segment-queue solve
  * (B * D / 8 >= 4 * SMs), one launch solves every 512-step segment of every
  * tile, each segment from the state the one before it converged to (stats
@@ -217,7 +216,10 @@ int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
  * max over both components.  With bf16 u and at least one 8-channel tile per
  * resident CTA of the segment-queue solve (B * D / 8 >= 4 * SMs), one launch
  * solves every 128-step segment of every tile (any T), each segment from the
- * (c, h) the one before it converged to.  Otherwise, with bf16 u and
+ * (c, h) the one before it converged to; there an iterate reached by an
+ * exact step from a residual at most sqrt(tol / 2) is checked by its residual
+ * alone and returned when that is below tol / 2 (a margin for the fp32
+ * rounding of a cell state, which is not bounded).  Otherwise, with bf16 u and
  * T <= 4096, a tile's sequence is
  * held by a cluster of k CTAs of 512 steps each; when a smaller cluster of
  * k' CTAs already puts one CTA on every SM (k' * B * D / 8 >= SMs), the

@@ -29,9 +29,12 @@
 // receiver's mbarrier, so a CTA waits only for the bytes it needs and no
 // cluster-wide barrier is taken per iteration.  The fix-up adds P_t ds_in.
 // Mailboxes and per-warp data are double-buffered by the parity of a phase
-// counter that runs on across tiles.  The cluster stops after the update of
-// the first iteration whose residual over the tile is below tol, or after a
-// residual-only evaluation at the cap; the state before each chunk is re-anchored every iteration to its
+// counter that runs on across tiles.  The cluster stops at the first exact
+// evaluation whose residual over the tile is below tol: after its update
+// when the evaluation formed the step, or on the iterate itself when it was
+// a residual-only check (the evaluation after an exact step from a residual
+// at most sqrt(tol)); at the cap it ends with a residual-only evaluation.
+// The state before each chunk is re-anchored every iteration to its
 // predecessor's pre-update last state plus the incoming delta.
 //
 // Data: bf16 u arrives by four TMA boxes of 256 steps into the top of the
@@ -332,22 +335,25 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       P[i] = f2(1.f, 1.f);
     }
     float hb = first ? h0v : 0.f;  // state before this chunk
-    int last_bad = -1, updates = 0, k = 0;
+    // last_bad: updates applied before the last evaluation that left the
+    // channel at or above tol (histogram); nupd: updates applied so far
+    int last_bad = -1, updates = 0, k = 0, nupd = 0;
     float final_m = 0.f;
     bool apx = p.apx_tau > 0.f;  // cluster-uniform: set from the tile's residual maximum
     // one Newton iteration of the tile (kMode 0: exact evaluation and update,
-    // 1: inexact evaluation and update, 2: exact residual only, at the cap);
-    // true when the tile is done
+    // 1: inexact evaluation and update, 2: exact residual only, at the cap or
+    // as a check that certifies the iterate); true when the tile is done
     auto iterate = [&](auto mode) -> bool {
       constexpr int kMode = decltype(mode)::value;
-      constexpr bool cap = kMode == 2, apx_eval = kMode == 1;
+      constexpr bool resid_only = kMode == 2, apx_eval = kMode == 1;
+      const bool cap = resid_only && k >= p.max_iters;
       const int par = phase & 1;
       const unsigned mpar = (phase >> 1) & 1;  // phase parity of mbar[par]
       ++phase;
       const float last_pre = H[kRowH - 1].y;
       float2 DL, PA;
       float m;
-      if constexpr (cap)
+      if constexpr (resid_only)
         m = row_pass<kRowH, false>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
       else if constexpr (apx_eval)
         m = row_pass_apx<kRowH>(base, c * 8, hb, H, P, AZ2, AR2, AC2, AZ, DL, PA);
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < kRowWarps; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (apx_eval || !(chm < p.tol)) last_bad = k;
+        if (apx_eval || !(chm < p.tol)) last_bad = nupd;
       }
       // maps of the warps before this one: CTA incoming delta -> delta
       // entering this warp; and the CTA's residual maximum
@@ -456,10 +462,10 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       // residual is at most apx_tau hands over to exact evaluations
       const bool own_ok = !apx_eval && tmax < p.tol;
       if (apx_eval && tmax <= p.apx_tau) apx = false;
-      if constexpr (cap) {
-        updates = k;
-        if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        return true;
+      if constexpr (resid_only) {
+        updates = nupd;
+        if (cap && !own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
+        return cap || own_ok;
       }
       const float cin = fmaf(cP, din_cta, cd);  // delta entering this warp
       const float din = first ? 0.f : fmaf(xP, cin, xd);
@@ -470,18 +476,30 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       const float2 DIN = f2(din, fmaf(PA.x, din, DL.x));
 #pragma unroll
       for (int i = 0; i < kRowH; ++i) H[i] = ffma2(P[i], DIN, H[i]);
-      updates = k + 1;
+      updates = ++nupd;
       return own_ok;
     };
     // inexact iterations while the residual is large, then exact ones to
-    // convergence or the cap (k: the evaluation's index)
+    // convergence or the cap (k: the evaluation's index).  An exact step
+    // from a residual at most spec_tau (sqrt(tol)) lands below tol with
+    // quadratic convergence, so the evaluation after it is a residual-only
+    // check: if it certifies, the tile ends on that iterate without forming
+    // the step; if not, the next evaluation forms the step at the same
+    // iterate.
     for (; apx && k < p.max_iters; ++k) iterate(std::integral_constant<int, 1>{});
+    bool spec = false;
     for (;; ++k) {
       if (k >= p.max_iters) {
         iterate(std::integral_constant<int, 2>{});
         break;
       }
+      if (spec) {
+        spec = false;
+        if (iterate(std::integral_constant<int, 2>{})) break;
+        continue;
+      }
       if (iterate(std::integral_constant<int, 0>{})) break;
+      spec = final_m <= p.spec_tau;
     }
     // every thread of the CTA is past its last pass of this tile (the
     // barrier of the last exchange): the staging area takes the next tile
