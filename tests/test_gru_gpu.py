@@ -111,6 +111,35 @@ def test_capped_iterates_match_oracle_newton(cuda_ok, n):
     assert st["max_residual"] == pytest.approx(r["trace"][n], rel=1e-2)
 
 
+def _tile_copies(x, n):
+    # every 8-channel tile holds the same 8 channels (D is the last axis of
+    # every input), so each tile stops as the whole problem does
+    return {k: v.repeat(*([1] * (v.dim() - 1)), n) for k, v in x.items()}
+
+
+@pytest.mark.parametrize("D", [8, 4736])
+def test_certified_iterate_is_the_oracle_newton_result(cuda_ok, D):
+    # the solve ends on the first iterate whose residual is below tol, the
+    # oracle's rule.  After an exact step from a residual at most sqrt(tol)
+    # the next evaluation is a residual-only check, and the solve returns the
+    # oracle's iterate itself (n updates); otherwise the certifying
+    # evaluation also forms its step (n + 1).  D = 8 is one tile on the
+    # whole-sequence kernel, D = 4736 is 592 copies of it on the queue (one
+    # 512-step segment).  Exact steps throughout.
+    tol = 1e-6
+    x = make_inputs(WORKLOADS[2].scaled(B=1, T=512, D=8))
+    r = oracle.gru_newton(x["u"], x["a"], x["bias"], x["h0"], tol=tol, max_iters=64)
+    n, tr = r["iters"], r["trace"]
+    # the oracle's residuals sit far from the thresholds the fp32 kernels test
+    assert n >= 2 and tr[n] < 0.5 * tol and (tr[: n - 1] > 2 * np.sqrt(tol)).all()
+    assert not 0.5 * np.sqrt(tol) < tr[n - 1] < 2 * np.sqrt(tol)
+    expect = n if tr[n - 1] <= np.sqrt(tol) else n + 1
+    h, st, _ = _solve(_tile_copies(x, D // 8), tol=tol, flags=pr.PARARNN_FLAG_EXACT_STEPS)
+    assert st["status"] == "converged" and st["max_residual"] < tol, st
+    assert st["iters"] == expect and st["evals"] == n + 1, (st, n, expect)
+    assert np.abs(h - np.tile(r["h"], (1, 1, D // 8))).max() < TOL_STATE
+
+
 def test_withheld_record_times_out_without_hanging(cuda_ok):
     # host-injected fault: cluster chunk 0 of the first tile never publishes
     # (T = 5000 needs two 16-CTA cluster chunks), so its successor's bounded
