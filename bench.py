@@ -23,7 +23,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import torch
@@ -206,8 +205,38 @@ def rank_seed(rank):
 
 
 # ---------------------------------------------------------------- clocks --
+_SAMPLER_CHILD = r"""
+import select, sys, time
+import pynvml
+pynvml.nvmlInit()
+bus = sys.argv[1]
+h = (pynvml.nvmlDeviceGetHandleByPciBusId(bus) if bus
+     else pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[2])))
+for _ in range(5):  # the first queries are slow: take them before the timed region
+    pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+print("ready", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+period = float(sys.argv[3])
+rows = []
+# sample until the parent closes stdin, then write every sample at once
+while not select.select([sys.stdin], [], [], 0)[0]:
+    t = time.monotonic()
+    rows.append("%.6f %d %d" % (t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
+    time.sleep(period)
+sys.stdout.write("\n".join(rows) + "\n")
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """Samples SM clock and throttle reasons through NVML while running.
+
+    The sampling loop runs in a child process (its own interpreter, so the
+    timed loop's Python thread cannot starve it), stamping each sample with
+    the system's monotonic clock; the samples kept are those inside the
+    host-time bracket of the `with` block, which encloses the synchronised
+    timed region.  The device is found by its PCI bus id (NVML does not
+    follow CUDA_VISIBLE_DEVICES)."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
@@ -216,45 +245,57 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index, period=0.001):
-        # a 1 ms period: a timed region of 20 steps of under 1 ms still
-        # carries several samples (one NVML query takes well under 1 ms)
-        self.index, self.period = index, period
+    def __init__(self, index, period=0.0002):
+        import subprocess
         self.mhz, self.reasons = [], set()
         self.max_mhz = None
-        self._stop = threading.Event()
-        self._th = None
+        self.proc = None
+        self.t0 = self.t1 = None
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            pr_ = torch.cuda.get_device_properties(index)
+            bus = "%08x:%02x:%02x.0" % (pr_.pci_domain_id, pr_.pci_bus_id, pr_.pci_device_id)
+        except Exception:
+            bus = ""
+        try:
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", _SAMPLER_CHILD, bus, str(index), str(period)],
+                stdin=subprocess.PIPE, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            line = self.proc.stdout.readline().split()
+            if len(line) != 2 or line[0] != "ready":
+                raise RuntimeError("clock sampler did not start")
+            self.max_mhz = int(line[1])
         except Exception:  # no NVML: clocks stay unreported
-            self.nv = None
+            self._stop_child()
 
-    def _run(self):
-        while not self._stop.is_set():
+    def _stop_child(self):
+        """Closes the child's stdin (its signal to stop) -> its samples."""
+        out = ""
+        if self.proc is not None:
             try:
-                self.mhz.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if r & bit and name != "gpu_idle":
-                        self.reasons.add(name)
+                out = self.proc.communicate(input="", timeout=30)[0] or ""
             except Exception:
-                pass
-            time.sleep(self.period)
+                self.proc.kill()
+                self.proc.communicate()
+            self.proc = None
+        return out
 
     def __enter__(self):
-        if self.nv is not None:
-            self._th = threading.Thread(target=self._run, daemon=True)
-            self._th.start()
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
-        self._stop.set()
-        if self._th is not None:
-            self._th.join()
+        self.t1 = time.monotonic()
+        for ln in self._stop_child().splitlines():
+            f = ln.split()
+            if len(f) != 3:
+                continue
+            t, mhz, r = float(f[0]), int(f[1]), int(f[2])
+            if self.t0 <= t <= self.t1:
+                self.mhz.append(mhz)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
 
     def summary(self):
         if not self.mhz:
