@@ -498,7 +498,9 @@ __global__ void __launch_bounds__(NW * 32, MINB)
 // (512-step segments), 4 CTAs per SM.  Measured on configuration 2 (B200,
 // CUDA events): 345 us, against 354 us for 16-step chunks at 5 CTAs per SM
 // (96 registers) and 366 us at 6 (80 registers, a few spills): more resident
-// warps did not pay for the doubled per-step scan work
+// warps did not pay for the doubled per-step scan work.  8 warps per CTA
+// (1024-step segments, 2 CTAs per SM) measured 6% slower: the per-item work
+// halves per step, but every iteration's barrier spans twice the warps.
 constexpr int kQW = 4, kQL = 32, kQMinB = 4;
 using QRun = QCfg<kQW, kQL>;
 
