@@ -216,16 +216,16 @@ int pararnn_gru_solve(const void* u, int u_dtype, const float* a,
  * max over both components.  With bf16 u and at least one 8-channel tile per
  * resident CTA of the segment-queue solve (B * D / 8 >= 4 * SMs), one launch
  * solves every 128-step segment of every tile (any T), each segment from the
- * (c, h) the one before it converged to; there an iterate reached by an
- * exact step from a residual at most sqrt(tol / 2) is checked by its residual
- * alone and returned when that is below tol / 2 (a margin for the fp32
- * rounding of a cell state, which is not bounded).  Otherwise, with bf16 u and
- * T <= 4096, a tile's sequence is
- * held by a cluster of k CTAs of 512 steps each; when a smaller cluster of
- * k' CTAs already puts one CTA on every SM (k' * B * D / 8 >= SMs), the
- * sequence is solved in segments of k' * 512 steps instead, each starting
- * from the (c, h) the one before it converged to; stats and iter_hist then
- * take the maximum over the segments. */
+ * (c, h) the one before it converged to.  Otherwise, with bf16 u and
+ * T <= 4096, a tile's sequence is held by a cluster of k CTAs of 512 steps
+ * each; when a smaller cluster of k' CTAs already puts one CTA on every SM
+ * (k' * B * D / 8 >= SMs), the sequence is solved in segments of k' * 512
+ * steps instead, each starting from the (c, h) the one before it converged
+ * to; stats and iter_hist then take the maximum over the segments.  The
+ * segment-queue and whole-sequence solves check an iterate reached by an
+ * exact step from a residual at most sqrt(tol / 2) by its residual alone and
+ * return it when that is below tol / 2 (a margin for the fp32 rounding of a
+ * cell state, which is not bounded). */
 int pararnn_lstm_solve(const void* u, int u_dtype, const float* a,
                        const float* bias, const float* c0, const float* h0,
                        float* c, float* h, int B, int T, int D,

@@ -299,7 +299,10 @@ int forward(int cell, const void* u, int u_dtype, const float* a, const float* b
   p.tol = tol;
   p.flags = opts ? opts->flags : 0u;
   p.apx_tau = (p.flags & PARARNN_FLAG_EXACT_STEPS) ? 0.f : kApxTau;
-  p.spec_tau = tol > 0.f ? std::sqrt(tol) : -1.f;
+  // the row kernels' certifying check: ParaLSTM certifies below tol / 2 (a
+  // margin for the fp32 rounding of a cell state that is not bounded)
+  p.chk_tol = cell == PARARNN_LSTM ? 0.5f * tol : tol;
+  p.spec_tau = tol > 0.f ? std::sqrt(p.chk_tol) : -1.f;
   p.inject_chunk = opts ? opts->inject_chunk : -1;
   p.timeout_ns = 1000ull * ((opts && opts->timeout_us) ? opts->timeout_us : kDefaultTimeoutUs);
   p.hdr = reinterpret_cast<WsHeader*>(ws);

@@ -241,7 +241,8 @@ struct FwdParams {
   int max_iters;
   float tol;
   float apx_tau;      // ParaGRU row kernel: inexact evaluations above this residual (0: none)
-  float spec_tau;     // ParaGRU row kernel: a residual-only check follows an exact step from at most this
+  float spec_tau;     // row kernels: a residual-only check follows an exact step from at most this
+  float chk_tol;      // and certifies the iterate below this
   unsigned flags;
   int inject_chunk;
   uint64_t timeout_ns;

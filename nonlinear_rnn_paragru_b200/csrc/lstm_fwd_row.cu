@@ -30,11 +30,14 @@
 // mailboxes (the CTA's map and last state to the CTAs after it, its residual
 // maximum to all), each completing on the receiver's mbarrier.  The fix-up
 // adds P_t ds_in.  Mailboxes and per-warp data are double-buffered by the
-// parity of a phase counter that runs on across tiles.  The cluster stops
-// after the update of the first iteration whose residual over the tile is
-// below tol, or after a residual-only evaluation at the cap; the state before
-// each chunk is re-anchored every iteration to its predecessor's pre-update
-// last state plus the incoming delta.
+// parity of a phase counter that runs on across tiles.  The cluster stops at
+// the first exact evaluation whose residual over the tile is below tol: after
+// its update when the evaluation formed the step, or on the iterate itself
+// when it was a residual-only check below tol / 2 (the evaluation after a
+// step from a residual at most sqrt(tol / 2)); at the cap it ends with a
+// residual-only evaluation.  The state before each chunk is re-anchored
+// every iteration to its predecessor's pre-update last state plus the
+// incoming delta.
 //
 // Data: the tile's u arrives bf16 by two TMA boxes of 256 steps into a
 // staging area (a, bias, c0 and h0 of the next tile's channels are read with
@@ -383,10 +386,16 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       P00[i] = P01[i] = P10[i] = P11[i] = lf2(0.f, 0.f);
     }
     float cb = first ? c0v : 0.f, hb = first ? h0v : 0.f;  // state before this chunk
-    int last_bad = -1, updates = 0, kit = 0;
+    // last_bad: updates applied before the last evaluation that left the
+    // channel at or above tol (histogram); nupd: updates applied so far.
+    // spec: the last step started from a residual at most spec_tau, so this
+    // evaluation is a residual-only check that may certify the iterate.
+    int last_bad = -1, updates = 0, kit = 0, nupd = 0;
     float final_m = 0.f;
+    bool spec = false;
     for (;; ++kit) {
       const bool cap = (kit >= p.max_iters);
+      const bool ronly = cap || spec;
       const int par = phase & 1;
       const unsigned mpar = (phase >> 1) & 1;  // phase parity of mbar[par]
       ++phase;
@@ -394,7 +403,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       float2 DC, DH;
       Aff2 Mx, My;
       float m;
-      if (cap)
+      if (ronly)
         m = lr_pass<false>(base, c * 8, cb, hb, C, H, P00, P01, P10, P11, k, DC, DH, Mx, My);
       else
         m = lr_pass<true>(base, c * 8, cb, hb, C, H, P00, P01, P10, P11, k, DC, DH, Mx, My);
@@ -428,7 +437,7 @@ __global__ void __launch_bounds__(kLrThreads, 1)
         float chm = 0.f;
 #pragma unroll
         for (int w = 0; w < kLrWarps; ++w) chm = fmax_nan(chm, sh.wcm[par][w][c]);
-        if (!(chm < p.tol)) last_bad = kit;
+        if (!(chm < p.tol)) last_bad = nupd;
       }
       // maps of the warps before this one: CTA incoming delta -> delta
       // entering this warp; and the CTA's residual maximum
@@ -483,10 +492,17 @@ __global__ void __launch_bounds__(kLrThreads, 1)
       }
       final_m = tmax;
       const bool own_ok = tmax < p.tol;
-      if (cap) {
-        updates = kit;
-        if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
-        break;
+      if (ronly) {
+        updates = nupd;
+        if (cap) {
+          if (!own_ok && status == 0) status = PARARNN_STATUS_NOT_CONVERGED;
+          break;
+        }
+        // the check: certified below chk_tol, else the next evaluation forms
+        // the step at the same iterate
+        spec = false;
+        if (tmax < p.chk_tol) break;
+        continue;
       }
       const float2 cin = cw.apply(din_cta);             // delta entering this warp
       const float2 din = first ? lf2(0.f, 0.f) : xm.apply(cin);
@@ -509,8 +525,9 @@ __global__ void __launch_bounds__(kLrThreads, 1)
         C[i] = lfma(P00[i], DINC, lfma(P01[i], DINH, C[i]));
         H[i] = lfma(P10[i], DINC, lfma(P11[i], DINH, H[i]));
       }
-      updates = kit + 1;
+      updates = ++nupd;
       if (own_ok) break;
+      spec = tmax <= p.spec_tau;
     }
 
     if (pj >= 0 && pj < 10 * kLrC) (&sh.par[pb ^ 1][0][0])[pj] = pnext;

@@ -38,11 +38,12 @@ def _check(x, **kw):
 @pytest.mark.parametrize("wl,D", [(3, 8), (3, 4736), (5, 4736)])
 def test_certified_iterate_is_the_oracle_newton_result(cuda_ok, wl, D):
     # the oracle returns the first iterate whose residual is below tol.  The
-    # segment queue (D = 4736: 592 copies of one 8-channel tile, one 128-step
-    # segment) checks the residual alone after an exact step from at most
+    # solve checks the residual alone after an exact step from at most
     # sqrt(tol / 2) and returns that iterate when it is below tol / 2 (n
-    # updates); the whole-sequence kernel (D = 8) forms the step of the
-    # certifying evaluation too (n + 1).  Exact steps throughout.
+    # updates); otherwise the certifying evaluation forms its step too
+    # (n + 1).  D = 8 is one tile on the whole-sequence kernel, D = 4736 is
+    # 592 copies of it on the segment queue (one 128-step segment).  Exact
+    # steps throughout.
     tol = 1e-6
     x = make_inputs(WORKLOADS[wl].scaled(B=1, T=128, D=8))
     r = oracle.lstm_newton(x["u"], x["a"], x["bias"], x["c0"], x["h0"], tol=tol,
@@ -52,8 +53,7 @@ def test_certified_iterate_is_the_oracle_newton_result(cuda_ok, wl, D):
     # the oracle's residuals sit far from the thresholds the fp32 kernels test
     assert n >= 2 and tr[n] < 0.25 * tol and (tr[: n - 1] > 2 * spec).all()
     assert not 0.5 * spec < tr[n - 1] < 2 * spec
-    queue = D > 8
-    expect = n if queue and tr[n - 1] <= spec else n + 1
+    expect = n if tr[n - 1] <= spec else n + 1
     xr = {k: v.repeat(*([1] * (v.dim() - 1)), D // 8) for k, v in x.items()}
     c, h, st, _ = _solve(xr, tol=tol, flags=pr.PARARNN_FLAG_EXACT_STEPS)
     assert st["status"] == "converged" and st["max_residual"] < tol, st
