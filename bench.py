@@ -91,7 +91,7 @@ def fwd_plan(w, sms=None):
         return "gru_newton_queue", 3.75, 512
     if w.cell == "lstm":
         if w.u_dtype == "bf16" and tiles8 >= QUEUE_CTAS_PER_SM * sms and not FORCE_ROW:
-            return "lstm_newton_queue", 6.5, 128
+            return "lstm_newton_queue", 10.0, 128
         if w.u_dtype == "bf16" and w.T <= 4096:
             cls, seg = 1, w.T
             while cls * 512 < w.T:

@@ -21,10 +21,12 @@
 //
 // Inexact early evaluations.  While the item's max |r| is above 0.1 the cell
 // is evaluated with the one-instruction tanh (sigma(x) = 1/2 + 1/2 tanh(x/2);
-// gates within about 2^-11 relative), then exactly: with ex2 and reciprocals,
-// one serving the six sigmoids i, f, o of a step pair, one its two tanh(g)
-// and one its two tanh(c'), every exponent argument clamped at 21 (a product
-// of six (1 + 2^x) stays below 2^127; the clamp moves a gate by under 5e-7).
+// gates within about 2^-11 relative), then exactly: an ex2 and a reciprocal
+// per gate and per tanh(c'), sigma(x) = 1 / (1 + 2^(-x log2 e)) and
+// tanh(y) = 1 - 2 / (1 + 2^(2y log2 e)).  Unclamped, a saturating argument
+// gives 2^x = inf and a reciprocal of 0, the gate's limit, and a NaN stays
+// NaN.  (Sharing one reciprocal between the six sigmoids of a step pair
+// needed a clamp per argument and a longer dependency chain: 1% slower.)
 // Only exact evaluations decide convergence.  PARARNN_FLAG_EXACT_STEPS makes
 // every evaluation exact.
 //
@@ -129,10 +131,9 @@ __device__ __forceinline__ float2 qf2(float x, float y) { return make_float2(x, 
 __device__ __forceinline__ float2 qfma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 qmul(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 qadd(float2 a, float2 b) { return __fadd2_rn(a, b); }
-__device__ __forceinline__ float2 qex2c(float2 a) {  // 2^min(a, 21), NaN kept
-  return qf2(ex2(fmin_nan(a.x, 21.f)), ex2(fmin_nan(a.y, 21.f)));
-}
 __device__ __forceinline__ float2 qtanh(float2 a) { return qf2(tanh_apx(a.x), tanh_apx(a.y)); }
+__device__ __forceinline__ float2 qex2(float2 a) { return qf2(ex2(a.x), ex2(a.y)); }
+__device__ __forceinline__ float2 qrcp(float2 a) { return qf2(rcp(a.x), rcp(a.y)); }
 
 struct LqPar {
   float2 ai2, af2, ag2, ao2;  // h coefficients of the stored arguments
@@ -183,26 +184,17 @@ __device__ __forceinline__ float lq_pass(const unsigned char* __restrict__ base,
         DT = qfma(qmul(TC, M1), TC, ONE);
       }
     } else {
-      const float2 EI = qex2c(qfma(k.ai2, HP, UI));
-      const float2 EF = qex2c(qfma(k.af2, HP, UF));
-      const float2 EO = qex2c(qfma(k.ao2, HP, UO));
-      const float2 EG = qex2c(qfma(k.ag2, HP, UG));
-      const float2 PI = qadd(ONE, EI), PF = qadd(ONE, EF), PO = qadd(ONE, EO);
-      const float2 PFO = qmul(PF, PO), PIO = qmul(PI, PO), PIF = qmul(PI, PF);
-      const float2 Q = qmul(PI, PFO);
-      const float iq = rcp(Q.x * Q.y);
-      const float2 IQ = qf2(Q.y * iq, Q.x * iq);            // 1/(pi pf po) per step
-      I = qmul(PFO, IQ);
-      F = qmul(PIO, IQ);
-      O = qmul(PIF, IQ);
-      const float2 PG = qadd(ONE, EG);
-      const float ig = rcp(PG.x * PG.y);
-      const float2 TG = qf2(PG.y * ig, PG.x * ig);          // 1/(1+e^{2y})
+      const float2 PI = qadd(ONE, qex2(qfma(k.ai2, HP, UI)));
+      const float2 PF = qadd(ONE, qex2(qfma(k.af2, HP, UF)));
+      const float2 PO = qadd(ONE, qex2(qfma(k.ao2, HP, UO)));
+      const float2 PG = qadd(ONE, qex2(qfma(k.ag2, HP, UG)));
+      I = qrcp(PI);
+      F = qrcp(PF);
+      O = qrcp(PO);
+      const float2 TG = qrcp(PG);                           // 1/(1+e^{2y})
       G = qfma(M2, TG, ONE);                                // tanh(y_g)
       CN = qfma(F, CP, qmul(I, G));
-      const float2 PC = qadd(ONE, qex2c(qmul(TL, CN)));
-      const float icn = rcp(PC.x * PC.y);
-      const float2 TC1 = qf2(PC.y * icn, PC.x * icn);
+      const float2 TC1 = qrcp(qadd(ONE, qex2(qmul(TL, CN))));
       TC = qfma(M2, TC1, ONE);                              // tanh(c')
       if constexpr (kMode != 2) {
         DG = qmul(TG, qfma(TG, M4, F4));                    // 1 - g^2 = 4t(1-t)
