@@ -45,26 +45,23 @@ struct ArCell {
 
 // The cell at a step pair: from the previous state HP and the pre-scaled
 // arguments UZ, UR, UC, the Jacobian A = df/dh and the pieces
-// GZ = df/du_z, GR = df/du_r, GC = df/du_c, RH = r h.
+// GZ = df/du_z, GR = df/du_r, GC = df/du_c, RH = r h.  Each sigmoid and the
+// tanh take their own ex2 and reciprocal, unclamped (a saturating argument
+// gives the gate's limit, a NaN stays NaN): 2% faster in the queue adjoint
+// than one reciprocal shared by a step pair's four sigmoids.
 __device__ __forceinline__ void ar_cell(const ArCell& k, float2 HP, float2 UZ, float2 UR,
                                         float2 UC, float2& A, float2& GZ, float2& GR,
                                         float2& GC, float2& RH) {
   const float2 ONE = af2(1.f, 1.f), M1 = af2(-1.f, -1.f), M2 = af2(-2.f, -2.f);
   const float2 F4 = af2(4.f, 4.f), M4 = af2(-4.f, -4.f);
   const float2 TZ = afma(k.AZ2, HP, UZ), TR = afma(k.AR2, HP, UR);
-  const float2 EZ = af2(ex2(fmin_nan(TZ.x, 31.f)), ex2(fmin_nan(TZ.y, 31.f)));
-  const float2 ER = af2(ex2(fmin_nan(TR.x, 31.f)), ex2(fmin_nan(TR.y, 31.f)));
-  const float2 PZ = aadd(ONE, EZ), PR = aadd(ONE, ER);
-  const float2 PP = amul(PZ, PR);
-  const float inv = rcp(PP.x * PP.y);
-  const float2 INV = af2(PP.y * inv, PP.x * inv);
-  const float2 Z = amul(PR, INV), R = amul(PZ, INV);
+  const float2 PZ = aadd(ONE, af2(ex2(TZ.x), ex2(TZ.y)));
+  const float2 PR = aadd(ONE, af2(ex2(TR.x), ex2(TR.y)));
+  const float2 Z = af2(rcp(PZ.x), rcp(PZ.y)), R = af2(rcp(PR.x), rcp(PR.y));
   RH = amul(R, HP);
   const float2 TC = afma(k.AC2, RH, UC);
-  const float2 EC = af2(ex2(fmin_nan(TC.x, 31.f)), ex2(fmin_nan(TC.y, 31.f)));
-  const float2 PC = aadd(ONE, EC);
-  const float ic = rcp(PC.x * PC.y);
-  const float2 TT = af2(PC.y * ic, PC.x * ic);
+  const float2 PC = aadd(ONE, af2(ex2(TC.x), ex2(TC.y)));
+  const float2 TT = af2(rcp(PC.x), rcp(PC.y));
   const float2 C = afma(M2, TT, ONE);                 // tanh
   const float2 CMH = afma(HP, M1, C);
   const float2 OMZ = afma(Z, M1, ONE);
