@@ -113,9 +113,9 @@ def test_bench_plan_follows_the_library_dispatch_rules():
     # fewer tiles than resident queue CTAs: the row kernel, launch by segment
     assert bench.fwd_plan(WORKLOADS[2].scaled(B=2), sms=148) == ("gru_newton_row", 3.75, 2048)
     assert bench.fwd_launches(WORKLOADS[2].scaled(B=2), sms=148) == 2
-    assert plan[3] == ("lstm_newton_queue", 6.5, 128)  # 1024 tiles >= 4 x 148
+    assert plan[3] == ("lstm_newton_queue", 10.0, 128)  # 1024 tiles >= 4 x 148
     assert plan[4] == ("gru_newton_row", 3.75, 4096)     # T > 4096, 256 tiles >= 148
-    assert plan[5] == ("lstm_newton_queue", 6.5, 128)  # 2048 tiles
+    assert plan[5] == ("lstm_newton_queue", 10.0, 128)  # 2048 tiles
     assert bench.fwd_launches(WORKLOADS[3], sms=148) == 1
     assert bench.fwd_plan(WORKLOADS[3].scaled(B=1, D=512), sms=148) == ("lstm_newton_row", 6.5, 2048)
     assert len(bench.fwd_segments(WORKLOADS[4], sms=148)) == 16
