@@ -43,8 +43,8 @@ NCU_TRAFFIC_BYTES = {
 }
 # Special-function (MUFU) work per element and cell evaluation.  The roofline
 # counts the cell in its plain form, the algorithmic figure: ParaGRU 3 exp + 3
-# reciprocals, ParaLSTM 5 exp + 5 reciprocals.  The kernels issue fewer, and
-# the second element of fwd_plan() is that issued count for an exact
+# reciprocals, ParaLSTM 5 exp + 5 reciprocals.  Most kernels issue fewer, and
+# the second element of fwd_plan() is the issued count for an exact
 # evaluation:
 #   gru_newton_queue (ParaGRU with bf16 u and at least one 8-channel tile per
 #     resident CTA, four CTAs per SM: every 512-step segment of every tile in
@@ -57,8 +57,8 @@ NCU_TRAFFIC_BYTES = {
 #   gru_newton_fused (ParaGRU otherwise): 3 ex2 + 2 rcp;
 #   lstm_newton_queue (ParaLSTM, bf16 u, at least one 8-channel tile per
 #     resident CTA, four CTAs per SM: every 128-step segment in one launch):
-#     5 ex2 + 1.5 rcp for an exact evaluation; the inexact early evaluations
-#     issue 5 tanh;
+#     5 ex2 + 5 rcp for an exact evaluation (one reciprocal per gate and per
+#     tanh(c')); the inexact early evaluations issue 5 tanh;
 #   lstm_newton_row (ParaLSTM, bf16 u, T <= 4096, in segments where
 #     smaller clusters fill the SMs): 5 ex2 + 1.5 rcp (one
 #     reciprocal per step pair for the six sigmoids, one for the two tanh(g),
